@@ -1,0 +1,463 @@
+"""Pins for the CPU oracle: each check ties it to something other than itself
+(brute-force enumeration, closed forms, independent library routines, values
+the pages state).  CPU only."""
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import scipy.special as sps
+import torch
+
+from oracle import oracle as O
+from mixture_experts_routing_top_b200 import synth, workloads as W
+
+RNG = np.random.default_rng(12345)
+
+
+# ---------------------------------------------------------------- top-k
+def _beats(la, ea, lb, eb):
+    """(logit desc, index asc): does expert ea beat expert eb?"""
+    return la > lb or (la == lb and ea < eb)
+
+
+@pytest.mark.parametrize("E", [1, 2, 3, 5, 8])
+def test_topk_matches_subset_enumeration(E):
+    # small integer logits make exact ties common
+    T = 150
+    logits = RNG.integers(-2, 3, size=(T, E)).astype(np.float32)
+    for k in range(1, E + 1):
+        idx, _ = O.route_topk(logits, k)
+        for t in range(T):
+            l = logits[t]
+            winners = [S for S in itertools.combinations(range(E), k)
+                       if all(_beats(l[a], a, l[b], b) for a in S for b in range(E) if b not in S)]
+            assert len(winners) == 1
+            S = winners[0]
+            assert set(idx[t].tolist()) == set(S)
+            # slot order: best first
+            for j in range(k - 1):
+                assert _beats(l[idx[t, j]], idx[t, j], l[idx[t, j + 1]], idx[t, j + 1])
+
+
+def test_topk_all_equal_logits():
+    T, E, k = 7, 6, 3
+    logits = np.full((T, E), 0.25, np.float32)
+    idx, gate = O.route_topk(logits, k)
+    assert (idx == np.arange(k)[None, :]).all()
+    np.testing.assert_allclose(gate, 1.0 / E, rtol=1e-7)
+    _, gate_n = O.route_topk(logits, k, norm_topk=True)
+    np.testing.assert_allclose(gate_n, 1.0 / k, rtol=1e-7)
+
+
+def test_gate_two_experts_is_logistic():
+    T = 64
+    logits = RNG.normal(size=(T, 2)).astype(np.float32) * 3
+    idx, gate = O.route_topk(logits, 2)
+    for t in range(T):
+        a, b = float(logits[t, idx[t, 0]]), float(logits[t, idx[t, 1]])
+        p = 1.0 / (1.0 + math.exp(b - a))
+        assert gate[t, 0] == pytest.approx(p, rel=1e-7)
+        assert gate[t, 1] == pytest.approx(1.0 - p, rel=1e-6)
+
+
+def test_gates_are_softmax_probabilities():
+    T, E, k = 300, 16, 4
+    logits = RNG.normal(size=(T, E)).astype(np.float32) * 2
+    idx, gate = O.route_topk(logits, k)
+    p = sps.softmax(logits.astype(np.float64), axis=1)
+    np.testing.assert_allclose(gate, np.take_along_axis(p, idx, 1), rtol=2e-7, atol=0)
+    _, gate_n = O.route_topk(logits, k, norm_topk=True)
+    sel = np.take_along_axis(p, idx, 1)
+    np.testing.assert_allclose(gate_n, sel / sel.sum(1, keepdims=True), rtol=2e-7, atol=0)
+    np.testing.assert_allclose(gate_n.astype(np.float64).sum(1), 1.0, atol=1e-6)
+    _, gate_all = O.route_topk(logits, E)
+    np.testing.assert_allclose(gate_all.astype(np.float64).sum(1), 1.0, atol=1e-6)
+
+
+def test_topk_rejects_bad_k():
+    with pytest.raises(ValueError):
+        O.route_topk(np.zeros((2, 4), np.float32), 5)
+
+
+# ------------------------------------------------------------- capacity
+def test_capacity_golden(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "capacity_factor.json")))
+    for c in g["cases"]:
+        assert c["T"] * c["k"] / c["E"] == c["average_load"]
+        assert O.capacity(c["capacity_factor"], c["T"], c["k"], c["E"]) == c["capacity"]
+
+
+@pytest.mark.parametrize("w", [W.TINY, W.MIXTRAL, W.FINE])
+def test_capacity_is_exact_ceiling(w):
+    q = Fraction(w.capacity_factor) * w.T * w.k / w.E
+    cap = O.capacity(w.capacity_factor, w.T, w.k, w.E)
+    assert cap - 1 < q <= cap
+    assert cap == {"tiny_fp32": 80, "mixtral_top2_bf16": 2560, "fine_top6_shared_bf16": 2304}[w.name]
+
+
+def test_capacity_unbounded():
+    assert O.capacity(0.0, 100, 3, 7) >= 300
+    assert O.capacity(-1.0, 100, 3, 7) >= 300
+
+
+# -------------------------------------------------------------- permute
+def _brute_ranks(idx):
+    flat = idx.reshape(-1)
+    seen = {}
+    ranks = np.empty(flat.size, np.int64)
+    for s, e in enumerate(flat):
+        ranks[s] = seen.get(e, 0)
+        seen[e] = ranks[s] + 1
+    return ranks.reshape(idx.shape)
+
+
+@pytest.mark.parametrize("T,E,k,cf", [(64, 4, 2, 0.5), (97, 8, 3, 1.0), (33, 3, 1, 0.7), (50, 6, 6, 0.0)])
+def test_drops_match_brute_force_rank(T, E, k, cf):
+    logits = RNG.normal(size=(T, E)).astype(np.float32)
+    logits[:, 0] += 1.5                       # skew the load so experts overflow
+    idx, _ = O.route_topk(logits, k)
+    cap = O.capacity(cf, T, k, E)
+    p = O.permute(idx, E, cap)
+    ranks = _brute_ranks(idx)
+    assert ((p["row_map"] < 0) == (ranks >= cap)).all()
+    load = np.bincount(idx.reshape(-1), minlength=E)
+    assert (p["load"] == load).all()
+    assert (p["counts"] == np.minimum(load, cap)).all()
+    assert (p["counts"] <= cap).all()
+    assert p["counts"].sum() + p["dropped"] == T * k
+    assert p["R"] == p["counts"].sum()
+    if cf > 0 and cf < 1:
+        assert p["dropped"] > 0
+
+
+def test_expert_major_layout_and_round_trip():
+    T, E, k, d = 120, 5, 1, 9
+    logits = RNG.normal(size=(T, E)).astype(np.float32)
+    logits[:, 2] += 1.0
+    idx, _ = O.route_topk(logits, k)
+    cap = O.capacity(1.0, T, k, E)
+    p = O.permute(idx, E, cap)
+    off, rt = p["offsets"], p["row_token"]
+    assert off[0] == 0 and (np.diff(off) == p["counts"]).all()
+    for e in range(E):
+        toks = rt[off[e]:off[e + 1]]
+        assert (np.diff(toks) > 0).all()                      # ascending token order
+        assert (idx[toks, 0] == e).all()
+    x = RNG.normal(size=(T, d)).astype(np.float32)
+    buf = O.gather_rows(x, rt)
+    for r in range(p["R"]):
+        assert buf[r].tobytes() == x[rt[r]].tobytes()
+    # identity experts, unit gates: unpermute(permute(x)) == x for kept tokens, 0 for dropped
+    y = O.unpermute(buf, p["row_map"], np.ones((T, k), np.float32))
+    kept = p["row_map"][:, 0] >= 0
+    assert (y[kept] == x[kept].astype(np.float64)).all()
+    assert (y[~kept] == 0).all()
+    assert (~kept).sum() == p["dropped"] > 0
+
+
+@pytest.mark.parametrize("cf", [0.0, 0.6])
+def test_group_major_with_identity_groups_is_expert_major(cf):
+    T, E, k = 80, 6, 2
+    idx, _ = O.route_topk(RNG.normal(size=(T, E)).astype(np.float32), k)
+    cap = O.capacity(cf, T, k, E)
+    a = O.permute(idx, E, cap)
+    b = O.permute(idx, E, cap, group_of_expert=np.arange(E, dtype=np.int32))
+    for key in ("row_map", "row_token", "counts", "offsets", "dropped", "R"):
+        assert np.array_equal(np.asarray(a[key]), np.asarray(b[key])), key
+
+
+@pytest.mark.parametrize("G,cf", [(2, 0.0), (4, 0.0), (4, 0.8), (8, 1.0)])
+def test_group_major_matches_distinct_pairs(G, cf):
+    T, E, k = 90, 8, 3
+    idx, _ = O.route_topk(RNG.normal(size=(T, E)).astype(np.float32), k)
+    goe = W.equal_groups(E, G)
+    cap = O.capacity(cf, T, k, E)
+    p = O.permute(idx, E, cap, group_of_expert=goe)
+    kept = _brute_ranks(idx) < cap
+    pairs = sorted({(int(goe[idx[t, j]]), t) for t in range(T) for j in range(k) if kept[t, j]})
+    assert p["R"] == len(pairs)
+    row_of = {pair: r for r, pair in enumerate(pairs)}
+    assert [t for _, t in pairs] == p["row_token"].tolist()
+    for t in range(T):
+        for j in range(k):
+            want = row_of[(int(goe[idx[t, j]]), t)] if kept[t, j] else -1
+            assert p["row_map"][t, j] == want
+    starts = [next((r for r, (g, _) in enumerate(pairs) if g == gg), None) for gg in range(G)]
+    for gg in range(G):
+        n_g = sum(1 for g, _ in pairs if g == gg)
+        assert p["offsets"][gg + 1] - p["offsets"][gg] == n_g
+        if n_g:
+            assert p["offsets"][gg] == starts[gg]
+
+
+def _expected_group_rows_per_slot(E, k, G):
+    L = E // G
+    return G * (1.0 - math.comb(E - L, k) / math.comb(E, k)) / k
+
+
+@pytest.mark.parametrize("G,expected", [(8, 0.662), (32, 0.908), (64, 0.959)])
+def test_group_major_row_count_under_uniform_routing(G, expected):
+    E, k, T = 256, 8, 4096
+    assert _expected_group_rows_per_slot(E, k, G) == pytest.approx(expected, abs=1e-3)
+    logits = synth.normal_f32(7, 1, (T, E))
+    idx, _ = O.route_topk(logits, k)
+    p = O.permute(idx, E, O.capacity(0.0, T, k, E), group_of_expert=W.equal_groups(E, G))
+    ratio = p["R"] / (T * k)
+    # per-token row count has std < sqrt(k)/2 rows; 4 sigma over T tokens
+    tol = 4 * (math.sqrt(k) / 2) / math.sqrt(T) / k
+    assert abs(ratio - _expected_group_rows_per_slot(E, k, G)) < tol
+
+
+def test_local_fraction_golden(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "local_fraction.json")))
+    for c in g["cases"]:
+        E, G = c["E"], c["G"]
+        assert E // G == c["L"]
+        T, k = 20000, 2
+        idx, _ = O.route_topk(synth.normal_f32(3, 1, (T, E)), k)
+        f = O.local_fraction(idx, W.equal_groups(E, G), G)
+        # binomial standard error over T*k slots (slots of one token are dependent: use T)
+        tol = 4 * math.sqrt(c["expected_local_fraction"] * (1 - c["expected_local_fraction"]) / T)
+        assert abs(f - c["expected_local_fraction"]) < tol
+
+
+def test_local_fraction_extremes():
+    T, E, G = 40, 4, 2
+    goe = W.equal_groups(E, G)
+    home = (np.arange(T) * G) // T
+    idx = (home * 2).astype(np.int32)[:, None]           # every token in its home group
+    assert O.local_fraction(idx, goe, G) == 1.0
+    idx = ((1 - home) * 2).astype(np.int32)[:, None]     # every token away
+    assert O.local_fraction(idx, goe, G) == 0.0
+
+
+# ------------------------------------------------------------------ FFN
+def test_activation_values():
+    assert O.silu(0.0) == 0.0
+    assert O.gelu(0.0) == 0.0
+    assert O.gelu(1.0) == pytest.approx(0.8413447460685429, rel=1e-15)   # Phi(1)
+    for z in (-3.1, -0.4, 0.7, 2.5, 9.0):
+        assert O.silu(z) - O.silu(-z) == pytest.approx(z, abs=1e-14)
+        assert O.gelu(-z) == pytest.approx(O.gelu(z) - z, abs=1e-14)
+        assert O.silu(z) == pytest.approx(z * sps.expit(z), rel=1e-14)
+        assert O.gelu(z) == pytest.approx(z * sps.ndtr(z), rel=1e-13, abs=1e-300)
+
+
+def test_round_bf16():
+    assert O.round_bf16(1.0 + 2 ** -8) == 1.0                       # tie -> even
+    assert O.round_bf16(1.0 + 3 * 2 ** -8) == 1.0 + 2 ** -6          # tie -> even (up)
+    assert O.round_bf16(1.0 + 2 ** -8 + 2 ** -30) == 1.0 + 2 ** -7   # just above the tie
+    assert O.round_bf16(1.0 / 3.0) == 0.333984375
+    assert O.round_bf16(-2.0 ** -130) == -(2.0 ** -130)              # subnormal, exact
+    vals = RNG.normal(size=5000).astype(np.float32) * np.float32(10.0) ** RNG.integers(-30, 30, 5000).astype(np.float32)
+    ref = torch.from_numpy(vals).to(torch.bfloat16).to(torch.float64).numpy()
+    got = np.array([O.round_bf16(float(v)) for v in vals])
+    assert np.array_equal(got, ref)
+
+
+def test_ffn_scalar_closed_form():
+    x = np.array([[1.5], [-0.75]], np.float32)
+    W1 = np.array([[[0.5]], [[-2.0]]], np.float32)
+    W3 = np.array([[[3.0]], [[0.25]]], np.float32)
+    W2 = np.array([[[-1.25]], [[4.0]]], np.float32)
+    for e in (0, 1):
+        y = O.expert_ffn_rows(x, np.array([e, e], np.int32), W1, W3, W2)
+        for i in range(2):
+            a = float(W1[e, 0, 0] * x[i, 0])
+            want = float(W2[e, 0, 0]) * (a / (1 + math.exp(-a))) * float(W3[e, 0, 0] * x[i, 0])
+            assert y[i, 0] == pytest.approx(want, rel=1e-15)
+        yg = O.expert_ffn_rows(x, np.array([e, e], np.int32), W1, None, W2, act="gelu")
+        for i in range(2):
+            a = float(W1[e, 0, 0] * x[i, 0])
+            assert yg[i, 0] == pytest.approx(float(W2[e, 0, 0]) * a * sps.ndtr(a), rel=1e-13)
+
+
+def test_ffn_one_hot_rows_pick_columns():
+    E, F, d = 3, 5, 4
+    W1 = RNG.normal(size=(E, F, d)).astype(np.float32)
+    W3 = RNG.normal(size=(E, F, d)).astype(np.float32)
+    W2 = RNG.normal(size=(E, d, F)).astype(np.float32)
+    for e in range(E):
+        for c in range(d):
+            x = np.zeros((1, d), np.float32)
+            x[0, c] = 1.0
+            y = O.expert_ffn_rows(x, np.array([e], np.int32), W1, W3, W2)[0]
+            a, b = W1[e, :, c].astype(np.float64), W3[e, :, c].astype(np.float64)
+            h = a * sps.expit(a) * b
+            np.testing.assert_allclose(y, W2[e].astype(np.float64) @ h, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("act", ["swiglu", "gelu"])
+def test_ffn_matches_float64_matmul(act):
+    E, F, d, n = 4, 24, 16, 30
+    x = RNG.normal(size=(n, d)).astype(np.float32)
+    W1 = RNG.normal(size=(E, F, d)).astype(np.float32) * 0.3
+    W3 = RNG.normal(size=(E, F, d)).astype(np.float32) * 0.3
+    W2 = RNG.normal(size=(E, d, F)).astype(np.float32) * 0.3
+    re = RNG.integers(0, E, n).astype(np.int32)
+    y = O.expert_ffn_rows(x, re, W1, W3 if act == "swiglu" else None, W2, act=act)
+    for i in range(n):
+        xe = x[i].astype(np.float64)
+        a = W1[re[i]].astype(np.float64) @ xe
+        h = a * sps.expit(a) * (W3[re[i]].astype(np.float64) @ xe) if act == "swiglu" else a * sps.ndtr(a)
+        np.testing.assert_allclose(y[i], W2[re[i]].astype(np.float64) @ h, rtol=1e-11, atol=1e-13)
+
+
+def test_ffn_bf16_rounds_hidden_and_output():
+    # small integers: every product and sum before the nonlinearity is exact
+    E, F, d, n = 2, 6, 8, 5
+    x = synth.f32_to_bf16(RNG.integers(-3, 4, (n, d)).astype(np.float32))
+    W1 = synth.f32_to_bf16(RNG.integers(-2, 3, (E, F, d)).astype(np.float32) * 0.25)
+    W3 = synth.f32_to_bf16(RNG.integers(-2, 3, (E, F, d)).astype(np.float32) * 0.25)
+    W2 = synth.f32_to_bf16(RNG.integers(-2, 3, (E, d, F)).astype(np.float32) * 0.25)
+    re = np.array([0, 1, 1, 0, 1], np.int32)
+    y = O.expert_ffn_rows(x, re, W1, W3, W2)
+    f = lambda a: synth.bf16_to_f32(a).astype(np.float64)
+    for i in range(n):
+        a = f(W1)[re[i]] @ f(x)[i]
+        b = f(W3)[re[i]] @ f(x)[i]
+        h = np.array([O.round_bf16(v) for v in a * sps.expit(a) * b])
+        want = np.array([O.round_bf16(v) for v in f(W2)[re[i]] @ h])
+        np.testing.assert_allclose(y[i], want, rtol=1e-15, atol=0)
+        # every value is a bf16 number
+        assert np.array_equal(y[i], synth.bf16_to_f32(synth.f32_to_bf16(y[i].astype(np.float32))))
+
+
+# -------------------------------------------------------------- combine
+def test_combine_identity_experts_closed_form():
+    T, E, k, d = 70, 6, 3, 5
+    logits = RNG.normal(size=(T, E)).astype(np.float32)
+    logits[:, 1] += 1.0
+    idx, gate = O.route_topk(logits, k)
+    cap = O.capacity(0.8, T, k, E)
+    p = O.permute(idx, E, cap)
+    x = RNG.normal(size=(T, d)).astype(np.float32)
+    y = O.unpermute(O.gather_rows(x, p["row_token"]), p["row_map"], gate)
+    kept_gate = np.where(p["row_map"] >= 0, gate.astype(np.float64), 0.0).sum(1)
+    np.testing.assert_allclose(y, kept_gate[:, None] * x.astype(np.float64), rtol=1e-15, atol=0)
+    sh = RNG.normal(size=(T, d)).astype(np.float32)
+    y2 = O.unpermute(O.gather_rows(x, p["row_token"]), p["row_map"], gate, shared=sh)
+    np.testing.assert_allclose(y2, y + sh.astype(np.float64), rtol=1e-15, atol=1e-15)
+
+
+def test_combine_group_major_identity_experts():
+    T, E, k, d, G = 60, 8, 4, 3, 4
+    idx, gate = O.route_topk(RNG.normal(size=(T, E)).astype(np.float32), k, norm_topk=True)
+    p = O.permute(idx, E, O.capacity(0.0, T, k, E), group_of_expert=W.equal_groups(E, G))
+    x = RNG.normal(size=(T, d)).astype(np.float32)
+    y = O.unpermute(O.gather_rows(x, p["row_token"]), p["row_map"], gate)
+    # renormalised gates sum to 1 and nothing is dropped: y == x
+    np.testing.assert_allclose(y, x.astype(np.float64), rtol=1e-6, atol=1e-7)
+
+
+# --------------------------------------------------------- expert choice
+@pytest.mark.parametrize("T,E,C", [(40, 4, 10), (33, 5, 33), (25, 3, 1)])
+def test_expert_choice_matches_sort(T, E, C):
+    logits = RNG.normal(size=(T, E)).astype(np.float32)
+    ec_token, ec_gate, tok_ptr, tok_row = O.route_ec(logits, C)
+    p = sps.softmax(logits.astype(np.float64), axis=1)
+    for e in range(E):
+        order = np.lexsort((np.arange(T), -p[:, e]))        # prob desc, token asc
+        want = np.sort(order[:C])
+        assert (ec_token[e] == want).all()
+        np.testing.assert_allclose(ec_gate[e], p[want, e], rtol=1e-6)
+    assert tok_ptr[0] == 0 and tok_ptr[-1] == E * C
+    assert sorted(tok_row.tolist()) == list(range(E * C))
+    for t in range(T):
+        rows = tok_row[tok_ptr[t]:tok_ptr[t + 1]]
+        assert (np.diff(rows // C) > 0).all()               # ascending expert
+        assert all(ec_token.reshape(-1)[r] == t for r in rows)
+        assert len(rows) == sum(t in set(ec_token[e].tolist()) for e in range(E))
+
+
+def test_expert_choice_ties_prefer_lower_token():
+    T, E, C = 12, 2, 5
+    logits = np.zeros((T, E), np.float32)                    # all scores equal
+    ec_token, ec_gate, _, _ = O.route_ec(logits, C)
+    assert (ec_token == np.arange(C)[None, :]).all()
+    np.testing.assert_allclose(ec_gate, 0.5, rtol=1e-7)
+
+
+def test_expert_choice_combine():
+    T, E, C, d = 30, 4, 9, 6
+    logits = RNG.normal(size=(T, E)).astype(np.float32)
+    ec_token, ec_gate, tok_ptr, tok_row = O.route_ec(logits, C)
+    x = RNG.normal(size=(T, d)).astype(np.float32)
+    Y = O.gather_rows(x, ec_token.reshape(-1))               # identity experts
+    y = O.unpermute_ec(Y, tok_ptr, tok_row, ec_gate)
+    gsum = np.zeros(T)
+    for e in range(E):
+        for i in range(C):
+            gsum[ec_token[e, i]] += ec_gate[e, i]
+    np.testing.assert_allclose(y, gsum[:, None] * x.astype(np.float64), rtol=1e-14, atol=1e-15)
+
+
+# ------------------------------------------------------------ histograms
+@pytest.mark.parametrize("E,k", [(8, 2), (16, 6), (5, 5)])
+def test_coselect_properties_and_brute_force(E, k):
+    T = 200
+    idx, _ = O.route_topk(RNG.normal(size=(T, E)).astype(np.float32), k)
+    C = O.coselect(idx, E)
+    assert (C == C.T).all()
+    load = np.bincount(idx.reshape(-1), minlength=E)
+    assert (np.diag(C) == load).all()
+    off = C - np.diag(np.diag(C))
+    assert off.sum() == T * k * (k - 1)
+    assert (off.sum(1) == (k - 1) * load).all()
+    want = np.zeros((E, E), np.int64)
+    for t in range(T):
+        s = set(idx[t].tolist())
+        for a in range(E):
+            for b in range(E):
+                want[a, b] += (a in s) and (b in s)
+    assert (C == want).all()
+    C2 = O.coselect(idx, E, into=C.copy())                   # accumulates
+    assert (C2 == 2 * C).all()
+
+
+def test_transition_properties_and_brute_force():
+    T, E = 300, 12
+    for k1, k2 in ((1, 1), (2, 3)):
+        i1, _ = O.route_topk(RNG.normal(size=(T, E)).astype(np.float32), k1)
+        i2, _ = O.route_topk(RNG.normal(size=(T, E)).astype(np.float32), k2)
+        M = O.transition(i1, i2, E)
+        assert M.sum() == T * k1 * k2
+        assert (M.sum(1) == k2 * np.bincount(i1.reshape(-1), minlength=E)).all()
+        assert (M.sum(0) == k1 * np.bincount(i2.reshape(-1), minlength=E)).all()
+        want = np.zeros((E, E), np.int64)
+        for t in range(T):
+            for a in i1[t]:
+                for b in i2[t]:
+                    want[a, b] += 1
+        assert (M == want).all()
+
+
+def test_transition_detects_correlation():
+    # layer-2 logits built from layer-1's top-1: the transition matrix is
+    # concentrated (its top entry per row holds far more than 1/E of the row)
+    w = W.EXPERT_CHOICE.with_(T=4096)
+    l1 = W.make_logits(w)
+    l2 = W.make_layer2_logits(w, l1)
+    a, _ = O.route_topk(l1, 1)
+    b, _ = O.route_topk(l2, 1)
+    M = O.transition(a, b, w.E)
+    rows = M.sum(1)
+    nz = rows > 0
+    assert (M.max(1)[nz] / rows[nz]).mean() > 5.0 / w.E
+
+
+# ---------------------------------------------------------------- inputs
+def test_generator_deterministic_and_distribution():
+    a = synth.normal_f32(0, 1, (1000, 37))
+    b = synth.normal_f32(0, 1, (1000, 37))
+    assert a.tobytes() == b.tobytes()
+    assert abs(a.mean()) < 0.01 and abs(a.std() - 1) < 0.01
+    c = synth.normal_f32(0, 1, (500, 37))                    # prefix property
+    assert c.tobytes() == a[:500].tobytes()
+    h = synth.normal_bf16(0, 1, (1000, 37))
+    assert np.array_equal(h, synth.f32_to_bf16(a))
+    assert not np.array_equal(synth.u64(0, 1, 10), synth.u64(0, 2, 10))
