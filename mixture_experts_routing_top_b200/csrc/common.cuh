@@ -1,0 +1,89 @@
+// common.cuh - small helpers shared by the libmoe kernels (sm_100a).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/libmoe.h"
+
+namespace moe {
+
+// Device fault word bits (see moe_device_error).
+constexpr unsigned kErrTimeout = 1u;
+constexpr unsigned kErrIndex = 2u;
+
+// Address of the current device's fault word (defined in api.cu).
+unsigned* device_error_word();
+
+// Counts kernel launches made by the library (moe_kernel_launches).
+void count_launch();
+
+__device__ __forceinline__ void raise_error(unsigned* err, unsigned bits) {
+    if (err) atomicOr(err, bits);
+}
+
+__device__ __forceinline__ unsigned lane_id() {
+    unsigned r;
+    asm volatile("mov.u32 %0, %%laneid;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ unsigned lanemask_lt() {
+    unsigned r;
+    asm volatile("mov.u32 %0, %%lanemask_lt;" : "=r"(r));
+    return r;
+}
+
+// 16-byte vector loads/stores.  Inputs read once take the non-coherent path
+// without allocating in L1; outputs are written with the streaming (.cs)
+// hint so a large copy does not flush useful lines from L2.
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint4 ld_keep(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void st_stream(uint4* p, uint4 v) {
+    asm volatile("st.global.cs.v4.u32 [%0], {%1,%2,%3,%4};"
+                 :: "l"(p), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w) : "memory");
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Round-to-nearest-even packing of two floats into a bf16x2 word (lo first).
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+template <typename T>
+__device__ __forceinline__ T warp_sum(T v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+}  // namespace moe
+
+// Launch-error check used right after each kernel launch in host code;
+// also counts the launch.
+#define MOE_LAUNCH_CHECK()                                  \
+    do {                                                    \
+        moe::count_launch();                                \
+        if (cudaPeekAtLastError() != cudaSuccess) {         \
+            (void)cudaGetLastError();                       \
+            return MOE_ERR_CUDA;                            \
+        }                                                   \
+    } while (0)

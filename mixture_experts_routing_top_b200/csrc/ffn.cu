@@ -1,0 +1,578 @@
+// ffn.cu - the grouped expert MLP ("MoELayer" step 2 of "How MegaDLMs
+// Implements Mixture of Experts (MoE) Architectures": each expert held on
+// the device runs its MLP on the rows routed to it).
+//
+// bf16: two persistent tcgen05 grouped GEMMs per call.
+//   GEMM1  H[r, :] = act(X[r] W1[e]^T (, X[r] W3[e]^T))   (bf16 H in workspace)
+//   GEMM2  Y[r, :] = H[r] W2[e]^T
+// Each CTA owns one SM: a TMA warp streams 128x64 A tiles and 256x64 B tiles
+// (128-byte swizzle) into a 4-stage shared-memory ring; one thread issues
+// tcgen05.mma (M=128, N=256, K=16, bf16 in, fp32 accumulate in TMEM); four
+// epilogue warps drain the accumulator with tcgen05.ld, apply the
+// activation and store bf16.  Two TMEM accumulators (2 x 256 columns) let
+// the epilogue of one tile overlap the MMAs of the next.  For SwiGLU the B
+// tile stacks 128 rows of W1 over the same 128 rows of W3, so one MMA chain
+// yields both projections and silu(a) * b is formed in registers.
+//
+// Ragged experts: offsets[] stays on the device.  Every CTA derives the
+// per-expert tile counts from it at start; tile t -> (expert, n-tile,
+// m-tile), m fastest, so CTAs working at the same time share weight tiles
+// through L2.  Rows of a 128-row tile past the expert's end belong to the
+// next expert or lie past the buffer (TMA fills zeros); the epilogue never
+// stores them.
+//
+// Every wait on an mbarrier is bounded (a few seconds of %globaltimer):
+// on expiry the CTA records MOE_ERR_TIMEOUT in the device fault word, all
+// roles leave their loops, and TMEM is still freed.
+//
+// fp32: a plain FMA kernel pair for small fp32 layers (no fp32-input
+// tensor-core kind keeps fp32 accuracy).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace moe {
+namespace tc {
+
+constexpr int BM = 128;              // rows per tile (TMEM lanes)
+constexpr int BK = 64;               // K per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int ACC_N = 256;           // accumulator columns per tile
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;         // 16 KB
+constexpr int B_BYTES = ACC_N * BK * 2;      // 32 KB
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int THREADS = 192;                 // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int MAX_E = 1024;
+constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/ + 4 * (MAX_E + 1);
+constexpr long long WAIT_NS = 4000000000LL;  // 4 s
+
+enum { MODE_SWIGLU = 0, MODE_GELU = 1, MODE_PLAIN = 2 };
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ long long globaltimer() {
+    long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+
+// Bounded parity wait.  Returns false on timeout or when another role of
+// this CTA has already given up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag) {
+    long long t0 = 0;
+    for (uint32_t i = 1;; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+        if (done) return true;
+        if ((i & 255u) == 0) {
+            if (*abort_flag) return false;
+            const long long now = globaltimer();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > WAIT_NS) return false;
+        }
+    }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// UMMA shared-memory descriptor: K-major operand, 128-byte swizzle, rows
+// of 128 bytes, 8-row groups 1024 bytes apart (SBO), LBO 16 bytes,
+// descriptor version 1.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t addr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;                    // LBO = 16 B
+    d |= (uint64_t)(1024u >> 4) << 32;          // SBO = 1024 B
+    d |= (uint64_t)1u << 46;                    // version
+    d |= (uint64_t)2u << 61;                    // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor, kind::f16: D fp32, A/B bf16, both K-major, M x N.
+__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc) : "memory");
+}
+
+// Arrives on `bar` once every tcgen05.mma issued so far by this thread is done.
+__device__ __forceinline__ void umma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 lanes x 32 consecutive fp32 columns: thread = lane (row), v[i] = column i.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
+__device__ __forceinline__ float gelu_f(float z) { return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f)); }
+
+// Store 32 consecutive bf16 values (64 bytes) of one output row.
+__device__ __forceinline__ void store_row32(uint16_t* dst, const float* v) {
+    uint4* p = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+        w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+        w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+        w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+        p[q] = w;
+    }
+}
+
+struct GemmArgs {
+    const int32_t* offsets;   // [E+1] device
+    int E;
+    int K;                    // reduction length (multiple of 64)
+    int N_out;                // output columns (multiple of 32)
+    int w_rows;               // rows per expert in the B tensor(s)
+    int R_max;                // rows of A / out
+    uint16_t* out;            // bf16 [R_max, N_out]
+    unsigned* err;
+};
+
+template <int MODE>
+__global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
+                                                                  const __grid_constant__ CUtensorMap map_b0,
+                                                                  const __grid_constant__ CUtensorMap map_b1,
+                                                                  GemmArgs args) {
+    constexpr int BN_OUT = (MODE == MODE_SWIGLU) ? 128 : 256;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t* stage_base = smem;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* full = bars;                     // [STAGES]
+    uint64_t* empty = bars + STAGES;           // [STAGES]
+    uint64_t* tfull = bars + 2 * STAGES;       // [2]
+    uint64_t* tempty = bars + 2 * STAGES + 2;  // [2]
+    uint64_t* drain = bars + 2 * STAGES + 4;   // [1] MMA completion before TMEM is freed
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* tile_prefix = reinterpret_cast<int*>(smem + STAGES * STAGE_BYTES + 256);   // [E+1]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int E = args.E;
+    const int n_tiles = (args.N_out + BN_OUT - 1) / BN_OUT;
+    const int nk = args.K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), 128);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&map_a);
+        tma_prefetch_desc(&map_b0);
+        if (MODE == MODE_SWIGLU) tma_prefetch_desc(&map_b1);
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(tmem_slot)), "r"(2 * ACC_N) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (warp == 2 && lane == 0) {
+        int acc = 0;
+        tile_prefix[0] = 0;
+        for (int e = 0; e < E; ++e) {
+            int b = min(max(args.offsets[e], 0), args.R_max);
+            int en = min(max(args.offsets[e + 1], 0), args.R_max);
+            int cnt = max(en - b, 0);
+            acc += ((cnt + BM - 1) / BM) * n_tiles;
+            tile_prefix[e + 1] = acc;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = tile_prefix[E];
+
+    // tile -> expert, row range, n offset
+    auto decode = [&](int t, int& row0, int& row_end, int& brow, int& n0) {
+        int lo = 0, hi = E;
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (tile_prefix[mid] <= t) lo = mid; else hi = mid - 1;
+        }
+        const int e = lo;
+        const int b = min(max(args.offsets[e], 0), args.R_max);
+        const int en = min(max(args.offsets[e + 1], 0), args.R_max);
+        const int mt = (en - b + BM - 1) / BM;
+        const int local = t - tile_prefix[e];
+        const int n_idx = local / mt, m_idx = local - n_idx * mt;
+        row0 = b + m_idx * BM;
+        row_end = en;
+        n0 = n_idx * BN_OUT;
+        brow = e * args.w_rows + n0;
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, fill_parity = 0;     // per stage: any fill issued, parity of the last one
+            for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x) {
+                int row0, row_end, brow, n0;
+                decode(t, row0, row_end, brow, n0);
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) {
+                        *abort_flag = 1;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full[stage]);
+                    const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+                    const uint32_t sb = sa + A_BYTES;
+                    mbar_expect_tx(fb, STAGE_BYTES);
+                    issued |= 1u << stage;
+                    fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+                    tma_load_2d(sa, &map_a, kb * BK, row0, fb);
+                    if (MODE == MODE_SWIGLU) {
+                        tma_load_2d(sb, &map_b0, kb * BK, brow, fb);
+                        tma_load_2d(sb + B_BYTES / 2, &map_b1, kb * BK, brow, fb);
+                    } else {
+                        tma_load_2d(sb, &map_b0, kb * BK, brow, fb);
+                    }
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // every issued fill has landed before the CTA may exit (immediate
+            // on the normal path: the MMA thread consumed them all)
+            int never = 0;
+            for (int st = 0; st < STAGES; ++st)
+                if (issued & (1u << st)) mbar_wait(smem_u32(&full[st]), (fill_parity >> st) & 1u, &never);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16(BM, ACC_N);
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            for (int t = blockIdx.x; t < total && !*abort_flag; t += gridDim.x, ++it) {
+                const int acc = it & 1;
+                const uint32_t acc_phase = (it >> 1) & 1;
+                if (!mbar_wait(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag)) { *abort_flag = 1; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * ACC_N;
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&full[stage]), phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+                    const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        umma_bf16(d_tmem, umma_desc_sw128(sa + kk * 32), umma_desc_sw128(sb + kk * 32), idesc,
+                                  (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(smem_u32(&empty[stage]));
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) { *abort_flag = 1; break; }
+                umma_commit(smem_u32(&tfull[acc]));
+            }
+            // no tcgen05.mma of this CTA may still be running when TMEM is freed
+            umma_commit(smem_u32(drain));
+            int never = 0;
+            if (!mbar_wait(smem_u32(drain), 0, &never)) *abort_flag = 1;
+        }
+    } else {
+        // epilogue: warps 2..5 -> TMEM lane quarter (warp % 4)
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        int it = 0;
+        for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
+            int row0, row_end, brow, n0;
+            decode(t, row0, row_end, brow, n0);
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag)) { *abort_flag = 1; break; }
+            tc_fence_after();
+            const int grow = row0 + r;
+            const bool valid = grow < row_end;
+            const uint32_t taddr = tmem_base + acc * ACC_N + ((uint32_t)(q * 32) << 16);
+            uint16_t* orow = args.out + (long long)grow * args.N_out;
+            if (MODE == MODE_SWIGLU) {
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float a[32], b[32];
+                    tmem_ld32(taddr + c * 32, a);
+                    tmem_ld32(taddr + 128 + c * 32, b);
+                    tmem_ld_wait();
+                    const int col = n0 + c * 32;
+                    if (valid && col < args.N_out) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) a[i] = silu_f(a[i]) * b[i];
+                        store_row32(orow + col, a);
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                    float a[32];
+                    tmem_ld32(taddr + c * 32, a);
+                    tmem_ld_wait();
+                    const int col = n0 + c * 32;
+                    if (valid && col < args.N_out) {
+                        if (MODE == MODE_GELU) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) a[i] = gelu_f(a[i]);
+                        }
+                        store_row32(orow + col, a);
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(smem_u32(&tempty[acc]));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag && threadIdx.x == 0) raise_error(args.err, kErrTimeout);
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem_base), "r"(2 * ACC_N) : "memory");
+    }
+}
+
+}  // namespace tc
+
+// ------------------------------------------------------------- fp32 SIMT
+// H[r, f] = act(x_r . W1[e, f] (, x_r . W3[e, f])), one thread per (r, f);
+// Y[r, c] = H[r] . W2[e, c], one thread per (r, c).  e from offsets.
+__device__ __forceinline__ int expert_of_row(const int32_t* __restrict__ offsets, int E, int r) {
+    int lo = 0, hi = E - 1;
+    while (lo < hi) {
+        int mid = (lo + hi + 1) >> 1;
+        if (offsets[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+}
+
+__global__ void ffn_f32_hidden_kernel(const float* __restrict__ x, int d, int F, int E, const int32_t* __restrict__ offsets,
+                                      int R_max, const float* __restrict__ W1, const float* __restrict__ W3, int act,
+                                      float* __restrict__ H) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int R = min(offsets[E], R_max);
+    if (i >= (long long)R * F) return;
+    const int r = (int)(i / F), f = (int)(i % F);
+    if (r < offsets[0]) return;
+    const int e = expert_of_row(offsets, E, r);
+    const float* xr = x + (long long)r * d;
+    const float* w1 = W1 + ((long long)e * F + f) * d;
+    float a = 0.0f;
+    for (int c = 0; c < d; ++c) a = __fmaf_rn(w1[c], xr[c], a);
+    float h;
+    if (act == MOE_ACT_SWIGLU) {
+        const float* w3 = W3 + ((long long)e * F + f) * d;
+        float b = 0.0f;
+        for (int c = 0; c < d; ++c) b = __fmaf_rn(w3[c], xr[c], b);
+        h = tc::silu_f(a) * b;
+    } else {
+        h = tc::gelu_f(a);
+    }
+    H[i] = h;
+}
+
+__global__ void ffn_f32_out_kernel(const float* __restrict__ H, int d, int F, int E, const int32_t* __restrict__ offsets,
+                                   int R_max, const float* __restrict__ W2, float* __restrict__ y) {
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int R = min(offsets[E], R_max);
+    if (i >= (long long)R * d) return;
+    const int r = (int)(i / d), c = (int)(i % d);
+    if (r < offsets[0]) return;
+    const int e = expert_of_row(offsets, E, r);
+    const float* hr = H + (long long)r * F;
+    const float* w2 = W2 + ((long long)e * d + c) * F;
+    float acc = 0.0f;
+    for (int f = 0; f < F; ++f) acc = __fmaf_rn(w2[f], hr[f], acc);
+    y[i] = acc;
+}
+
+// --------------------------------------------------------------- host side
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::mutex g_encode_mu;
+
+bool get_encoder() {
+    std::lock_guard<std::mutex> lk(g_encode_mu);
+    if (g_encode) return true;
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || !fn)
+        return false;
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    return true;
+}
+
+// 2-D bf16 tensor [rows, K] (K contiguous), box = 64 x box_rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, long long rows, int K, int box_rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)tc::BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (n <= 0) n = 148;
+    }
+    return n;
+}
+
+template <int MODE>
+moe_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, const tc::GemmArgs& a,
+                       cudaStream_t s) {
+    static bool attr_done = false;
+    if (!attr_done) {
+        if (cudaFuncSetAttribute(tc::grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc::SMEM_BYTES) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_done = true;
+    }
+    const int bn_out = MODE == tc::MODE_SWIGLU ? 128 : 256;
+    const long long n_tiles = (a.N_out + bn_out - 1) / bn_out;
+    const long long m_tiles_max = (a.R_max + tc::BM - 1) / tc::BM + a.E;
+    long long tiles_max = n_tiles * m_tiles_max;
+    int grid = sm_count();
+    if (tiles_max < grid) grid = (int)(tiles_max > 0 ? tiles_max : 1);
+    tc::grouped_gemm_kernel<MODE><<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(ma, mb0, mb1, a);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" size_t moe_expert_ffn_workspace_bytes(int R_max, int d, int F, int dtype) {
+    (void)d;
+    if (R_max < 0 || F < 1) return 0;
+    const size_t esz = dtype == MOE_BF16 ? 2 : 4;
+    return al256((size_t)R_max * F * esz) + 256;
+}
+
+extern "C" moe_status moe_expert_ffn(const void* buffer, int dtype, int R_max, int d, int F, int E,
+                                     const int32_t* offsets, const void* W1, const void* W3, const void* W2, int act,
+                                     void* y, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+    if (R_max < 0 || d < 1 || F < 1 || E < 1) return MOE_ERR_ARG;
+    if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_ARG;
+    if (act != MOE_ACT_SWIGLU && act != MOE_ACT_GELU) return MOE_ERR_ARG;
+    if (E > tc::MAX_E) return MOE_ERR_SHAPE;
+    if (R_max == 0) return MOE_OK;
+    if (!buffer || !offsets || !W1 || !W2 || !y || (act == MOE_ACT_SWIGLU && !W3)) return MOE_ERR_ARG;
+    const size_t need = moe_expert_ffn_workspace_bytes(R_max, d, F, dtype);
+    if (!workspace || workspace_bytes < need || ((uintptr_t)workspace & 255)) return MOE_ERR_WORKSPACE;
+    if (dtype == MOE_BF16) {
+        if (d % 64 != 0 || F % 64 != 0) return MOE_ERR_SHAPE;
+        auto al16 = [](const void* p) { return ((uintptr_t)p & 15) == 0; };
+        if (!al16(buffer) || !al16(W1) || !al16(W2) || !al16(y) || (W3 && !al16(W3))) return MOE_ERR_SHAPE;
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+
+    if (dtype == MOE_F32) {
+        float* H = (float*)workspace;
+        const long long nh = (long long)R_max * F, ny = (long long)R_max * d;
+        ffn_f32_hidden_kernel<<<(int)((nh + 255) / 256), 256, 0, s>>>((const float*)buffer, d, F, E, offsets, R_max,
+                                                                      (const float*)W1, (const float*)W3, act, H);
+        MOE_LAUNCH_CHECK();
+        ffn_f32_out_kernel<<<(int)((ny + 255) / 256), 256, 0, s>>>(H, d, F, E, offsets, R_max, (const float*)W2,
+                                                                   (float*)y);
+        MOE_LAUNCH_CHECK();
+        return MOE_OK;
+    }
+
+    // bf16 tensor-core path
+    if (!get_encoder()) return MOE_ERR_CUDA;
+    uint16_t* H = (uint16_t*)workspace;
+    CUtensorMap m_x, m_w1, m_w3, m_h, m_w2;
+    const bool swiglu = act == MOE_ACT_SWIGLU;
+    if (!make_map(&m_x, buffer, R_max, d, tc::BM)) return MOE_ERR_CUDA;
+    if (!make_map(&m_w1, W1, (long long)E * F, d, swiglu ? 128 : 256)) return MOE_ERR_CUDA;
+    if (swiglu && !make_map(&m_w3, W3, (long long)E * F, d, 128)) return MOE_ERR_CUDA;
+    if (!make_map(&m_h, H, R_max, F, tc::BM)) return MOE_ERR_CUDA;
+    if (!make_map(&m_w2, W2, (long long)E * d, F, 256)) return MOE_ERR_CUDA;
+
+    tc::GemmArgs g1{offsets, E, d, F, F, R_max, H, err};
+    moe_status st = swiglu ? launch_gemm<tc::MODE_SWIGLU>(m_x, m_w1, m_w3, g1, s)
+                           : launch_gemm<tc::MODE_GELU>(m_x, m_w1, m_w1, g1, s);
+    if (st != MOE_OK) return st;
+    tc::GemmArgs g2{offsets, E, F, d, d, R_max, (uint16_t*)y, err};
+    return launch_gemm<tc::MODE_PLAIN>(m_h, m_w2, m_w2, g2, s);
+}

@@ -1,0 +1,112 @@
+"""One MoE layer as a chain of libmoe calls, with every buffer preallocated.
+
+Top-k layer ("MoELayer" of "How MegaDLMs Implements Mixture of Experts (MoE)
+Architectures"): route -> permute -> expert MLPs -> unpermute, plus the
+shared expert when one is configured.  Expert-choice layer
+("MoELayerExpertChoice"): route_ec -> gather rows -> expert MLPs ->
+unpermute_ec.  Nothing here computes: it owns device memory and calls the
+library on one stream, with no host synchronisation inside a forward.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import libmoe as M
+
+
+class TopKLayer:
+    def __init__(self, T: int, d: int, E: int, k: int, F: int, capacity_factor: float, dtype: torch.dtype,
+                 W1, W3, W2, act: str = "swiglu", norm_topk: bool = False, shared_weights=None,
+                 group_of_expert: Optional[torch.Tensor] = None, G: int = 0, out_dtype=None, device="cuda"):
+        self.T, self.d, self.E, self.k, self.F = T, d, E, k, F
+        self.cf, self.dtype, self.act, self.norm_topk = capacity_factor, dtype, act, norm_topk
+        self.W1, self.W3, self.W2 = W1, W3, W2
+        self.goe, self.G = group_of_expert, (G if group_of_expert is not None else 0)
+        self.out_dtype = out_dtype or dtype
+        dev = torch.device(device)
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+        self.gate = torch.empty((T, k), dtype=torch.float32, device=dev)
+        R_max = M.permute_max_rows(T, k, E, capacity_factor, self.G)
+        self.R_max = max(R_max, 1)
+        self.perm = dict(buffer=torch.empty((self.R_max, d), dtype=dtype, device=dev),
+                         row_map=torch.empty((T, k), dtype=torch.int32, device=dev),
+                         row_token=torch.empty(self.R_max, dtype=torch.int32, device=dev),
+                         counts=torch.empty(E, dtype=torch.int32, device=dev),
+                         offsets=torch.empty((self.G or E) + 1, dtype=torch.int32, device=dev),
+                         dropped=torch.empty(1, dtype=torch.int32, device=dev))
+        self.perm_ws = M._ws(M.permute_workspace_bytes(T, k, E, self.G), dev)
+        self.identity = F == 0 or W1 is None
+        if not self.identity:
+            self.y = torch.empty((self.R_max, d), dtype=dtype, device=dev)
+            self.ffn_ws = M._ws(M.expert_ffn_workspace_bytes(self.R_max, d, F, dtype), dev)
+        self.shared_weights = shared_weights
+        if shared_weights is not None:
+            sW1 = shared_weights[0]
+            self.F_shared = sW1.shape[1]
+            self.shared_offsets = torch.tensor([0, T], dtype=torch.int32, device=dev)
+            self.shared_y = torch.empty((T, d), dtype=dtype, device=dev)
+            self.shared_ws = M._ws(M.expert_ffn_workspace_bytes(T, d, self.F_shared, dtype), dev)
+        self.out = torch.empty((T, d), dtype=self.out_dtype, device=dev)
+
+    def route(self, logits, stream=None):
+        return M.route_topk(logits, self.k, self.norm_topk, self.idx, self.gate, stream=stream)
+
+    def dispatch(self, x, stream=None):
+        return M.permute(x, self.idx, self.E, self.cf, self.goe, self.G, out=self.perm, workspace=self.perm_ws,
+                         stream=stream)
+
+    def experts(self, stream=None):
+        if self.identity:
+            return self.perm["buffer"]
+        return M.expert_ffn(self.perm["buffer"], self.perm["offsets"], self.W1, self.W3, self.W2, self.act,
+                            y=self.y, workspace=self.ffn_ws, stream=stream)
+
+    def shared_expert(self, x, stream=None):
+        if self.shared_weights is None:
+            return None
+        sW1, sW3, sW2 = self.shared_weights
+        return M.expert_ffn(x, self.shared_offsets, sW1, sW3, sW2, "swiglu", y=self.shared_y,
+                            workspace=self.shared_ws, stream=stream)
+
+    def combine(self, y, shared=None, stream=None):
+        return M.unpermute(y, self.perm["row_map"], self.gate, shared, self.out_dtype, out=self.out, stream=stream)
+
+    def forward(self, logits: torch.Tensor, x: torch.Tensor, stream=None) -> torch.Tensor:
+        self.route(logits, stream)
+        self.dispatch(x, stream)
+        y = self.experts(stream)
+        sh = self.shared_expert(x, stream)
+        return self.combine(y, sh, stream)
+
+
+class ExpertChoiceLayer:
+    def __init__(self, T: int, d: int, E: int, C: int, F: int, dtype: torch.dtype, W1, W3, W2, act: str = "gelu",
+                 out_dtype=None, device="cuda"):
+        self.T, self.d, self.E, self.C, self.F = T, d, E, C, F
+        self.dtype, self.act = dtype, act
+        self.W1, self.W3, self.W2 = W1, W3, W2
+        self.out_dtype = out_dtype or dtype
+        dev = torch.device(device)
+        R = E * C
+        self.R = R
+        self.routing = (torch.empty((E, C), dtype=torch.int32, device=dev),
+                        torch.empty((E, C), dtype=torch.float32, device=dev),
+                        torch.empty(T + 1, dtype=torch.int32, device=dev),
+                        torch.empty(R, dtype=torch.int32, device=dev))
+        self.route_ws = M._ws(M.route_ec_workspace_bytes(T, E, C), dev)
+        self.buffer = torch.empty((R, d), dtype=dtype, device=dev)
+        self.offsets = torch.arange(0, R + 1, C, dtype=torch.int32, device=dev)
+        self.y = torch.empty((R, d), dtype=dtype, device=dev)
+        self.ffn_ws = M._ws(M.expert_ffn_workspace_bytes(R, d, F, dtype), dev)
+        self.out = torch.empty((T, d), dtype=self.out_dtype, device=dev)
+
+    def forward(self, logits: torch.Tensor, x: torch.Tensor, stream=None) -> torch.Tensor:
+        ec_token, ec_gate, tok_ptr, tok_row = M.route_ec(logits, self.C, workspace=self.route_ws, out=self.routing,
+                                                         stream=stream)
+        M.gather_rows(x, tok_ptr, tok_row, self.R, buffer=self.buffer, stream=stream)
+        M.expert_ffn(self.buffer, self.offsets, self.W1, self.W3, self.W2, self.act, y=self.y,
+                     workspace=self.ffn_ws, stream=stream)
+        return M.unpermute_ec(self.y, tok_ptr, tok_row, ec_gate.view(-1), self.out_dtype, out=self.out,
+                              stream=stream)

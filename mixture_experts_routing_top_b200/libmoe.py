@@ -1,0 +1,297 @@
+"""Python binding of the libmoe C ABI (``include/libmoe.h``).
+
+Argument marshalling only: every function checks dtypes/devices/shapes of
+torch tensors, allocates outputs and workspaces with torch (device memory
+is PyTorch's job here), and calls the C entry point of the same name on the
+current CUDA stream.  Every step of the MoE layer runs in the library's
+CUDA kernels; there is no CPU or PyTorch fallback: a missing library or a
+non-zero status raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+SO_PATH = os.path.join(_HERE, "lib", "libmoe.so")
+
+MOE_F32, MOE_BF16 = 0, 1
+MOE_ACT_SWIGLU, MOE_ACT_GELU = 0, 1
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_ARG", 2: "MOE_ERR_SHAPE", 3: "MOE_ERR_DTYPE", 4: "MOE_ERR_WORKSPACE",
+          5: "MOE_ERR_CUDA", 6: "MOE_ERR_UNSUPPORTED", 7: "MOE_ERR_TIMEOUT", 8: "MOE_ERR_DEVICE_INDEX"}
+
+# name -> (restype, argtypes)
+_vp, _i32, _i64, _dbl, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double, ctypes.c_size_t
+SIGNATURES = {
+    "moe_status_string": (ctypes.c_char_p, [_i32]),
+    "moe_abi_version": (_i32, []),
+    "moe_device_error": (_i32, [_i32]),
+    "moe_kernel_launches": (ctypes.c_uint64, []),
+    "moe_route_topk": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moe_route_ec_workspace_bytes": (_sz, [_i32, _i32, _i32]),
+    "moe_route_ec": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
+    "moe_capacity": (_i64, [_dbl, _i32, _i32, _i32]),
+    "moe_permute_max_rows": (_i64, [_i32, _i32, _i32, _dbl, _i32]),
+    "moe_permute_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
+    "moe_permute": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32, _i32, _dbl, _vp, _i32, _vp, _vp, _vp, _vp, _vp,
+                           _vp, _vp, _sz, _vp]),
+    "moe_gather_rows": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp]),
+    "moe_expert_ffn_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
+    "moe_expert_ffn": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp]),
+    "moe_unpermute": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp]),
+    "moe_unpermute_ec": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp]),
+    "moe_coselect": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
+    "moe_transition": (_i32, [_vp, _i32, _vp, _i32, _i32, _i32, _vp, _vp]),
+}
+
+_lib = None
+
+
+class MoeError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__("%s failed: %s (%d)" % (fn, STATUS.get(status, "?"), status))
+        self.status = status
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libmoe.so; raises if it was never built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(SO_PATH):
+            raise RuntimeError("libmoe.so is missing (%s): build it first with "
+                               "`python -m mixture_experts_routing_top_b200.build`" % SO_PATH)
+        L = ctypes.CDLL(SO_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(L, name)
+            f.restype, f.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise MoeError(fn, status)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _dev(t: torch.Tensor, dtype=None, name="tensor"):
+    if not t.is_cuda:
+        raise ValueError("%s must be a CUDA tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    return t
+
+
+def _act_dtype(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return MOE_F32
+    if t.dtype == torch.bfloat16:
+        return MOE_BF16
+    raise ValueError("activations must be float32 or bfloat16, got %s" % t.dtype)
+
+
+def _ws(nbytes: int, device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+# ------------------------------------------------------------- routing
+def route_topk(logits: torch.Tensor, k: int, norm_topk: bool = False, expert_idx=None, gate=None, stream=None):
+    _dev(logits, torch.float32, "logits")
+    T, E = logits.shape
+    if expert_idx is None:
+        expert_idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
+    if gate is None:
+        gate = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    _check("moe_route_topk", lib().moe_route_topk(_p(logits), T, E, k, int(bool(norm_topk)), _p(expert_idx),
+                                                  _p(gate), _stream(stream)))
+    return expert_idx, gate
+
+
+def route_ec_workspace_bytes(T: int, E: int, C: int) -> int:
+    return int(lib().moe_route_ec_workspace_bytes(T, E, C))
+
+
+def route_ec(logits: torch.Tensor, C: int, workspace=None, out=None, stream=None):
+    """Returns (ec_token [E,C], ec_gate [E,C], tok_ptr [T+1], tok_row [E*C])."""
+    _dev(logits, torch.float32, "logits")
+    T, E = logits.shape
+    dev = logits.device
+    if out is None:
+        out = (torch.empty((E, C), dtype=torch.int32, device=dev), torch.empty((E, C), dtype=torch.float32, device=dev),
+               torch.empty(T + 1, dtype=torch.int32, device=dev), torch.empty(E * C, dtype=torch.int32, device=dev))
+    ec_token, ec_gate, tok_ptr, tok_row = out
+    nbytes = route_ec_workspace_bytes(T, E, C)
+    if workspace is None:
+        workspace = _ws(nbytes, dev)
+    _check("moe_route_ec", lib().moe_route_ec(_p(logits), T, E, C, _p(ec_token), _p(ec_gate), _p(tok_ptr),
+                                              _p(tok_row), _p(workspace), workspace.numel(), _stream(stream)))
+    return ec_token, ec_gate, tok_ptr, tok_row
+
+
+# --------------------------------------------------------- permutation
+def capacity(capacity_factor: float, T: int, k: int, E: int) -> int:
+    return int(lib().moe_capacity(float(capacity_factor), T, k, E))
+
+
+def permute_max_rows(T: int, k: int, E: int, capacity_factor: float, G: int = 0) -> int:
+    return int(lib().moe_permute_max_rows(T, k, E, float(capacity_factor), G))
+
+
+def permute_workspace_bytes(T: int, k: int, E: int, G: int = 0) -> int:
+    return int(lib().moe_permute_workspace_bytes(T, k, E, G))
+
+
+def permute(x: Optional[torch.Tensor], expert_idx: torch.Tensor, E: int, capacity_factor: float,
+            group_of_expert: Optional[torch.Tensor] = None, G: int = 0, out=None, workspace=None, stream=None):
+    """token_permutation.  Returns dict(buffer, row_map, row_token, counts,
+    offsets, dropped); buffer is [R_max, d] (R = offsets[-1] rows used)."""
+    _dev(expert_idx, torch.int32, "expert_idx")
+    T, k = expert_idx.shape
+    dev = expert_idx.device
+    if group_of_expert is not None:
+        _dev(group_of_expert, torch.int32, "group_of_expert")
+        if G <= 0:
+            raise ValueError("G must be given with group_of_expert")
+    else:
+        G = 0
+    R_max = permute_max_rows(T, k, E, capacity_factor, G)
+    dtype = MOE_F32
+    d = 0
+    if x is not None:
+        _dev(x, None, "x")
+        dtype = _act_dtype(x)
+        d = x.shape[1]
+    if out is None:
+        out = dict(
+            buffer=None if x is None else torch.empty((max(R_max, 1), d), dtype=x.dtype, device=dev),
+            row_map=torch.empty((T, k), dtype=torch.int32, device=dev),
+            row_token=torch.empty(max(R_max, 1), dtype=torch.int32, device=dev),
+            counts=torch.empty(E, dtype=torch.int32, device=dev),
+            offsets=torch.empty((G if G else E) + 1, dtype=torch.int32, device=dev),
+            dropped=torch.empty(1, dtype=torch.int32, device=dev))
+    if workspace is None:
+        workspace = _ws(permute_workspace_bytes(T, k, E, G), dev)
+    _check("moe_permute", lib().moe_permute(
+        _p(x), dtype, T, d, _p(expert_idx), k, E, float(capacity_factor), _p(group_of_expert), G,
+        _p(out["buffer"]), _p(out["row_map"]), _p(out["row_token"]), _p(out["counts"]), _p(out["offsets"]),
+        _p(out["dropped"]), _p(workspace), workspace.numel(), _stream(stream)))
+    out["R_max"] = R_max
+    return out
+
+
+def gather_rows(x: torch.Tensor, tok_ptr: torch.Tensor, tok_row: torch.Tensor, R: int, buffer=None, stream=None):
+    _dev(x, None, "x")
+    T, d = x.shape
+    if buffer is None:
+        buffer = torch.empty((R, d), dtype=x.dtype, device=x.device)
+    _check("moe_gather_rows", lib().moe_gather_rows(_p(x), _act_dtype(x), T, d, _p(tok_ptr), _p(tok_row), R,
+                                                    _p(buffer), _stream(stream)))
+    return buffer
+
+
+# --------------------------------------------------------- expert MLPs
+def expert_ffn_workspace_bytes(R_max: int, d: int, F: int, dtype: torch.dtype) -> int:
+    return int(lib().moe_expert_ffn_workspace_bytes(R_max, d, F, MOE_BF16 if dtype == torch.bfloat16 else MOE_F32))
+
+
+def expert_ffn(buffer: torch.Tensor, offsets: torch.Tensor, W1: torch.Tensor, W3: Optional[torch.Tensor],
+               W2: torch.Tensor, act: str = "swiglu", y=None, workspace=None, stream=None):
+    _dev(buffer, None, "buffer")
+    _dev(offsets, torch.int32, "offsets")
+    dtype = _act_dtype(buffer)
+    R_max, d = buffer.shape
+    E, F, d1 = W1.shape
+    if d1 != d or tuple(W2.shape) != (E, d, F):
+        raise ValueError("weight shapes: W1 [E,F,d], W2 [E,d,F]")
+    for name, w in (("W1", W1), ("W2", W2)) + ((("W3", W3),) if W3 is not None else ()):
+        _dev(w, buffer.dtype, name)
+    a = MOE_ACT_SWIGLU if act == "swiglu" else MOE_ACT_GELU
+    if y is None:
+        y = torch.empty_like(buffer)
+    if workspace is None:
+        workspace = _ws(expert_ffn_workspace_bytes(R_max, d, F, buffer.dtype), buffer.device)
+    _check("moe_expert_ffn", lib().moe_expert_ffn(
+        _p(buffer), dtype, R_max, d, F, E, _p(offsets), _p(W1), _p(W3), _p(W2), a, _p(y), _p(workspace),
+        workspace.numel(), _stream(stream)))
+    return y
+
+
+# ----------------------------------------------------- unpermutation
+def unpermute(y: torch.Tensor, row_map: torch.Tensor, gate: torch.Tensor, shared: Optional[torch.Tensor] = None,
+              out_dtype: Optional[torch.dtype] = None, out=None, stream=None):
+    _dev(y, None, "y")
+    _dev(row_map, torch.int32, "row_map")
+    _dev(gate, torch.float32, "gate")
+    T, k = row_map.shape
+    d = y.shape[1]
+    out_dtype = out_dtype or y.dtype
+    if shared is not None:
+        _dev(shared, y.dtype, "shared")
+    if out is None:
+        out = torch.empty((T, d), dtype=out_dtype, device=y.device)
+    _check("moe_unpermute", lib().moe_unpermute(
+        _p(y), _act_dtype(y), y.shape[0], T, d, k, _p(row_map), _p(gate), _p(shared), _p(out), _act_dtype(out),
+        _stream(stream)))
+    return out
+
+
+def unpermute_ec(y: torch.Tensor, tok_ptr: torch.Tensor, tok_row: torch.Tensor, ec_gate: torch.Tensor,
+                 out_dtype: Optional[torch.dtype] = None, out=None, stream=None):
+    _dev(y, None, "y")
+    T = tok_ptr.numel() - 1
+    d = y.shape[1]
+    out_dtype = out_dtype or y.dtype
+    if out is None:
+        out = torch.empty((T, d), dtype=out_dtype, device=y.device)
+    _check("moe_unpermute_ec", lib().moe_unpermute_ec(
+        _p(y), _act_dtype(y), y.shape[0], T, d, _p(tok_ptr), _p(tok_row), _p(ec_gate), _p(out), _act_dtype(out),
+        _stream(stream)))
+    return out
+
+
+# ---------------------------------------------------------- statistics
+def coselect(expert_idx: torch.Tensor, E: int, into: Optional[torch.Tensor] = None, stream=None):
+    _dev(expert_idx, torch.int32, "expert_idx")
+    T, k = expert_idx.shape
+    if into is None:
+        into = torch.zeros((E, E), dtype=torch.int32, device=expert_idx.device)
+    _check("moe_coselect", lib().moe_coselect(_p(expert_idx), T, k, E, _p(into), _stream(stream)))
+    return into
+
+
+def transition(idx1: torch.Tensor, idx2: torch.Tensor, E: int, into: Optional[torch.Tensor] = None, stream=None):
+    _dev(idx1, torch.int32, "idx1")
+    _dev(idx2, torch.int32, "idx2")
+    T, k1 = idx1.shape
+    T2, k2 = idx2.shape
+    if T != T2:
+        raise ValueError("idx1 and idx2 need the same token count")
+    if into is None:
+        into = torch.zeros((E, E), dtype=torch.int32, device=idx1.device)
+    _check("moe_transition", lib().moe_transition(_p(idx1), k1, _p(idx2), k2, T, E, _p(into), _stream(stream)))
+    return into
+
+
+def device_error(clear: bool = True) -> int:
+    """Device fault word of the current device (synchronises): 0 if clean."""
+    return int(lib().moe_device_error(int(bool(clear))))
+
+
+def kernel_launches() -> int:
+    """Kernels libmoe has launched in this process so far."""
+    return int(lib().moe_kernel_launches())

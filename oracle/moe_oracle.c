@@ -15,8 +15,9 @@
  *                Constraints" (no token dropping).
  *  [Coupling]  "Expert Coupling in MoE Pretraining: Reducing All-to-All
  *              Overhead with Correlated Placement and Token Shuffling" - Abstract
- *              (pairs selected together, layer-to-layer prediction, a
- *              dispatcher that sends each token to each GPU once).
+ *              (expert pairs chosen by the same token, layer-to-layer
+ *              prediction, a dispatcher that ships a token to a given GPU
+ *              at most one time).
  *  [EPKey]     "Expert Parallelism > Key Parameters" (top_k, capacity_factor,
  *              dropped tokens contribute zero, shared expert, L/E local share).
  *
@@ -70,7 +71,7 @@ static double load_elem(const void* p, int dtype, int64_t i) {
     return (double)((const float*)p)[i];
 }
 
-/* ------------------------------------------------------- TopKRouter (S1) */
+/* ------------------------------------------------------- TopKRouter */
 /* [MegaDLMs] "Routing Mechanisms": softmax over the expert logits, then the
  * top-k experts of each token; returns the probability weights (gates) and
  * the routing map (expert indices).  Slot j holds the (j+1)-th best expert
@@ -107,7 +108,7 @@ int oracle_route_topk(const float* logits, int64_t T, int E, int k, int norm_top
     return 0;
 }
 
-/* ---------------------------------------------------- capacity (S4) */
+/* ---------------------------------------------------- capacity */
 /* [EPKey] "capacity_factor": each expert is given capacity_factor times the
  * average load T*k/E (rounded up to whole rows).  cf <= 0: unbounded, the
  * no-dropping mode of [MegaDLMs] "Activation Checkpointing and Constraints". */
@@ -116,15 +117,15 @@ int64_t oracle_capacity(double capacity_factor, int64_t T, int k, int E) {
     return (int64_t)ceil(capacity_factor * (double)T * (double)k / (double)E);
 }
 
-/* ------------------------------------------- token_permutation (S3-S5) */
+/* ------------------------------------------- token_permutation */
 /* [MegaDLMs] "MoELayer" step 1 and "Token Dispatching": tokens are placed
  * into per-expert buckets.  [EPKey]: assignments beyond an expert's capacity
  * are dropped (row_map = -1).  Expert-major layout, packed: expert e owns
  * rows [offsets[e], offsets[e] + counts[e]) in ascending token order.
  *
- * Group-major layout (group_of_expert != NULL): [Coupling] Abstract, "a
- * dispatcher that sends each token to each GPU once", on one device: one row
- * per distinct (token, group) with at least one kept assignment into that
+ * Group-major layout (group_of_expert != NULL): [Coupling] Abstract, the
+ * dispatcher that ships a token to a given GPU at most one time, on one
+ * device: one row per distinct (token, group) with at least one kept assignment into that
  * group, ordered by group then token; every kept slot of the token into that
  * group maps to the row.  offsets has G+1 entries.
  *
@@ -191,8 +192,8 @@ void oracle_gather_rows(const void* x, int64_t row_bytes, const int32_t* row_tok
         memcpy((char*)buffer + r * row_bytes, (const char*)x + (int64_t)row_token[r] * row_bytes, (size_t)row_bytes);
 }
 
-/* -------------------------------------------------- expert FFN (S6) */
-/* [MegaDLMs] "MoELayer" step 2, local experts process the dispatched tokens;
+/* -------------------------------------------------- expert FFN */
+/* [MegaDLMs] "MoELayer" step 2: each expert on the device runs on its rows;
  * the experts are MLPs.  SwiGLU MLP: h = silu(W1 x) * (W3 x), y = W2 h;
  * GELU MLP: h = gelu(W1 x), y = W2 h, gelu(z) = z * Phi(z) (erf form).
  * [EPKey] "shared expert": the same MLP applied to every token.
@@ -237,7 +238,7 @@ void oracle_expert_ffn_rows(const void* x, int dtype, int64_t n, int d, int F,
     free(h);
 }
 
-/* ---------------------------------------------- token_unpermutation (S7) */
+/* ---------------------------------------------- token_unpermutation */
 /* [MegaDLMs] "MoELayer" step 3: the output sequence is rebuilt from the
  * expert outputs, each token's expert outputs weighted by its gates and
  * summed (slot order j = 0..k-1).  [EPKey]: a dropped assignment
@@ -259,9 +260,9 @@ void oracle_unpermute(const void* Y, int dtype, int64_t T, int d, int k, const i
     }
 }
 
-/* ---------------------------------------------- ExpertChoiceRouter (S2) */
-/* [MegaDLMs] "Routing Mechanisms": each expert chooses its preferred tokens
- * based on the routing scores.  Scores: per-token softmax over experts,
+/* ---------------------------------------------- ExpertChoiceRouter */
+/* [MegaDLMs] "Routing Mechanisms": the selection is inverted, every expert
+ * picking the tokens that score highest for it.  Scores: per-token softmax over experts,
  * compared through key = logit - logsumexp (same order as the probability,
  * computed in double, sum over e in ascending order).  Expert e keeps the C
  * tokens with the largest key (lower token index on equal keys), stored in
@@ -342,8 +343,8 @@ void oracle_unpermute_ec(const void* Y, int dtype, int64_t T, int d, const int32
         }
 }
 
-/* ------------------------------------------------ co-selection (S8) */
-/* [Coupling] Abstract: expert pairs selected together by the same token.
+/* ------------------------------------------------ co-selection */
+/* [Coupling] Abstract: pairs of experts that one token picks jointly.
  * cosel[a][b] += 1 for every ordered pair of the token's slots (a from slot
  * i, b from slot j); the diagonal (i == j) is each expert's load.  Counts are
  * accumulated into cosel [E, E] and use the routing decisions before
@@ -355,9 +356,9 @@ void oracle_coselect(const int32_t* expert_idx, int64_t T, int k, int E, int32_t
                 cosel[(int64_t)expert_idx[t * k + i] * E + expert_idx[t * k + j]] += 1;
 }
 
-/* ------------------------------------------ layer transition (S9) */
-/* [Coupling] Abstract: the experts a token selects at one layer predict the
- * experts it selects at the next.  trans[a][b] += 1 for every a among the
+/* ------------------------------------------ layer transition */
+/* [Coupling] Abstract: a token's expert choices in one layer are predictive
+ * of its choices in the following layer.  trans[a][b] += 1 for every a among the
  * token's layer-1 experts and b among its layer-2 experts (accumulated). */
 void oracle_transition(const int32_t* idx1, int k1, const int32_t* idx2, int k2, int64_t T, int E,
                        int32_t* trans) {

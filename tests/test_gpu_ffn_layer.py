@@ -1,0 +1,145 @@
+"""GPU vs oracle: grouped expert MLPs and whole MoE layers.
+
+Tolerance (bf16 layers): max|y - y_ref| <= 2e-2 * max|y_ref|; the fp32
+layer must also meet a 1e-4 bound (fp32 FMA against the fp64 oracle)."""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_routing_top_b200 import libmoe as M, layer as Lyr, synth, workloads as W
+from oracle import oracle as O
+from tests.helpers import as_f64, assert_layer_close, needs_gpu, to_dev, to_np
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+
+def ffn_case(counts, d, F, act, bf16=True, seed=0):
+    E = len(counts)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    R = int(offsets[-1])
+    R_max = R + 37                                   # rows past R must stay untouched
+    gen = (lambda s, shp, std: synth.normal_bf16(seed, s, shp, 0.0, std)) if bf16 else \
+          (lambda s, shp, std: synth.normal_f32(seed, s, shp, 0.0, std))
+    x = gen(1, (R_max, d), 1.0)
+    W1 = gen(2, (E, F, d), 0.05)
+    W3 = gen(3, (E, F, d), 0.05) if act == "swiglu" else None
+    W2 = gen(4, (E, d, F), 0.05)
+    y = torch.full((R_max, d), 7.0, dtype=torch.bfloat16 if bf16 else torch.float32, device="cuda")
+    M.expert_ffn(to_dev(x), to_dev(offsets), to_dev(W1), None if W3 is None else to_dev(W3), to_dev(W2), act, y=y)
+    assert M.device_error() == 0
+    got = to_np(y)
+    row_e = np.repeat(np.arange(E, dtype=np.int32), counts)
+    ref = O.expert_ffn_rows(x[:R], row_e, W1, W3, W2, act)
+    assert (as_f64(got[R:]) == 7.0).all()
+    return got[:R], ref
+
+
+@pytest.mark.parametrize("counts,d,F,act", [
+    ([0, 130, 300], 128, 192, "swiglu"),           # empty expert, ragged tiles, partial n-tiles
+    ([257, 1, 128, 0, 64], 256, 128, "swiglu"),
+    ([200, 333], 512, 1024, "swiglu"),             # several k-blocks and n-tiles
+    ([0, 130, 300], 128, 256, "gelu"),
+    ([129, 511], 320, 448, "gelu"),
+    ([1000], 64, 64, "swiglu")])
+def test_expert_ffn_bf16(counts, d, F, act):
+    got, ref = ffn_case(counts, d, F, act)
+    assert_layer_close(got, ref)
+
+
+def test_expert_ffn_fp32():
+    got, ref = ffn_case([70, 0, 90, 100], 64, 128, "swiglu", bf16=False)
+    assert_layer_close(got, ref, rel=1e-4)
+    got, ref = ffn_case([10, 20], 24, 40, "gelu", bf16=False)
+    assert_layer_close(got, ref, rel=1e-4)
+
+
+# ------------------------------------------------------------------ layers
+def weights_dev(ws):
+    return tuple(None if a is None else to_dev(a) for a in ws)
+
+
+def test_layer_tiny_fp32_all_tokens():
+    w = W.TINY
+    logits, x = W.make_logits(w), W.make_x(w)
+    Wt = W.make_weights(w)
+    L = Lyr.TopKLayer(w.T, w.d, w.E, w.k, w.F, w.capacity_factor, torch.float32, *weights_dev(Wt))
+    got = to_np(L.forward(to_dev(logits), to_dev(x)))
+    ref, info = O.topk_layer_tokens(w, logits, x, Wt, None, np.arange(w.T))
+    assert_layer_close(got, ref, rel=1e-4)
+
+
+def test_layer_tiny_forced_drops():
+    w = W.TINY.with_(T=999, capacity_factor=0.5)
+    logits, x = W.make_logits(w), W.make_x(w)
+    Wt = W.make_weights(w)
+    L = Lyr.TopKLayer(w.T, w.d, w.E, w.k, w.F, w.capacity_factor, torch.float32, *weights_dev(Wt))
+    got = to_np(L.forward(to_dev(logits), to_dev(x)))
+    ref, info = O.topk_layer_tokens(w, logits, x, Wt, None, np.arange(w.T))
+    assert info["perm"]["dropped"] > 0
+    assert int(L.perm["dropped"][0]) == info["perm"]["dropped"]
+    assert_layer_close(got, ref, rel=1e-4)
+    all_dropped = (info["perm"]["row_map"] < 0).all(1)
+    assert all_dropped.any() and (got[all_dropped] == 0).all()
+
+
+def sampled_tokens(info, T, n, seed=0):
+    """n tokens: some with dropped slots first, the rest uniform."""
+    rng = np.random.default_rng(seed)
+    dropped = np.nonzero((info["perm"]["row_map"] < 0).any(1))[0]
+    pick = list(rng.choice(dropped, size=min(n // 2, dropped.size), replace=False)) if dropped.size else []
+    rest = rng.choice(T, size=n - len(pick), replace=False)
+    return np.unique(np.concatenate([np.asarray(pick, np.int64), rest, [0, T - 1]]))
+
+
+@pytest.mark.parametrize("w", [W.MIXTRAL, W.FINE], ids=lambda w: w.name)
+def test_layer_full_size_sampled(w):
+    logits, x = W.make_logits(w), W.make_x(w)
+    Wt = W.make_weights(w)
+    Ws = W.make_shared_weights(w)
+    L = Lyr.TopKLayer(w.T, w.d, w.E, w.k, w.F, w.capacity_factor, torch.bfloat16, *weights_dev(Wt),
+                      shared_weights=None if Ws is None else weights_dev(Ws))
+    got = to_np(L.forward(to_dev(logits), to_dev(x)))
+    assert M.device_error() == 0
+    _, info = O.topk_layer_tokens(w, logits, x, Wt, Ws, [])
+    toks = sampled_tokens(info, w.T, 12)
+    ref, _ = O.topk_layer_tokens(w, logits, x, Wt, Ws, toks)
+    assert_layer_close(got[toks], ref)
+    # co-selection of this layer's routing, bit-exact
+    assert np.array_equal(to_np(M.coselect(L.idx, w.E)), O.coselect(info["idx"], w.E))
+
+
+@pytest.mark.parametrize("G", W.SWEEP_G)
+def test_layer_dispatch_combine_identity(G):
+    w = W.SWEEP.with_(T=4096)
+    logits, x = W.make_logits(w), W.make_x(w)
+    goe = W.equal_groups(w.E, G)
+    L = Lyr.TopKLayer(w.T, w.d, w.E, w.k, 0, 0.0, torch.bfloat16, None, None, None, norm_topk=True,
+                      group_of_expert=to_dev(goe), G=G, out_dtype=torch.float32)
+    got = as_f64(to_np(L.forward(to_dev(logits), to_dev(x))))
+    idx, gate = O.route_topk(logits, w.k, True)
+    p = O.permute(idx, w.E, O.capacity(0.0, w.T, w.k, w.E), goe)
+    ref = O.unpermute(O.gather_rows(x, p["row_token"]), p["row_map"], gate)
+    np.testing.assert_allclose(got, ref, rtol=1e-5, atol=1e-6)
+    np.testing.assert_allclose(got, as_f64(x), rtol=1e-5, atol=1e-6)   # renormalised gates: y == x
+
+
+def test_layer_expert_choice_sampled():
+    w = W.EXPERT_CHOICE
+    logits, x = W.make_logits(w), W.make_x(w)
+    W1, _, W2 = W.make_weights(w)
+    L = Lyr.ExpertChoiceLayer(w.T, w.d, w.E, w.C, w.F, torch.bfloat16, to_dev(W1), None, to_dev(W2), "gelu")
+    got = to_np(L.forward(to_dev(logits), to_dev(x)))
+    assert M.device_error() == 0
+    ec_token, ec_gate, tok_ptr, tok_row = O.route_ec(logits, w.C)
+    rng = np.random.default_rng(0)
+    chosen = np.nonzero(np.diff(tok_ptr) > 0)[0]
+    unchosen = np.nonzero(np.diff(tok_ptr) == 0)[0]
+    toks = np.unique(np.concatenate([rng.choice(chosen, 10, replace=False), unchosen[:3]]))
+    ref = np.zeros((toks.size, w.d))
+    for i, t in enumerate(toks):
+        rows = tok_row[tok_ptr[t]:tok_ptr[t + 1]]
+        if rows.size:
+            y = O.expert_ffn_rows(x[[t] * rows.size], (rows // w.C).astype(np.int32), W1, None, W2, "gelu")
+            ref[i] = (ec_gate.reshape(-1)[rows].astype(np.float64)[:, None] * y).sum(0)
+    assert_layer_close(got[toks], ref)
+    assert (as_f64(got[unchosen]) == 0).all()

@@ -1,0 +1,81 @@
+"""GPU vs oracle: top-k and expert-choice routing (bit-exact indices)."""
+import numpy as np
+import pytest
+import torch
+
+from mixture_experts_routing_top_b200 import libmoe as M, synth, workloads as W
+from oracle import oracle as O
+from tests.helpers import needs_gpu, to_dev, to_np
+
+pytestmark = [pytest.mark.gpu, needs_gpu]
+
+GATE_RTOL = 1e-6   # expf (<= 2 ulp) + fp32 rounding; the sum and the ratio are fp64
+
+
+def check_topk(logits, k, norm=False):
+    idx, gate = M.route_topk(to_dev(logits), k, norm)
+    ridx, rgate = O.route_topk(logits, k, norm)
+    gi, gg = to_np(idx), to_np(gate)
+    bad = np.nonzero((gi != ridx).any(1))[0]
+    assert bad.size == 0, "token %d: gpu %s oracle %s" % (bad[0], gi[bad[0]], ridx[bad[0]])
+    np.testing.assert_allclose(gg, rgate, rtol=GATE_RTOL, atol=1e-30)
+
+
+@pytest.mark.parametrize("T,E,k", [(1, 1, 1), (7, 3, 2), (1000, 8, 2), (333, 33, 5), (512, 64, 6), (300, 100, 7),
+                                   (1025, 256, 8), (200, 1024, 32), (64, 160, 32), (50, 5, 5)])
+@pytest.mark.parametrize("norm", [False, True])
+def test_topk_random(T, E, k, norm):
+    check_topk(synth.normal_f32(11, 1, (T, E), 0.0, 2.0), k, norm)
+
+
+def test_topk_ties_lower_index_wins():
+    rng = np.random.default_rng(0)
+    for E, k in ((8, 3), (40, 6), (256, 8)):
+        logits = rng.integers(-2, 3, size=(2000, E)).astype(np.float32)
+        check_topk(logits, k)
+    check_topk(np.zeros((10, 70), np.float32), 7, True)
+
+
+def test_topk_empty():
+    idx, gate = M.route_topk(torch.empty((0, 8), dtype=torch.float32, device="cuda"), 2)
+    assert idx.shape == (0, 2)
+
+
+@pytest.mark.parametrize("w", [W.TINY, W.MIXTRAL, W.FINE, W.SWEEP], ids=lambda w: w.name)
+def test_topk_workloads(w):
+    check_topk(W.make_logits(w), w.k, w.norm_topk)
+
+
+def test_top1_both_layers_of_expert_choice_workload():
+    w = W.EXPERT_CHOICE
+    l1 = W.make_logits(w)
+    check_topk(l1, 1)
+    check_topk(W.make_layer2_logits(w, l1), 1)
+
+
+def check_ec(logits, C):
+    out = M.route_ec(to_dev(logits), C)
+    ec_token, ec_gate, tok_ptr, tok_row = [to_np(t) for t in out]
+    r_token, r_gate, r_ptr, r_row = O.route_ec(logits, C)
+    bad = np.nonzero((ec_token != r_token).any(1))[0]
+    assert bad.size == 0, "expert %d differs" % bad[0]
+    np.testing.assert_allclose(ec_gate, r_gate, rtol=GATE_RTOL, atol=1e-30)
+    assert np.array_equal(tok_ptr, r_ptr)
+    assert np.array_equal(tok_row, r_row)
+
+
+@pytest.mark.parametrize("T,E,C", [(1, 1, 1), (40, 4, 10), (1000, 7, 333), (3000, 64, 100), (2048, 33, 2048),
+                                   (5000, 128, 79)])
+def test_expert_choice_random(T, E, C):
+    check_ec(synth.normal_f32(5, 1, (T, E)), C)
+
+
+def test_expert_choice_ties():
+    rng = np.random.default_rng(1)
+    check_ec(rng.integers(-1, 2, size=(3000, 16)).astype(np.float32), 700)
+    check_ec(np.zeros((257, 3), np.float32), 100)
+
+
+def test_expert_choice_workload():
+    w = W.EXPERT_CHOICE
+    check_ec(W.make_logits(w), w.C)
