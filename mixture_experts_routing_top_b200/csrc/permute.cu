@@ -410,7 +410,17 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
     if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_ARG;
     if (k > 32 || E > 1024) return MOE_ERR_SHAPE;
     if (group_of_expert && (G < 1 || G > 1024)) return (G < 1) ? MOE_ERR_ARG : MOE_ERR_SHAPE;
-    if (!expert_idx || !row_map || !row_token || !counts || !offsets || !dropped) return MOE_ERR_ARG;
+    if (!counts || !offsets || !dropped) return MOE_ERR_ARG;
+    if (T == 0) {
+        // nothing routed: zero counts, offsets, dropped
+        cudaStream_t s0 = (cudaStream_t)stream;
+        if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s0) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * ((group_of_expert ? G : E) + 1), s0) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        if (cudaMemsetAsync(dropped, 0, sizeof(int32_t), s0) != cudaSuccess) return MOE_ERR_CUDA;
+        return MOE_OK;
+    }
+    if (!expert_idx || !row_map || !row_token) return MOE_ERR_ARG;
     if ((x == nullptr) != (buffer == nullptr)) return MOE_ERR_ARG;
     const int esz = dtype == MOE_BF16 ? 2 : 4;
     const long long row_bytes = (long long)d * esz;
@@ -428,13 +438,6 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
     int32_t* base = (int32_t*)(ws + L.base);
     int32_t* total = (int32_t*)(ws + L.total);
     const int nw = kIdxThreads / 32;
-    if (T == 0) {
-        // nothing routed: zero counts, offsets, dropped
-        if (cudaMemsetAsync(counts, 0, sizeof(int32_t) * E, s) != cudaSuccess) return MOE_ERR_CUDA;
-        if (cudaMemsetAsync(offsets, 0, sizeof(int32_t) * ((group_of_expert ? G : E) + 1), s) != cudaSuccess) return MOE_ERR_CUDA;
-        if (cudaMemsetAsync(dropped, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
-        return MOE_OK;
-    }
     // expert pass: counts, scan, capacity
     perm_count_kernel<<<nblk, kIdxThreads, sizeof(int) * E, s>>>(0, expert_idx, nullptr, nullptr, T, k, E, E, nblk, cnt, err);
     MOE_LAUNCH_CHECK();

@@ -52,7 +52,7 @@ def test_expert_major(T, E, k, cf, d, bf16):
     idx = routed(T, E, k, skew=1.0)
     x = synth.normal_bf16(1, 2, (T, d)) if bf16 else synth.normal_f32(1, 2, (T, d))
     _, ref = run(x, idx, E, cf)
-    if 0 < cf < 1:
+    if 0 < cf < 1 and T >= 100:
         assert ref["dropped"] > 0
 
 
