@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--cpu-rows", type=int, default=24, help="expert-MLP rows in the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
+                    help="override a workload field (e.g. T=4096) - for smaller profiling cases, not bench lines")
     return ap.parse_args()
 
 
@@ -429,6 +431,12 @@ def main():
     from mixture_experts_routing_top_b200 import workloads as W
 
     w = W.BY_NAME[args.workload]
+    for kv in args.set:
+        key, val = kv.split("=", 1)
+        cur = getattr(w, key)
+        w = w.with_(**{key: type(cur)(val)})
+    if args.set:
+        w = w.with_(name=w.name + "[" + ",".join(args.set) + "]")
     if w.routing != "topk":
         raise SystemExit("bench.py times top-k layers; %s is measured by its tests" % w.name)
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -150,6 +150,28 @@ moe_status moe_permute(const void* x, int dtype, int T, int d,
                        int32_t* counts, int32_t* offsets, int32_t* dropped,
                        void* workspace, size_t workspace_bytes, moe_stream_t stream);
 
+/* moe_permute without a caller workspace, for callers that cannot allocate
+ * device memory: a host framework that owns all device memory and forbids
+ * allocation once running (inference plugins, serving loops with a fixed
+ * memory plan), or a hot path that cannot take cudaMalloc's implicit
+ * synchronisation.  The pages have no counterpart to this call; it exists
+ * for deployment only.  Arguments and results are those of moe_permute.
+ * Scratch: a fixed MOE_PERMUTE_NOALLOC_SCRATCH_BYTES array in device memory,
+ * held by every GPU that loads the library until the process exits.
+ * Limit: moe_permute_workspace_bytes(T, k, E, G) must not exceed it
+ * (e.g. T = 131072, k = 8, E = 256, G = 64 needs 2.25 MiB); larger problems
+ * return MOE_ERR_WORKSPACE and launch nothing.  The first call on a device
+ * looks up the array's device address (cudaGetSymbolAddress) and caches it;
+ * make that first call before any stream capture.  All calls share the one
+ * array, so calls whose kernels overlap on the GPU (different streams, no
+ * ordering between them) race and give wrong results; serialise them. */
+#define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (4u << 20)
+moe_status moe_permute_noalloc(const void* x, int dtype, int T, int d,
+                               const int32_t* expert_idx, int k, int E, double capacity_factor,
+                               const int32_t* group_of_expert, int G,
+                               void* buffer, int32_t* row_map, int32_t* row_token,
+                               int32_t* counts, int32_t* offsets, int32_t* dropped, moe_stream_t stream);
+
 /* Expert-choice dispatch: buffer rows from the token CSR of moe_route_ec,
  * each token read once: buffer[tok_row[p]] = x[t] for p in
  * [tok_ptr[t], tok_ptr[t+1]).  buffer has R rows (E*C) and tok_row R

@@ -22,6 +22,8 @@
 //               same count/scan/rank over the (token, group) head slots.
 //   5. copy:    one token per warp, x[t] read once (16-byte vectors) and
 //               written to each distinct row the token owns.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moe {
@@ -501,4 +503,52 @@ extern "C" moe_status moe_gather_rows(const void* x, int dtype, int T, int d, co
     else copy_rows_csr_kernel<4><<<grid, 256, 0, s>>>((const uint4*)x, T, vpr, tok_ptr, tok_row, R, (uint4*)buffer, err);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
+}
+
+// ------------------------------------------------ allocation-free variant
+// For callers that may not allocate device memory at all: code running
+// inside a host framework that owns every device byte and forbids
+// allocation after start-up (an inference plugin's enqueue, a real-time
+// serving loop with a pre-planned memory budget), or code that cannot
+// afford cudaMalloc's implicit device synchronisation on its hot path.
+// Such callers still pass their inputs and outputs; the permutation's
+// scratch comes from this fixed array instead of a caller workspace.  Every
+// GPU that loads the library holds it until the process exits.
+static __device__ __align__(256) unsigned char g_permute_noalloc_scratch[MOE_PERMUTE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_scratch[64] = {nullptr};
+
+// Device address of this device's scratch array.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up
+// once per device (with that device current) and cached.
+void* noalloc_scratch_address() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_scratch[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_permute_noalloc_scratch) != cudaSuccess) return nullptr;
+        g_noalloc_scratch[dev] = p;
+    }
+    return g_noalloc_scratch[dev];
+}
+}  // namespace
+
+extern "C" moe_status moe_permute_noalloc(const void* x, int dtype, int T, int d, const int32_t* expert_idx, int k,
+                                          int E, double capacity_factor, const int32_t* group_of_expert, int G,
+                                          void* buffer, int32_t* row_map, int32_t* row_token, int32_t* counts,
+                                          int32_t* offsets, int32_t* dropped, moe_stream_t stream) {
+    if (T < 0 || k < 1 || E < 1 || G < 0) return MOE_ERR_ARG;
+    const size_t need = moe_permute_workspace_bytes(T, k, E, group_of_expert ? G : 0);
+    if (need > (size_t)MOE_PERMUTE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
+    void* scratch = noalloc_scratch_address();
+    if (!scratch) return MOE_ERR_CUDA;
+    // Nothing in the permutation's scratch needs to start at zero: every
+    // count, base and flag it reads is written earlier in the same call, so
+    // what a previous call left there is never used.
+    return moe_permute(x, dtype, T, d, expert_idx, k, E, capacity_factor, group_of_expert, G, buffer, row_map,
+                       row_token, counts, offsets, dropped, scratch, (size_t)MOE_PERMUTE_NOALLOC_SCRATCH_BYTES,
+                       stream);
 }

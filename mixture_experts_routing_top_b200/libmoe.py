@@ -38,6 +38,8 @@ SIGNATURES = {
     "moe_permute_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
     "moe_permute": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32, _i32, _dbl, _vp, _i32, _vp, _vp, _vp, _vp, _vp,
                            _vp, _vp, _sz, _vp]),
+    "moe_permute_noalloc": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32, _i32, _dbl, _vp, _i32, _vp, _vp, _vp, _vp,
+                                   _vp, _vp, _vp]),
     "moe_gather_rows": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _vp]),
     "moe_expert_ffn_workspace_bytes": (_sz, [_i32, _i32, _i32, _i32]),
     "moe_expert_ffn": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp]),
