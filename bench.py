@@ -112,13 +112,40 @@ class Clocks:
                 "reasons": reasons, "samples": len(rows)}
 
 
+# ---------------------------------------------------------- ranks
+def rank_batch(w, rank):
+    """Workload of one rank: its own batch (seed = rank), same shapes."""
+    return w.with_(seed=rank)
+
+
+def reduce_over_ranks(elapsed_ms, launches, device):
+    """Slowest rank's time and total launches over all ranks (identity on one
+    process).  Runs on any torch.distributed backend (NCCL on GPUs, gloo on
+    CPU in the tests)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(elapsed_ms), int(launches)
+    t = torch.tensor([float(elapsed_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    c = torch.tensor([int(launches)], dtype=torch.int64, device=device)
+    dist.all_reduce(c, op=dist.ReduceOp.SUM)
+    return float(t.item()), int(c.item())
+
+
+def throughput(world, tokens_per_rank, steps, max_elapsed_ms):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return world * tokens_per_rank * steps / (max_elapsed_ms / 1e3)
+
+
 # ------------------------------------------------------------ libmoe arm
 def make_problem(w, rank, device):
     import torch
 
     from mixture_experts_routing_top_b200 import workloads as W
 
-    wr = w.with_(seed=rank)                    # this rank's batch
+    wr = rank_batch(w, rank)                   # this rank's batch
     logits = W.make_logits(wr)
     x = W.make_x(wr)
     Wt = W.make_weights(w)                     # one model on every rank
@@ -284,13 +311,7 @@ def run_libmoe(args, w, rank, world, local_rank):
         raise RuntimeError("device fault word set during the timed steps")
 
     # max over ranks (slowest rank), total launches
-    if world > 1:
-        t = torch.tensor([elapsed_ms], dtype=torch.float64, device=device)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
-        c = torch.tensor([launches], dtype=torch.int64, device=device)
-        dist.all_reduce(c, op=dist.ReduceOp.SUM)
-        launches = int(c.item())
+    elapsed_ms, launches = reduce_over_ranks(elapsed_ms, launches, device)
 
     # end to end through the public API: pinned host inputs -> layer -> host output
     e2e = None
@@ -319,12 +340,8 @@ def run_libmoe(args, w, rank, world, local_rank):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = a.elapsed_time(b)
-        if world > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=device)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": world * w.T * args.e2e_steps / (e_ms / 1e3), "unit": "tokens/s",
+        e_ms, _ = reduce_over_ranks(a.elapsed_time(b), 0, device)
+        e2e = {"value": throughput(world, w.T, args.e2e_steps, e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": lg_h.numel() * 4 + x_h.numel() * x_h.element_size(),
                "d2h_bytes_per_step": out_h.numel() * out_h.element_size()}
 
@@ -344,7 +361,7 @@ def run_libmoe(args, w, rank, world, local_rank):
         for s in stages}
     stage_report["ffn"].update({"TFLOP/s": round(achieved, 1), "flops": flops,
                                 "frac_burst": round(achieved / pk["bf16_tflops"], 3)})
-    value = world * w.T * args.steps / (elapsed_ms / 1e3)
+    value = throughput(world, w.T, args.steps, elapsed_ms)
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
