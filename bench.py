@@ -1,11 +1,14 @@
 #!/usr/bin/env python
 """Benchmark of one MoE layer step on B200 through libmoe.
 
-A step is one pass of the whole hot path over one batch: top-k routing,
-capacity-bounded permutation, the grouped expert MLPs (tcgen05 GEMMs), the
-gate-weighted combine and the co-selection histogram.  Default workload:
+A step is one pass of the whole hot path over one batch.  Default workload:
 the Mixtral-shaped top-2 layer (T=8192 tokens, d=4096, E=8 experts, SwiGLU
-4096->14336->4096, capacity factor 1.25, bf16 with fp32 accumulation).
+4096->14336->4096, capacity factor 1.25, bf16 with fp32 accumulation); its
+step is top-k routing -> capacity-bounded permutation -> grouped expert MLPs
+(tcgen05 GEMMs) -> gate-weighted combine -> co-selection histogram.  Other
+workloads (``--workload``): the fine-grained top-6 layer with a shared expert,
+the dispatch/combine sweep (identity experts, group-major rows), and the
+expert-choice layer with its layer-to-layer transition histogram.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libmoe|reference]
 
@@ -13,7 +16,7 @@ One JSON line on rank 0.  Under torchrun each rank runs its own batch (its
 own seed) against the same expert weights: independent replicas, no
 collective on the data path, weak scaling; the timed region is bracketed by
 a barrier and a device synchronise on both sides and the slowest rank's
-time is taken.  `--impl reference` times the CPU oracle (single-threaded C)
+time is taken.  ``--impl reference`` times the CPU oracle (single-threaded C)
 on a bounded sample of the same workload.
 """
 from __future__ import annotations
@@ -36,11 +39,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer tokens/s; permute/combine HBM GB/s and grouped-GEMM TFLOP/s vs peak"
 PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "ffn_traffic.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
@@ -52,15 +56,32 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
                     help="override a workload field (e.g. T=4096) - for smaller profiling cases, not bench lines")
-    return ap.parse_args()
+    return ap.parse_args(argv)
 
 
 def peaks():
     if os.path.exists(PEAKS_FILE):
         with open(PEAKS_FILE) as f:
-            p = json.load(f)
-        return p, "measured"
+            return json.load(f), "measured"
     return FALLBACK_PEAKS, "fallback"
+
+
+def workload_from_args(args):
+    from mixture_experts_routing_top_b200 import workloads as W
+
+    w = W.BY_NAME[args.workload]
+    for kv in args.set:
+        key, val = kv.split("=", 1)
+        w = w.with_(**{key: type(getattr(w, key))(val)})
+    if args.set:
+        w = w.with_(name=w.name + "[" + ",".join(args.set) + "]")
+    return w
+
+
+def kind_of(w):
+    if w.routing == "ec":
+        return "ec"
+    return "sweep" if w.F == 0 else "topk"
 
 
 # ------------------------------------------------------------- clocks
@@ -84,7 +105,7 @@ class Clocks:
         except (OSError, ValueError):
             self.proc = None
 
-    def stop(self, gpu_index=None):
+    def stop(self):
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -96,20 +117,19 @@ class Clocks:
         with open(self.path) as f:
             for line in f:
                 parts = [p.strip() for p in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                if gpu_index is not None and parts[0] != str(gpu_index):
-                    continue
-                rows.append(parts)
+                if len(parts) >= 9:
+                    rows.append(parts)
         os.unlink(self.path)
         if not rows:
             return {"samples": 0}
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        num = lambda v: v.replace(".", "", 1).isdigit()
+        sm = [float(r[1]) for r in rows if num(r[1])]
+        mx = [float(r[2]) for r in rows if num(r[2])]
+        pw = [float(r[3]) for r in rows if num(r[3])]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+                "power_w_max": max(pw) if pw else None, "reasons": reasons, "samples": len(rows)}
 
 
 # ---------------------------------------------------------- ranks
@@ -139,96 +159,18 @@ def throughput(world, tokens_per_rank, steps, max_elapsed_ms):
     return world * tokens_per_rank * steps / (max_elapsed_ms / 1e3)
 
 
-# ------------------------------------------------------------ libmoe arm
-def make_problem(w, rank, device):
-    import torch
-
-    from mixture_experts_routing_top_b200 import workloads as W
-
-    wr = rank_batch(w, rank)                   # this rank's batch
-    logits = W.make_logits(wr)
-    x = W.make_x(wr)
-    Wt = W.make_weights(w)                     # one model on every rank
-    Ws = W.make_shared_weights(w)
-
-    def dev(a):
-        if a is None:
-            return None
-        a = np.ascontiguousarray(a)
-        if a.dtype == np.uint16:
-            return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
-        return torch.from_numpy(a).to(device)
-
-    return dict(logits_np=logits, x_np=x, weights_np=Wt, shared_np=Ws, logits=dev(logits), x=dev(x),
-                weights=tuple(dev(a) for a in Wt), shared=None if Ws is None else tuple(dev(a) for a in Ws))
-
-
-def stage_bytes(w, R, b):
-    """Algorithmic bytes per launch of the memory-bound stages (kept rows only)."""
-    T, d, E, k = w.T, w.d, w.E, w.k
-    return {
-        "route": T * E * 4 + T * k * 8,
-        "permute": T * d * b + R * d * b + T * k * (4 + 4) + R * 4,
-        "combine": R * d * b + T * d * b + T * k * (4 + 4) + (T * d * b if w.F_shared else 0),
-        "coselect": T * k * 4 + E * E * 4,
-    }
-
-
-def ffn_flops(w, R):
-    mats = 3 if w.act == "swiglu" else 2
-    f = 2.0 * R * w.d * w.F * mats
-    if w.F_shared:
-        f += 2.0 * w.T * w.d * w.F_shared * 3
-    return f
-
-
-def traffic_of_ffn():
-    """Per-launch DRAM bytes of the FFN stage from the committed ncu summary,
-    or None if missing or taken on another version of the kernel source."""
+def traffic_for(kernel_key):
+    """Per-step DRAM bytes of a stage from the committed ncu summary, or None
+    if missing or taken on another version of the kernel's source."""
     try:
         with open(TRAFFIC_FILE) as f:
-            t = json.load(f)
-        src = open(os.path.join(ROOT, "mixture_experts_routing_top_b200", "csrc", "ffn.cu"), "rb").read()
-        if t.get("source_sha256") != hashlib.sha256(src).hexdigest():
+            entry = json.load(f)[kernel_key]
+        src = open(os.path.join(ROOT, entry["source"]), "rb").read()
+        if entry.get("source_sha256") != hashlib.sha256(src).hexdigest():
             return None
-        return t.get("bytes_per_step")
-    except (OSError, ValueError):
+        return entry.get("bytes_per_step")
+    except (OSError, ValueError, KeyError):
         return None
-
-
-def cpu_baseline(w, prob, n_rows):
-    """The oracle as it stands, single-threaded, on a bounded sample."""
-    from oracle import oracle as O
-    from mixture_experts_routing_top_b200 import synth
-
-    logits, x = prob["logits_np"], prob["x_np"]
-    t0 = time.perf_counter()
-    idx, gate = O.route_topk(logits, w.k, w.norm_topk)
-    p = O.permute(idx, w.E, O.capacity(w.capacity_factor, w.T, w.k, w.E))
-    buf = O.gather_rows(x, p["row_token"])
-    t_rp = time.perf_counter() - t0
-    R = p["R"]
-    rows = np.linspace(0, R - 1, num=min(n_rows, R)).astype(np.int64)
-    row_e = np.searchsorted(p["offsets"], rows, side="right").astype(np.int32) - 1
-    W1, W3, W2 = prob["weights_np"]
-    t0 = time.perf_counter()
-    O.expert_ffn_rows(buf[rows], row_e, W1, W3, W2, w.act)
-    t_row = (time.perf_counter() - t0) / len(rows)
-    Y = synth.normal_bf16(99, 1, (R, w.d)) if w.dtype == "bf16" else synth.normal_f32(99, 1, (R, w.d))
-    t0 = time.perf_counter()
-    O.unpermute(Y, p["row_map"], gate)
-    t_comb = time.perf_counter() - t0
-    t_shared_row = 0.0
-    if prob["shared_np"] is not None:
-        sW1, sW3, sW2 = prob["shared_np"]
-        t0 = time.perf_counter()
-        O.expert_ffn_rows(x[:2], np.zeros(2, np.int32), sW1, sW3, sW2, "swiglu")
-        t_shared_row = (time.perf_counter() - t0) / 2
-    per_token = (t_rp + t_comb) / w.T + t_row * R / w.T + t_shared_row
-    return {"value": 1.0 / per_token, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": "route, capacity, permute and combine on all %d tokens (%.2f s); expert MLP on %d of %d "
-                      "rows, %.3f s per row, extrapolated to all rows" % (w.T, t_rp + t_comb, len(rows), R, t_row),
-            "cpu": _cpu_name()}
 
 
 def _cpu_name():
@@ -242,47 +184,288 @@ def _cpu_name():
     return "unknown"
 
 
+def _dev(a, device):
+    import torch
+
+    if a is None:
+        return None
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        return torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(device)
+    return torch.from_numpy(a).to(device)
+
+
+def _pinned(a):
+    import torch
+
+    a = np.ascontiguousarray(a)
+    t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16) if a.dtype == np.uint16 else torch.from_numpy(a)
+    return t.pin_memory()
+
+
+# ----------------------------------------------------------- runners
+class TopKRunner:
+    """Top-k layers (with or without experts/shared expert) and the
+    dispatch/combine sweep (identity experts, group-major rows)."""
+
+    def __init__(self, w, rank, device):
+        import torch
+
+        from mixture_experts_routing_top_b200 import layer as Lyr, libmoe as M, workloads as W
+
+        self.w, self.M = w, M
+        wr = rank_batch(w, rank)
+        self.logits_np, self.x_np = W.make_logits(wr), W.make_x(wr)
+        self.weights_np = W.make_weights(w) if w.F else (None, None, None)
+        self.shared_np = W.make_shared_weights(w)
+        self.logits, self.x = _dev(self.logits_np, device), _dev(self.x_np, device)
+        weights = tuple(_dev(a, device) for a in self.weights_np)
+        shared = None if self.shared_np is None else tuple(_dev(a, device) for a in self.shared_np)
+        self.goe = W.equal_groups(w.E, w.G) if (w.G and not w.F) else None
+        dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        self.L = Lyr.TopKLayer(w.T, w.d, w.E, w.k, w.F, w.capacity_factor, dt, *weights, act=w.act,
+                               norm_topk=w.norm_topk, shared_weights=shared,
+                               group_of_expert=None if self.goe is None else _dev(self.goe, device),
+                               G=w.G if self.goe is not None else 0, device=device)
+        self.cosel = torch.zeros((w.E, w.E), dtype=torch.int32, device=device)
+        self.resident_bytes = (sum(t.numel() * t.element_size() for t in weights if t is not None) +
+                               self.logits.numel() * 4 + self.x.numel() * self.x.element_size())
+        self.stages = [("route", lambda: self.L.route(self.logits)),
+                       ("permute", lambda: self.L.dispatch(self.x))]
+        if w.F:
+            self.stages.append(("ffn", self._ffn))
+        self.stages.append(("combine", self._combine))
+        self.stages.append(("coselect", lambda: M.coselect(self.L.idx, w.E, into=self.cosel)))
+        self._y = self._sh = None
+
+    def _ffn(self):
+        self._y = self.L.experts()
+        self._sh = self.L.shared_expert(self.x)
+
+    def _combine(self):
+        y = self._y if self.w.F else self.L.perm["buffer"]
+        self.L.combine(y, self._sh)
+
+    def after_warmup(self):
+        self.R = int(self.L.perm["offsets"][-1].item())
+        self.dropped = int(self.L.perm["dropped"][0].item())
+
+    def work(self):
+        """Algorithmic bytes (memory stages) and FLOPs (expert MLPs) per step."""
+        w, R = self.w, self.R
+        b = 2 if w.dtype == "bf16" else 4
+        T, d, E, k = w.T, w.d, w.E, w.k
+        shared = T * d * b if w.F_shared else 0
+        out = {"route": ("bytes", T * E * 4 + T * k * 8),
+               "permute": ("bytes", T * d * b + R * d * b + T * k * 8 + R * 4),
+               "combine": ("bytes", R * d * b + T * d * b + T * k * 8 + shared),
+               "coselect": ("bytes", T * k * 4 + E * E * 4)}
+        if w.F:
+            f = 2.0 * R * d * w.F * (3 if w.act == "swiglu" else 2)
+            if w.F_shared:
+                f += 2.0 * T * d * w.F_shared * 3
+            out["ffn"] = ("flops", f)
+        return out
+
+    def e2e_setup(self):
+        import torch
+
+        self.h_in = [(_pinned(self.logits_np), self.logits), (_pinned(self.x_np), self.x)]
+        self.h_out = torch.empty(self.L.out.shape, dtype=self.L.out.dtype).pin_memory()
+
+    def e2e_step(self):
+        for h, d in self.h_in:
+            d.copy_(h, non_blocking=True)
+        for _, fn in self.stages[:-1]:          # the layer (the statistic is not part of its output)
+            fn()
+        self.h_out.copy_(self.L.out, non_blocking=True)
+
+    def e2e_bytes(self):
+        return (sum(h.numel() * h.element_size() for h, _ in self.h_in),
+                self.h_out.numel() * self.h_out.element_size())
+
+    def extra(self):
+        return {"rows": self.R, "dropped": self.dropped}
+
+    def cpu_baseline(self, n_rows):
+        """The oracle as it stands, single-threaded, on a bounded sample."""
+        from oracle import oracle as O
+        from mixture_experts_routing_top_b200 import synth
+
+        w = self.w
+        Ts = min(w.T, 8192)                    # token sample for the routing/permute/combine part
+        logits, x = self.logits_np[:Ts], self.x_np[:Ts]
+        t0 = time.perf_counter()
+        idx, gate = O.route_topk(logits, w.k, w.norm_topk)
+        p = O.permute(idx, w.E, O.capacity(w.capacity_factor, Ts, w.k, w.E), self.goe)
+        buf = O.gather_rows(x, p["row_token"])
+        t_rp = time.perf_counter() - t0
+        R = p["R"]
+        Y = buf if not w.F else (synth.normal_bf16(99, 1, (R, w.d)) if w.dtype == "bf16"
+                                 else synth.normal_f32(99, 1, (R, w.d)))
+        t0 = time.perf_counter()
+        O.unpermute(Y, p["row_map"], gate)
+        t_comb = time.perf_counter() - t0
+        per_token = (t_rp + t_comb) / Ts
+        sample = "route, capacity, permute, row copy and combine on %d of %d tokens (%.2f s)" % (
+            Ts, w.T, t_rp + t_comb)
+        if w.F:
+            rows = np.linspace(0, R - 1, num=min(n_rows, R)).astype(np.int64)
+            row_e = np.searchsorted(p["offsets"], rows, side="right").astype(np.int32) - 1
+            W1, W3, W2 = self.weights_np
+            t0 = time.perf_counter()
+            O.expert_ffn_rows(buf[rows], row_e, W1, W3, W2, w.act)
+            t_row = (time.perf_counter() - t0) / len(rows)
+            per_token += t_row * R / Ts
+            sample += "; expert MLP on %d of %d rows, %.3f s per row, extrapolated to all rows" % (
+                len(rows), R, t_row)
+            if self.shared_np is not None:
+                t0 = time.perf_counter()
+                O.expert_ffn_rows(x[:2], np.zeros(2, np.int32), *self.shared_np, "swiglu")
+                per_token += (time.perf_counter() - t0) / 2
+                sample += "; shared expert on 2 tokens"
+        return {"value": 1.0 / per_token, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": sample,
+                "cpu": _cpu_name()}
+
+
+class ExpertChoiceRunner:
+    """Expert-choice layer plus the two top-1 routings and the layer-to-layer
+    transition histogram."""
+
+    def __init__(self, w, rank, device):
+        import torch
+
+        from mixture_experts_routing_top_b200 import layer as Lyr, libmoe as M, workloads as W
+
+        self.w, self.M = w, M
+        wr = rank_batch(w, rank)
+        self.logits_np, self.x_np = W.make_logits(wr), W.make_x(wr)
+        self.logits2_np = W.make_layer2_logits(wr, self.logits_np)
+        self.weights_np = W.make_weights(w)
+        self.logits, self.logits2 = _dev(self.logits_np, device), _dev(self.logits2_np, device)
+        self.x = _dev(self.x_np, device)
+        W1, W3, W2 = (_dev(a, device) for a in self.weights_np)
+        self.L = Lyr.ExpertChoiceLayer(w.T, w.d, w.E, w.C, w.F, torch.bfloat16, W1, W3, W2, w.act, device=device)
+        self.top1 = [torch.empty((w.T, 1), dtype=torch.int32, device=device) for _ in range(2)]
+        self.g1 = [torch.empty((w.T, 1), dtype=torch.float32, device=device) for _ in range(2)]
+        self.trans = torch.zeros((w.E, w.E), dtype=torch.int32, device=device)
+        self.resident_bytes = (sum(t.numel() * t.element_size() for t in (W1, W2)) + 2 * self.logits.numel() * 4 +
+                               self.x.numel() * 2)
+        L = self.L
+        self.stages = [("route_ec", lambda: M.route_ec(self.logits, w.C, workspace=L.route_ws, out=L.routing)),
+                       ("dispatch", lambda: M.gather_rows(self.x, L.routing[2], L.routing[3], L.R, buffer=L.buffer)),
+                       ("ffn", lambda: M.expert_ffn(L.buffer, L.offsets, L.W1, L.W3, L.W2, w.act, y=L.y,
+                                                    workspace=L.ffn_ws)),
+                       ("combine", lambda: M.unpermute_ec(L.y, L.routing[2], L.routing[3], L.routing[1].view(-1),
+                                                          out=L.out)),
+                       ("transition", self._transition)]
+
+    def _transition(self):
+        M = self.M
+        M.route_topk(self.logits, 1, False, self.top1[0], self.g1[0])
+        M.route_topk(self.logits2, 1, False, self.top1[1], self.g1[1])
+        M.transition(self.top1[0], self.top1[1], self.w.E, into=self.trans)
+
+    def after_warmup(self):
+        tp = self.L.routing[2]
+        self.chosen = int((tp[1:] > tp[:-1]).sum().item())
+
+    def work(self):
+        w = self.w
+        T, d, E, C = w.T, w.d, w.E, w.C
+        R = E * C
+        return {"route_ec": ("bytes", T * E * 4 + R * 12 + (T + 1) * 4),
+                "dispatch": ("bytes", self.chosen * d * 2 + R * d * 2 + (T + 1 + R) * 4),
+                "ffn": ("flops", 2.0 * R * d * w.F * (3 if w.act == "swiglu" else 2)),
+                "combine": ("bytes", R * d * 2 + T * d * 2 + (T + 1 + 2 * R) * 4),
+                "transition": ("bytes", 2 * T * E * 4 + 2 * T * 8)}
+
+    def e2e_setup(self):
+        import torch
+
+        self.h_in = [(_pinned(self.logits_np), self.logits), (_pinned(self.x_np), self.x)]
+        self.h_out = torch.empty(self.L.out.shape, dtype=self.L.out.dtype).pin_memory()
+
+    def e2e_step(self):
+        for h, d in self.h_in:
+            d.copy_(h, non_blocking=True)
+        for _, fn in self.stages[:-1]:
+            fn()
+        self.h_out.copy_(self.L.out, non_blocking=True)
+
+    def e2e_bytes(self):
+        return (sum(h.numel() * h.element_size() for h, _ in self.h_in),
+                self.h_out.numel() * self.h_out.element_size())
+
+    def extra(self):
+        return {"rows": self.w.E * self.w.C, "tokens_chosen": self.chosen}
+
+    def cpu_baseline(self, n_rows):
+        from oracle import oracle as O
+        from mixture_experts_routing_top_b200 import synth
+
+        w = self.w
+        t0 = time.perf_counter()
+        ec_token, ec_gate, tok_ptr, tok_row = O.route_ec(self.logits_np, w.C)
+        buf = O.gather_rows(self.x_np, ec_token.reshape(-1))
+        R = w.E * w.C
+        Y = synth.normal_bf16(99, 1, (R, w.d))
+        O.unpermute_ec(Y, tok_ptr, tok_row, ec_gate)
+        a, _ = O.route_topk(self.logits_np, 1)
+        b, _ = O.route_topk(self.logits2_np, 1)
+        O.transition(a, b, w.E)
+        t_rest = time.perf_counter() - t0
+        rows = np.linspace(0, R - 1, num=min(n_rows, R)).astype(np.int64)
+        W1, W3, W2 = self.weights_np
+        t0 = time.perf_counter()
+        O.expert_ffn_rows(buf[rows], (rows // w.C).astype(np.int32), W1, W3, W2, w.act)
+        t_row = (time.perf_counter() - t0) / len(rows)
+        per_token = t_rest / w.T + t_row * R / w.T
+        return {"value": 1.0 / per_token, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                "sample": "expert-choice routing, dispatch, combine and both top-1 routings + transitions on all "
+                          "%d tokens (%.2f s); expert MLP on %d of %d rows, %.3f s per row, extrapolated"
+                          % (w.T, t_rest, len(rows), R, t_row), "cpu": _cpu_name()}
+
+
+def make_runner(w, rank, device):
+    return ExpertChoiceRunner(w, rank, device) if kind_of(w) == "ec" else TopKRunner(w, rank, device)
+
+
+# ------------------------------------------------------------ libmoe arm
 def run_libmoe(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
 
-    from mixture_experts_routing_top_b200 import build as B, layer as Lyr, libmoe as M
+    from mixture_experts_routing_top_b200 import build as B, libmoe as M
 
     B.build()
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    prob = make_problem(w, rank, device)
-    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    L = Lyr.TopKLayer(w.T, w.d, w.E, w.k, w.F, w.capacity_factor, dt, *prob["weights"], act=w.act,
-                      norm_topk=w.norm_topk, shared_weights=prob["shared"], device=device)
-    cosel = torch.zeros((w.E, w.E), dtype=torch.int32, device=device)
+    run = make_runner(w, rank, device)
     stream = torch.cuda.current_stream(device)
-    stages = ["route", "permute", "ffn", "shared", "combine", "coselect"]
+    names = [n for n, _ in run.stages]
+    ns = len(names)
+    # inputs smaller than L2: flush it between timed steps (outside the events)
+    flush = None
+    if run.resident_bytes < 2 * L2_BYTES:
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=device)
 
     def step(ev=None):
-        if ev: ev[0].record(stream)
-        L.route(prob["logits"])
-        if ev: ev[1].record(stream)
-        L.dispatch(prob["x"])
-        if ev: ev[2].record(stream)
-        y = L.experts()
-        if ev: ev[3].record(stream)
-        sh = L.shared_expert(prob["x"])
-        if ev: ev[4].record(stream)
-        L.combine(y, sh)
-        if ev: ev[5].record(stream)
-        M.coselect(L.idx, w.E, into=cosel)
-        if ev: ev[6].record(stream)
+        for j, (_, fn) in enumerate(run.stages):
+            if ev:
+                ev[j].record(stream)
+            fn()
+        if ev:
+            ev[ns].record(stream)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     if M.device_error() != 0:
         raise RuntimeError("device fault word set during warm-up")
-    R = int(L.perm["offsets"][-1].item())
-    dropped = int(L.perm["dropped"][0].item())
+    run.after_warmup()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(args.steps)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(ns + 1)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = Clocks()
     if world > 1:
@@ -297,6 +480,8 @@ def run_libmoe(args, w, rank, world, local_rank):
     n0 = M.kernel_launches()
     t_start.record(stream)
     for i in range(args.steps):
+        if flush is not None:
+            flush.zero_()
         step(evs[i])
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -305,86 +490,89 @@ def run_libmoe(args, w, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize()
     clk = clocks.stop() if rank == 0 else None
-    elapsed_ms = t_start.elapsed_time(t_end)
-    stage_ms = {s: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, s in enumerate(stages)}
+    if flush is None:
+        elapsed_ms = t_start.elapsed_time(t_end)
+    else:
+        elapsed_ms = sum(e[0].elapsed_time(e[ns]) for e in evs)
+    stage_ms = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in enumerate(names)}
     if M.device_error() != 0:
         raise RuntimeError("device fault word set during the timed steps")
-
-    # max over ranks (slowest rank), total launches
     elapsed_ms, launches = reduce_over_ranks(elapsed_ms, launches, device)
 
     # end to end through the public API: pinned host inputs -> layer -> host output
     e2e = None
     if args.e2e_steps > 0:
-        lg_h = torch.from_numpy(prob["logits_np"]).pin_memory()
-        xn = prob["x_np"]
-        x_h = (torch.from_numpy(xn.view(np.int16)).view(torch.bfloat16) if xn.dtype == np.uint16
-               else torch.from_numpy(xn)).pin_memory()
-        out_h = torch.empty(L.out.shape, dtype=L.out.dtype).pin_memory()
-        lg_d, x_d = torch.empty_like(prob["logits"]), torch.empty_like(prob["x"])
-
-        def e2e_step():
-            lg_d.copy_(lg_h, non_blocking=True)
-            x_d.copy_(x_h, non_blocking=True)
-            out = L.forward(lg_d, x_d)
-            out_h.copy_(out, non_blocking=True)
-
+        run.e2e_setup()
         for _ in range(3):
-            e2e_step()
+            run.e2e_step()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(args.e2e_steps):
-            e2e_step()
+            run.e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
         e_ms, _ = reduce_over_ranks(a.elapsed_time(b), 0, device)
-        e2e = {"value": throughput(world, w.T, args.e2e_steps, e_ms), "unit": "tokens/s",
-               "h2d_bytes_per_step": lg_h.numel() * 4 + x_h.numel() * x_h.element_size(),
-               "d2h_bytes_per_step": out_h.numel() * out_h.element_size()}
+        hb, db = run.e2e_bytes()
+        e2e = {"value": round(throughput(world, w.T, args.e2e_steps, e_ms), 1), "unit": "tokens/s",
+               "h2d_bytes_per_step": hb, "d2h_bytes_per_step": db}
 
     if rank != 0:
         return None
     pk, pk_kind = peaks()
-    b = 2 if w.dtype == "bf16" else 4
-    sb = stage_bytes(w, R, b)
-    flops = ffn_flops(w, R)
-    ffn_ms = stage_ms["ffn"] + stage_ms["shared"]
-    achieved = flops / (ffn_ms / 1e3) / 1e12
-    peak_s = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-    stage_report = {
-        s: {"ms": round(stage_ms[s], 4),
-            **({"GB/s": round(sb[s] / (stage_ms[s] / 1e3) / 1e9, 1),
-                "frac_hbm": round(sb[s] / (stage_ms[s] / 1e3) / 1e9 / pk["hbm_gbs"], 3)} if s in sb else {})}
-        for s in stages}
-    stage_report["ffn"].update({"TFLOP/s": round(achieved, 1), "flops": flops,
-                                "frac_burst": round(achieved / pk["bf16_tflops"], 3)})
+    work = run.work()
+    report = {}
+    for n in names:
+        kind, amount = work[n]
+        ms = stage_ms[n]
+        r = {"ms": round(ms, 4)}
+        if kind == "bytes":
+            gbs = amount / (ms / 1e3) / 1e9
+            r.update({"GB/s": round(gbs, 1), "frac_hbm": round(gbs / pk["hbm_gbs"], 3), "bytes": amount})
+        else:
+            tf = amount / (ms / 1e3) / 1e12
+            r.update({"TFLOP/s": round(tf, 1), "flops": amount,
+                      "frac_burst": round(tf / pk["bf16_tflops"], 3)})
+        report[n] = r
+    dom = max(names, key=lambda n: stage_ms[n])
+    kind, amount = work[dom]
+    if kind == "flops":
+        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        ach = report[dom]["TFLOP/s"]
+        roof = {"bound": "tensor", "stage": dom, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": round(ach / peak, 4), "peak_kind": pk_kind + " sustained bf16 (cuBLAS, 4 s loop)"}
+    else:
+        peak = pk["hbm_gbs"]
+        ach = report[dom]["GB/s"]
+        roof = {"bound": "hbm", "stage": dom, "achieved": ach, "peak": peak, "unit": "GB/s",
+                "frac": round(ach / peak, 4), "peak_kind": pk_kind + " HBM copy"}
+    roof["traffic"] = traffic_for("%s/%s" % (w.name, dom))
     value = throughput(world, w.T, args.steps, elapsed_ms)
+    cfg = {"workload": w.name, "T": w.T, "d": w.d, "E": w.E}
+    cfg.update({"k": w.k, "capacity_factor": w.capacity_factor} if w.routing == "topk" else {"C": w.C})
+    if w.F:
+        cfg.update({"F": w.F, "act": w.act})
+    if w.F_shared:
+        cfg["F_shared"] = w.F_shared
+    if w.G and not w.F:
+        cfg["G"] = w.G
+    cfg.update({"global_batch": world * w.T, "parallelism": "independent replicas, one batch per GPU",
+                "l2": ("flushed between timed steps (256 MB write outside the events)" if flush is not None else
+                       "inputs larger than L2: %.2f GB resident inputs read every step" % (run.resident_bytes / 1e9))})
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic: seeded normals (logits, activations) and random-init expert weights",
-        "config": {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "F": w.F, "F_shared": w.F_shared,
-                   "capacity_factor": w.capacity_factor, "act": w.act, "global_batch": world * w.T,
-                   "parallelism": "independent replicas, one batch per GPU",
-                   "l2": "inputs larger than L2: %.2f GB of expert weights read every step" %
-                         (sum(t.numel() * t.element_size() for t in prob["weights"] if t is not None) / 1e9)},
-        "roofline": {"bound": "tensor", "kernel": "expert MLP (2 tcgen05 grouped-GEMM launches)",
-                     "achieved": round(achieved, 1), "peak": peak_s, "unit": "TFLOP/s",
-                     "frac": round(achieved / peak_s, 4), "peak_kind": pk_kind + " sustained bf16 (cuBLAS)",
-                     "traffic": traffic_of_ffn()},
-        "stages": stage_report,
-        "rows": R, "dropped": dropped,
-        "gpu_launches": launches,
-        "clocks": clk,
+        "config": cfg, "roofline": roof, "stages": report, "gpu_launches": launches, "clocks": clk,
     }
+    res.update(run.extra())
     if e2e:
         res["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(w, prob, args.cpu_rows)
+        res["cpu_baseline"] = run.cpu_baseline(args.cpu_rows)
     return res
 
 
@@ -392,52 +580,66 @@ def run_libmoe(args, w, rank, world, local_rank):
 def run_reference(args, w):
     """The oracle as it stands (single-threaded C) on the host cores.  Each
     step: routing, capacity, permutation (with the row copy) and the combine
-    over all T tokens, plus the expert MLP of one buffer row (rotating);
+    over a token sample, plus the expert MLP of one buffer row (rotating);
     throughput is extrapolated per token from those parts."""
     from oracle import oracle as O
     from mixture_experts_routing_top_b200 import synth, workloads as W
 
-    logits, x = W.make_logits(w), W.make_x(w)
-    W1, W3, W2 = W.make_weights(w)
+    Ts = min(w.T, 8192)
+    logits, x = W.make_logits(w)[:Ts], W.make_x(w)[:Ts]
+    is_ec = kind_of(w) == "ec"
+    Wt = W.make_weights(w) if w.F else None
     Ws = W.make_shared_weights(w)
-    R_probe = O.permute(O.route_topk(logits, w.k, w.norm_topk)[0], w.E,
-                        O.capacity(w.capacity_factor, w.T, w.k, w.E))["R"]
+    goe = W.equal_groups(w.E, w.G) if (w.G and not w.F) else None
+    if is_ec:
+        C = max(1, w.C * Ts // w.T)
+        R_probe = w.E * C
+    else:
+        R_probe = O.permute(O.route_topk(logits, w.k, w.norm_topk)[0], w.E,
+                            O.capacity(w.capacity_factor, Ts, w.k, w.E), goe)["R"]
     Y = synth.normal_bf16(99, 1, (R_probe, w.d)) if w.dtype == "bf16" else synth.normal_f32(99, 1, (R_probe, w.d))
 
     def step(i):
         t0 = time.perf_counter()
-        idx, gate = O.route_topk(logits, w.k, w.norm_topk)
-        p = O.permute(idx, w.E, O.capacity(w.capacity_factor, w.T, w.k, w.E))
-        buf = O.gather_rows(x, p["row_token"])
-        O.unpermute(Y, p["row_map"], gate)
+        if is_ec:
+            ec_token, ec_gate, tok_ptr, tok_row = O.route_ec(logits, C)
+            buf = O.gather_rows(x, ec_token.reshape(-1))
+            O.unpermute_ec(Y, tok_ptr, tok_row, ec_gate)
+            R = w.E * C
+            row_e = lambda r: r // C
+        else:
+            idx, gate = O.route_topk(logits, w.k, w.norm_topk)
+            p = O.permute(idx, w.E, O.capacity(w.capacity_factor, Ts, w.k, w.E), goe)
+            buf = O.gather_rows(x, p["row_token"])
+            O.unpermute(Y if w.F else buf, p["row_map"], gate)
+            R = p["R"]
+            row_e = lambda r: int(np.searchsorted(p["offsets"], r, side="right") - 1)
         t1 = time.perf_counter()
-        r = (i * 7919) % p["R"]
-        e = int(np.searchsorted(p["offsets"], r, side="right") - 1)
-        O.expert_ffn_rows(buf[r:r + 1], np.array([e], np.int32), W1, W3, W2, w.act)
-        if Ws is not None:
-            O.expert_ffn_rows(x[:1], np.zeros(1, np.int32), *Ws, "swiglu")
+        if w.F:
+            r = (i * 7919) % R
+            O.expert_ffn_rows(buf[r:r + 1], np.array([row_e(r)], np.int32), *Wt, w.act)
+            if Ws is not None:
+                O.expert_ffn_rows(x[:1], np.zeros(1, np.int32), *Ws, "swiglu")
         t2 = time.perf_counter()
-        shared_t = 0.0
-        return (t1 - t0) / w.T + (t2 - t1) * p["R"] / w.T, t2 - t0, shared_t
+        return (t1 - t0) / Ts + (t2 - t1) * (R / Ts if w.F else 0.0), t2 - t0
 
     for i in range(args.warmup):
         step(i)
     per_token, wall = [], []
     for i in range(args.steps):
-        pt, wt, _ = step(args.warmup + i)
+        pt, wt = step(args.warmup + i)
         per_token.append(pt)
         wall.append(wt)
     value = len(per_token) / sum(per_token)
+    sample = ("per step: routing, capacity, permutation, row copy and combine over %d of %d tokens%s, "
+              "extrapolated per token" % (Ts, w.T, ", plus the expert MLP of one buffer row" if w.F else ""))
     return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(wall), 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic: seeded normals and random-init expert weights",
-            "config": {"workload": w.name, "T": w.T, "d": w.d, "E": w.E, "k": w.k, "F": w.F,
-                       "capacity_factor": w.capacity_factor},
+            "config": {"workload": w.name, "T": w.T, "d": w.d, "E": w.E},
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": "per step: route, capacity, permute, row copy and combine over all %d "
-                                       "tokens, expert MLP of one buffer row, extrapolated per token" % w.T,
-                             "cpu": _cpu_name()},
+                             "sample": sample, "cpu": _cpu_name()},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
@@ -445,17 +647,7 @@ def main():
     args = parse()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
-    from mixture_experts_routing_top_b200 import workloads as W
-
-    w = W.BY_NAME[args.workload]
-    for kv in args.set:
-        key, val = kv.split("=", 1)
-        cur = getattr(w, key)
-        w = w.with_(**{key: type(cur)(val)})
-    if args.set:
-        w = w.with_(name=w.name + "[" + ",".join(args.set) + "]")
-    if w.routing != "topk":
-        raise SystemExit("bench.py times top-k layers; %s is measured by its tests" % w.name)
+    w = workload_from_args(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
