@@ -82,22 +82,97 @@ __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict
     }
 }
 
+// Vectorised variant for E % 4 == 0 (16-byte rows): lane l loads float4
+// number l + 32 j, i.e. experts 128 j + 4 l + q.  Logits become
+// order-preserving integer keys (-0 folded into +0 so that equal values tie
+// exactly as floats do), and each selection round is two warp reductions:
+// redux.sync max over the lanes' best keys, then redux.sync min over the
+// expert indices holding that key (lowest index wins ties).  The winning
+// value is recovered from its key, so no shuffles are needed.  The softmax
+// denominator uses the hardware exp2 for each term, accumulated in fp64 (the
+// sum is dominated by the terms nearest the maximum, where that exp is within
+// a few ulp); the k gates themselves use expf with the TwoSum correction.
+__device__ __forceinline__ unsigned f2key(float v) {
+    unsigned u = __float_as_uint(__fadd_rn(v, 0.0f));
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key2f(unsigned k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+template <int NV4>
+__global__ void __launch_bounds__(256) route_topk_vec_kernel(const float* __restrict__ logits, int T, int E, int k,
+                                                             int norm_topk, int32_t* __restrict__ expert_idx,
+                                                             float* __restrict__ gate) {
+    constexpr int NV = 4 * NV4;
+    const int lane = threadIdx.x & 31;
+    const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+    const int E4 = E >> 2;
+    for (long long t = warp; t < T; t += nwarps) {
+        const uint4* row = reinterpret_cast<const uint4*>(logits + t * E);
+        float v[NV];
+        unsigned key[NV];
+        unsigned taken = 0;
+#pragma unroll
+        for (int j = 0; j < NV4; ++j) {
+            const int e4 = lane + 32 * j;
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+            if (e4 < E4) w = ld_stream(row + e4);
+            else taken |= 0xFu << (4 * j);
+            v[4 * j + 0] = __uint_as_float(w.x);
+            v[4 * j + 1] = __uint_as_float(w.y);
+            v[4 * j + 2] = __uint_as_float(w.z);
+            v[4 * j + 3] = __uint_as_float(w.w);
+        }
+#pragma unroll
+        for (int i = 0; i < NV; ++i) key[i] = f2key(v[i]);
+        float m = 0.0f, my_val = 0.0f;
+        int my_idx = -1;
+        for (int j = 0; j < k; ++j) {
+            unsigned bk = 0;                     // 0 is below every real key
+            int bi = -1;
+#pragma unroll
+            for (int i = 0; i < NV; ++i)
+                if (!((taken >> i) & 1u) && (bi < 0 || key[i] > bk)) { bk = key[i]; bi = i; }
+            const unsigned mk = __reduce_max_sync(0xffffffffu, bk);
+            const unsigned cand = (bi >= 0 && bk == mk) ? (unsigned)(128 * (bi >> 2) + 4 * lane + (bi & 3)) : 0xFFFFFFFFu;
+            const unsigned win = __reduce_min_sync(0xffffffffu, cand);
+            if ((int)((win >> 2) & 31u) == lane) taken |= 1u << (4 * (win >> 7) + (win & 3u));
+            const float wv = key2f(mk);
+            if (j == 0) m = wv;
+            if (lane == j) { my_val = wv; my_idx = (int)win; }
+        }
+        auto expdiff = [m](float l) -> float {
+            float hi = __fsub_rn(l, m);
+            float bb = __fsub_rn(hi, l);                     // TwoSum(l, -m)
+            float lo = __fadd_rn(__fsub_rn(l, __fsub_rn(hi, bb)), __fsub_rn(-m, bb));
+            float e = expf(hi);
+            return __fmaf_rn(e, lo, e);
+        };
+        const float my_e = lane < k ? expdiff(my_val) : 0.0f;
+        double s = 0.0;
+        if (norm_topk) {
+            s = (double)my_e;
+        } else {
+#pragma unroll
+            for (int i = 0; i < NV; ++i)
+                if (128 * (i >> 2) + 4 * lane + (i & 3) < E) s += (double)__expf(__fsub_rn(v[i], m));
+        }
+        s = warp_sum(s);
+        if (lane < k) {
+            expert_idx[t * k + lane] = my_idx;
+            gate[t * k + lane] = (float)((double)my_e / s);
+        }
+    }
+}
+
 // ---------------------------------------------------------- expert choice
 // Scores compare as key = logit - lse, lse = m + log(sum_e exp(logit - m)),
 // all in fp64 with the sum taken over e in ascending order (one thread per
 // token), so the keys are those of the plain definition up to the last ulp
 // of exp/log.
-
-__global__ void ec_lse_kernel(const float* __restrict__ logits, int T, int E, double* __restrict__ lse) {
-    int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= T) return;
-    const float* row = logits + (long long)t * E;
-    double m = -INFINITY;
-    for (int e = 0; e < E; ++e) m = fmax(m, (double)__ldg(row + e));
-    double s = 0.0;
-    for (int e = 0; e < E; ++e) s += exp((double)__ldg(row + e) - m);
-    lse[t] = m + log(s);
-}
 
 // Order-preserving map of a double onto uint64 (larger double -> larger key).
 __device__ __forceinline__ unsigned long long key_bits(double x) {
@@ -105,22 +180,65 @@ __device__ __forceinline__ unsigned long long key_bits(double x) {
     return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
 }
 
-// keysT[e][t] = key_bits(logit[t][e] - lse[t]), transposed through shared
-// memory so that both the read and the write are coalesced.
-__global__ void ec_keys_kernel(const float* __restrict__ logits, const double* __restrict__ lse, int T, int E,
-                               unsigned long long* __restrict__ keysT) {
-    __shared__ unsigned long long tile[32][33];
-    const int t0 = blockIdx.x * 32, e0 = blockIdx.y * 32;
-    const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // 32 x 8 threads
-    for (int r = ty; r < 32; r += 8) {
-        int t = t0 + r, e = e0 + tx;
-        if (t < T && e < E) tile[r][tx] = key_bits((double)logits[(long long)t * E + e] - lse[t]);
+// A CTA takes `tpb` consecutive tokens (one contiguous span of logits).
+// Everything order-independent runs in parallel over the CTA's tokens x
+// experts: the copy into shared memory, each row's max, every
+// exp(l - m) in fp64; only the additions run one thread per token, over the
+// experts in ascending order (the order of the logsumexp definition), from
+// the staged exps.  Keys are then written transposed, keysT[e][t], with
+// consecutive threads on consecutive tokens.
+constexpr int kEcThreads = 256;
+
+__global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __restrict__ logits, int T, int E, int tpb,
+                                                                 double* __restrict__ lse_out,
+                                                                 unsigned long long* __restrict__ keysT) {
+    extern __shared__ double ex[];                 // [tpb][E+1] exps (padded rows), then [tpb] row max / lse
+    const int ld = E + 1;
+    double* rowv = ex + (size_t)tpb * ld;
+    const long long t0 = (long long)blockIdx.x * tpb;
+    const int rows = (int)min((long long)tpb, (long long)T - t0);
+    const float* src = logits + t0 * E;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    // row max (exact in any order): one warp per row
+    for (int r = wid; r < rows; r += nw) {
+        float m = -INFINITY;
+        for (int c = lane; c < E; c += 32) m = fmaxf(m, __ldg(src + (long long)r * E + c));
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) rowv[r] = (double)m;
     }
     __syncthreads();
-    for (int r = ty; r < 32; r += 8) {
-        int e = e0 + r, t = t0 + tx;
-        if (t < T && e < E) keysT[(long long)e * T + t] = tile[tx][r];
+    // every exp(l - m) in fp64, in parallel
+    const int n = rows * E;
+#pragma unroll 4
+    for (int f = threadIdx.x; f < n; f += blockDim.x) {
+        const int r = f / E, c = f - r * E;
+        ex[r * ld + c] = exp((double)__ldg(src + f) - rowv[r]);
     }
+    __syncthreads();
+    // ascending-expert sums, one thread per token
+    for (int r = threadIdx.x; r < rows; r += blockDim.x) {
+        const double* er = ex + (size_t)r * ld;
+        double sum = 0.0;
+#pragma unroll 8
+        for (int c = 0; c < E; ++c) sum += er[c];
+        const double l = rowv[r] + log(sum);
+        rowv[r] = l;
+        lse_out[t0 + r] = l;
+    }
+    __syncthreads();
+    // keys, transposed and coalesced
+#pragma unroll 4
+    for (int f = threadIdx.x; f < rows * E; f += blockDim.x) {
+        const int c = f / rows, r = f - c * rows;
+        keysT[(long long)c * T + t0 + r] = key_bits((double)__ldg(src + (long long)r * E + c) - rowv[r]);
+    }
+}
+
+int ec_tokens_per_block(int E) {
+    int tpb = 32;                                   // ~33 KB at E = 128: several CTAs per SM
+    while (tpb > 1 && (size_t)tpb * (E + 2) * sizeof(double) > 96 * 1024) tpb >>= 1;
+    return tpb;
 }
 
 // Block-wide exclusive scan of one int per thread (blockDim = 1024).
@@ -151,73 +269,352 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* total, int* sh /
     return base + x - v;
 }
 
-// One 1024-thread CTA per expert: radix-select the C-th largest key
-// (8 passes of 8 bits, stopping early once the boundary bucket is taken
-// whole), then a stable compaction in token order; equal keys at the
-// boundary go to the lowest token indices.  Also marks token membership
-// bits for the CSR build.
+// One 1024-thread CTA per expert: radix-select the C-th largest key, then a
+// stable compaction in token order (equal keys at the boundary go to the
+// lowest token indices).  The leading bits all keys share (from their min
+// and max) are skipped; each pass histograms the next 8 bits of the keys
+// still matching the chosen prefix, with one shared-memory atomic per
+// distinct digit per warp (__match_any_sync); the search stops once the
+// boundary bucket is taken whole.  Also sets the token-membership bits used
+// to build the token CSR.
 __global__ void __launch_bounds__(1024) ec_select_kernel(const unsigned long long* __restrict__ keysT,
                                                          const float* __restrict__ logits, const double* __restrict__ lse,
                                                          int T, int E, int C, int32_t* __restrict__ ec_token,
                                                          float* __restrict__ ec_gate, unsigned* __restrict__ tokmask,
                                                          int mask_words) {
     __shared__ int hist[256];
-    __shared__ int sh_scan[32];
-    __shared__ unsigned long long s_prefix, s_mask;
-    __shared__ int s_need, s_done;
+    __shared__ unsigned long long s_prefix, s_mask, s_min, s_max;
+    __shared__ int s_need, s_done, s_hi;
     const int e = blockIdx.x;
+    const int lane = threadIdx.x & 31;
     const unsigned long long* keys = keysT + (long long)e * T;
-    if (threadIdx.x == 0) { s_prefix = 0; s_mask = 0; s_need = C; s_done = 0; }
+    if (threadIdx.x == 0) { s_min = ~0ull; s_max = 0ull; }
     __syncthreads();
-    for (int pass = 0; pass < 8; ++pass) {
-        if (s_done) break;
-        const int shift = 56 - 8 * pass;
+    unsigned long long lmin = ~0ull, lmax = 0ull;
+    for (int t = threadIdx.x; t < T; t += blockDim.x) {
+        const unsigned long long u = keys[t];
+        lmin = min(lmin, u);
+        lmax = max(lmax, u);
+    }
+    atomicMin(&s_min, lmin);
+    atomicMax(&s_max, lmax);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned long long diff = s_min ^ s_max;
+        s_need = C;
+        if (diff == 0) {                          // every key equal: the C lowest tokens
+            s_prefix = s_min; s_mask = ~0ull; s_done = 1; s_hi = -1;
+        } else {
+            const int hi = 63 - __clzll(diff);    // highest differing bit
+            const unsigned long long low = (hi == 63) ? ~0ull : ((1ull << (hi + 1)) - 1ull);
+            s_mask = ~low;
+            s_prefix = s_min & ~low;
+            s_done = 0;
+            s_hi = hi;
+        }
+    }
+    __syncthreads();
+    while (!s_done && s_hi >= 0) {
+        const int hi = s_hi;
+        const int shift = max(hi - 7, 0);
+        const int width = hi - shift + 1;
+        const unsigned bins_mask = (1u << width) - 1u;
         for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
         __syncthreads();
         const unsigned long long prefix = s_prefix, mask = s_mask;
-        for (int t = threadIdx.x; t < T; t += blockDim.x) {
-            unsigned long long u = keys[t];
-            if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255], 1);
+        for (int t0 = 0; t0 < T; t0 += blockDim.x) {
+            const int t = t0 + threadIdx.x;
+            int digit = -1;
+            if (t < T) {
+                const unsigned long long u = keys[t];
+                if ((u & mask) == prefix) digit = (int)((u >> shift) & bins_mask);
+            }
+            const unsigned peers = __match_any_sync(0xffffffffu, digit);
+            if (digit >= 0 && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[digit], __popc(peers));
         }
         __syncthreads();
         if (threadIdx.x == 0) {
-            int need = s_need, cum = 0, dgt = 255;
+            int need = s_need, cum = 0, dgt = (int)bins_mask;
             for (; dgt > 0; --dgt) {
                 if (cum + hist[dgt] >= need) break;
                 cum += hist[dgt];
             }
             need -= cum;
+            const unsigned long long field = (unsigned long long)bins_mask << shift;
             s_prefix = prefix | ((unsigned long long)dgt << shift);
-            s_mask = mask | (255ull << shift);
+            s_mask = mask | field;
             s_need = need;
-            if (hist[dgt] == need) s_done = 1;       // the whole boundary bucket is taken
+            if (hist[dgt] == need || shift == 0) s_done = 1;   // boundary bucket taken whole, or key fully resolved
+            s_hi = shift - 1;
         }
         __syncthreads();
     }
+    // stable compaction: warp w owns tokens [w*S, (w+1)*S); pass 1 counts the
+    // keys above the threshold prefix and the ties per warp, one scan over
+    // the 32 warps gives each warp its bases, pass 2 writes in token order.
     const unsigned long long prefix = s_prefix, mask = s_mask;
     const int need = s_need;
-    int ties_before = 0, taken_before = 0;
-    for (int t0 = 0; t0 < T; t0 += blockDim.x) {
-        int t = t0 + threadIdx.x;
-        int above = 0, tie = 0;
-        if (t < T) {
-            unsigned long long u = keys[t] & mask;
+    __shared__ int w_above[32], w_tie[32];
+    const int wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int S = (T + nw - 1) / nw;
+    const int seg0 = min(wid * S, T), seg1 = min(seg0 + S, T);
+    const unsigned lt = (1u << lane) - 1u;
+    int n_above = 0, n_tie = 0;
+    for (int c = seg0; c < seg1; c += 32) {
+        const int t = c + lane;
+        bool above = false, tie = false;
+        if (t < seg1) {
+            const unsigned long long u = keys[t] & mask;
             above = u > prefix;
             tie = u == prefix;
         }
-        int tie_total;
-        int tie_rank = ties_before + block_exclusive_scan(tie, &tie_total, sh_scan);
-        int sel = above || (tie && tie_rank < need);
-        int sel_total;
-        int pos = taken_before + block_exclusive_scan(sel, &sel_total, sh_scan);
+        n_above += __popc(__ballot_sync(0xffffffffu, above));
+        n_tie += __popc(__ballot_sync(0xffffffffu, tie));
+    }
+    if (lane == 0) { w_above[wid] = n_above; w_tie[wid] = n_tie; }
+    __syncthreads();
+    int above_base = 0, tie_base = 0;
+    for (int q = 0; q < wid; ++q) { above_base += w_above[q]; tie_base += w_tie[q]; }
+    int sel_base = above_base + min(tie_base, need);
+    for (int c = seg0; c < seg1; c += 32) {
+        const int t = c + lane;
+        bool above = false, tie = false;
+        if (t < seg1) {
+            const unsigned long long u = keys[t] & mask;
+            above = u > prefix;
+            tie = u == prefix;
+        }
+        const unsigned tie_mask = __ballot_sync(0xffffffffu, tie);
+        const int tie_rank = tie_base + __popc(tie_mask & lt);
+        const bool sel = above || (tie && tie_rank < need);
+        const unsigned sel_mask = __ballot_sync(0xffffffffu, sel);
         if (sel) {
-            long long r = (long long)e * C + pos;
+            const long long r = (long long)e * C + sel_base + __popc(sel_mask & lt);
             ec_token[r] = t;
-            ec_gate[r] = (float)exp((double)logits[(long long)t * E + e] - lse[t]);
             atomicOr(&tokmask[(long long)t * mask_words + (e >> 5)], 1u << (e & 31));
         }
-        ties_before += tie_total;
-        taken_before += sel_total;
+        tie_base += __popc(tie_mask);
+        sel_base += __popc(sel_mask);
+    }
+}
+
+// Warp 0: scanning digit bins from the top, find the bin where the running
+// count first reaches `need` (nbins <= 256, 8 bins per lane, one warp scan).
+// Writes the bin and the count still needed inside it.
+__device__ __forceinline__ void warp_find_boundary(const int* hist, int nbins, int need, int* out_bin,
+                                                   int* out_need, int* out_count) {
+    const int lane = threadIdx.x & 31;
+    int c[8], sum = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int b = nbins - 1 - 8 * lane - j;
+        c[j] = b >= 0 ? hist[b] : 0;
+        sum += c[j];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const unsigned hit = __ballot_sync(0xffffffffu, incl >= need);
+    const int L = hit ? __ffs(hit) - 1 : 31;
+    if (lane == L) {
+        int cum = incl - sum, bin = nbins - 1 - 8 * lane, cnt = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int b = nbins - 1 - 8 * lane - j;
+            if (b < 0) break;
+            bin = b;
+            cnt = c[j];
+            if (cum + c[j] >= need) break;
+            cum += c[j];
+        }
+        *out_bin = bin;
+        *out_need = need - cum;
+        *out_count = cnt;
+    }
+}
+
+// Shared-memory-resident variant (T <= kEcSmemTokens): the high 32 bits of
+// expert e's T keys are loaded once (coalesced, 8 loads in flight per
+// thread) and every radix pass and both compaction passes read them from
+// shared memory.  The threshold is resolved on the high half first; only if
+// the boundary bucket still has to be split are the low halves of the keys
+// whose high half equals the threshold's read from global memory (a second
+// radix over those tokens).  Same selection as ec_select_kernel.
+constexpr int kEcSmemTokens = 49152;
+
+__global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned long long* __restrict__ keysT,
+                                                              const float* __restrict__ logits,
+                                                              const double* __restrict__ lse, int T, int E, int C,
+                                                              int32_t* __restrict__ ec_token, float* __restrict__ ec_gate,
+                                                              unsigned* __restrict__ tokmask, int mask_words) {
+    extern __shared__ unsigned hi_keys[];          // [T]
+    __shared__ int hist[256];
+    __shared__ unsigned s_min, s_max, s_prefix, s_mask;
+    __shared__ unsigned s_lprefix, s_lmask;
+    __shared__ int s_need, s_done, s_hi, s_level, s_bin, s_bneed, s_bcount;
+    __shared__ int w_above[32], w_tie[32];
+    const int e = blockIdx.x;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const unsigned long long* keys = keysT + (long long)e * T;
+    if (threadIdx.x == 0) { s_min = 0xFFFFFFFFu; s_max = 0u; }
+    __syncthreads();
+    unsigned lmin = 0xFFFFFFFFu, lmax = 0u;
+    for (int t0 = 0; t0 < T; t0 += 8 * blockDim.x) {
+        unsigned long long u[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int t = t0 + q * blockDim.x + threadIdx.x;
+            u[q] = t < T ? keys[t] : 0ull;
+        }
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            const int t = t0 + q * blockDim.x + threadIdx.x;
+            if (t < T) {
+                const unsigned h = (unsigned)(u[q] >> 32);
+                hi_keys[t] = h;
+                lmin = min(lmin, h);
+                lmax = max(lmax, h);
+            }
+        }
+    }
+    atomicMin(&s_min, lmin);
+    atomicMax(&s_max, lmax);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        s_need = C;
+        s_level = 0;
+        const unsigned diff = s_min ^ s_max;
+        if (diff == 0) { s_prefix = s_min; s_mask = 0xFFFFFFFFu; s_hi = -1; }
+        else {
+            const int hb = 31 - __clz(diff);
+            const unsigned low = (hb == 31) ? 0xFFFFFFFFu : ((1u << (hb + 1)) - 1u);
+            s_mask = ~low;
+            s_prefix = s_min & ~low;
+            s_hi = hb;
+        }
+        s_done = 0;
+        s_lprefix = 0; s_lmask = 0;
+    }
+    __syncthreads();
+    // level 0: radix on the high halves (shared memory only)
+    while (!s_done && s_hi >= 0) {
+        const int hb = s_hi;
+        const int shift = max(hb - 7, 0);
+        const unsigned bins_mask = (1u << (hb - shift + 1)) - 1u;
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+        __syncthreads();
+        const unsigned prefix = s_prefix, mask = s_mask;
+        for (int t0 = 0; t0 < T; t0 += 4 * blockDim.x) {
+            int digit[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int t = t0 + q * blockDim.x + threadIdx.x;
+                digit[q] = -1;
+                if (t < T) {
+                    const unsigned h = hi_keys[t];
+                    if ((h & mask) == prefix) digit[q] = (int)((h >> shift) & bins_mask);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const unsigned peers = __match_any_sync(0xffffffffu, digit[q]);
+                if (digit[q] >= 0 && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[digit[q]], __popc(peers));
+            }
+        }
+        __syncthreads();
+        if (wid == 0) warp_find_boundary(hist, (int)bins_mask + 1, s_need, &s_bin, &s_bneed, &s_bcount);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const int dgt = s_bin;
+            s_prefix = prefix | ((unsigned)dgt << shift);
+            s_mask = mask | (bins_mask << shift);
+            s_need = s_bneed;
+            if (s_bcount == s_bneed) s_done = 1;
+            s_hi = shift - 1;
+        }
+        __syncthreads();
+    }
+    // level 1: split the boundary bucket on the low halves (global loads of
+    // the few tokens whose high half equals the threshold's)
+    if (!s_done) {
+        if (threadIdx.x == 0) { s_level = 1; s_hi = 31; s_lprefix = 0; s_lmask = 0; }
+        __syncthreads();
+        const unsigned hprefix = s_prefix;
+        while (!s_done && s_hi >= 0) {
+            const int hb = s_hi;
+            const int shift = max(hb - 7, 0);
+            const unsigned bins_mask = (1u << (hb - shift + 1)) - 1u;
+            for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+            __syncthreads();
+            const unsigned lprefix = s_lprefix, lmask = s_lmask;
+            for (int t0 = 0; t0 < T; t0 += blockDim.x) {
+                const int t = t0 + threadIdx.x;
+                int digit = -1;
+                if (t < T && hi_keys[t] == hprefix) {
+                    const unsigned lo = (unsigned)keys[t];
+                    if ((lo & lmask) == lprefix) digit = (int)((lo >> shift) & bins_mask);
+                }
+                const unsigned peers = __match_any_sync(0xffffffffu, digit);
+                if (digit >= 0 && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[digit], __popc(peers));
+            }
+            __syncthreads();
+            if (wid == 0) warp_find_boundary(hist, (int)bins_mask + 1, s_need, &s_bin, &s_bneed, &s_bcount);
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                const int dgt = s_bin;
+                s_lprefix = lprefix | ((unsigned)dgt << shift);
+                s_lmask = lmask | (bins_mask << shift);
+                s_need = s_bneed;
+                if (s_bcount == s_bneed || shift == 0) s_done = 1;
+                s_hi = shift - 1;
+            }
+            __syncthreads();
+        }
+    }
+    const unsigned prefix = s_prefix, mask = s_mask, lprefix = s_lprefix, lmask = s_lmask;
+    const int need = s_need, level = s_level;
+    // classify a token: 1 above the threshold, 2 tie at it, 0 below
+    auto classify = [&](int t) -> int {
+        const unsigned h = hi_keys[t] & mask;
+        if (h != prefix) return h > prefix ? 1 : 0;
+        if (level == 0) return 2;
+        if (hi_keys[t] != prefix) return hi_keys[t] > prefix ? 1 : 0;   // differs below the high mask
+        const unsigned lo = (unsigned)keys[t] & lmask;
+        if (lo != lprefix) return lo > lprefix ? 1 : 0;
+        return 2;
+    };
+    const int S = (T + nw - 1) / nw;
+    const int seg0 = min(wid * S, T), seg1 = min(seg0 + S, T);
+    const unsigned lt = (1u << lane) - 1u;
+    int n_above = 0, n_tie = 0;
+    for (int c = seg0; c < seg1; c += 32) {
+        const int t = c + lane;
+        const int cl = t < seg1 ? classify(t) : 0;
+        n_above += __popc(__ballot_sync(0xffffffffu, cl == 1));
+        n_tie += __popc(__ballot_sync(0xffffffffu, cl == 2));
+    }
+    if (lane == 0) { w_above[wid] = n_above; w_tie[wid] = n_tie; }
+    __syncthreads();
+    int above_base = 0, tie_base = 0;
+    for (int q = 0; q < wid; ++q) { above_base += w_above[q]; tie_base += w_tie[q]; }
+    int sel_base = above_base + min(tie_base, need);
+    for (int c = seg0; c < seg1; c += 32) {
+        const int t = c + lane;
+        const int cl = t < seg1 ? classify(t) : 0;
+        const unsigned tie_mask = __ballot_sync(0xffffffffu, cl == 2);
+        const int tie_rank = tie_base + __popc(tie_mask & lt);
+        const bool sel = cl == 1 || (cl == 2 && tie_rank < need);
+        const unsigned sel_mask = __ballot_sync(0xffffffffu, sel);
+        if (sel) {
+            const long long r = (long long)e * C + sel_base + __popc(sel_mask & lt);
+            ec_token[r] = t;
+            atomicOr(&tokmask[(long long)t * mask_words + (e >> 5)], 1u << (e & 31));
+        }
+        tie_base += __popc(tie_mask);
+        sel_base += __popc(sel_mask);
     }
 }
 
@@ -262,13 +659,18 @@ __global__ void scan_add_kernel(int32_t* __restrict__ out, int n, const int32_t*
     if (i < n) out[i] += block_base[i >> 10];
 }
 
-// tok_row[tok_ptr[t] + (#experts below e that chose t)] = row, for every row.
-__global__ void ec_fill_kernel(const int32_t* __restrict__ ec_token, int E, int C, const unsigned* __restrict__ tokmask,
-                               int mask_words, const int32_t* __restrict__ tok_ptr, int32_t* __restrict__ tok_row) {
+// For every buffer row r = e*C + i holding token t: its gate exp(key) and
+// tok_row[tok_ptr[t] + (#experts below e that chose t)] = r.
+__global__ void ec_fill_kernel(const int32_t* __restrict__ ec_token, int T, int E, int C,
+                               const unsigned* __restrict__ tokmask, int mask_words,
+                               const int32_t* __restrict__ tok_ptr, const float* __restrict__ logits,
+                               const double* __restrict__ lse, float* __restrict__ ec_gate,
+                               int32_t* __restrict__ tok_row) {
     long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (r >= (long long)E * C) return;
     int e = (int)(r / C);
     int t = ec_token[r];
+    ec_gate[r] = (float)exp((double)logits[(long long)t * E + e] - lse[t]);
     const unsigned* m = tokmask + (long long)t * mask_words;
     int below = 0;
     for (int w = 0; w < (e >> 5); ++w) below += __popc(m[w]);
@@ -294,6 +696,20 @@ extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, i
     int blocks = (int)((warps_needed + 7) / 8);
     if (blocks > 148 * 16) blocks = 148 * 16;
     const int nv = (E + 31) / 32;
+    if (E % 4 == 0 && ((uintptr_t)logits & 15) == 0) {
+        const int nv4 = (E + 127) / 128;
+#define MOE_TOPKV_CASE(N) \
+    case N: route_topk_vec_kernel<N><<<blocks, threads, 0, s>>>(logits, T, E, k, norm_topk, expert_idx, gate); break;
+        switch (nv4 <= 1 ? 1 : nv4 <= 2 ? 2 : nv4 <= 4 ? 4 : 8) {
+            MOE_TOPKV_CASE(1)
+            MOE_TOPKV_CASE(2)
+            MOE_TOPKV_CASE(4)
+            MOE_TOPKV_CASE(8)
+        }
+#undef MOE_TOPKV_CASE
+        MOE_LAUNCH_CHECK();
+        return MOE_OK;
+    }
 #define MOE_TOPK_CASE(N) \
     case N: route_topk_kernel<N><<<blocks, threads, 0, s>>>(logits, T, E, k, norm_topk, expert_idx, gate); break;
     switch (nv <= 1 ? 1 : nv <= 2 ? 2 : nv <= 4 ? 4 : nv <= 8 ? 8 : nv <= 16 ? 16 : 32) {
@@ -351,11 +767,25 @@ extern "C" moe_status moe_route_ec(const float* logits, int T, int E, int C, int
     int32_t* btot = (int32_t*)(ws + L.btot);
     const int mw = (E + 31) / 32;
     if (cudaMemsetAsync(mask, 0, sizeof(unsigned) * (size_t)T * mw, s) != cudaSuccess) return MOE_ERR_CUDA;
-    ec_lse_kernel<<<ceil_div(T, 128), 128, 0, s>>>(logits, T, E, lse);
-    MOE_LAUNCH_CHECK();
-    ec_keys_kernel<<<dim3(ceil_div(T, 32), ceil_div(E, 32)), 256, 0, s>>>(logits, lse, T, E, keys);
-    MOE_LAUNCH_CHECK();
-    ec_select_kernel<<<E, 1024, 0, s>>>(keys, logits, lse, T, E, C, ec_token, ec_gate, mask, mw);
+    {
+        const int tpb = ec_tokens_per_block(E);
+        const size_t smem = (size_t)tpb * (E + 2) * sizeof(double);
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(ec_lse_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        ec_lse_keys_kernel<<<ceil_div(T, tpb), kEcThreads, smem, s>>>(logits, T, E, tpb, lse, keys);
+        MOE_LAUNCH_CHECK();
+    }
+    if (T <= kEcSmemTokens) {
+        const size_t smem = sizeof(unsigned) * (size_t)T;
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(ec_select_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+                cudaSuccess)
+            return MOE_ERR_CUDA;
+        ec_select_smem_kernel<<<E, 1024, smem, s>>>(keys, logits, lse, T, E, C, ec_token, ec_gate, mask, mw);
+    } else {
+        ec_select_kernel<<<E, 1024, 0, s>>>(keys, logits, lse, T, E, C, ec_token, ec_gate, mask, mw);
+    }
     MOE_LAUNCH_CHECK();
     ec_count_kernel<<<ceil_div(T, 256), 256, 0, s>>>(mask, T, mw, cnt);
     MOE_LAUNCH_CHECK();
@@ -370,7 +800,8 @@ extern "C" moe_status moe_route_ec(const float* logits, int T, int E, int C, int
     scan_add_kernel<<<ceil_div(n, 256), 256, 0, s>>>(tok_ptr, n, btot);
     MOE_LAUNCH_CHECK();
     const long long rows = (long long)E * C;
-    ec_fill_kernel<<<(int)((rows + 255) / 256), 256, 0, s>>>(ec_token, E, C, mask, mw, tok_ptr, tok_row);
+    ec_fill_kernel<<<(int)((rows + 255) / 256), 256, 0, s>>>(ec_token, T, E, C, mask, mw, tok_ptr, logits, lse, ec_gate,
+                                                              tok_row);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }
