@@ -29,6 +29,7 @@
 // tensor-core kind keeps fp32 accuracy).
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
@@ -398,6 +399,311 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
 
 }  // namespace tc
 
+// ------------------------------------------------------ 2-CTA (CTA pair)
+// The same grouped GEMM with tcgen05.mma.cta_group::2: a cluster of two
+// CTAs on the two SMs of a TPC computes a 256-row x 256-column tile.  Each
+// CTA stages its own 128 rows of A and one half of B (N rows 0-127 in the
+// even CTA, 128-255 in the odd one; for SwiGLU that is the W1 tile and the
+// W3 tile), so per SM a k-block costs 32 KB of shared memory instead of 48
+// and six stages fit.  The even CTA's thread issues the MMAs (M=256); its
+// accumulator rows live in the even CTA's TMEM, the odd half in the odd
+// CTA's.  Both CTAs' TMA loads complete on the even CTA's stage barrier
+// (address mapped with mapa; plain loads, no multicast); tcgen05.commit
+// multicasts each stage release and each accumulator-ready signal to both
+// CTAs; the odd CTA's epilogue arrives remotely on the even CTA's
+// accumulator-empty barrier.  Waits are bounded as in the one-CTA kernel.
+namespace tc2 {
+using namespace tc;
+
+constexpr int BM = 256;                       // rows per tile (pair)
+constexpr int STAGES = 6;
+constexpr int A_BYTES = 128 * BK * 2;         // 16 KB per CTA
+constexpr int B_BYTES = 128 * BK * 2;         // 16 KB per CTA (half of N = 256)
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + 4 * (MAX_E + 1);
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+    uint32_t out;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(addr), "r"(rank));
+    return out;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void arrive_remote(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" :: "r"(cluster_addr) : "memory");
+}
+
+// Bounded wait with cluster-scope acquire (for barriers other CTAs arrive on).
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const volatile int* abort_flag) {
+    long long t0 = 0;
+    for (uint32_t i = 1;; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done) : "r"(bar), "r"(parity) : "memory");
+        if (done) return true;
+        if ((i & 255u) == 0) {
+            if (*abort_flag) return false;
+            const long long now = globaltimer();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > WAIT_NS) return false;
+        }
+    }
+}
+
+// TMA into this CTA's shared memory, completing on the barrier at `bar_cluster`
+// (a shared::cluster address: the even CTA's stage barrier).
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar_cluster) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster) : "memory");
+}
+
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc) : "memory");
+}
+
+// Arrives on the barrier at this shared offset in every CTA of `mask`.
+__device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t mask) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 :: "r"(bar), "h"(mask) : "memory");
+}
+
+template <int MODE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b0,
+                     const __grid_constant__ CUtensorMap map_b1, GemmArgs args) {
+    constexpr int BN_OUT = (MODE == MODE_SWIGLU) ? 128 : 256;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    uint8_t* stage_base = smem;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* full = bars;                     // [STAGES] (used in the even CTA)
+    uint64_t* empty = bars + STAGES;           // [STAGES]
+    uint64_t* tfull = bars + 2 * STAGES;       // [2]
+    uint64_t* tempty = bars + 2 * STAGES + 2;  // [2] (used in the even CTA)
+    uint64_t* drain = bars + 2 * STAGES + 4;   // [1]
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* tile_prefix = reinterpret_cast<int*>(smem + STAGES * STAGE_BYTES + 256);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_rank();
+    const bool leader = rank == 0;
+    const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+    const int E = args.E;
+    const int n_tiles = (args.N_out + BN_OUT - 1) / BN_OUT;
+    const int nk = args.K / BK;
+
+    if (threadIdx.x == 0) {
+        for (int st = 0; st < STAGES; ++st) {
+            mbar_init(smem_u32(&full[st]), 1);
+            mbar_init(smem_u32(&empty[st]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull[a]), 1);
+            mbar_init(smem_u32(&tempty[a]), 256);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 0 && lane == 0) {
+        tma_prefetch_desc(&map_a);
+        tma_prefetch_desc(&map_b0);
+        if (MODE == MODE_SWIGLU) tma_prefetch_desc(&map_b1);
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_u32(tmem_slot)), "r"(2 * ACC_N) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+    }
+    if (warp == 2 && lane == 0) {
+        int acc = 0;
+        tile_prefix[0] = 0;
+        for (int e = 0; e < E; ++e) {
+            int b = min(max(args.offsets[e], 0), args.R_max);
+            int en = min(max(args.offsets[e + 1], 0), args.R_max);
+            int cnt = max(en - b, 0);
+            acc += ((cnt + BM - 1) / BM) * n_tiles;
+            tile_prefix[e + 1] = acc;
+        }
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+    const int total = tile_prefix[E];
+
+    auto decode = [&](int t, int& row0, int& row_end, int& n0, int& e_out) {
+        int lo = 0, hi = E;
+        while (lo < hi) {
+            int mid = (lo + hi + 1) >> 1;
+            if (tile_prefix[mid] <= t) lo = mid; else hi = mid - 1;
+        }
+        const int e = lo;
+        const int b = min(max(args.offsets[e], 0), args.R_max);
+        const int en = min(max(args.offsets[e + 1], 0), args.R_max);
+        const int mt = (en - b + BM - 1) / BM;
+        const int local = t - tile_prefix[e];
+        const int n_idx = local / mt, m_idx = local - n_idx * mt;
+        row0 = b + m_idx * BM;
+        row_end = en;
+        n0 = n_idx * BN_OUT;
+        e_out = e;
+    };
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            uint32_t issued = 0, fill_parity = 0;
+            for (int t = pair; t < total && !*abort_flag; t += npairs) {
+                int row0, row_end, n0, e;
+                decode(t, row0, row_end, n0, e);
+                const int arow = row0 + (int)rank * 128;
+                int brow;
+                const CUtensorMap* bmap = &map_b0;
+                if (MODE == MODE_SWIGLU) {
+                    brow = e * args.w_rows + n0;
+                    if (!leader) bmap = &map_b1;
+                } else {
+                    brow = e * args.w_rows + n0 + (int)rank * 128;
+                }
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) { *abort_flag = 1; break; }
+                    const uint32_t fb_local = smem_u32(&full[stage]);
+                    const uint32_t fb = map_to_rank(fb_local, 0);
+                    const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+                    const uint32_t sb = sa + A_BYTES;
+                    if (leader) mbar_expect_tx(fb_local, 2 * STAGE_BYTES);
+                    issued |= 1u << stage;
+                    fill_parity = (fill_parity & ~(1u << stage)) | (phase << stage);
+                    tma_load_2d_pair(sa, &map_a, kb * BK, arow, fb);
+                    tma_load_2d_pair(sb, bmap, kb * BK, brow, fb);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+            }
+            // the even CTA's own fills have landed before it may exit; the
+            // odd CTA's fills complete on the even CTA's barriers, which the
+            // even CTA's MMA thread consumed (or which time out)
+            int never = 0;
+            if (leader)
+                for (int st = 0; st < STAGES; ++st)
+                    if (issued & (1u << st)) mbar_wait(smem_u32(&full[st]), (fill_parity >> st) & 1u, &never);
+        }
+    } else if (warp == 1) {
+        if (lane == 0 && leader) {
+            constexpr uint32_t idesc = umma_idesc_bf16(BM, ACC_N);
+            int stage = 0;
+            uint32_t phase = 0;
+            int it = 0;
+            for (int t = pair; t < total && !*abort_flag; t += npairs, ++it) {
+                const int acc = it & 1;
+                const uint32_t acc_phase = (it >> 1) & 1;
+                if (!mbar_wait_cluster(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag)) { *abort_flag = 1; break; }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + acc * ACC_N;
+                bool ok = true;
+                for (int kb = 0; kb < nk; ++kb) {
+                    if (!mbar_wait_cluster(smem_u32(&full[stage]), phase, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t sa = smem_u32(stage_base + stage * STAGE_BYTES);
+                    const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk)
+                        umma_bf16_pair(d_tmem, umma_desc_sw128(sa + kk * 32), umma_desc_sw128(sb + kk * 32), idesc,
+                                       (kb | kk) != 0 ? 1u : 0u);
+                    umma_commit_pair(smem_u32(&empty[stage]), 0x3);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+                }
+                if (!ok) { *abort_flag = 1; break; }
+                umma_commit_pair(smem_u32(&tfull[acc]), 0x3);
+            }
+            umma_commit_pair(smem_u32(drain), 0x1);
+            int never = 0;
+            if (!mbar_wait(smem_u32(drain), 0, &never)) *abort_flag = 1;
+        }
+    } else {
+        const int q = warp & 3;
+        const int r = q * 32 + lane;
+        const uint32_t tempty_leader0 = map_to_rank(smem_u32(&tempty[0]), 0);
+        const uint32_t tempty_leader1 = map_to_rank(smem_u32(&tempty[1]), 0);
+        int it = 0;
+        for (int t = pair; t < total; t += npairs, ++it) {
+            int row0, row_end, n0, e;
+            decode(t, row0, row_end, n0, e);
+            const int acc = it & 1;
+            const uint32_t acc_phase = (it >> 1) & 1;
+            if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag)) { *abort_flag = 1; break; }
+            tc_fence_after();
+            const int grow = row0 + (int)rank * 128 + r;
+            const bool valid = grow < row_end;
+            const uint32_t taddr = tmem_base + acc * ACC_N + ((uint32_t)(q * 32) << 16);
+            uint16_t* orow = args.out + (long long)grow * args.N_out;
+            if (MODE == MODE_SWIGLU) {
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    float a[32], b[32];
+                    tmem_ld32(taddr + c * 32, a);
+                    tmem_ld32(taddr + 128 + c * 32, b);
+                    tmem_ld_wait();
+                    const int col = n0 + c * 32;
+                    if (valid && col < args.N_out) {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) a[i] = silu_f(a[i]) * b[i];
+                        store_row32(orow + col, a);
+                    }
+                }
+            } else {
+#pragma unroll 1
+                for (int c = 0; c < 8; ++c) {
+                    float a[32];
+                    tmem_ld32(taddr + c * 32, a);
+                    tmem_ld_wait();
+                    const int col = n0 + c * 32;
+                    if (valid && col < args.N_out) {
+                        if (MODE == MODE_GELU) {
+#pragma unroll
+                            for (int i = 0; i < 32; ++i) a[i] = gelu_f(a[i]);
+                        }
+                        store_row32(orow + col, a);
+                    }
+                }
+            }
+            tc_fence_before();
+            arrive_remote(acc ? tempty_leader1 : tempty_leader0);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag && threadIdx.x == 0) raise_error(args.err, kErrTimeout);
+    cluster_sync();                              // no remote arrival may target an exited CTA
+    if (warp == 1) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" :: "r"(tmem_base), "r"(2 * ACC_N) : "memory");
+    }
+}
+
+}  // namespace tc2
+
 // ------------------------------------------------------------- fp32 SIMT
 // H[r, f] = act(x_r . W1[e, f] (, x_r . W3[e, f])), one thread per (r, f);
 // Y[r, c] = H[r] . W2[e, c], one thread per (r, c).  e from offsets.
@@ -512,6 +818,35 @@ moe_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUte
     return MOE_OK;
 }
 
+template <int MODE>
+moe_status launch_gemm2(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, const tc::GemmArgs& a,
+                        cudaStream_t s) {
+    static bool attr_done = false;
+    if (!attr_done) {
+        if (cudaFuncSetAttribute(tc2::grouped_gemm2_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 tc2::SMEM_BYTES) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        attr_done = true;
+    }
+    const int bn_out = MODE == tc::MODE_SWIGLU ? 128 : 256;
+    const long long n_tiles = (a.N_out + bn_out - 1) / bn_out;
+    const long long m_tiles_max = (a.R_max + tc2::BM - 1) / tc2::BM + a.E;
+    const long long tiles_max = n_tiles * m_tiles_max;
+    int pairs = sm_count() / 2;
+    if (tiles_max < pairs) pairs = (int)(tiles_max > 0 ? tiles_max : 1);
+    tc2::grouped_gemm2_kernel<MODE><<<2 * pairs, tc::THREADS, tc2::SMEM_BYTES, s>>>(ma, mb0, mb1, a);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+// CTA-pair kernels when experts average at least 512 rows (256-row tiles
+// waste little); one-CTA kernels otherwise.  LIBMOE_GEMM_PAIR=0/1 forces it.
+bool use_pair_kernels(int R_max, int E) {
+    const char* env = getenv("LIBMOE_GEMM_PAIR");
+    if (env && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
+    return (long long)R_max >= 512LL * E;
+}
+
 size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 }  // namespace
@@ -563,13 +898,24 @@ extern "C" moe_status moe_expert_ffn(const void* buffer, int dtype, int R_max, i
     uint16_t* H = (uint16_t*)workspace;
     CUtensorMap m_x, m_w1, m_w3, m_h, m_w2;
     const bool swiglu = act == MOE_ACT_SWIGLU;
-    if (!make_map(&m_x, buffer, R_max, d, tc::BM)) return MOE_ERR_CUDA;
-    if (!make_map(&m_w1, W1, (long long)E * F, d, swiglu ? 128 : 256)) return MOE_ERR_CUDA;
+    const bool pair = use_pair_kernels(R_max, E);
+    // per-CTA boxes: A is always 128 rows; B is 128 rows per CTA in the pair
+    // kernels, and 128 (SwiGLU halves) or 256 rows in the one-CTA kernels
+    const int bbox = pair ? 128 : 256;
+    if (!make_map(&m_x, buffer, R_max, d, 128)) return MOE_ERR_CUDA;
+    if (!make_map(&m_w1, W1, (long long)E * F, d, swiglu ? 128 : bbox)) return MOE_ERR_CUDA;
     if (swiglu && !make_map(&m_w3, W3, (long long)E * F, d, 128)) return MOE_ERR_CUDA;
-    if (!make_map(&m_h, H, R_max, F, tc::BM)) return MOE_ERR_CUDA;
-    if (!make_map(&m_w2, W2, (long long)E * d, F, 256)) return MOE_ERR_CUDA;
+    if (!make_map(&m_h, H, R_max, F, 128)) return MOE_ERR_CUDA;
+    if (!make_map(&m_w2, W2, (long long)E * d, F, bbox)) return MOE_ERR_CUDA;
 
     tc::GemmArgs g1{offsets, E, d, F, F, R_max, H, err};
+    if (pair) {
+        moe_status st = swiglu ? launch_gemm2<tc::MODE_SWIGLU>(m_x, m_w1, m_w3, g1, s)
+                               : launch_gemm2<tc::MODE_GELU>(m_x, m_w1, m_w1, g1, s);
+        if (st != MOE_OK) return st;
+        tc::GemmArgs g2{offsets, E, F, d, d, R_max, (uint16_t*)y, err};
+        return launch_gemm2<tc::MODE_PLAIN>(m_h, m_w2, m_w2, g2, s);
+    }
     moe_status st = swiglu ? launch_gemm<tc::MODE_SWIGLU>(m_x, m_w1, m_w3, g1, s)
                            : launch_gemm<tc::MODE_GELU>(m_x, m_w1, m_w1, g1, s);
     if (st != MOE_OK) return st;

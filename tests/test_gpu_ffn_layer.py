@@ -13,6 +13,13 @@ from tests.helpers import as_f64, assert_layer_close, needs_gpu, to_dev, to_np
 pytestmark = [pytest.mark.gpu, needs_gpu]
 
 
+@pytest.fixture(params=["pair", "single"])
+def gemm_kind(request, monkeypatch):
+    """Run a test with the CTA-pair grouped GEMMs and with the one-CTA ones."""
+    monkeypatch.setenv("LIBMOE_GEMM_PAIR", "1" if request.param == "pair" else "0")
+    return request.param
+
+
 def ffn_case(counts, d, F, act, bf16=True, seed=0):
     E = len(counts)
     offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
@@ -40,8 +47,10 @@ def ffn_case(counts, d, F, act, bf16=True, seed=0):
     ([200, 333], 512, 1024, "swiglu"),             # several k-blocks and n-tiles
     ([0, 130, 300], 128, 256, "gelu"),
     ([129, 511], 320, 448, "gelu"),
-    ([1000], 64, 64, "swiglu")])
-def test_expert_ffn_bf16(counts, d, F, act):
+    ([1000], 64, 64, "swiglu"),
+    ([600, 0, 900, 257], 256, 320, "swiglu"),     # 256-row tiles with ragged tails, partial n-tiles
+    ([513, 1100], 320, 256, "gelu")])
+def test_expert_ffn_bf16(counts, d, F, act, gemm_kind):
     got, ref = ffn_case(counts, d, F, act)
     assert_layer_close(got, ref)
 
@@ -92,7 +101,7 @@ def sampled_tokens(info, T, n, seed=0):
 
 
 @pytest.mark.parametrize("w", [W.MIXTRAL, W.FINE], ids=lambda w: w.name)
-def test_layer_full_size_sampled(w):
+def test_layer_full_size_sampled(w, gemm_kind):
     logits, x = W.make_logits(w), W.make_x(w)
     Wt = W.make_weights(w)
     Ws = W.make_shared_weights(w)
@@ -123,7 +132,7 @@ def test_layer_dispatch_combine_identity(G):
     np.testing.assert_allclose(got, as_f64(x), rtol=1e-5, atol=1e-6)   # renormalised gates: y == x
 
 
-def test_layer_expert_choice_sampled():
+def test_layer_expert_choice_sampled(gemm_kind):
     w = W.EXPERT_CHOICE
     logits, x = W.make_logits(w), W.make_x(w)
     W1, _, W2 = W.make_weights(w)
