@@ -159,7 +159,7 @@ moe_status moe_permute(const void* x, int dtype, int T, int d,
  * Scratch: a fixed MOE_PERMUTE_NOALLOC_SCRATCH_BYTES array in device memory,
  * held by every GPU that loads the library until the process exits.
  * Limit: moe_permute_workspace_bytes(T, k, E, G) must not exceed it
- * (e.g. T = 131072, k = 8, E = 256, G = 64 needs 2.25 MiB); larger problems
+ * (e.g. T = 131072, k = 8, E = 256, G = 64 needs 3.25 MiB); larger problems
  * return MOE_ERR_WORKSPACE and launch nothing.  The first call on a device
  * looks up the array's device address (cudaGetSymbolAddress) and caches it;
  * make that first call before any stream capture.  All calls share the one

@@ -8,7 +8,7 @@
 // Each CTA owns one SM: a TMA warp streams 128x64 A tiles and 256x64 B tiles
 // (128-byte swizzle) into a 4-stage shared-memory ring; one thread issues
 // tcgen05.mma (M=128, N=256, K=16, bf16 in, fp32 accumulate in TMEM); four
-// epilogue warps drain the accumulator with tcgen05.ld, apply the
+// epilogue warps (one per TMEM lane quarter) drain the accumulator with tcgen05.ld, apply the
 // activation and store bf16.  Two TMEM accumulators (2 x 256 columns) let
 // the epilogue of one tile overlap the MMAs of the next.  For SwiGLU the B
 // tile stacks 128 rows of W1 over the same 128 rows of W3, so one MMA chain
@@ -44,7 +44,8 @@ constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;         // 16 KB
 constexpr int B_BYTES = ACC_N * BK * 2;      // 32 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int THREADS = 192;                 // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
+constexpr int EPI_WARPS = 4;                 // one warp per TMEM lane quarter (EPI_WARPS = 8 splits the columns in half)
+constexpr int THREADS = 64 + 32 * EPI_WARPS;  // warp 0 TMA, warp 1 MMA, then the epilogue warps
 constexpr int MAX_E = 1024;
 constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/ + 4 * (MAX_E + 1);
 constexpr long long WAIT_NS = 4000000000LL;  // 4 s
@@ -215,7 +216,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&tfull[a]), 1);
-            mbar_init(smem_u32(&tempty[a]), 128);
+            mbar_init(smem_u32(&tempty[a]), 32 * EPI_WARPS);
         }
         mbar_init(smem_u32(drain), 1);
         *abort_flag = 0;
@@ -338,8 +339,9 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
             if (!mbar_wait(smem_u32(drain), 0, &never)) *abort_flag = 1;
         }
     } else {
-        // epilogue: warps 2..5 -> TMEM lane quarter (warp % 4)
+        // epilogue: warps 2.. -> TMEM lane quarter (warp % 4), column part
         const int q = warp & 3;
+        const int half = (EPI_WARPS == 8) ? ((warp - 2) >> 2) : 0;
         const int r = q * 32 + lane;
         int it = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
@@ -355,7 +357,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
             uint16_t* orow = args.out + (long long)grow * args.N_out;
             if (MODE == MODE_SWIGLU) {
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = (16 / EPI_WARPS) * half; c < (16 / EPI_WARPS) * half + 16 / EPI_WARPS; ++c) {
                     float a[32], b[32];
                     tmem_ld32(taddr + c * 32, a);
                     tmem_ld32(taddr + 128 + c * 32, b);
@@ -369,7 +371,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                 }
             } else {
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
+                for (int c = (32 / EPI_WARPS) * half; c < (32 / EPI_WARPS) * half + 32 / EPI_WARPS; ++c) {
                     float a[32];
                     tmem_ld32(taddr + c * 32, a);
                     tmem_ld_wait();
@@ -517,7 +519,7 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&tfull[a]), 1);
-            mbar_init(smem_u32(&tempty[a]), 256);
+            mbar_init(smem_u32(&tempty[a]), 2 * 32 * EPI_WARPS);
         }
         mbar_init(smem_u32(drain), 1);
         *abort_flag = 0;
@@ -642,6 +644,7 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
         }
     } else {
         const int q = warp & 3;
+        const int half = (EPI_WARPS == 8) ? ((warp - 2) >> 2) : 0;
         const int r = q * 32 + lane;
         const uint32_t tempty_leader0 = map_to_rank(smem_u32(&tempty[0]), 0);
         const uint32_t tempty_leader1 = map_to_rank(smem_u32(&tempty[1]), 0);
@@ -659,7 +662,7 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
             uint16_t* orow = args.out + (long long)grow * args.N_out;
             if (MODE == MODE_SWIGLU) {
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
+                for (int c = (16 / EPI_WARPS) * half; c < (16 / EPI_WARPS) * half + 16 / EPI_WARPS; ++c) {
                     float a[32], b[32];
                     tmem_ld32(taddr + c * 32, a);
                     tmem_ld32(taddr + 128 + c * 32, b);
@@ -673,7 +676,7 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
                 }
             } else {
 #pragma unroll 1
-                for (int c = 0; c < 8; ++c) {
+                for (int c = (32 / EPI_WARPS) * half; c < (32 / EPI_WARPS) * half + 32 / EPI_WARPS; ++c) {
                     float a[32];
                     tmem_ld32(taddr + c * 32, a);
                     tmem_ld_wait();

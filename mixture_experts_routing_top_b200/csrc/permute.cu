@@ -10,16 +10,20 @@
 //
 // Plan (all int32, no atomics on the ordering path, so results are
 // deterministic):
-//   1. count:   per token block b and key (expert or group), how many slots
-//               of the block carry the key  -> cnt[key][b]
-//   2. scan:    per key, exclusive scan over blocks -> base[key][b], total
-//   3. offsets: capacity clamp per expert, exclusive scan over keys,
+//   1. count:   per token block b and expert, how many slots of the block
+//               carry the expert -> cnt[e][b]
+//   2. scan:    per expert, exclusive scan over blocks -> base[e][b], total
+//   3. offsets: capacity clamp per expert, exclusive scan over experts,
 //               dropped = sum(load - kept)
+//      (1-3 run as one launch whose last CTA does the scans when experts x
+//      blocks is small; as three launches otherwise)
 //   4. rank:    per block, the stable (token-order) rank of each slot among
-//               the block's slots with the same key, plus base: the global
-//               token-order rank.  Expert-major: row = offsets[e] + rank if
-//               rank < capacity.  Group-major: kept flags first, then the
-//               same count/scan/rank over the (token, group) head slots.
+//               the block's slots with the same expert, plus base: the
+//               global token-order rank; row = offsets[e] + rank if rank <
+//               capacity.  Group-major instead: one kernel derives the kept
+//               slots, each token's group heads and the per-block group
+//               counts (its last CTA scanning them), one kernel ranks the
+//               heads per group and gives every kept slot its head's row.
 //   5. copy:    one token per warp, x[t] read once (16-byte vectors) and
 //               written to each distinct row the token owns.
 #include <mutex>
@@ -31,42 +35,21 @@ namespace moe {
 constexpr int kTB = 256;       // tokens per block in the index kernels
 constexpr int kIdxThreads = 256;
 
-// Key of slot s.  mode 0: the expert.  mode 1: the group of the expert if
-// the slot is the first kept slot of its token into that group, else -1.
-__device__ __forceinline__ int slot_key(int mode, const int32_t* __restrict__ idx, const uint8_t* __restrict__ kept,
-                                        const int32_t* __restrict__ goe, long long s, int k, int E, int nkeys,
-                                        unsigned* err) {
-    int e = idx[s];
-    if (e < 0 || e >= E) { raise_error(err, kErrIndex); return -1; }
-    if (mode == 0) return e;
-    if (!kept[s]) return -1;
-    int g = goe[e];
-    if (g < 0 || g >= nkeys) { raise_error(err, kErrIndex); return -1; }
-    long long t0 = (s / k) * k;
-    for (long long q = t0; q < s; ++q) {
-        int eq = idx[q];
-        if (eq >= 0 && eq < E && kept[q] && goe[eq] == g) return -1;   // an earlier slot already owns the row
-    }
-    return g;
-}
-
-// 1. per-block histogram of keys, stored key-major: cnt[key * nblk + b]
-__global__ void __launch_bounds__(kIdxThreads) perm_count_kernel(int mode, const int32_t* __restrict__ idx,
-                                                                 const uint8_t* __restrict__ kept,
-                                                                 const int32_t* __restrict__ goe, int T, int k, int E,
-                                                                 int nkeys, int nblk, int32_t* __restrict__ cnt,
-                                                                 unsigned* err) {
+// 1. per-block histogram of experts, stored expert-major: cnt[e * nblk + b]
+__global__ void __launch_bounds__(kIdxThreads) perm_count_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
+                                                                 int nblk, int32_t* __restrict__ cnt, unsigned* err) {
     extern __shared__ int hist[];
-    for (int i = threadIdx.x; i < nkeys; i += blockDim.x) hist[i] = 0;
+    for (int i = threadIdx.x; i < E; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     const long long s0 = (long long)blockIdx.x * kTB * k;
     const long long s1 = min((long long)(blockIdx.x + 1) * kTB, (long long)T) * k;
     for (long long s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
-        int key = slot_key(mode, idx, kept, goe, s, k, E, nkeys, err);
-        if (key >= 0 && key < nkeys) atomicAdd(&hist[key], 1);
+        const int e = idx[s];
+        if (e < 0 || e >= E) { raise_error(err, kErrIndex); continue; }
+        atomicAdd(&hist[e], 1);
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < nkeys; i += blockDim.x) cnt[(long long)i * nblk + blockIdx.x] = hist[i];
+    for (int i = threadIdx.x; i < E; i += blockDim.x) cnt[(long long)i * nblk + blockIdx.x] = hist[i];
 }
 
 // 2. one CTA per key: exclusive scan over the blocks, total per key.
@@ -156,36 +139,28 @@ __global__ void __launch_bounds__(1024) perm_offsets_kernel(const int32_t* __res
     }
 }
 
-// 4. stable in-block ranks.  The block's slots are split into 8 contiguous
-// runs, one per warp; a warp walks its run 32 slots at a time and ranks
-// equal keys with __match_any_sync.  Per-warp, per-key counts are scanned
+// Stable in-block ranks: the block's slots [s0, s1) are split into one
+// contiguous run per warp; a warp walks its run 32 slots at a time and ranks
+// equal keys with __match_any_sync; per-warp, per-key counts are scanned
 // across warps so that ranks follow slot order over the whole block.
-// out_mode 0 (expert-major rows), 1 (kept flags only), 2 (group rows).
-template <int OUT>
-__global__ void __launch_bounds__(kIdxThreads) perm_rank_kernel(int mode, const int32_t* __restrict__ idx,
-                                                                uint8_t* __restrict__ kept,
-                                                                const int32_t* __restrict__ goe, int T, int k, int E,
-                                                                int nkeys, int nblk, const int32_t* __restrict__ base,
-                                                                long long cap, const int32_t* __restrict__ offsets,
-                                                                int32_t* __restrict__ row_map, int32_t* __restrict__ row_token,
-                                                                unsigned* err) {
-    extern __shared__ int sm[];
-    int* wcnt = sm;                              // [8][nkeys]: counts, then exclusive warp bases
-    const int nw = kIdxThreads / 32;
+// rank = base_s[key] (the count of the key in earlier blocks) + position
+// among this block's earlier slots with the same key.  key_of(s) < 0 skips a
+// slot.  Called by the whole block.
+template <typename KeyOf, typename OnRank>
+__device__ __forceinline__ void block_stable_ranks(long long s0, long long s1, int nkeys, const int* base_s, int* wcnt,
+                                                   KeyOf key_of, OnRank on_rank) {
+    const int nw = blockDim.x >> 5;
     const int wid = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < nw * nkeys; i += blockDim.x) wcnt[i] = 0;
     __syncthreads();
-    const long long s0 = (long long)blockIdx.x * kTB * k;
-    const long long s1 = min((long long)(blockIdx.x + 1) * kTB, (long long)T) * k;
     const long long n = s1 - s0;
     const long long per = (n + nw - 1) / nw;
     const long long w0 = s0 + min(n, per * wid), w1 = s0 + min(n, per * (wid + 1));
-    // pass 1: per-warp counts
     for (long long c = w0; c < w1; c += 32) {
-        long long s = c + lane;
-        int key = s < w1 ? slot_key(mode, idx, kept, goe, s, k, E, nkeys, err) : -1;
-        unsigned act = __ballot_sync(0xffffffffu, key >= 0);
-        unsigned peers = __match_any_sync(0xffffffffu, key);
+        const long long s = c + lane;
+        const int key = s < w1 ? key_of(s) : -1;
+        const unsigned act = __ballot_sync(0xffffffffu, key >= 0);
+        const unsigned peers = __match_any_sync(0xffffffffu, key);
         if (key >= 0 && (peers & act & lanemask_lt()) == 0) wcnt[wid * nkeys + key] += __popc(peers & act);
         __syncwarp();
     }
@@ -193,63 +168,223 @@ __global__ void __launch_bounds__(kIdxThreads) perm_rank_kernel(int mode, const 
     for (int key = threadIdx.x; key < nkeys; key += blockDim.x) {
         int run = 0;
         for (int w = 0; w < nw; ++w) {
-            int c = wcnt[w * nkeys + key];
+            const int c = wcnt[w * nkeys + key];
             wcnt[w * nkeys + key] = run;
             run += c;
         }
     }
     __syncthreads();
-    // pass 2: ranks
     for (long long c = w0; c < w1; c += 32) {
-        long long s = c + lane;
-        int key = s < w1 ? slot_key(mode, idx, kept, goe, s, k, E, nkeys, err) : -1;
-        unsigned act = __ballot_sync(0xffffffffu, key >= 0);
-        unsigned peers = __match_any_sync(0xffffffffu, key) & act;
+        const long long s = c + lane;
+        const int key = s < w1 ? key_of(s) : -1;
+        const unsigned act = __ballot_sync(0xffffffffu, key >= 0);
+        const unsigned peers = __match_any_sync(0xffffffffu, key) & act;
         int rank = 0;
-        if (key >= 0) rank = base[(long long)key * nblk + blockIdx.x] + wcnt[wid * nkeys + key] + __popc(peers & lanemask_lt());
+        if (key >= 0) rank = base_s[key] + wcnt[wid * nkeys + key] + __popc(peers & lanemask_lt());
         __syncwarp();
         if (key >= 0 && (peers & lanemask_lt()) == 0) wcnt[wid * nkeys + key] += __popc(peers);
         __syncwarp();
-        if (s < w1) {
-            if (OUT == 0) {
-                if (key >= 0 && rank < cap) {
-                    int r = offsets[key] + rank;
-                    row_map[s] = r;
-                    row_token[r] = (int32_t)(s / k);
-                } else {
-                    row_map[s] = -1;
-                }
-            } else if (OUT == 1) {
-                kept[s] = (key >= 0 && rank < cap) ? 1 : 0;
-            } else {
-                if (key >= 0) {
-                    int r = offsets[key] + rank;
-                    row_map[s] = r;
-                    row_token[r] = (int32_t)(s / k);
-                }
-            }
-        }
+        if (s < w1) on_rank(s, key, rank);
     }
 }
 
-// Group-major: kept slots that are not their group's head take the head's row.
-__global__ void perm_group_fill_kernel(const int32_t* __restrict__ idx, const uint8_t* __restrict__ kept,
-                                       const int32_t* __restrict__ goe, int T, int k, int E, int G,
-                                       int32_t* __restrict__ row_map) {
-    long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= T) return;
-    const long long s0 = t * k;
-    for (int j = 0; j < k; ++j) {
-        long long s = s0 + j;
-        int e = idx[s];
-        if (e < 0 || e >= E || !kept[s]) { row_map[s] = -1; continue; }
-        int g = goe[e];
-        if (g < 0 || g >= G) { row_map[s] = -1; continue; }
-        for (int q = 0; q < j; ++q) {
-            int eq = idx[s0 + q];
-            if (eq >= 0 && eq < E && kept[s0 + q] && goe[eq] == g) { row_map[s] = row_map[s0 + q]; break; }
+// Each block's view of the scans, into shared memory: base_s[key] = the
+// key's count in the blocks before this one; off_s[key] = exclusive scan over
+// keys of the clamped totals min(total, cap).  `fused`: computed here from
+// cnt[key][block] (for small keys x blocks, one pass over cnt per block);
+// otherwise read from the outputs of the scan kernels (base[key][block],
+// offsets).  With `fused`, block 0 also writes counts, offsets
+// ([nkeys] = rows) and dropped, each when non-null.
+__device__ void block_scan_prologue(bool fused, const int32_t* __restrict__ cnt, const int32_t* __restrict__ base,
+                                    const int32_t* offsets_in, int nkeys, int nblk, long long cap,
+                                    int* base_s, int* off_s, int32_t* __restrict__ counts,
+                                    int32_t* offsets_out, int32_t* __restrict__ dropped) {
+    __shared__ int wsum[32];
+    __shared__ long long wdrop[32];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    if (!fused) {
+        for (int key = threadIdx.x; key < nkeys; key += blockDim.x) {
+            base_s[key] = base[(long long)key * nblk + blockIdx.x];
+            off_s[key] = offsets_in ? offsets_in[key] : 0;
+        }
+        __syncthreads();
+        return;
+    }
+    long long drop = 0;
+    for (int key = threadIdx.x; key < nkeys; key += blockDim.x) {
+        const int32_t* c = cnt + (long long)key * nblk;
+        int before = 0, tot = 0;
+        for (int i = 0; i < nblk; ++i) {
+            const int v = c[i];
+            if (i < (int)blockIdx.x) before += v;
+            tot += v;
+        }
+        base_s[key] = before;
+        const int kept = (int)min((long long)tot, cap);
+        off_s[key] = kept;                      // scanned below
+        if (blockIdx.x == 0 && counts) counts[key] = kept;
+        drop += tot - kept;
+    }
+    drop = warp_sum(drop);
+    if (lane == 0) wdrop[wid] = drop;
+    __syncthreads();
+    int carry = 0;
+    for (int k0 = 0; k0 < nkeys; k0 += blockDim.x) {
+        const int key = k0 + threadIdx.x;
+        const int v = key < nkeys ? off_s[key] : 0;
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) wsum[wid] = x;
+        __syncthreads();
+        int wb = 0, tot = 0;
+        for (int w = 0; w < nw; ++w) {
+            if (w < wid) wb += wsum[w];
+            tot += wsum[w];
+        }
+        if (key < nkeys) {
+            off_s[key] = carry + wb + x - v;
+            if (blockIdx.x == 0 && offsets_out) offsets_out[key] = off_s[key];
+        }
+        carry += tot;
+        __syncthreads();
+    }
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        if (offsets_out) offsets_out[nkeys] = carry;
+        if (dropped) {
+            long long d = 0;
+            for (int w = 0; w < nw; ++w) d += wdrop[w];
+            *dropped = (int32_t)d;
         }
     }
+    __syncthreads();
+}
+
+// Group-major, part 1 (one CTA per kTB tokens): expert ranks -> kept slots;
+// then, one thread per token, each kept slot's group, whether it is the
+// first kept slot of its token in that group (the row's "head"), and the
+// per-block head count of every group.  code[s]: group id for a head,
+// -2 - j for a kept slot whose head is slot j of the same token, -1 for a
+// dropped slot.
+__global__ void __launch_bounds__(kIdxThreads) perm_group_heads_kernel(
+    const int32_t* __restrict__ idx, const int32_t* __restrict__ goe, int T, int k, int E, int G, int nblk, int fused,
+    const int32_t* __restrict__ ecnt, const int32_t* __restrict__ ebase, long long cap, int32_t* __restrict__ counts,
+    int32_t* __restrict__ dropped, int16_t* __restrict__ code, int32_t* __restrict__ gcnt, unsigned* err) {
+    extern __shared__ int sm[];
+    int* wcnt = sm;                                          // [8][E]
+    int* base_s = wcnt + (kIdxThreads / 32) * E;             // [E]
+    int* off_s = base_s + E;                                 // [E]
+    int* ghist = off_s + E;                                  // [G]
+    uint8_t* kept_s = reinterpret_cast<uint8_t*>(ghist + G); // [kTB * k]
+    const long long s0 = (long long)blockIdx.x * kTB * k;
+    const long long s1 = min((long long)(blockIdx.x + 1) * kTB, (long long)T) * k;
+    for (int i = threadIdx.x; i < G; i += blockDim.x) ghist[i] = 0;
+    block_scan_prologue(fused, ecnt, ebase, nullptr, E, nblk, cap, base_s, off_s, counts, nullptr, dropped);
+    block_stable_ranks(
+        s0, s1, E, base_s, wcnt,
+        [&](long long s) -> int {
+            const int e = idx[s];
+            if (e < 0 || e >= E) { raise_error(err, kErrIndex); return -1; }
+            return e;
+        },
+        [&](long long s, int key, int rank) { kept_s[s - s0] = (key >= 0 && rank < cap) ? 1 : 0; });
+    __syncthreads();
+    const long long t0 = (long long)blockIdx.x * kTB;
+    const int ntok = (int)((s1 - s0) / k);
+    for (int tl = threadIdx.x; tl < ntok; tl += blockDim.x) {
+        const long long sb = (t0 + tl) * k;
+        for (int j = 0; j < k; ++j) {
+            const long long s = sb + j;
+            int c = -1;
+            if (kept_s[s - s0]) {
+                const int g = goe[idx[s]];
+                if (g < 0 || g >= G) {
+                    raise_error(err, kErrIndex);
+                } else {
+                    int jh = -1;
+                    for (int q = 0; q < j; ++q)
+                        if (kept_s[sb + q - s0] && goe[idx[sb + q]] == g) { jh = q; break; }
+                    if (jh < 0) { c = g; atomicAdd(&ghist[g], 1); }
+                    else c = -2 - jh;
+                }
+            }
+            code[s] = (int16_t)c;
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < G; i += blockDim.x) gcnt[(long long)i * nblk + blockIdx.x] = ghist[i];
+}
+
+// Group-major, part 2: head slots get stable per-group ranks (token order)
+// and their rows; every other kept slot takes its head's row.
+__global__ void __launch_bounds__(kIdxThreads) perm_group_rows_kernel(
+    const int16_t* __restrict__ code, int T, int k, int G, int nblk, int fused, const int32_t* __restrict__ gcnt,
+    const int32_t* __restrict__ gbase, const int32_t* __restrict__ goffsets_in, int32_t* __restrict__ offsets,
+    int32_t* __restrict__ row_map, int32_t* __restrict__ row_token) {
+    extern __shared__ int sm[];
+    int* wcnt = sm;                                          // [8][G]
+    int* base_s = wcnt + (kIdxThreads / 32) * G;             // [G]
+    int* off_s = base_s + G;                                 // [G]
+    int* rows_s = off_s + G;                                 // [kTB * k]
+    const long long s0 = (long long)blockIdx.x * kTB * k;
+    const long long s1 = min((long long)(blockIdx.x + 1) * kTB, (long long)T) * k;
+    block_scan_prologue(fused, gcnt, gbase, goffsets_in, G, nblk, (long long)T * k, base_s, off_s, nullptr, offsets,
+                        nullptr);
+    block_stable_ranks(
+        s0, s1, G, base_s, wcnt, [&](long long s) -> int { return (int)code[s]; },
+        [&](long long s, int key, int rank) {
+            int r = -1;
+            if (key >= 0) {
+                r = off_s[key] + rank;
+                row_token[r] = (int32_t)(s / k);
+            }
+            rows_s[s - s0] = r;
+        });
+    __syncthreads();
+    for (long long s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
+        const int c = code[s];
+        int r = -1;
+        if (c >= 0) r = rows_s[s - s0];
+        else if (c <= -2) r = rows_s[(s / k) * k + (-2 - c) - s0];
+        row_map[s] = r;
+    }
+}
+
+// 4. expert-major rows: stable ranks per expert (token order); a slot is
+// kept if its rank is below the capacity, at row offsets[e] + rank.
+__global__ void __launch_bounds__(kIdxThreads) perm_rank_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
+                                                                int nblk, int fused, const int32_t* __restrict__ cnt,
+                                                                const int32_t* __restrict__ base, long long cap,
+                                                                int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                                int32_t* __restrict__ dropped,
+                                                                int32_t* __restrict__ row_map,
+                                                                int32_t* __restrict__ row_token, unsigned* err) {
+    extern __shared__ int sm[];
+    int* wcnt = sm;                              // [8][E]
+    int* base_s = wcnt + (kIdxThreads / 32) * E; // [E]
+    int* off_s = base_s + E;                     // [E]
+    const long long s0 = (long long)blockIdx.x * kTB * k;
+    const long long s1 = min((long long)(blockIdx.x + 1) * kTB, (long long)T) * k;
+    block_scan_prologue(fused, cnt, base, offsets, E, nblk, cap, base_s, off_s, counts, offsets, dropped);
+    block_stable_ranks(
+        s0, s1, E, base_s, wcnt,
+        [&](long long s) -> int {
+            const int e = idx[s];
+            if (e < 0 || e >= E) { raise_error(err, kErrIndex); return -1; }
+            return e;
+        },
+        [&](long long s, int key, int rank) {
+            if (key >= 0 && rank < cap) {
+                const int r = off_s[key] + rank;
+                row_map[s] = r;
+                row_token[r] = (int32_t)(s / k);
+            } else {
+                row_map[s] = -1;
+            }
+        });
 }
 
 // 5. token-major row copy: warp per token, x[t] read once, written to each
@@ -351,8 +486,10 @@ namespace {
 size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 struct PermWs {
-    size_t cnt, base, total, kept, gcnt, gbase, gtotal, bytes;
+    size_t cnt, base, total, code, gcnt, gbase, gtotal, bytes;
 };
+
+constexpr long long kFuseLimit = 16384;   // keys x blocks each consumer block scans itself
 
 PermWs perm_layout(int T, int k, int E, int G) {
     const int nblk = ceil_div(T, kTB) > 0 ? ceil_div(T, kTB) : 1;
@@ -360,18 +497,23 @@ PermWs perm_layout(int T, int k, int E, int G) {
     w.cnt = 0;
     w.base = w.cnt + al256(sizeof(int32_t) * (size_t)E * nblk);
     w.total = w.base + al256(sizeof(int32_t) * (size_t)E * nblk);
-    w.kept = w.total + al256(sizeof(int32_t) * (size_t)E);
-    size_t end = w.kept;
+    size_t end = w.total + al256(sizeof(int32_t) * (size_t)E);
     if (G > 0) {
-        w.gcnt = w.kept + al256((size_t)T * k);
+        w.code = end;
+        w.gcnt = w.code + al256(sizeof(int16_t) * (size_t)T * k);
         w.gbase = w.gcnt + al256(sizeof(int32_t) * (size_t)G * nblk);
         w.gtotal = w.gbase + al256(sizeof(int32_t) * (size_t)G * nblk);
         end = w.gtotal + al256(sizeof(int32_t) * (size_t)G);
     } else {
-        w.gcnt = w.gbase = w.gtotal = end;
+        w.code = w.gcnt = w.gbase = w.gtotal = end;
     }
     w.bytes = end;
     return w;
+}
+
+bool set_smem(const void* fn, size_t bytes) {
+    if (bytes <= 48 * 1024) return true;
+    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
 }
 
 moe_status launch_copy_slots(const void* x, int T, int row_bytes, const int32_t* row_map, int k, void* buffer,
@@ -440,45 +582,48 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
     int32_t* base = (int32_t*)(ws + L.base);
     int32_t* total = (int32_t*)(ws + L.total);
     const int nw = kIdxThreads / 32;
-    // expert pass: counts, scan, capacity
-    perm_count_kernel<<<nblk, kIdxThreads, sizeof(int) * E, s>>>(0, expert_idx, nullptr, nullptr, T, k, E, E, nblk, cnt, err);
+    // 1. per-block expert counts
+    perm_count_kernel<<<nblk, kIdxThreads, sizeof(int) * E, s>>>(expert_idx, T, k, E, nblk, cnt, err);
     MOE_LAUNCH_CHECK();
-    perm_scan_blocks_kernel<<<E, 1024, 0, s>>>(cnt, nblk, base, total);
-    MOE_LAUNCH_CHECK();
-    const size_t rank_smem = sizeof(int) * (size_t)nw * (group_of_expert ? (E > G ? E : G) : E);
-    if (rank_smem > 48 * 1024) {
-        if (cudaFuncSetAttribute(perm_rank_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rank_smem) != cudaSuccess ||
-            cudaFuncSetAttribute(perm_rank_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rank_smem) != cudaSuccess ||
-            cudaFuncSetAttribute(perm_rank_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)rank_smem) != cudaSuccess)
-            return MOE_ERR_CUDA;
+    // 2-3. the scans: done by every consumer block itself when experts x
+    // blocks is small, else by two kernels
+    const int fused_e = (long long)E * nblk <= kFuseLimit;
+    int32_t* eoffsets = group_of_expert ? nullptr : offsets;
+    if (!fused_e) {
+        perm_scan_blocks_kernel<<<E, 1024, 0, s>>>(cnt, nblk, base, total);
+        MOE_LAUNCH_CHECK();
+        perm_offsets_kernel<<<1, 1024, 0, s>>>(total, E, cap, counts, eoffsets, dropped);
+        MOE_LAUNCH_CHECK();
     }
     if (!group_of_expert) {
-        perm_offsets_kernel<<<1, 1024, 0, s>>>(total, E, cap, counts, offsets, dropped);
-        MOE_LAUNCH_CHECK();
-        perm_rank_kernel<0><<<nblk, kIdxThreads, rank_smem, s>>>(0, expert_idx, nullptr, nullptr, T, k, E, E, nblk, base,
-                                                                 cap, offsets, row_map, row_token, err);
+        // 4. ranks and rows (its block 0 writes counts, offsets and dropped when fused)
+        const size_t rank_smem = sizeof(int) * ((size_t)nw * E + 2 * (size_t)E);
+        if (!set_smem((const void*)perm_rank_kernel, rank_smem)) return MOE_ERR_CUDA;
+        perm_rank_kernel<<<nblk, kIdxThreads, rank_smem, s>>>(expert_idx, T, k, E, nblk, fused_e, cnt, base, cap,
+                                                              counts, offsets, dropped, row_map, row_token, err);
         MOE_LAUNCH_CHECK();
     } else {
-        uint8_t* kept = (uint8_t*)(ws + L.kept);
+        int16_t* code = (int16_t*)(ws + L.code);
         int32_t* gcnt = (int32_t*)(ws + L.gcnt);
         int32_t* gbase = (int32_t*)(ws + L.gbase);
         int32_t* gtotal = (int32_t*)(ws + L.gtotal);
-        perm_offsets_kernel<<<1, 1024, 0, s>>>(total, E, cap, counts, nullptr, dropped);
+        const size_t heads_smem = sizeof(int) * ((size_t)nw * E + 2 * (size_t)E + G) + (size_t)kTB * k;
+        if (!set_smem((const void*)perm_group_heads_kernel, heads_smem)) return MOE_ERR_CUDA;
+        perm_group_heads_kernel<<<nblk, kIdxThreads, heads_smem, s>>>(expert_idx, group_of_expert, T, k, E, G, nblk,
+                                                                        fused_e, cnt, base, cap, counts, dropped, code,
+                                                                        gcnt, err);
         MOE_LAUNCH_CHECK();
-        perm_rank_kernel<1><<<nblk, kIdxThreads, rank_smem, s>>>(0, expert_idx, kept, nullptr, T, k, E, E, nblk, base,
-                                                                 cap, nullptr, nullptr, nullptr, err);
-        MOE_LAUNCH_CHECK();
-        perm_count_kernel<<<nblk, kIdxThreads, sizeof(int) * G, s>>>(1, expert_idx, kept, group_of_expert, T, k, E, G,
-                                                                       nblk, gcnt, err);
-        MOE_LAUNCH_CHECK();
-        perm_scan_blocks_kernel<<<G, 1024, 0, s>>>(gcnt, nblk, gbase, gtotal);
-        MOE_LAUNCH_CHECK();
-        perm_offsets_kernel<<<1, 1024, 0, s>>>(gtotal, G, (long long)T * k, nullptr, offsets, nullptr);
-        MOE_LAUNCH_CHECK();
-        perm_rank_kernel<2><<<nblk, kIdxThreads, rank_smem, s>>>(1, expert_idx, kept, group_of_expert, T, k, E, G, nblk,
-                                                                 gbase, (long long)T * k, offsets, row_map, row_token, err);
-        MOE_LAUNCH_CHECK();
-        perm_group_fill_kernel<<<ceil_div(T, 256), 256, 0, s>>>(expert_idx, kept, group_of_expert, T, k, E, G, row_map);
+        const int fused_g = (long long)G * nblk <= kFuseLimit;
+        if (!fused_g) {
+            perm_scan_blocks_kernel<<<G, 1024, 0, s>>>(gcnt, nblk, gbase, gtotal);
+            MOE_LAUNCH_CHECK();
+            perm_offsets_kernel<<<1, 1024, 0, s>>>(gtotal, G, (long long)T * k, nullptr, offsets, nullptr);
+            MOE_LAUNCH_CHECK();
+        }
+        const size_t rows_smem = sizeof(int) * ((size_t)nw * G + 2 * (size_t)G + (size_t)kTB * k);
+        if (!set_smem((const void*)perm_group_rows_kernel, rows_smem)) return MOE_ERR_CUDA;
+        perm_group_rows_kernel<<<nblk, kIdxThreads, rows_smem, s>>>(code, T, k, G, nblk, fused_g, gcnt, gbase, offsets,
+                                                                      offsets, row_map, row_token);
         MOE_LAUNCH_CHECK();
     }
     if (x && d > 0) return launch_copy_slots(x, T, (int)row_bytes, row_map, k, buffer, s);
