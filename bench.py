@@ -270,19 +270,18 @@ class TopKRunner:
     def e2e_setup(self):
         import torch
 
-        self.h_in = [(_pinned(self.logits_np), self.logits), (_pinned(self.x_np), self.x)]
-        self.h_out = torch.empty(self.L.out.shape, dtype=self.L.out.dtype).pin_memory()
+        from mixture_experts_routing_top_b200 import layer as Lyr
 
-    def e2e_step(self):
-        for h, d in self.h_in:
-            d.copy_(h, non_blocking=True)
-        for _, fn in self.stages[:-1]:          # the layer (the statistic is not part of its output)
-            fn()
-        self.h_out.copy_(self.L.out, non_blocking=True)
+        self.h_in = [_pinned(self.logits_np), _pinned(self.x_np)]
+        self.h_out = torch.empty(self.L.out.shape, dtype=self.L.out.dtype).pin_memory()
+        self.pipe = Lyr.HostPipeline(lambda lg, x, out: self.L.forward(lg, x, out=out), [self.logits, self.x],
+                                     self.L.out)
+
+    def e2e_run(self, n):
+        self.pipe.run([self.h_in] * n, [self.h_out] * n)
 
     def e2e_bytes(self):
-        return (sum(h.numel() * h.element_size() for h, _ in self.h_in),
-                self.h_out.numel() * self.h_out.element_size())
+        return (sum(h.numel() * h.element_size() for h in self.h_in), self.h_out.numel() * self.h_out.element_size())
 
     def extra(self):
         return {"rows": self.R, "dropped": self.dropped}
@@ -383,19 +382,18 @@ class ExpertChoiceRunner:
     def e2e_setup(self):
         import torch
 
-        self.h_in = [(_pinned(self.logits_np), self.logits), (_pinned(self.x_np), self.x)]
-        self.h_out = torch.empty(self.L.out.shape, dtype=self.L.out.dtype).pin_memory()
+        from mixture_experts_routing_top_b200 import layer as Lyr
 
-    def e2e_step(self):
-        for h, d in self.h_in:
-            d.copy_(h, non_blocking=True)
-        for _, fn in self.stages[:-1]:
-            fn()
-        self.h_out.copy_(self.L.out, non_blocking=True)
+        self.h_in = [_pinned(self.logits_np), _pinned(self.x_np)]
+        self.h_out = torch.empty(self.L.out.shape, dtype=self.L.out.dtype).pin_memory()
+        self.pipe = Lyr.HostPipeline(lambda lg, x, out: self.L.forward(lg, x, out=out), [self.logits, self.x],
+                                     self.L.out)
+
+    def e2e_run(self, n):
+        self.pipe.run([self.h_in] * n, [self.h_out] * n)
 
     def e2e_bytes(self):
-        return (sum(h.numel() * h.element_size() for h, _ in self.h_in),
-                self.h_out.numel() * self.h_out.element_size())
+        return (sum(h.numel() * h.element_size() for h in self.h_in), self.h_out.numel() * self.h_out.element_size())
 
     def extra(self):
         return {"rows": self.w.E * self.w.C, "tokens_chosen": self.chosen}
@@ -503,15 +501,13 @@ def run_libmoe(args, w, rank, world, local_rank):
     e2e = None
     if args.e2e_steps > 0:
         run.e2e_setup()
-        for _ in range(3):
-            run.e2e_step()
+        run.e2e_run(3)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        for _ in range(args.e2e_steps):
-            run.e2e_step()
+        run.e2e_run(args.e2e_steps)               # each step: its inputs in, the layer, its output out
         b.record(stream)
         torch.cuda.synchronize()
         e_ms, _ = reduce_over_ranks(a.elapsed_time(b), 0, device)

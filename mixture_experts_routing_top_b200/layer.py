@@ -70,15 +70,16 @@ class TopKLayer:
         return M.expert_ffn(x, self.shared_offsets, sW1, sW3, sW2, "swiglu", y=self.shared_y,
                             workspace=self.shared_ws, stream=stream)
 
-    def combine(self, y, shared=None, stream=None):
-        return M.unpermute(y, self.perm["row_map"], self.gate, shared, self.out_dtype, out=self.out, stream=stream)
+    def combine(self, y, shared=None, stream=None, out=None):
+        return M.unpermute(y, self.perm["row_map"], self.gate, shared, self.out_dtype,
+                           out=self.out if out is None else out, stream=stream)
 
-    def forward(self, logits: torch.Tensor, x: torch.Tensor, stream=None) -> torch.Tensor:
+    def forward(self, logits: torch.Tensor, x: torch.Tensor, stream=None, out=None) -> torch.Tensor:
         self.route(logits, stream)
         self.dispatch(x, stream)
         y = self.experts(stream)
         sh = self.shared_expert(x, stream)
-        return self.combine(y, sh, stream)
+        return self.combine(y, sh, stream, out)
 
 
 class ExpertChoiceLayer:
@@ -102,11 +103,58 @@ class ExpertChoiceLayer:
         self.ffn_ws = M._ws(M.expert_ffn_workspace_bytes(R, d, F, dtype), dev)
         self.out = torch.empty((T, d), dtype=self.out_dtype, device=dev)
 
-    def forward(self, logits: torch.Tensor, x: torch.Tensor, stream=None) -> torch.Tensor:
+    def forward(self, logits: torch.Tensor, x: torch.Tensor, stream=None, out=None) -> torch.Tensor:
         ec_token, ec_gate, tok_ptr, tok_row = M.route_ec(logits, self.C, workspace=self.route_ws, out=self.routing,
                                                          stream=stream)
         M.gather_rows(x, tok_ptr, tok_row, self.R, buffer=self.buffer, stream=stream)
         M.expert_ffn(self.buffer, self.offsets, self.W1, self.W3, self.W2, self.act, y=self.y,
                      workspace=self.ffn_ws, stream=stream)
-        return M.unpermute_ec(self.y, tok_ptr, tok_row, ec_gate.view(-1), self.out_dtype, out=self.out,
-                              stream=stream)
+        return M.unpermute_ec(self.y, tok_ptr, tok_row, ec_gate.view(-1), self.out_dtype,
+                              out=self.out if out is None else out, stream=stream)
+
+
+class HostPipeline:
+    """Runs a layer over a sequence of batches held in pinned host memory.
+
+    Each batch's inputs are copied to the device on one stream, the layer
+    runs on the current stream, and its output is copied back on a third, so
+    the copies of batch i+1 and of batch i-1 overlap the compute of batch i.
+    Device inputs and outputs are double-buffered; events order every reuse.
+    forward(*device_inputs, out=device_output) is the layer call.
+    """
+
+    def __init__(self, forward, device_inputs, device_output):
+        self.forward = forward
+        self.din = [list(device_inputs), [torch.empty_like(t) for t in device_inputs]]
+        self.dout = [device_output, torch.empty_like(device_output)]
+        self.s_in, self.s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]       # inputs landed
+        self.ev_used = [torch.cuda.Event() for _ in range(2)]     # compute finished with the inputs
+        self.ev_out = [torch.cuda.Event() for _ in range(2)]      # output written
+        self.ev_drained = [torch.cuda.Event() for _ in range(2)]  # output copied back
+
+    def run(self, host_inputs, host_outputs):
+        """host_inputs[i]: the pinned input tensors of batch i; host_outputs[i]:
+        its pinned output tensor.  Returns once everything is enqueued; work
+        enqueued on the current stream afterwards runs after the last copy."""
+        s_c = torch.cuda.current_stream()
+        self.s_in.wait_stream(s_c)
+        for i, (hin, hout) in enumerate(zip(host_inputs, host_outputs)):
+            b = i & 1
+            with torch.cuda.stream(self.s_in):
+                if i >= 2:
+                    self.s_in.wait_event(self.ev_used[b])
+                for h, d in zip(hin, self.din[b]):
+                    d.copy_(h, non_blocking=True)
+                self.ev_in[b].record(self.s_in)
+            s_c.wait_event(self.ev_in[b])
+            if i >= 2:
+                s_c.wait_event(self.ev_drained[b])
+            self.forward(*self.din[b], out=self.dout[b])
+            self.ev_used[b].record(s_c)
+            self.ev_out[b].record(s_c)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(self.ev_out[b])
+                hout.copy_(self.dout[b], non_blocking=True)
+                self.ev_drained[b].record(self.s_out)
+        s_c.wait_stream(self.s_out)

@@ -386,3 +386,80 @@ double oracle_local_fraction(const int32_t* expert_idx, int64_t T, int k, const 
 double oracle_silu(double z) { return silu(z); }
 double oracle_gelu(double z) { return gelu(z); }
 double oracle_round_bf16(double x) { return round_to_bf16(x); }
+
+/* -------------------------------------------- correlated placement */
+/* [Coupling] Abstract: experts that tokens often pick together are placed on
+ * the same GPU.  The pages give no algorithm; this is a plain greedy reading
+ * on the co-selection counts C (symmetric, E x E) for G groups of L = E/G:
+ * each group starts from the unassigned expert with the largest off-diagonal
+ * co-selection mass and grows by the unassigned expert with the largest
+ * summed co-selection with the group's members; ties go to the lower index.
+ * Returns 0, or 1 if G does not divide E. */
+int oracle_place_experts(const int32_t* cosel, int E, int G, int32_t* group_of_expert) {
+    if (G < 1 || E % G != 0) return 1;
+    const int L = E / G;
+    int64_t* mass = (int64_t*)calloc((size_t)E, sizeof(int64_t));
+    int64_t* aff = (int64_t*)calloc((size_t)E, sizeof(int64_t));
+    for (int x = 0; x < E; ++x) {
+        group_of_expert[x] = -1;
+        for (int y = 0; y < E; ++y)
+            if (y != x) mass[x] += cosel[(int64_t)x * E + y];
+    }
+    for (int g = 0; g < G; ++g) {
+        int seed = -1;
+        for (int x = 0; x < E; ++x)
+            if (group_of_expert[x] < 0 && (seed < 0 || mass[x] > mass[seed])) seed = x;
+        group_of_expert[seed] = g;
+        for (int x = 0; x < E; ++x) aff[x] = cosel[(int64_t)x * E + seed];
+        for (int m = 1; m < L; ++m) {
+            int best = -1;
+            for (int x = 0; x < E; ++x)
+                if (group_of_expert[x] < 0 && (best < 0 || aff[x] > aff[best])) best = x;
+            group_of_expert[best] = g;
+            for (int x = 0; x < E; ++x) aff[x] += cosel[(int64_t)x * E + best];
+        }
+    }
+    free(mass);
+    free(aff);
+    return 0;
+}
+
+/* ------------------------------------------ token shuffling statistic */
+/* [Coupling] Abstract: a token is moved to the GPU predicted to hold its
+ * next-layer experts.  Prediction from the layer-to-layer transition counts
+ * M: affinity[a][g] = sum of M[a][b] over the experts b of group g. */
+void oracle_group_affinity(const int32_t* trans, int E, const int32_t* group_of_expert, int G, int64_t* affinity) {
+    for (int64_t i = 0; i < (int64_t)E * G; ++i) affinity[i] = 0;
+    for (int a = 0; a < E; ++a)
+        for (int b = 0; b < E; ++b)
+            affinity[(int64_t)a * G + group_of_expert[b]] += trans[(int64_t)a * E + b];
+}
+
+/* A token's predicted home group: the group with the largest summed affinity
+ * over its layer-1 experts (lower group on ties). */
+void oracle_predict_home(const int32_t* idx1, int64_t T, int k1, const int64_t* affinity, int G, int32_t* home) {
+    for (int64_t t = 0; t < T; ++t) {
+        int best = 0;
+        int64_t best_v = 0;
+        for (int g = 0; g < G; ++g) {
+            int64_t v = 0;
+            for (int i = 0; i < k1; ++i) v += affinity[(int64_t)idx1[t * k1 + i] * G + g];
+            if (g == 0 || v > best_v) { best = g; best_v = v; }
+        }
+        home[t] = best;
+    }
+}
+
+/* Slots served on the token's own GPU: assignments whose expert lies in the
+ * token's home group; home == NULL means the sequence-sharded home
+ * floor(t * G / T) ([EPKey] L/E baseline; [Coupling] 12.5% on one node). */
+int64_t oracle_count_local(const int32_t* expert_idx, int64_t T, int k, const int32_t* group_of_expert, int G,
+                           const int32_t* home) {
+    int64_t local = 0;
+    for (int64_t t = 0; t < T; ++t) {
+        const int64_t h = home ? home[t] : t * G / T;
+        for (int j = 0; j < k; ++j)
+            if (group_of_expert[expert_idx[t * k + j]] == h) ++local;
+    }
+    return local;
+}

@@ -50,6 +50,10 @@ def _load():
         "oracle_coselect": (None, [vp, i64, i32, i32, vp]),
         "oracle_transition": (None, [vp, i32, vp, i32, i64, i32, vp]),
         "oracle_local_fraction": (dbl, [vp, i64, i32, vp, i32]),
+        "oracle_place_experts": (i32, [vp, i32, i32, vp]),
+        "oracle_group_affinity": (None, [vp, i32, vp, i32, vp]),
+        "oracle_predict_home": (None, [vp, i64, i32, vp, i32, vp]),
+        "oracle_count_local": (i64, [vp, i64, i32, vp, i32, vp]),
         "oracle_silu": (dbl, [dbl]),
         "oracle_gelu": (dbl, [dbl]),
         "oracle_round_bf16": (dbl, [dbl]),
@@ -216,6 +220,45 @@ def local_fraction(expert_idx: np.ndarray, group_of_expert: np.ndarray, G: int) 
     T, k = idx.shape
     goe = _c(group_of_expert, np.int32)
     return float(_load().oracle_local_fraction(idx.ctypes.data, T, k, goe.ctypes.data, G))
+
+
+def place_experts(cosel: np.ndarray, G: int) -> np.ndarray:
+    """Greedy correlated placement: group_of_expert [E]."""
+    C = _c(cosel, np.int32)
+    E = C.shape[0]
+    goe = np.empty(E, np.int32)
+    if _load().oracle_place_experts(C.ctypes.data, E, G, goe.ctypes.data):
+        raise ValueError("G must divide E")
+    return goe
+
+
+def group_affinity(trans: np.ndarray, group_of_expert: np.ndarray, G: int) -> np.ndarray:
+    M = _c(trans, np.int32)
+    E = M.shape[0]
+    goe = _c(group_of_expert, np.int32)
+    aff = np.empty((E, G), np.int64)
+    _load().oracle_group_affinity(M.ctypes.data, E, goe.ctypes.data, G, aff.ctypes.data)
+    return aff
+
+
+def predict_home(idx1: np.ndarray, affinity: np.ndarray) -> np.ndarray:
+    i1 = _c(idx1, np.int32)
+    T, k1 = i1.shape
+    aff = _c(affinity, np.int64)
+    home = np.empty(T, np.int32)
+    _load().oracle_predict_home(i1.ctypes.data, T, k1, aff.ctypes.data, aff.shape[1], home.ctypes.data)
+    return home
+
+
+def count_local(expert_idx: np.ndarray, group_of_expert: np.ndarray, G: int, home=None) -> int:
+    idx = _c(expert_idx, np.int32)
+    T, k = idx.shape
+    goe = _c(group_of_expert, np.int32)
+    hp = None
+    if home is not None:
+        home = _c(home, np.int32)
+        hp = home.ctypes.data
+    return int(_load().oracle_count_local(idx.ctypes.data, T, k, goe.ctypes.data, G, hp))
 
 
 def silu(z: float) -> float:

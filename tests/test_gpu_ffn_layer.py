@@ -152,3 +152,22 @@ def test_layer_expert_choice_sampled(gemm_kind):
             ref[i] = (ec_gate.reshape(-1)[rows].astype(np.float64)[:, None] * y).sum(0)
     assert_layer_close(got[toks], ref)
     assert (as_f64(got[unchosen]) == 0).all()
+
+
+def test_host_pipeline_matches_plain_forward():
+    """Batches streamed through HostPipeline (copies overlapped with compute)
+    give exactly the outputs of one forward per batch."""
+    w = W.TINY
+    Wt = weights_dev(W.make_weights(w))
+    L = Lyr.TopKLayer(w.T, w.d, w.E, w.k, w.F, w.capacity_factor, torch.float32, *Wt)
+    batches = [w.with_(seed=s) for s in (3, 4, 5, 6, 7)]
+    h_in = [[torch.from_numpy(W.make_logits(b)).pin_memory(), torch.from_numpy(W.make_x(b)).pin_memory()]
+            for b in batches]
+    h_out = [torch.empty((w.T, w.d), dtype=torch.float32).pin_memory() for _ in batches]
+    d_lg, d_x = torch.empty((w.T, w.E), device="cuda"), torch.empty((w.T, w.d), device="cuda")
+    pipe = Lyr.HostPipeline(lambda lg, x, out: L.forward(lg, x, out=out), [d_lg, d_x], torch.empty_like(L.out))
+    pipe.run(h_in, h_out)
+    torch.cuda.synchronize()
+    for (lg, x), got in zip(h_in, h_out):
+        want = L.forward(lg.cuda(), x.cuda()).cpu()
+        assert torch.equal(got, want)

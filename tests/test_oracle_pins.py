@@ -461,3 +461,90 @@ def test_generator_deterministic_and_distribution():
     h = synth.normal_bf16(0, 1, (1000, 37))
     assert np.array_equal(h, synth.f32_to_bf16(a))
     assert not np.array_equal(synth.u64(0, 1, 10), synth.u64(0, 2, 10))
+
+
+# ------------------------------------------------ placement and shuffling
+def test_place_experts_hand_traced():
+    # off-diagonal masses 4, 3, 2, 3 -> seed 0; affinities to {0}: 3, 0, 1 -> add 1;
+    # remaining {2, 3}: masses 2, 3 -> seed 3, then 2
+    C = np.array([[5, 3, 0, 1], [3, 4, 0, 0], [0, 0, 6, 2], [1, 0, 2, 3]], np.int32)
+    assert O.place_experts(C, 2).tolist() == [0, 0, 1, 1]
+    # all ties: lowest indices first
+    assert O.place_experts(np.zeros((6, 6), np.int32), 2).tolist() == [0, 0, 0, 1, 1, 1]
+    with pytest.raises(ValueError):
+        O.place_experts(np.zeros((6, 6), np.int32), 4)
+
+
+def test_place_experts_is_a_balanced_partition():
+    for E, G in ((12, 3), (64, 16), (32, 1), (10, 10)):
+        idx, _ = O.route_topk(RNG.normal(size=(500, E)).astype(np.float32), min(4, E))
+        goe = O.place_experts(O.coselect(idx, E), G)
+        assert (np.bincount(goe, minlength=G) == E // G).all()
+
+
+def test_place_experts_recovers_planted_clusters():
+    # the clustered top-6 recipe with expert ids scrambled: each group found
+    # must be exactly one of the 16 planted clusters
+    w = W.FINE.with_(T=4096)
+    idx, _ = O.route_topk(W.make_logits(w), w.k)
+    perm = np.random.default_rng(7).permutation(w.E).astype(np.int32)
+    scrambled = perm[idx]
+    goe = O.place_experts(O.coselect(scrambled, w.E), w.n_clusters)
+    inv = np.argsort(perm)
+    for g in range(w.n_clusters):
+        members = inv[np.nonzero(goe == g)[0]]
+        assert len(set((members // 4).tolist())) == 1
+    # so the group-major layout needs exactly the rows of the true clusters,
+    # fewer than contiguous groups of the scrambled ids
+    cap = O.capacity(0.0, w.T, w.k, w.E)
+    rows_placed = O.permute(scrambled, w.E, cap, goe)["R"]
+    rows_true = O.permute(idx, w.E, cap, W.equal_groups(w.E, w.n_clusters))["R"]
+    rows_contig = O.permute(scrambled, w.E, cap, W.equal_groups(w.E, w.n_clusters))["R"]
+    assert rows_placed == rows_true
+    assert rows_placed < 0.8 * rows_contig
+
+
+def test_group_affinity_and_home_brute_force():
+    T, E, G = 400, 12, 3
+    i1, _ = O.route_topk(RNG.normal(size=(T, E)).astype(np.float32), 2)
+    i2, _ = O.route_topk(RNG.normal(size=(T, E)).astype(np.float32), 3)
+    M = O.transition(i1, i2, E)
+    goe = RNG.permutation(np.repeat(np.arange(G), E // G)).astype(np.int32)
+    aff = O.group_affinity(M, goe, G)
+    want = np.zeros((E, G), np.int64)
+    for a in range(E):
+        for b in range(E):
+            want[a, goe[b]] += M[a, b]
+    assert (aff == want).all()
+    assert (aff.sum(1) == M.sum(1)).all()
+    home = O.predict_home(i1, aff)
+    score = aff[i1].sum(1)                                   # [T, G]
+    assert (home == np.argmax(score, axis=1)).all()           # argmax: first maximum
+    local = O.count_local(i2, goe, G, home)
+    assert local == sum(int(goe[i2[t, j]] == home[t]) for t in range(T) for j in range(3))
+
+
+def test_count_local_closed_forms():
+    T, E, G = 240, 8, 4
+    goe = W.equal_groups(E, G)
+    idx, _ = O.route_topk(RNG.normal(size=(T, E)).astype(np.float32), 1)
+    # sequence-sharded home: same as the local-fraction definition
+    assert O.count_local(idx, goe, G) == round(O.local_fraction(idx, goe, G) * T)
+    # next layer identical to this one: the transition matrix is diagonal and
+    # every token's predicted home holds its expert
+    aff = O.group_affinity(O.transition(idx, idx, E), goe, G)
+    assert O.count_local(idx, goe, G, O.predict_home(idx, aff)) == T
+
+
+def test_shuffling_raises_local_share_on_correlated_layers():
+    w = W.EXPERT_CHOICE.with_(T=8192)
+    l1 = W.make_logits(w)
+    a, _ = O.route_topk(l1, 1)
+    b, _ = O.route_topk(W.make_layer2_logits(w, l1), 1)
+    G = 8
+    goe = W.equal_groups(w.E, G)
+    before = O.count_local(b, goe, G) / w.T
+    home = O.predict_home(a, O.group_affinity(O.transition(a, b, w.E), goe, G))
+    after = O.count_local(b, goe, G, home) / w.T
+    assert abs(before - 1 / G) < 0.02
+    assert after > 2 * before
