@@ -241,6 +241,41 @@ moe_status moe_coselect(const int32_t* expert_idx, int T, int k, int E, int32_t*
 moe_status moe_transition(const int32_t* idx1, int k1, const int32_t* idx2, int k2, int T, int E,
                           int32_t* trans, moe_stream_t stream);
 
+/* ------------------------------- placement and token shuffling */
+
+/* Correlated expert placement ("Expert Coupling in MoE Pretraining",
+ * Abstract: experts often picked together go to the same GPU).  The pages
+ * give no algorithm; this is a greedy on the co-selection counts cosel
+ * [E, E] (as moe_coselect produces): each of the G groups (L = E/G experts)
+ * starts from the unassigned expert with the largest off-diagonal
+ * co-selection mass and grows by the unassigned expert with the largest
+ * co-selection summed over the group's members (column reads cosel[x][m]);
+ * lower index on ties.  group_of_expert [E] int32 out, in [0, G).  One CTA.
+ * Limits: G divides E, E <= 1024. */
+moe_status moe_place_experts(const int32_t* cosel, int E, int G, int32_t* group_of_expert, moe_stream_t stream);
+
+/* Affinity of each expert's next-layer traffic to each group (same Abstract:
+ * tokens are moved to the GPU predicted to hold their next-layer experts):
+ * affinity[a][g] = sum over experts b of group g of trans[a][b], with trans
+ * the layer-to-layer transition counts [E, E] of moe_transition.
+ * affinity [E, G] int64 out.  Limits: E, G <= 1024. */
+moe_status moe_group_affinity(const int32_t* trans, int E, const int32_t* group_of_expert, int G,
+                              int64_t* affinity, moe_stream_t stream);
+
+/* Predicted home group of each token: the group with the largest affinity
+ * summed over the token's layer-1 experts idx1 [T, k1] (lower group on
+ * ties).  home [T] int32 out.  Limits: k1 <= 32, E, G <= 1024. */
+moe_status moe_predict_home(const int32_t* idx1, int T, int k1, const int64_t* affinity, int E, int G,
+                            int32_t* home, moe_stream_t stream);
+
+/* Assignments served on the token's own GPU: count += the slots of
+ * expert_idx [T, k] whose expert's group equals the token's home group;
+ * home [T] (moe_predict_home) or NULL for the sequence-sharded home
+ * floor(t * G / T) ("Expert Parallelism > Key Parameters": L/E of the
+ * assignments under uniform routing).  count [1] uint64, accumulated. */
+moe_status moe_count_local(const int32_t* expert_idx, int T, int k, const int32_t* group_of_expert, int E, int G,
+                           const int32_t* home, uint64_t* count, moe_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

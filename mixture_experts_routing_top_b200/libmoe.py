@@ -47,6 +47,10 @@ SIGNATURES = {
     "moe_unpermute_ec": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp]),
     "moe_coselect": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
     "moe_transition": (_i32, [_vp, _i32, _vp, _i32, _i32, _i32, _vp, _vp]),
+    "moe_place_experts": (_i32, [_vp, _i32, _i32, _vp, _vp]),
+    "moe_group_affinity": (_i32, [_vp, _i32, _vp, _i32, _vp, _vp]),
+    "moe_predict_home": (_i32, [_vp, _i32, _i32, _vp, _i32, _i32, _vp, _vp]),
+    "moe_count_local": (_i32, [_vp, _i32, _i32, _vp, _i32, _i32, _vp, _vp, _vp]),
 }
 
 _lib = None
@@ -286,6 +290,51 @@ def transition(idx1: torch.Tensor, idx2: torch.Tensor, E: int, into: Optional[to
     if into is None:
         into = torch.zeros((E, E), dtype=torch.int32, device=idx1.device)
     _check("moe_transition", lib().moe_transition(_p(idx1), k1, _p(idx2), k2, T, E, _p(into), _stream(stream)))
+    return into
+
+
+# ------------------------------------------- placement and shuffling
+def place_experts(cosel: torch.Tensor, G: int, out=None, stream=None):
+    _dev(cosel, torch.int32, "cosel")
+    E = cosel.shape[0]
+    if out is None:
+        out = torch.empty(E, dtype=torch.int32, device=cosel.device)
+    _check("moe_place_experts", lib().moe_place_experts(_p(cosel), E, G, _p(out), _stream(stream)))
+    return out
+
+
+def group_affinity(trans: torch.Tensor, group_of_expert: torch.Tensor, G: int, out=None, stream=None):
+    _dev(trans, torch.int32, "trans")
+    _dev(group_of_expert, torch.int32, "group_of_expert")
+    E = trans.shape[0]
+    if out is None:
+        out = torch.empty((E, G), dtype=torch.int64, device=trans.device)
+    _check("moe_group_affinity", lib().moe_group_affinity(_p(trans), E, _p(group_of_expert), G, _p(out),
+                                                          _stream(stream)))
+    return out
+
+
+def predict_home(idx1: torch.Tensor, affinity: torch.Tensor, out=None, stream=None):
+    _dev(idx1, torch.int32, "idx1")
+    _dev(affinity, torch.int64, "affinity")
+    T, k1 = idx1.shape
+    E, G = affinity.shape
+    if out is None:
+        out = torch.empty(T, dtype=torch.int32, device=idx1.device)
+    _check("moe_predict_home", lib().moe_predict_home(_p(idx1), T, k1, _p(affinity), E, G, _p(out), _stream(stream)))
+    return out
+
+
+def count_local(expert_idx: torch.Tensor, group_of_expert: torch.Tensor, G: int, home=None, into=None,
+                stream=None):
+    _dev(expert_idx, torch.int32, "expert_idx")
+    _dev(group_of_expert, torch.int32, "group_of_expert")
+    T, k = expert_idx.shape
+    E = group_of_expert.numel()
+    if into is None:
+        into = torch.zeros(1, dtype=torch.int64, device=expert_idx.device)
+    _check("moe_count_local", lib().moe_count_local(_p(expert_idx), T, k, _p(group_of_expert), E, G, _p(home),
+                                                    _p(into), _stream(stream)))
     return into
 
 
