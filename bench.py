@@ -284,7 +284,39 @@ class TopKRunner:
         return (sum(h.numel() * h.element_size() for h in self.h_in), self.h_out.numel() * self.h_out.element_size())
 
     def extra(self):
-        return {"rows": self.R, "dropped": self.dropped}
+        out = {"rows": self.R, "dropped": self.dropped}
+        if self.w.cluster_bias:
+            out["correlated_placement"] = self.placement_stat()
+        return out
+
+    def placement_stat(self):
+        """Correlated placement on this batch: the expert ids are scrambled
+        by a fixed seeded permutation (so that contiguous groups no longer
+        coincide with the routing clusters), the co-selection counts feed
+        moe_place_experts, and the group-major row counts with the placed
+        and with contiguous groups are compared (one group per cluster)."""
+        import torch
+
+        M, w = self.M, self.w
+        dev = self.L.idx.device
+        G = w.n_clusters
+        perm = torch.from_numpy(np.random.default_rng(7).permutation(w.E).astype(np.int32)).to(dev)
+        scr = perm[self.L.idx.long()].contiguous()
+        cosel = M.coselect(scr, w.E)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        goe = M.place_experts(cosel, G)
+        b.record()
+        torch.cuda.synchronize()
+        contig = torch.arange(w.E, dtype=torch.int32, device=dev) // (w.E // G)
+        rows = {}
+        for name, g in (("placed", goe), ("contiguous", contig)):
+            p = M.permute(None, scr, w.E, 0.0, g, G)
+            rows[name] = int(p["offsets"][-1].item())
+        return {"G": G, "rows_placed": rows["placed"], "rows_contiguous": rows["contiguous"],
+                "rows_removed": round(1.0 - rows["placed"] / rows["contiguous"], 4),
+                "assignments": w.T * w.k, "place_us": round(1e3 * a.elapsed_time(b), 1),
+                "inputs": "this batch's routing, expert ids scrambled (seed 7)"}
 
     def cpu_baseline(self, n_rows):
         """The oracle as it stands, single-threaded, on a bounded sample."""
@@ -396,7 +428,26 @@ class ExpertChoiceRunner:
         return (sum(h.numel() * h.element_size() for h in self.h_in), self.h_out.numel() * self.h_out.element_size())
 
     def extra(self):
-        return {"rows": self.w.E * self.w.C, "tokens_chosen": self.chosen}
+        return {"rows": self.w.E * self.w.C, "tokens_chosen": self.chosen, "token_shuffling": self.shuffle_stat()}
+
+    def shuffle_stat(self, G=8):
+        """Share of layer-2 assignments served in the token's home group of
+        G contiguous expert groups: sequence-sharded homes vs homes predicted
+        from this batch's layer-1 -> layer-2 transition counts."""
+        import torch
+
+        M, w = self.M, self.w
+        goe = torch.arange(w.E, dtype=torch.int32, device=self.x.device) // (w.E // G)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        home = M.predict_home(self.top1[0], M.group_affinity(self.trans, goe, G))
+        b.record()
+        before = int(M.count_local(self.top1[1], goe, G)[0].item())
+        after = int(M.count_local(self.top1[1], goe, G, home)[0].item())
+        torch.cuda.synchronize()
+        return {"G": G, "local_before": round(before / w.T, 4), "local_after": round(after / w.T, 4),
+                "predict_us": round(1e3 * a.elapsed_time(b), 1),
+                "note": "transition counts accumulated over all timed steps (identical batches)"}
 
     def cpu_baseline(self, n_rows):
         from oracle import oracle as O
