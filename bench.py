@@ -221,7 +221,7 @@ class TopKRunner:
         self.logits, self.x = _dev(self.logits_np, device), _dev(self.x_np, device)
         weights = tuple(_dev(a, device) for a in self.weights_np)
         shared = None if self.shared_np is None else tuple(_dev(a, device) for a in self.shared_np)
-        self.goe = W.equal_groups(w.E, w.G) if (w.G and not w.F) else None
+        self.goe = W.equal_groups(w.E, w.G) if w.G else None
         dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
         self.L = Lyr.TopKLayer(w.T, w.d, w.E, w.k, w.F, w.capacity_factor, dt, *weights, act=w.act,
                                norm_topk=w.norm_topk, shared_weights=shared,
@@ -232,15 +232,23 @@ class TopKRunner:
                                self.logits.numel() * 4 + self.x.numel() * self.x.element_size())
         self.stages = [("route", lambda: self.L.route(self.logits)),
                        ("permute", lambda: self.L.dispatch(self.x))]
+        if self.L.grouped:
+            # send-once dispatcher with experts: group rows -> expert rows -> MLPs -> group rows
+            self.stages.append(("local_permute", lambda: self.L.local_permute()))
         if w.F:
             self.stages.append(("ffn", self._ffn))
+        if self.L.grouped:
+            self.stages.append(("precombine", self._precombine))
         self.stages.append(("combine", self._combine))
         self.stages.append(("coselect", lambda: M.coselect(self.L.idx, w.E, into=self.cosel)))
         self._y = self._sh = None
 
     def _ffn(self):
-        self._y = self.L.experts()
+        self._y = self.L.expert_mlps() if self.L.grouped else self.L.experts()
         self._sh = self.L.shared_expert(self.x)
+
+    def _precombine(self):
+        self._y = self.L.precombine(self._y)
 
     def _combine(self):
         y = self._y if self.w.F else self.L.perm["buffer"]
@@ -249,19 +257,27 @@ class TopKRunner:
     def after_warmup(self):
         self.R = int(self.L.perm["offsets"][-1].item())
         self.dropped = int(self.L.perm["dropped"][0].item())
+        self.R_e = int(self.L.perm_e["offsets"][-1].item()) if self.L.grouped else self.R
 
     def work(self):
-        """Algorithmic bytes (memory stages) and FLOPs (expert MLPs) per step."""
-        w, R = self.w, self.R
+        """Algorithmic bytes (memory stages) and FLOPs (expert MLPs) per step.
+        With groups, R counts the (token, group) rows and R_e the expert rows."""
+        w, R, R_e = self.w, self.R, self.R_e
         b = 2 if w.dtype == "bf16" else 4
         T, d, E, k = w.T, w.d, w.E, w.k
         shared = T * d * b if w.F_shared else 0
         out = {"route": ("bytes", T * E * 4 + T * k * 8),
                "permute": ("bytes", T * d * b + R * d * b + T * k * 8 + R * 4),
-               "combine": ("bytes", R * d * b + T * d * b + T * k * 8 + shared),
                "coselect": ("bytes", T * k * 4 + E * E * 4)}
+        if self.L.grouped:
+            out["permute"] = ("bytes", out["permute"][1] + T * k * 8 + R_e * 4)     # + the index-only permute
+            out["local_permute"] = ("bytes", 2 * R_e * d * b + T * k * 8)
+            out["precombine"] = ("bytes", R_e * d * b + R * d * b + T * k * 12)
+            out["combine"] = ("bytes", R * d * b + T * d * b + T * k * 4 + shared)
+        else:
+            out["combine"] = ("bytes", R * d * b + T * d * b + T * k * 8 + shared)
         if w.F:
-            f = 2.0 * R * d * w.F * (3 if w.act == "swiglu" else 2)
+            f = 2.0 * R_e * d * w.F * (3 if w.act == "swiglu" else 2)
             if w.F_shared:
                 f += 2.0 * T * d * w.F_shared * 3
             out["ffn"] = ("flops", f)
@@ -285,6 +301,8 @@ class TopKRunner:
 
     def extra(self):
         out = {"rows": self.R, "dropped": self.dropped}
+        if self.L.grouped:
+            out.update(expert_rows=self.R_e, G=self.w.G, rows_removed=round(1.0 - self.R / max(self.R_e, 1), 4))
         if self.w.cluster_bias:
             out["correlated_placement"] = self.placement_stat()
         return out
@@ -326,23 +344,33 @@ class TopKRunner:
         w = self.w
         Ts = min(w.T, 8192)                    # token sample for the routing/permute/combine part
         logits, x = self.logits_np[:Ts], self.x_np[:Ts]
+        grouped = self.L.grouped
         t0 = time.perf_counter()
         idx, gate = O.route_topk(logits, w.k, w.norm_topk)
-        p = O.permute(idx, w.E, O.capacity(w.capacity_factor, Ts, w.k, w.E), self.goe)
+        cap = O.capacity(w.capacity_factor, Ts, w.k, w.E)
+        p = O.permute(idx, w.E, cap, self.goe)
         buf = O.gather_rows(x, p["row_token"])
+        pe = p
+        if grouped:                            # the group's local permutation to expert rows
+            pe = O.permute(idx, w.E, cap)
+            buf = O.copy_slot_rows(buf, p["row_map"], pe["row_map"], np.empty((pe["R"], w.d), buf.dtype))
         t_rp = time.perf_counter() - t0
-        R = p["R"]
+        R = pe["R"]
         Y = buf if not w.F else (synth.normal_bf16(99, 1, (R, w.d)) if w.dtype == "bf16"
                                  else synth.normal_f32(99, 1, (R, w.d)))
         t0 = time.perf_counter()
-        O.unpermute(Y, p["row_map"], gate)
+        if grouped:
+            P = O.group_precombine(Y, pe["row_map"], p["row_map"], gate, p["R"])
+            O.unpermute_groups(O.to_dtype_bits(P, Y), p["row_map"])
+        else:
+            O.unpermute(Y, p["row_map"], gate)
         t_comb = time.perf_counter() - t0
         per_token = (t_rp + t_comb) / Ts
         sample = "route, capacity, permute, row copy and combine on %d of %d tokens (%.2f s)" % (
             Ts, w.T, t_rp + t_comb)
         if w.F:
             rows = np.linspace(0, R - 1, num=min(n_rows, R)).astype(np.int64)
-            row_e = np.searchsorted(p["offsets"], rows, side="right").astype(np.int32) - 1
+            row_e = np.searchsorted(pe["offsets"], rows, side="right").astype(np.int32) - 1
             W1, W3, W2 = self.weights_np
             t0 = time.perf_counter()
             O.expert_ffn_rows(buf[rows], row_e, W1, W3, W2, w.act)
@@ -637,13 +665,14 @@ def run_reference(args, w):
     is_ec = kind_of(w) == "ec"
     Wt = W.make_weights(w) if w.F else None
     Ws = W.make_shared_weights(w)
-    goe = W.equal_groups(w.E, w.G) if (w.G and not w.F) else None
+    goe = W.equal_groups(w.E, w.G) if w.G else None
+    grouped = bool(w.G and w.F)                 # send-once dispatcher with experts
     if is_ec:
         C = max(1, w.C * Ts // w.T)
         R_probe = w.E * C
     else:
         R_probe = O.permute(O.route_topk(logits, w.k, w.norm_topk)[0], w.E,
-                            O.capacity(w.capacity_factor, Ts, w.k, w.E), goe)["R"]
+                            O.capacity(w.capacity_factor, Ts, w.k, w.E), None if grouped else goe)["R"]
     Y = synth.normal_bf16(99, 1, (R_probe, w.d)) if w.dtype == "bf16" else synth.normal_f32(99, 1, (R_probe, w.d))
 
     def step(i):
@@ -656,11 +685,19 @@ def run_reference(args, w):
             row_e = lambda r: r // C
         else:
             idx, gate = O.route_topk(logits, w.k, w.norm_topk)
-            p = O.permute(idx, w.E, O.capacity(w.capacity_factor, Ts, w.k, w.E), goe)
+            cap = O.capacity(w.capacity_factor, Ts, w.k, w.E)
+            p = O.permute(idx, w.E, cap, goe)
             buf = O.gather_rows(x, p["row_token"])
-            O.unpermute(Y if w.F else buf, p["row_map"], gate)
-            R = p["R"]
-            row_e = lambda r: int(np.searchsorted(p["offsets"], r, side="right") - 1)
+            pe = p
+            if grouped:
+                pe = O.permute(idx, w.E, cap)
+                buf = O.copy_slot_rows(buf, p["row_map"], pe["row_map"], np.empty((pe["R"], w.d), buf.dtype))
+                P = O.group_precombine(Y, pe["row_map"], p["row_map"], gate, p["R"])
+                O.unpermute_groups(O.to_dtype_bits(P, Y), p["row_map"])
+            else:
+                O.unpermute(Y if w.F else buf, p["row_map"], gate)
+            R = pe["R"]
+            row_e = lambda r: int(np.searchsorted(pe["offsets"], r, side="right") - 1)
         t1 = time.perf_counter()
         if w.F:
             r = (i * 7919) % R

@@ -11,6 +11,7 @@
  *
  *   moe_route_topk / moe_route_ec  ->  moe_permute / moe_gather_rows
  *   ->  moe_expert_ffn  ->  moe_unpermute / moe_unpermute_ec
+ *   group-major experts: moe_copy_slot_rows, moe_group_precombine, moe_unpermute_groups
  *   beside it: moe_coselect, moe_transition
  *
  * Conventions shared by every call:
@@ -223,6 +224,55 @@ moe_status moe_unpermute(const void* y, int dtype, int R, int T, int d, int k, c
 moe_status moe_unpermute_ec(const void* y, int dtype, int R, int T, int d, const int32_t* tok_ptr,
                             const int32_t* tok_row, const float* ec_gate, void* out, int out_dtype,
                             moe_stream_t stream);
+
+/* ------------------------------------ group-major expert path */
+
+/* The send-once dispatcher with real experts ("Expert Coupling in MoE
+ * Pretraining", Abstract: a token is shipped to a given GPU at most one
+ * time, however many of its experts live there).  On one device the path is
+ *   moe_permute (group-major, x)          one row per (token, group)
+ *   moe_permute (expert-major, x = NULL)  the local expert rows, indices only
+ *   moe_copy_slot_rows                    group rows -> expert rows
+ *   moe_expert_ffn                        on the expert rows
+ *   moe_group_precombine                  expert outputs -> one row per (token, group)
+ *   moe_unpermute_groups                  token = sum of its group rows
+ * Both permutes take the same expert_idx and capacity factor, so they keep
+ * the same assignments (capacity is per expert in both layouts).
+ *
+ * Row copy through two row maps: for every slot s in [0, S) with
+ * src_row[s] >= 0 and dst_row[s] >= 0, dst[dst_row[s]] = src[src_row[s]]
+ * (a byte copy).  With src_row = the group-major row_map and dst_row = the
+ * expert-major row_map ([T, k], S = T*k) this is each group's local
+ * permutation to its experts; a destination row reached from several slots
+ * must get the same source row (as here: one slot per expert row).
+ *   src [R_src, d], dst [R_dst, d], dtype; row size a multiple of 16 bytes.
+ *   A row >= R_src or >= R_dst is skipped and reported through
+ *   moe_device_error. */
+moe_status moe_copy_slot_rows(const void* src, int dtype, int R_src, int d, const int32_t* src_row,
+                              const int32_t* dst_row, int S, void* dst, int R_dst, moe_stream_t stream);
+
+/* Pre-combine inside a group (same Abstract, the receiving side of the
+ * send-once dispatcher): y_g[r] = sum over the slots j of token t with
+ * row_map_g[t, j] = r, in slot order, of gate[t, j] * y_e[row_map_e[t, j]],
+ * accumulated in fp32 and stored once in dtype.  Slots with
+ * row_map_g = -1 (dropped) are skipped.
+ *   y_e [R_e, d] (expert rows, moe_expert_ffn output); y_g [R_g, d] out;
+ *   row_map_e, row_map_g, gate [T, k].  d % 8 == 0, k <= 32.  Entries past
+ *   R_e or R_g are skipped and reported through moe_device_error. */
+moe_status moe_group_precombine(const void* y_e, int dtype, int R_e, int T, int d, int k,
+                                const int32_t* row_map_e, const int32_t* row_map_g, const float* gate,
+                                void* y_g, int R_g, moe_stream_t stream);
+
+/* Token output from its group rows: out[t] = sum, in fp32 and in the order
+ * the rows first appear among the token's slots, of its distinct group rows
+ * y_g[row_map_g[t, j]] (unit weight: the gates were applied by
+ * moe_group_precombine), plus shared[t] when not NULL; a token with every
+ * slot dropped gets shared[t] or 0.
+ *   y_g [R_g, d] dtype; shared [T, d] dtype or NULL; out [T, d] out_dtype.
+ *   d % 8 == 0, k <= 32. */
+moe_status moe_unpermute_groups(const void* y_g, int dtype, int R_g, int T, int d, int k,
+                                const int32_t* row_map_g, const void* shared, void* out, int out_dtype,
+                                moe_stream_t stream);
 
 /* -------------------------------------------- routing statistics */
 

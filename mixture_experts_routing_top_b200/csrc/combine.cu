@@ -233,6 +233,171 @@ __global__ void __launch_bounds__(256) unpermute_ec_scalar_kernel(const void* __
     }
 }
 
+// ------------------------------------------- group-major expert path
+// The send-once dispatcher with real experts ("Expert Coupling in MoE
+// Pretraining", Abstract), each step as one GPU of an expert-parallel group
+// would run it: the group-major rows (one per token and group) are copied
+// to expert-major rows (the group's local permutation), the experts run,
+// each token's expert outputs inside one group are pre-combined with their
+// gates into that group's row, and the token's output is the sum of its
+// group rows.
+
+// dst[dst_row[s]] = src[src_row[s]] for every slot with both rows valid.
+template <int NV>
+__global__ void __launch_bounds__(256) copy_slot_rows_kernel(const uint4* __restrict__ src, int R_src, int vec_per_row,
+                                                             const int32_t* __restrict__ src_row,
+                                                             const int32_t* __restrict__ dst_row, long long S,
+                                                             uint4* __restrict__ dst, int R_dst, unsigned* err) {
+    const int lane = threadIdx.x & 31;
+    const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+    for (long long s = warp; s < S; s += nwarps) {
+        const int sr = src_row[s], dr = dst_row[s];
+        if (sr < 0 || dr < 0) continue;
+        if (sr >= R_src || dr >= R_dst) { if (lane == 0) raise_error(err, kErrIndex); continue; }
+        const uint4* a = src + (long long)sr * vec_per_row;
+        uint4* b = dst + (long long)dr * vec_per_row;
+        for (int v0 = 0; v0 < vec_per_row; v0 += 32 * NV) {
+            uint4 buf[NV];
+#pragma unroll
+            for (int u = 0; u < NV; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < vec_per_row) buf[u] = ld_stream(a + v);
+            }
+#pragma unroll
+            for (int u = 0; u < NV; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < vec_per_row) st_stream(b + v, buf[u]);
+            }
+        }
+    }
+}
+
+// y_g[r] = sum over the token's slots j with row_map_g[t, j] = r (slot order)
+// of gate[t, j] * y_e[row_map_e[t, j]], fp32 accumulation, one write per
+// group row.  One warp per token.
+template <bool BF16, int NV>
+__global__ void __launch_bounds__(256) group_precombine_kernel(const void* __restrict__ y_e, int R_e, int T, int d, int k,
+                                                               const int32_t* __restrict__ row_map_e,
+                                                               const int32_t* __restrict__ row_map_g,
+                                                               const float* __restrict__ gate, void* __restrict__ y_g,
+                                                               int R_g, unsigned* err) {
+    const int lane = threadIdx.x & 31;
+    const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+    const int nvec = d >> 3;
+    for (long long t = warp; t < T; t += nwarps) {
+        int re = -1, rg = -1;
+        float g = 0.0f;
+        if (lane < k) {
+            re = row_map_e[t * k + lane];
+            rg = row_map_g[t * k + lane];
+            g = gate[t * k + lane];
+            if (re >= R_e || rg >= R_g) { raise_error(err, kErrIndex); re = -1; rg = -1; }
+        }
+        for (int j = 0; j < k; ++j) {
+            const int rgj = __shfl_sync(0xffffffffu, rg, j);
+            if (rgj < 0) continue;
+            const unsigned earlier = __ballot_sync(0xffffffffu, lane < j && rg == rgj);
+            if (earlier) continue;                          // this group row was written for an earlier slot
+            for (int v0 = 0; v0 < nvec; v0 += 32 * NV) {
+                float acc[NV][8];
+#pragma unroll
+                for (int u = 0; u < NV; ++u)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+                for (int q = j; q < k; ++q) {
+                    const int rgq = __shfl_sync(0xffffffffu, rg, q);
+                    const int req = __shfl_sync(0xffffffffu, re, q);
+                    const float gq = __shfl_sync(0xffffffffu, g, q);
+                    if (rgq != rgj || req < 0) continue;
+                    float f[NV][8];
+#pragma unroll
+                    for (int u = 0; u < NV; ++u) {
+                        const int v = v0 + u * 32 + lane;
+                        if (v < nvec) Vec8<BF16>::load(y_e, (long long)req * d + 8LL * v, f[u]);
+                    }
+#pragma unroll
+                    for (int u = 0; u < NV; ++u)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) acc[u][i] = __fmaf_rn(gq, f[u][i], acc[u][i]);
+                }
+#pragma unroll
+                for (int u = 0; u < NV; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec) Vec8<BF16>::store(y_g, (long long)rgj * d + 8LL * v, acc[u]);
+                }
+            }
+        }
+    }
+}
+
+// out[t] = sum of the token's distinct group rows (first-appearance order)
+// plus shared[t] when given.  One warp per token.
+template <bool IN_BF16, bool OUT_BF16, int NV>
+__global__ void __launch_bounds__(256) unpermute_groups_kernel(const void* __restrict__ y_g, int R_g, int T, int d, int k,
+                                                               const int32_t* __restrict__ row_map_g,
+                                                               const void* __restrict__ shared, void* __restrict__ out,
+                                                               unsigned* err) {
+    const int lane = threadIdx.x & 31;
+    const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+    const int nvec = d >> 3;
+    for (long long t = warp; t < T; t += nwarps) {
+        int rg = -1;
+        if (lane < k) {
+            rg = row_map_g[t * k + lane];
+            if (rg >= R_g) { raise_error(err, kErrIndex); rg = -1; }
+        }
+        unsigned first = 0;                                  // slots holding a row's first appearance
+        for (int j = 0; j < k; ++j) {
+            const int rgj = __shfl_sync(0xffffffffu, rg, j);
+            if (rgj < 0) continue;
+            if (!__ballot_sync(0xffffffffu, lane < j && rg == rgj)) first |= 1u << j;
+        }
+        for (int v0 = 0; v0 < nvec; v0 += 32 * NV) {
+            float acc[NV][8];
+#pragma unroll
+            for (int u = 0; u < NV; ++u)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+            unsigned m = first;
+            while (m) {
+                const int j = __ffs(m) - 1;
+                m &= m - 1;
+                const int r = __shfl_sync(0xffffffffu, rg, j);
+                float f[NV][8];
+#pragma unroll
+                for (int u = 0; u < NV; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec) Vec8<IN_BF16>::load(y_g, (long long)r * d + 8LL * v, f[u]);
+                }
+#pragma unroll
+                for (int u = 0; u < NV; ++u)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[u][i] += f[u][i];
+            }
+            if (shared) {
+#pragma unroll
+                for (int u = 0; u < NV; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec) {
+                        float f[8];
+                        Vec8<IN_BF16>::load(shared, t * d + 8LL * v, f);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) acc[u][i] += f[i];
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < NV; ++u) {
+                const int v = v0 + u * 32 + lane;
+                if (v < nvec) Vec8<OUT_BF16>::store(out, t * d + 8LL * v, acc[u]);
+            }
+        }
+    }
+}
+
 int token_grid(long long T) {
     long long blocks = (T + 7) / 8;
     long long cap = 148LL * 8;
@@ -304,6 +469,80 @@ extern "C" moe_status moe_unpermute_ec(const void* y, int dtype, int R, int T, i
     } else {
         unpermute_ec_scalar_kernel<<<grid, 256, 0, s>>>(y, in_bf16, R, T, d, tok_ptr, tok_row, ec_gate, out, out_bf16, err);
     }
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_copy_slot_rows(const void* src, int dtype, int R_src, int d, const int32_t* src_row,
+                                         const int32_t* dst_row, int S, void* dst, int R_dst, moe_stream_t stream) {
+    if (R_src < 0 || R_dst < 0 || d < 0 || S < 0) return MOE_ERR_ARG;
+    if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_ARG;
+    if (S == 0 || d == 0) return MOE_OK;
+    if (!src || !src_row || !dst_row || !dst) return MOE_ERR_ARG;
+    const long long row_bytes = (long long)d * (dtype == MOE_BF16 ? 2 : 4);
+    if (row_bytes % 16 || !aligned16(src) || !aligned16(dst)) return MOE_ERR_SHAPE;
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    const int vpr = (int)(row_bytes / 16);
+    const int grid = token_grid(S);
+    if (vpr <= 32) copy_slot_rows_kernel<1><<<grid, 256, 0, s>>>((const uint4*)src, R_src, vpr, src_row, dst_row, S, (uint4*)dst, R_dst, err);
+    else if (vpr <= 64) copy_slot_rows_kernel<2><<<grid, 256, 0, s>>>((const uint4*)src, R_src, vpr, src_row, dst_row, S, (uint4*)dst, R_dst, err);
+    else copy_slot_rows_kernel<4><<<grid, 256, 0, s>>>((const uint4*)src, R_src, vpr, src_row, dst_row, S, (uint4*)dst, R_dst, err);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_group_precombine(const void* y_e, int dtype, int R_e, int T, int d, int k,
+                                           const int32_t* row_map_e, const int32_t* row_map_g, const float* gate,
+                                           void* y_g, int R_g, moe_stream_t stream) {
+    if (R_e < 0 || R_g < 0 || T < 0 || d < 0 || k < 1) return MOE_ERR_ARG;
+    if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_ARG;
+    if (k > 32) return MOE_ERR_SHAPE;
+    if (T == 0 || d == 0) return MOE_OK;
+    if (!y_e || !row_map_e || !row_map_g || !gate || !y_g) return MOE_ERR_ARG;
+    const int esz = dtype == MOE_BF16 ? 2 : 4;
+    if (d % 8 || (d * esz) % 16 || !aligned16(y_e) || !aligned16(y_g)) return MOE_ERR_SHAPE;
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    const int grid = token_grid(T);
+    const int nvec = d / 8;
+    const bool bf16 = dtype == MOE_BF16;
+#define MOE_PRE(NV)                                                                                                 \
+    do {                                                                                                            \
+        if (bf16) group_precombine_kernel<true, NV><<<grid, 256, 0, s>>>(y_e, R_e, T, d, k, row_map_e, row_map_g, gate, y_g, R_g, err); \
+        else group_precombine_kernel<false, NV><<<grid, 256, 0, s>>>(y_e, R_e, T, d, k, row_map_e, row_map_g, gate, y_g, R_g, err); \
+    } while (0)
+    if (nvec <= 32) MOE_PRE(1);
+    else if (nvec <= 64) MOE_PRE(2);
+    else MOE_PRE(4);
+#undef MOE_PRE
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_unpermute_groups(const void* y_g, int dtype, int R_g, int T, int d, int k,
+                                           const int32_t* row_map_g, const void* shared, void* out, int out_dtype,
+                                           moe_stream_t stream) {
+    if (R_g < 0 || T < 0 || d < 0 || k < 1) return MOE_ERR_ARG;
+    if ((dtype != MOE_F32 && dtype != MOE_BF16) || (out_dtype != MOE_F32 && out_dtype != MOE_BF16)) return MOE_ERR_ARG;
+    if (k > 32) return MOE_ERR_SHAPE;
+    if (T == 0 || d == 0) return MOE_OK;
+    if (!row_map_g || !out || (R_g > 0 && !y_g)) return MOE_ERR_ARG;
+    const bool in_bf16 = dtype == MOE_BF16, out_bf16 = out_dtype == MOE_BF16;
+    const int in_esz = in_bf16 ? 2 : 4, out_esz = out_bf16 ? 2 : 4;
+    if (d % 8 || (d * in_esz) % 16 || (d * out_esz) % 16 || (y_g && !aligned16(y_g)) || !aligned16(out) ||
+        (shared && !aligned16(shared)))
+        return MOE_ERR_SHAPE;
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    const int grid = token_grid(T);
+    const int nvec = d / 8;
+    if (nvec <= 32) MOE_DISPATCH_VEC(unpermute_groups_kernel, 1, y_g, R_g, T, d, k, row_map_g, shared, out, err);
+    else if (nvec <= 64) MOE_DISPATCH_VEC(unpermute_groups_kernel, 2, y_g, R_g, T, d, k, row_map_g, shared, out, err);
+    else MOE_DISPATCH_VEC(unpermute_groups_kernel, 4, y_g, R_g, T, d, k, row_map_g, shared, out, err);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }

@@ -2,7 +2,11 @@
 
 Top-k layer ("MoELayer" of "How MegaDLMs Implements Mixture of Experts (MoE)
 Architectures"): route -> permute -> expert MLPs -> unpermute, plus the
-shared expert when one is configured.  Expert-choice layer
+shared expert when one is configured.  With a group_of_expert and experts,
+the send-once dispatcher of "Expert Coupling in MoE Pretraining" (Abstract):
+one row per (token, group) -> the group's local permutation to its experts
+-> expert MLPs -> one gate-weighted row per (token, group) -> the token's
+sum of its group rows.  Expert-choice layer
 ("MoELayerExpertChoice"): route_ec -> gather rows -> expert MLPs ->
 unpermute_ec.  Nothing here computes: it owns device memory and calls the
 library on one stream, with no host synchronisation inside a forward.
@@ -38,9 +42,23 @@ class TopKLayer:
                          dropped=torch.empty(1, dtype=torch.int32, device=dev))
         self.perm_ws = M._ws(M.permute_workspace_bytes(T, k, E, self.G), dev)
         self.identity = F == 0 or W1 is None
+        self.grouped = self.G > 0 and not self.identity
+        R_ffn = self.R_max
+        if self.grouped:
+            # the local expert rows: an indices-only expert-major permute of the same routing
+            R_e = max(M.permute_max_rows(T, k, E, capacity_factor, 0), 1)
+            self.perm_e = dict(buffer=None, row_map=torch.empty((T, k), dtype=torch.int32, device=dev),
+                               row_token=torch.empty(R_e, dtype=torch.int32, device=dev),
+                               counts=torch.empty(E, dtype=torch.int32, device=dev),
+                               offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
+                               dropped=torch.empty(1, dtype=torch.int32, device=dev))
+            self.perm_e_ws = M._ws(M.permute_workspace_bytes(T, k, E, 0), dev)
+            self.x_e = torch.empty((R_e, d), dtype=dtype, device=dev)
+            self.y_g = torch.empty((self.R_max, d), dtype=dtype, device=dev)
+            R_ffn = R_e
         if not self.identity:
-            self.y = torch.empty((self.R_max, d), dtype=dtype, device=dev)
-            self.ffn_ws = M._ws(M.expert_ffn_workspace_bytes(self.R_max, d, F, dtype), dev)
+            self.y = torch.empty((R_ffn, d), dtype=dtype, device=dev)
+            self.ffn_ws = M._ws(M.expert_ffn_workspace_bytes(R_ffn, d, F, dtype), dev)
         self.shared_weights = shared_weights
         if shared_weights is not None:
             sW1 = shared_weights[0]
@@ -54,14 +72,37 @@ class TopKLayer:
         return M.route_topk(logits, self.k, self.norm_topk, self.idx, self.gate, stream=stream)
 
     def dispatch(self, x, stream=None):
-        return M.permute(x, self.idx, self.E, self.cf, self.goe, self.G, out=self.perm, workspace=self.perm_ws,
-                         stream=stream)
+        p = M.permute(x, self.idx, self.E, self.cf, self.goe, self.G, out=self.perm, workspace=self.perm_ws,
+                      stream=stream)
+        if self.grouped:
+            M.permute(None, self.idx, self.E, self.cf, out=self.perm_e, workspace=self.perm_e_ws, stream=stream)
+        return p
+
+    def local_permute(self, stream=None):
+        """Group rows -> expert rows (each group's local permutation)."""
+        return M.copy_slot_rows(self.perm["buffer"], self.perm["row_map"], self.perm_e["row_map"], self.x_e,
+                                stream=stream)
+
+    def expert_mlps(self, stream=None):
+        rows, offsets = (self.x_e, self.perm_e["offsets"]) if self.grouped else \
+            (self.perm["buffer"], self.perm["offsets"])
+        return M.expert_ffn(rows, offsets, self.W1, self.W3, self.W2, self.act, y=self.y, workspace=self.ffn_ws,
+                            stream=stream)
+
+    def precombine(self, y, stream=None):
+        """Expert outputs -> one gate-weighted row per (token, group)."""
+        return M.group_precombine(y, self.perm_e["row_map"], self.perm["row_map"], self.gate, self.y_g,
+                                  stream=stream)
 
     def experts(self, stream=None):
+        """Rows the combine reads: the expert outputs, or with groups the
+        pre-combined group rows."""
         if self.identity:
             return self.perm["buffer"]
-        return M.expert_ffn(self.perm["buffer"], self.perm["offsets"], self.W1, self.W3, self.W2, self.act,
-                            y=self.y, workspace=self.ffn_ws, stream=stream)
+        if not self.grouped:
+            return self.expert_mlps(stream)
+        self.local_permute(stream)
+        return self.precombine(self.expert_mlps(stream), stream)
 
     def shared_expert(self, x, stream=None):
         if self.shared_weights is None:
@@ -71,8 +112,10 @@ class TopKLayer:
                             workspace=self.shared_ws, stream=stream)
 
     def combine(self, y, shared=None, stream=None, out=None):
-        return M.unpermute(y, self.perm["row_map"], self.gate, shared, self.out_dtype,
-                           out=self.out if out is None else out, stream=stream)
+        out = self.out if out is None else out
+        if self.grouped:
+            return M.unpermute_groups(y, self.perm["row_map"], shared, self.out_dtype, out=out, stream=stream)
+        return M.unpermute(y, self.perm["row_map"], self.gate, shared, self.out_dtype, out=out, stream=stream)
 
     def forward(self, logits: torch.Tensor, x: torch.Tensor, stream=None, out=None) -> torch.Tensor:
         self.route(logits, stream)

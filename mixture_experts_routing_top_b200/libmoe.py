@@ -45,6 +45,9 @@ SIGNATURES = {
     "moe_expert_ffn": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _sz, _vp]),
     "moe_unpermute": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp]),
     "moe_unpermute_ec": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp]),
+    "moe_copy_slot_rows": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _i32, _vp, _i32, _vp]),
+    "moe_group_precombine": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _i32, _vp]),
+    "moe_unpermute_groups": (_i32, [_vp, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _i32, _vp]),
     "moe_coselect": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp]),
     "moe_transition": (_i32, [_vp, _i32, _vp, _i32, _i32, _i32, _vp, _vp]),
     "moe_place_experts": (_i32, [_vp, _i32, _i32, _vp, _vp]),
@@ -252,6 +255,55 @@ def unpermute(y: torch.Tensor, row_map: torch.Tensor, gate: torch.Tensor, shared
         out = torch.empty((T, d), dtype=out_dtype, device=y.device)
     _check("moe_unpermute", lib().moe_unpermute(
         _p(y), _act_dtype(y), y.shape[0], T, d, k, _p(row_map), _p(gate), _p(shared), _p(out), _act_dtype(out),
+        _stream(stream)))
+    return out
+
+
+# ------------------------------------------------ group-major expert path
+def copy_slot_rows(src: torch.Tensor, src_row: torch.Tensor, dst_row: torch.Tensor, dst: torch.Tensor, stream=None):
+    """dst[dst_row[s]] = src[src_row[s]] for the slots where both are >= 0."""
+    _dev(src, None, "src")
+    _dev(dst, src.dtype, "dst")
+    _dev(src_row, torch.int32, "src_row")
+    _dev(dst_row, torch.int32, "dst_row")
+    if src_row.numel() != dst_row.numel() or src.shape[1:] != dst.shape[1:]:
+        raise ValueError("copy_slot_rows: row maps or row sizes differ")
+    _check("moe_copy_slot_rows", lib().moe_copy_slot_rows(
+        _p(src), _act_dtype(src), src.shape[0], src.shape[1], _p(src_row), _p(dst_row), src_row.numel(), _p(dst),
+        dst.shape[0], _stream(stream)))
+    return dst
+
+
+def group_precombine(y_e: torch.Tensor, row_map_e: torch.Tensor, row_map_g: torch.Tensor, gate: torch.Tensor,
+                     y_g: torch.Tensor, stream=None):
+    """y_g[r] = sum of gate * y_e over the token's slots that map to group row r."""
+    _dev(y_e, None, "y_e")
+    _dev(y_g, y_e.dtype, "y_g")
+    for name, a, dt in (("row_map_e", row_map_e, torch.int32), ("row_map_g", row_map_g, torch.int32),
+                        ("gate", gate, torch.float32)):
+        _dev(a, dt, name)
+    T, k = row_map_g.shape
+    if tuple(row_map_e.shape) != (T, k) or tuple(gate.shape) != (T, k):
+        raise ValueError("group_precombine: row_map_e, row_map_g and gate must all be [T, k]")
+    _check("moe_group_precombine", lib().moe_group_precombine(
+        _p(y_e), _act_dtype(y_e), y_e.shape[0], T, y_e.shape[1], k, _p(row_map_e), _p(row_map_g), _p(gate),
+        _p(y_g), y_g.shape[0], _stream(stream)))
+    return y_g
+
+
+def unpermute_groups(y_g: torch.Tensor, row_map_g: torch.Tensor, shared: Optional[torch.Tensor] = None,
+                     out_dtype: Optional[torch.dtype] = None, out=None, stream=None):
+    """out[t] = sum of the token's distinct group rows (+ shared[t])."""
+    _dev(y_g, None, "y_g")
+    _dev(row_map_g, torch.int32, "row_map_g")
+    T, k = row_map_g.shape
+    d = y_g.shape[1]
+    if shared is not None:
+        _dev(shared, y_g.dtype, "shared")
+    if out is None:
+        out = torch.empty((T, d), dtype=out_dtype or y_g.dtype, device=y_g.device)
+    _check("moe_unpermute_groups", lib().moe_unpermute_groups(
+        _p(y_g), _act_dtype(y_g), y_g.shape[0], T, d, k, _p(row_map_g), _p(shared), _p(out), _act_dtype(out),
         _stream(stream)))
     return out
 

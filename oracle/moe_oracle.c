@@ -260,6 +260,74 @@ void oracle_unpermute(const void* Y, int dtype, int64_t T, int d, int k, const i
     }
 }
 
+/* ------------------------------------------- group-major expert path */
+/* [Coupling] Abstract: the dispatcher ships a token to a given GPU at most
+ * one time.  With real experts behind it, each GPU receives one row per
+ * (token, group), runs the token's experts that it holds, and returns one
+ * row: the gate-weighted sum of those experts' outputs.  The token's output
+ * is the sum of its returned rows - the same sum as the plain unpermutation,
+ * grouped by GPU.  The returned row is a tensor of the activation dtype, so
+ * for bf16 it is rounded to bf16 (as the expert outputs are).  */
+
+/* dst[dst_row[s]] = src[src_row[s]] byte for byte, for every slot with both
+ * rows valid (>= 0). */
+void oracle_copy_slot_rows(const void* src, int64_t row_bytes, const int32_t* src_row, const int32_t* dst_row,
+                           int64_t S, void* dst) {
+    for (int64_t s = 0; s < S; ++s) {
+        if (src_row[s] < 0 || dst_row[s] < 0) continue;
+        memcpy((char*)dst + (int64_t)dst_row[s] * row_bytes, (const char*)src + (int64_t)src_row[s] * row_bytes,
+               (size_t)row_bytes);
+    }
+}
+
+/* P[r] for each group row r = sum over the slots j of its token with
+ * row_map_g[t, j] = r (slot order) of gate[t, j] * Y_e[row_map_e[t, j]];
+ * rounded to bf16 when dtype is bf16.  Rows no slot maps to are left as
+ * they are.  Y_e: [R_e, d] dtype; P: [R_g, d] doubles. */
+void oracle_group_precombine(const void* Y_e, int dtype, int64_t T, int d, int k, const int32_t* row_map_e,
+                             const int32_t* row_map_g, const float* gate, double* P) {
+    for (int64_t t = 0; t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            const int32_t r = row_map_g[t * k + j];
+            if (r < 0) continue;
+            int first = 1;                       /* has an earlier slot of t already produced row r? */
+            for (int i = 0; i < j; ++i)
+                if (row_map_g[t * k + i] == r) first = 0;
+            if (!first) continue;
+            for (int c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (int q = j; q < k; ++q) {
+                    if (row_map_g[t * k + q] != r) continue;
+                    acc += (double)gate[t * k + q] * load_elem(Y_e, dtype, (int64_t)row_map_e[t * k + q] * d + c);
+                }
+                P[(int64_t)r * d + c] = (dtype == ORC_BF16) ? round_to_bf16(acc) : acc;
+            }
+        }
+    }
+}
+
+/* out[t] = sum of the token's distinct group rows (each once, in the order
+ * they first appear among its slots) + shared[t] (weight 1, may be NULL).
+ * Y_g: [R_g, d] dtype; out: [T, d] doubles. */
+void oracle_unpermute_groups(const void* Y_g, int dtype, int64_t T, int d, int k, const int32_t* row_map_g,
+                             const void* shared, double* out) {
+    for (int64_t t = 0; t < T; ++t) {
+        for (int c = 0; c < d; ++c) {
+            double acc = 0.0;
+            for (int j = 0; j < k; ++j) {
+                const int32_t r = row_map_g[t * k + j];
+                if (r < 0) continue;
+                int first = 1;
+                for (int i = 0; i < j; ++i)
+                    if (row_map_g[t * k + i] == r) first = 0;
+                if (first) acc += load_elem(Y_g, dtype, (int64_t)r * d + c);
+            }
+            if (shared) acc += load_elem(shared, dtype, t * d + c);
+            out[t * d + c] = acc;
+        }
+    }
+}
+
 /* ---------------------------------------------- ExpertChoiceRouter */
 /* [MegaDLMs] "Routing Mechanisms": the selection is inverted, every expert
  * picking the tokens that score highest for it.  Scores: per-token softmax over experts,

@@ -45,6 +45,9 @@ def _load():
         "oracle_gather_rows": (None, [vp, i64, vp, i64, vp]),
         "oracle_expert_ffn_rows": (None, [vp, i32, i64, i32, i32, vp, vp, vp, vp, i32, vp]),
         "oracle_unpermute": (None, [vp, i32, i64, i32, i32, vp, vp, vp, vp]),
+        "oracle_copy_slot_rows": (None, [vp, i64, vp, vp, i64, vp]),
+        "oracle_group_precombine": (None, [vp, i32, i64, i32, i32, vp, vp, vp, vp]),
+        "oracle_unpermute_groups": (None, [vp, i32, i64, i32, i32, vp, vp, vp]),
         "oracle_route_ec": (i32, [vp, i64, i32, i32, vp, vp, vp, vp]),
         "oracle_unpermute_ec": (None, [vp, i32, i64, i32, vp, vp, vp, vp]),
         "oracle_coselect": (None, [vp, i64, i32, i32, vp]),
@@ -165,6 +168,63 @@ def unpermute(Y: np.ndarray, row_map: np.ndarray, gate: np.ndarray, shared: Opti
     out = np.empty((T, d), np.float64)
     _load().oracle_unpermute(Y.ctypes.data, dt, T, d, k, rm.ctypes.data, g.ctypes.data, sp, out.ctypes.data)
     return out
+
+
+def copy_slot_rows(src: np.ndarray, src_row, dst_row, dst: np.ndarray) -> np.ndarray:
+    """dst[dst_row[s]] = src[src_row[s]] where both are >= 0 (dst updated in place)."""
+    src = np.ascontiguousarray(src)
+    assert dst.flags.c_contiguous and dst.dtype == src.dtype and dst.shape[1:] == src.shape[1:]
+    sr = _c(src_row, np.int32).reshape(-1)
+    dr = _c(dst_row, np.int32).reshape(-1)
+    assert sr.size == dr.size
+    _load().oracle_copy_slot_rows(src.ctypes.data, src[0].nbytes if src.shape[0] else 0, sr.ctypes.data,
+                                  dr.ctypes.data, sr.size, dst.ctypes.data)
+    return dst
+
+
+def group_precombine(Y_e: np.ndarray, row_map_e, row_map_g, gate, R_g: int) -> np.ndarray:
+    """One row per (token, group): float64 [R_g, d], bf16-rounded for bf16
+    inputs; rows no slot maps to are NaN."""
+    Y_e = np.ascontiguousarray(Y_e)
+    dt = _dt(Y_e)
+    re = _c(row_map_e, np.int32)
+    rg = _c(row_map_g, np.int32)
+    g = _c(gate, np.float32)
+    T, k = rg.shape
+    assert re.shape == (T, k) and g.shape == (T, k)
+    d = Y_e.shape[1]
+    P = np.full((R_g, d), np.nan)
+    _load().oracle_group_precombine(Y_e.ctypes.data, dt, T, d, k, re.ctypes.data, rg.ctypes.data, g.ctypes.data,
+                                    P.ctypes.data)
+    return P
+
+
+def unpermute_groups(Y_g: np.ndarray, row_map_g, shared: Optional[np.ndarray] = None) -> np.ndarray:
+    """Token outputs from their group rows: float64 [T, d]."""
+    Y_g = np.ascontiguousarray(Y_g)
+    dt = _dt(Y_g)
+    rg = _c(row_map_g, np.int32)
+    T, k = rg.shape
+    d = Y_g.shape[1]
+    sp = None
+    if shared is not None:
+        shared = np.ascontiguousarray(shared)
+        assert shared.dtype == Y_g.dtype
+        sp = shared.ctypes.data
+    out = np.empty((T, d), np.float64)
+    _load().oracle_unpermute_groups(Y_g.ctypes.data, dt, T, d, k, rg.ctypes.data, sp, out.ctypes.data)
+    return out
+
+
+def to_dtype_bits(v: np.ndarray, like: np.ndarray) -> np.ndarray:
+    """float64 values already representable in like's dtype -> that dtype
+    (float32, or bf16 bit patterns as uint16)."""
+    f = np.ascontiguousarray(v, np.float64).astype(np.float32)
+    if like.dtype == np.uint16:
+        u = f.view(np.uint32)
+        assert ((u & 0xFFFF) == 0).all(), "values are not bf16"
+        return (u >> 16).astype(np.uint16)
+    return f
 
 
 def route_ec(logits: np.ndarray, C: int):
@@ -304,4 +364,46 @@ def topk_layer_tokens(w, logits, x, weights, shared_weights, tokens):
         sW1, sW3, sW2 = shared_weights
         ys = expert_ffn_rows(x[tokens], np.zeros(len(tokens), np.int32), sW1, sW3, sW2, "swiglu")
         out += ys
+    return out, dict(idx=idx, gate=gate, cap=cap, perm=p)
+
+
+def topk_group_layer_tokens(w, logits, x, weights, shared_weights, group_of_expert, tokens):
+    """The top-k layer with the send-once dispatcher and real experts, for
+    the listed tokens only: float64 [len(tokens), d].  Per token, the kept
+    expert outputs of each group are gate-summed into one row (rounded to
+    the activation dtype, as a returned tensor is), and the token's output
+    is the sum of its group rows (+ the shared expert)."""
+    idx, gate = route_topk(logits, w.k, w.norm_topk)
+    cap = capacity(w.capacity_factor, w.T, w.k, w.E)
+    p = permute(idx, w.E, cap)
+    goe = np.asarray(group_of_expert, np.int32)
+    tokens = np.asarray(tokens, np.int64)
+    n = tokens.size
+    W1, W3, W2 = weights
+    rows, experts = [], []
+    rm_e = np.full((n, w.k), -1, np.int32)          # local expert rows of the listed tokens
+    rm_g = np.full((n, w.k), -1, np.int32)          # local group rows
+    n_g = 0
+    for i, t in enumerate(tokens):
+        seen = {}
+        for j in range(w.k):
+            if p["row_map"][t, j] < 0:
+                continue
+            rm_e[i, j] = len(rows)
+            rows.append(t)
+            experts.append(idx[t, j])
+            g = int(goe[idx[t, j]])
+            if g not in seen:
+                seen[g] = n_g
+                n_g += 1
+            rm_g[i, j] = seen[g]
+    out = np.zeros((n, w.d), np.float64)
+    if rows:
+        y = expert_ffn_rows(x[np.asarray(rows)], np.asarray(experts, np.int32), W1, W3, W2, w.act)
+        y_bits = to_dtype_bits(y, x)
+        P = group_precombine(y_bits, rm_e, rm_g, gate[tokens], n_g)
+        out = unpermute_groups(to_dtype_bits(P, x), rm_g)
+    if shared_weights is not None:
+        sW1, sW3, sW2 = shared_weights
+        out = out + expert_ffn_rows(x[tokens], np.zeros(n, np.int32), sW1, sW3, sW2, "swiglu")
     return out, dict(idx=idx, gate=gate, cap=cap, perm=p)

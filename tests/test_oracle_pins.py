@@ -354,6 +354,89 @@ def test_combine_group_major_identity_experts():
     np.testing.assert_allclose(y, x.astype(np.float64), rtol=1e-6, atol=1e-7)
 
 
+# ------------------------------------------------ group-major expert path
+def _two_group_example():
+    idx = np.array([[0, 2, 1], [3, 2, 0]], np.int32)
+    gate = np.array([[0.5, 0.25, 0.125], [0.5, 0.25, 0.25]], np.float32)
+    goe = np.array([0, 0, 1, 1], np.int32)
+    return idx, gate, goe
+
+
+def test_group_path_hand_example():
+    """Two tokens, experts {0,1} in group 0 and {2,3} in group 1; the output
+    of expert e for token t is (10e + t, e - t).  Group rows and token sums
+    worked out by hand."""
+    idx, gate, goe = _two_group_example()
+    E = 4
+    pe = O.permute(idx, E, O.capacity(0.0, 2, 3, E))
+    pg = O.permute(idx, E, O.capacity(0.0, 2, 3, E), group_of_expert=goe)
+    # group-major rows: group 0 (tokens 0, 1), then group 1 (tokens 0, 1)
+    assert pg["row_map"].tolist() == [[0, 2, 0], [3, 3, 1]]
+    row_e = np.repeat(np.arange(E), pe["counts"])
+    Y = np.stack([10.0 * row_e + pe["row_token"], row_e - pe["row_token"]], 1).astype(np.float32)
+    P = O.group_precombine(Y, pe["row_map"], pg["row_map"], gate, 4)
+    assert P.tolist() == [[1.25, 0.125], [0.25, -0.25], [5.0, 0.5], [20.75, 1.25]]
+    out = O.unpermute_groups(O.to_dtype_bits(P, Y), pg["row_map"])
+    assert out.tolist() == [[6.25, 0.625], [21.0, 1.0]]
+    sh = np.array([[1, 2], [3, 4]], np.float32)
+    assert O.unpermute_groups(O.to_dtype_bits(P, Y), pg["row_map"], shared=sh).tolist() == [[7.25, 2.625], [24.0, 5.0]]
+
+
+@pytest.mark.parametrize("cf,G", [(0.0, 4), (0.7, 4), (0.7, 16), (1.0, 1)])
+def test_group_path_equals_plain_unpermute(cf, G):
+    """Summing per group and then over groups is the plain gate-weighted sum."""
+    T, E, k, d = 300, 16, 4, 6
+    logits = RNG.normal(size=(T, E)).astype(np.float32)
+    logits[:, 3] += 1.5                             # a hot expert, so cf < 1 drops
+    idx, gate = O.route_topk(logits, k)
+    cap = O.capacity(cf, T, k, E)
+    goe = RNG.permutation(W.equal_groups(E, G)).astype(np.int32)
+    pe = O.permute(idx, E, cap)
+    pg = O.permute(idx, E, cap, group_of_expert=goe)
+    assert np.array_equal(pe["row_map"] >= 0, pg["row_map"] >= 0)      # same kept assignments
+    if cf > 0:
+        assert pe["dropped"] > 0
+    Y = RNG.normal(size=(int(pe["offsets"][-1]), d)).astype(np.float32)
+    R_g = int(pg["offsets"][-1])
+    P = O.group_precombine(Y, pe["row_map"], pg["row_map"], gate, R_g)
+    assert not np.isnan(P).any()                    # every group row is produced
+    got = O.unpermute_groups(O.to_dtype_bits(P, Y), pg["row_map"])
+    want = O.unpermute(Y, pe["row_map"], gate)
+    np.testing.assert_allclose(got, want, rtol=1e-6, atol=1e-6)
+
+
+def test_group_path_one_expert_per_group_is_one_rounding():
+    """G = E: each group row is one gated expert output, rounded once to bf16
+    (checked against torch's float64 -> bfloat16 conversion)."""
+    T, E, k, d = 64, 8, 3, 16
+    idx, gate = O.route_topk(RNG.normal(size=(T, E)).astype(np.float32), k)
+    cap = O.capacity(0.0, T, k, E)
+    pe = O.permute(idx, E, cap)
+    pg = O.permute(idx, E, cap, group_of_expert=np.arange(E, dtype=np.int32))
+    Yb = synth.f32_to_bf16(RNG.normal(size=(int(pe["offsets"][-1]), d)).astype(np.float32))
+    P = O.group_precombine(Yb, pe["row_map"], pg["row_map"], gate, int(pg["offsets"][-1]))
+    Yd = torch.from_numpy(synth.bf16_to_f32(Yb).astype(np.float64))
+    for t in range(T):
+        for j in range(k):
+            want = (float(gate[t, j]) * Yd[pe["row_map"][t, j]]).to(torch.bfloat16).to(torch.float64).numpy()
+            assert np.array_equal(P[pg["row_map"][t, j]], want)
+
+
+def test_copy_slot_rows_turns_group_rows_into_expert_rows():
+    T, E, k, d, G = 120, 8, 3, 5, 2
+    idx, _ = O.route_topk(RNG.normal(size=(T, E)).astype(np.float32), k)
+    cap = O.capacity(0.9, T, k, E)
+    goe = W.equal_groups(E, G)
+    pe = O.permute(idx, E, cap)
+    pg = O.permute(idx, E, cap, group_of_expert=goe)
+    x = RNG.normal(size=(T, d)).astype(np.float32)
+    xg = O.gather_rows(x, pg["row_token"][:pg["offsets"][-1]])
+    R_e = int(pe["offsets"][-1])
+    xe = np.full((R_e, d), np.nan, np.float32)
+    O.copy_slot_rows(xg, pg["row_map"], pe["row_map"], xe)
+    assert np.array_equal(xe, O.gather_rows(x, pe["row_token"][:R_e]))
+
+
 # --------------------------------------------------------- expert choice
 @pytest.mark.parametrize("T,E,C", [(40, 4, 10), (33, 5, 33), (25, 3, 1)])
 def test_expert_choice_matches_sort(T, E, C):
