@@ -219,6 +219,8 @@ class TopKRunner:
         self.weights_np = W.make_weights(w) if w.F else (None, None, None)
         self.shared_np = W.make_shared_weights(w)
         self.logits, self.x = _dev(self.logits_np, device), _dev(self.x_np, device)
+        self.Wr_np = W.make_router_weights(w) if w.router else None       # logits from x on the device
+        self.Wr = None if self.Wr_np is None else _dev(self.Wr_np, device)
         weights = tuple(_dev(a, device) for a in self.weights_np)
         shared = None if self.shared_np is None else tuple(_dev(a, device) for a in self.shared_np)
         self.goe = W.equal_groups(w.E, w.G) if w.G else None
@@ -226,12 +228,16 @@ class TopKRunner:
         self.L = Lyr.TopKLayer(w.T, w.d, w.E, w.k, w.F, w.capacity_factor, dt, *weights, act=w.act,
                                norm_topk=w.norm_topk, shared_weights=shared,
                                group_of_expert=None if self.goe is None else _dev(self.goe, device),
-                               G=w.G if self.goe is not None else 0, device=device)
+                               G=w.G if self.goe is not None else 0, device=device, W_r=self.Wr)
         self.cosel = torch.zeros((w.E, w.E), dtype=torch.int32, device=device)
+        route_in = self.Wr if w.router else self.logits
         self.resident_bytes = (sum(t.numel() * t.element_size() for t in weights if t is not None) +
-                               self.logits.numel() * 4 + self.x.numel() * self.x.element_size())
-        self.stages = [("route", lambda: self.L.route(self.logits)),
-                       ("permute", lambda: self.L.dispatch(self.x))]
+                               route_in.numel() * route_in.element_size() + self.x.numel() * self.x.element_size())
+        if w.router:
+            self.stages = [("route", lambda: self.L.route_x(self.x))]
+        else:
+            self.stages = [("route", lambda: self.L.route(self.logits))]
+        self.stages.append(("permute", lambda: self.L.dispatch(self.x)))
         if self.L.grouped:
             # send-once dispatcher with experts: group rows -> expert rows -> MLPs -> group rows
             self.stages.append(("local_permute", lambda: self.L.local_permute()))
@@ -266,7 +272,8 @@ class TopKRunner:
         b = 2 if w.dtype == "bf16" else 4
         T, d, E, k = w.T, w.d, w.E, w.k
         shared = T * d * b if w.F_shared else 0
-        out = {"route": ("bytes", T * E * 4 + T * k * 8),
+        route_bytes = (T * d * b + E * d * b if w.router else T * E * 4) + T * k * 8
+        out = {"route": ("bytes", route_bytes),
                "permute": ("bytes", T * d * b + R * d * b + T * k * 8 + R * 4),
                "coselect": ("bytes", T * k * 4 + E * E * 4)}
         if self.L.grouped:
@@ -288,10 +295,14 @@ class TopKRunner:
 
         from mixture_experts_routing_top_b200 import layer as Lyr
 
-        self.h_in = [_pinned(self.logits_np), _pinned(self.x_np)]
         self.h_out = torch.empty(self.L.out.shape, dtype=self.L.out.dtype).pin_memory()
-        self.pipe = Lyr.HostPipeline(lambda lg, x, out: self.L.forward(lg, x, out=out), [self.logits, self.x],
-                                     self.L.out)
+        if self.w.router:                      # the router runs on the device: x is the only input
+            self.h_in = [_pinned(self.x_np)]
+            self.pipe = Lyr.HostPipeline(lambda x, out: self.L.forward(None, x, out=out), [self.x], self.L.out)
+        else:
+            self.h_in = [_pinned(self.logits_np), _pinned(self.x_np)]
+            self.pipe = Lyr.HostPipeline(lambda lg, x, out: self.L.forward(lg, x, out=out), [self.logits, self.x],
+                                         self.L.out)
 
     def e2e_run(self, n):
         self.pipe.run([self.h_in] * n, [self.h_out] * n)
@@ -346,6 +357,8 @@ class TopKRunner:
         logits, x = self.logits_np[:Ts], self.x_np[:Ts]
         grouped = self.L.grouped
         t0 = time.perf_counter()
+        if w.router:
+            logits = O.router_logits(x, self.Wr_np).astype(np.float32)
         idx, gate = O.route_topk(logits, w.k, w.norm_topk)
         cap = O.capacity(w.capacity_factor, Ts, w.k, w.E)
         p = O.permute(idx, w.E, cap, self.goe)
@@ -366,8 +379,8 @@ class TopKRunner:
             O.unpermute(Y, p["row_map"], gate)
         t_comb = time.perf_counter() - t0
         per_token = (t_rp + t_comb) / Ts
-        sample = "route, capacity, permute, row copy and combine on %d of %d tokens (%.2f s)" % (
-            Ts, w.T, t_rp + t_comb)
+        sample = "%sroute, capacity, permute, row copy and combine on %d of %d tokens (%.2f s)" % (
+            "router gate, " if w.router else "", Ts, w.T, t_rp + t_comb)
         if w.F:
             rows = np.linspace(0, R - 1, num=min(n_rows, R)).astype(np.int64)
             row_e = np.searchsorted(pe["offsets"], rows, side="right").astype(np.int32) - 1
@@ -667,11 +680,13 @@ def run_reference(args, w):
     Ws = W.make_shared_weights(w)
     goe = W.equal_groups(w.E, w.G) if w.G else None
     grouped = bool(w.G and w.F)                 # send-once dispatcher with experts
+    Wr = W.make_router_weights(w) if w.router else None
     if is_ec:
         C = max(1, w.C * Ts // w.T)
         R_probe = w.E * C
     else:
-        R_probe = O.permute(O.route_topk(logits, w.k, w.norm_topk)[0], w.E,
+        lg0 = O.router_logits(x, Wr).astype(np.float32) if Wr is not None else logits
+        R_probe = O.permute(O.route_topk(lg0, w.k, w.norm_topk)[0], w.E,
                             O.capacity(w.capacity_factor, Ts, w.k, w.E), None if grouped else goe)["R"]
     Y = synth.normal_bf16(99, 1, (R_probe, w.d)) if w.dtype == "bf16" else synth.normal_f32(99, 1, (R_probe, w.d))
 
@@ -684,7 +699,8 @@ def run_reference(args, w):
             R = w.E * C
             row_e = lambda r: r // C
         else:
-            idx, gate = O.route_topk(logits, w.k, w.norm_topk)
+            lg = O.router_logits(x, Wr).astype(np.float32) if Wr is not None else logits
+            idx, gate = O.route_topk(lg, w.k, w.norm_topk)
             cap = O.capacity(w.capacity_factor, Ts, w.k, w.E)
             p = O.permute(idx, w.E, cap, goe)
             buf = O.gather_rows(x, p["row_token"])

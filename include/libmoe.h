@@ -9,6 +9,7 @@
  * correlation statistics follow "Expert Coupling in MoE Pretraining",
  * Abstract.  One call per step:
  *
+ *   moe_router_topk (x -> top-k) or
  *   moe_route_topk / moe_route_ec  ->  moe_permute / moe_gather_rows
  *   ->  moe_expert_ffn  ->  moe_unpermute / moe_unpermute_ec
  *   group-major experts: moe_copy_slot_rows, moe_group_precombine, moe_unpermute_groups
@@ -89,6 +90,25 @@ uint64_t moe_kernel_launches(void);
  * Limits: 1 <= k <= min(E, 32), E <= 1024, T >= 0. */
 moe_status moe_route_topk(const float* logits, int T, int E, int k, int norm_topk,
                           int32_t* expert_idx, float* gate, moe_stream_t stream);
+
+/* The router's linear gate fused with moe_route_topk ("Routing Mechanisms:
+ * Top-K vs Expert Choice": the TopKRouter scores each expert with a linear
+ * layer over the token's hidden state, then softmax and top-k as above):
+ * logits[t, e] = sum_c x[t, c] * W_r[e, c], then the top-k experts and
+ * gates of each logits row, with the ranking and gates of moe_route_topk.
+ *   x       [T, d] dtype;  W_r [E, d] dtype (one row per expert)
+ *   logits  [T, E] fp32 out, or NULL when not wanted (bf16 only)
+ *   expert_idx, gate  [T, k] out, as moe_route_topk
+ * bf16: one tcgen05 GEMM (fp32 accumulation in TMEM) whose epilogue ranks
+ * each token from TMEM; d % 64 == 0, E % 8 == 0, E <= 256, k <= 8, x, W_r
+ * and logits 16-byte aligned.  fp32: FMA logits into `logits` (required),
+ * then moe_route_topk on them; E <= 1024, k <= 32.
+ * The logits' rounding differs from an fp64 evaluation by the fp32
+ * accumulation error, so experts whose logits lie that close may rank
+ * differently from an exact evaluation; the ranking of the returned
+ * logits themselves is exact. */
+moe_status moe_router_topk(const void* x, int dtype, int T, int d, const void* W_r, int E, int k, int norm_topk,
+                           float* logits, int32_t* expert_idx, float* gate, moe_stream_t stream);
 
 /* ExpertChoiceRouter (same section): each expert chooses the C tokens with
  * the highest routing score, the score being the token's softmax

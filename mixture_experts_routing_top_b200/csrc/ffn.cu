@@ -27,12 +27,10 @@
 //
 // fp32: a plain FMA kernel pair for small fp32 layers (no fp32-input
 // tensor-core kind keeps fp32 accuracy).
-#include <cuda.h>
-#include <cudaTypedefs.h>
 #include <cstdlib>
-#include <mutex>
 
 #include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace moe {
 namespace tc {
@@ -48,114 +46,9 @@ constexpr int EPI_WARPS = 4;                 // one warp per TMEM lane quarter (
 constexpr int THREADS = 64 + 32 * EPI_WARPS;  // warp 0 TMA, warp 1 MMA, then the epilogue warps
 constexpr int MAX_E = 1024;
 constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/ + 4 * (MAX_E + 1);
-constexpr long long WAIT_NS = 4000000000LL;  // 4 s
 
 enum { MODE_SWIGLU = 0, MODE_GELU = 1, MODE_PLAIN = 2 };
 
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ long long globaltimer() {
-    long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
-}
-
-// Bounded parity wait.  Returns false on timeout or when another role of
-// this CTA has already given up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag) {
-    long long t0 = 0;
-    for (uint32_t i = 1;; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(done) : "r"(bar), "r"(parity) : "memory");
-        if (done) return true;
-        if ((i & 255u) == 0) {
-            if (*abort_flag) return false;
-            const long long now = globaltimer();
-            if (t0 == 0) t0 = now;
-            else if (now - t0 > WAIT_NS) return false;
-        }
-    }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        :: "r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
-    asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-// UMMA shared-memory descriptor: K-major operand, 128-byte swizzle, rows
-// of 128 bytes, 8-row groups 1024 bytes apart (SBO), LBO 16 bytes,
-// descriptor version 1.
-__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t addr) {
-    uint64_t d = 0;
-    d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-    d |= (uint64_t)1u << 16;                    // LBO = 16 B
-    d |= (uint64_t)(1024u >> 4) << 32;          // SBO = 1024 B
-    d |= (uint64_t)1u << 46;                    // version
-    d |= (uint64_t)2u << 61;                    // SWIZZLE_128B
-    return d;
-}
-
-// Instruction descriptor, kind::f16: D fp32, A/B bf16, both K-major, M x N.
-__host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
-    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
-}
-
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t acc) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        :: "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(acc) : "memory");
-}
-
-// Arrives on `bar` once every tcgen05.mma issued so far by this thread is done.
-__device__ __forceinline__ void umma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
-
-// 32 lanes x 32 consecutive fp32 columns: thread = lane (row), v[i] = column i.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
 __device__ __forceinline__ float gelu_f(float z) { return 0.5f * z * (1.0f + erff(z * 0.70710678118654752f)); }
@@ -762,44 +655,6 @@ __global__ void ffn_f32_out_kernel(const float* __restrict__ H, int d, int F, in
 // --------------------------------------------------------------- host side
 namespace {
 
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::mutex g_encode_mu;
-
-bool get_encoder() {
-    std::lock_guard<std::mutex> lk(g_encode_mu);
-    if (g_encode) return true;
-    void* fn = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
-        q != cudaDriverEntryPointSuccess || !fn)
-        return false;
-    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    return true;
-}
-
-// 2-D bf16 tensor [rows, K] (K contiguous), box = 64 x box_rows, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, long long rows, int K, int box_rows) {
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    cuuint32_t box[2] = {(cuuint32_t)tc::BK, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
-int sm_count() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
-    }
-    return n;
-}
-
 template <int MODE>
 moe_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, const tc::GemmArgs& a,
                        cudaStream_t s) {
@@ -814,7 +669,7 @@ moe_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUte
     const long long n_tiles = (a.N_out + bn_out - 1) / bn_out;
     const long long m_tiles_max = (a.R_max + tc::BM - 1) / tc::BM + a.E;
     long long tiles_max = n_tiles * m_tiles_max;
-    int grid = sm_count();
+    int grid = tc::sm_count();
     if (tiles_max < grid) grid = (int)(tiles_max > 0 ? tiles_max : 1);
     tc::grouped_gemm_kernel<MODE><<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(ma, mb0, mb1, a);
     MOE_LAUNCH_CHECK();
@@ -835,7 +690,7 @@ moe_status launch_gemm2(const CUtensorMap& ma, const CUtensorMap& mb0, const CUt
     const long long n_tiles = (a.N_out + bn_out - 1) / bn_out;
     const long long m_tiles_max = (a.R_max + tc2::BM - 1) / tc2::BM + a.E;
     const long long tiles_max = n_tiles * m_tiles_max;
-    int pairs = sm_count() / 2;
+    int pairs = tc::sm_count() / 2;
     if (tiles_max < pairs) pairs = (int)(tiles_max > 0 ? tiles_max : 1);
     tc2::grouped_gemm2_kernel<MODE><<<2 * pairs, tc::THREADS, tc2::SMEM_BYTES, s>>>(ma, mb0, mb1, a);
     MOE_LAUNCH_CHECK();
@@ -897,7 +752,7 @@ extern "C" moe_status moe_expert_ffn(const void* buffer, int dtype, int R_max, i
     }
 
     // bf16 tensor-core path
-    if (!get_encoder()) return MOE_ERR_CUDA;
+    if (!tc::tma_encoder_ready()) return MOE_ERR_CUDA;
     uint16_t* H = (uint16_t*)workspace;
     CUtensorMap m_x, m_w1, m_w3, m_h, m_w2;
     const bool swiglu = act == MOE_ACT_SWIGLU;
@@ -905,11 +760,11 @@ extern "C" moe_status moe_expert_ffn(const void* buffer, int dtype, int R_max, i
     // per-CTA boxes: A is always 128 rows; B is 128 rows per CTA in the pair
     // kernels, and 128 (SwiGLU halves) or 256 rows in the one-CTA kernels
     const int bbox = pair ? 128 : 256;
-    if (!make_map(&m_x, buffer, R_max, d, 128)) return MOE_ERR_CUDA;
-    if (!make_map(&m_w1, W1, (long long)E * F, d, swiglu ? 128 : bbox)) return MOE_ERR_CUDA;
-    if (swiglu && !make_map(&m_w3, W3, (long long)E * F, d, 128)) return MOE_ERR_CUDA;
-    if (!make_map(&m_h, H, R_max, F, 128)) return MOE_ERR_CUDA;
-    if (!make_map(&m_w2, W2, (long long)E * d, F, bbox)) return MOE_ERR_CUDA;
+    if (!tc::make_bf16_map(&m_x, buffer, R_max, d, 128)) return MOE_ERR_CUDA;
+    if (!tc::make_bf16_map(&m_w1, W1, (long long)E * F, d, swiglu ? 128 : bbox)) return MOE_ERR_CUDA;
+    if (swiglu && !tc::make_bf16_map(&m_w3, W3, (long long)E * F, d, 128)) return MOE_ERR_CUDA;
+    if (!tc::make_bf16_map(&m_h, H, R_max, F, 128)) return MOE_ERR_CUDA;
+    if (!tc::make_bf16_map(&m_w2, W2, (long long)E * d, F, bbox)) return MOE_ERR_CUDA;
 
     tc::GemmArgs g1{offsets, E, d, F, F, R_max, H, err};
     if (pair) {

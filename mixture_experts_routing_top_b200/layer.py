@@ -23,8 +23,10 @@ from . import libmoe as M
 class TopKLayer:
     def __init__(self, T: int, d: int, E: int, k: int, F: int, capacity_factor: float, dtype: torch.dtype,
                  W1, W3, W2, act: str = "swiglu", norm_topk: bool = False, shared_weights=None,
-                 group_of_expert: Optional[torch.Tensor] = None, G: int = 0, out_dtype=None, device="cuda"):
+                 group_of_expert: Optional[torch.Tensor] = None, G: int = 0, out_dtype=None, device="cuda",
+                 W_r: Optional[torch.Tensor] = None):
         self.T, self.d, self.E, self.k, self.F = T, d, E, k, F
+        self.W_r = W_r                     # router linear gate [E, d]: route from x instead of handed-in logits
         self.cf, self.dtype, self.act, self.norm_topk = capacity_factor, dtype, act, norm_topk
         self.W1, self.W3, self.W2 = W1, W3, W2
         self.goe, self.G = group_of_expert, (G if group_of_expert is not None else 0)
@@ -70,6 +72,10 @@ class TopKLayer:
 
     def route(self, logits, stream=None):
         return M.route_topk(logits, self.k, self.norm_topk, self.idx, self.gate, stream=stream)
+
+    def route_x(self, x, stream=None):
+        """The router's linear gate fused with top-k (needs W_r)."""
+        return M.router_topk(x, self.W_r, self.k, self.norm_topk, self.idx, self.gate, stream=stream)
 
     def dispatch(self, x, stream=None):
         p = M.permute(x, self.idx, self.E, self.cf, self.goe, self.G, out=self.perm, workspace=self.perm_ws,
@@ -117,8 +123,12 @@ class TopKLayer:
             return M.unpermute_groups(y, self.perm["row_map"], shared, self.out_dtype, out=out, stream=stream)
         return M.unpermute(y, self.perm["row_map"], self.gate, shared, self.out_dtype, out=out, stream=stream)
 
-    def forward(self, logits: torch.Tensor, x: torch.Tensor, stream=None, out=None) -> torch.Tensor:
-        self.route(logits, stream)
+    def forward(self, logits: Optional[torch.Tensor], x: torch.Tensor, stream=None, out=None) -> torch.Tensor:
+        """logits: the handed-in router logits, or None when the layer has W_r."""
+        if self.W_r is not None:
+            self.route_x(x, stream)
+        else:
+            self.route(logits, stream)
         self.dispatch(x, stream)
         y = self.experts(stream)
         sh = self.shared_expert(x, stream)

@@ -31,6 +31,7 @@ SIGNATURES = {
     "moe_device_error": (_i32, [_i32]),
     "moe_kernel_launches": (ctypes.c_uint64, []),
     "moe_route_topk": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "moe_router_topk": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
     "moe_route_ec_workspace_bytes": (_sz, [_i32, _i32, _i32]),
     "moe_route_ec": (_i32, [_vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp, _sz, _vp]),
     "moe_capacity": (_i64, [_dbl, _i32, _i32, _i32]),
@@ -129,6 +130,29 @@ def route_topk(logits: torch.Tensor, k: int, norm_topk: bool = False, expert_idx
     _check("moe_route_topk", lib().moe_route_topk(_p(logits), T, E, k, int(bool(norm_topk)), _p(expert_idx),
                                                   _p(gate), _stream(stream)))
     return expert_idx, gate
+
+
+
+def router_topk(x: torch.Tensor, W_r: torch.Tensor, k: int, norm_topk: bool = False, expert_idx=None, gate=None,
+                logits=None, want_logits: bool = False, stream=None):
+    """Router linear gate + TopKRouter: (expert_idx [T,k] int32, gate [T,k] fp32, logits [T,E] fp32 or None)."""
+    _dev(x, None, "x")
+    _dev(W_r, x.dtype, "W_r")
+    T, d = x.shape
+    E = W_r.shape[0]
+    if W_r.shape[1] != d:
+        raise ValueError("W_r must be [E, d]")
+    dev = x.device
+    if expert_idx is None:
+        expert_idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+    if gate is None:
+        gate = torch.empty((T, k), dtype=torch.float32, device=dev)
+    if logits is None and (want_logits or x.dtype == torch.float32):
+        logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+    _check("moe_router_topk", lib().moe_router_topk(
+        _p(x), _act_dtype(x), T, d, _p(W_r), E, k, int(bool(norm_topk)), _p(logits), _p(expert_idx), _p(gate),
+        _stream(stream)))
+    return expert_idx, gate, logits
 
 
 def route_ec_workspace_bytes(T: int, E: int, C: int) -> int:

@@ -23,7 +23,7 @@ from . import synth
 
 # generator stream ids, one per tensor
 S_LOGITS, S_X, S_W1, S_W3, S_W2, S_BIAS, S_CLUSTER = 1, 2, 3, 4, 5, 6, 7
-S_SW1, S_SW3, S_SW2, S_P, S_NOISE2 = 8, 9, 10, 11, 12
+S_SW1, S_SW3, S_SW2, S_P, S_NOISE2, S_WR = 8, 9, 10, 11, 12, 13
 
 
 @dataclasses.dataclass(frozen=True)
@@ -47,6 +47,7 @@ class Workload:
     n_clusters: int = 0
     transition_mix: float = 0.0     # layer-2 logits = mix * P[top1 of layer 1] + N(0, 1)
     w_std: float = 0.02
+    router: int = 0                 # 1: logits = x W_r^T on the device (the router's linear gate)
     seed: int = 0
 
     @property
@@ -125,6 +126,12 @@ def make_weights(w: Workload) -> Tuple[np.ndarray, Optional[np.ndarray], np.ndar
     W3 = _normal(w, S_W3, (w.E, w.F, w.d), w.w_std) if w.act == "swiglu" else None
     W2 = _normal(w, S_W2, (w.E, w.d, w.F), w.w_std)
     return W1, W3, W2
+
+
+def make_router_weights(w: Workload) -> np.ndarray:
+    """Router linear gate W_r [E, d], N(0, 1/d): with x ~ N(0, 1) the logits
+    are about N(0, 1), the spread of the handed-in logits."""
+    return _normal(w, S_WR, (w.E, w.d), std=1.0 / math.sqrt(w.d))
 
 
 def make_shared_weights(w: Workload):

@@ -71,6 +71,20 @@ static double load_elem(const void* p, int dtype, int64_t i) {
     return (double)((const float*)p)[i];
 }
 
+/* ------------------------------------------------ router linear gate */
+/* [MegaDLMs] "Routing Mechanisms": the TopKRouter's scores are a linear
+ * layer over the token's hidden state, one output per expert:
+ * logits[t][e] = sum_c x[t][c] * W_r[e][c] (c ascending, double).
+ * x: [T, d], W_r: [E, d] (dtype); logits: [T, E] doubles. */
+void oracle_router_logits(const void* x, int dtype, int64_t T, int d, const void* W_r, int E, double* logits) {
+    for (int64_t t = 0; t < T; ++t)
+        for (int e = 0; e < E; ++e) {
+            double acc = 0.0;
+            for (int c = 0; c < d; ++c) acc += load_elem(x, dtype, t * d + c) * load_elem(W_r, dtype, (int64_t)e * d + c);
+            logits[t * E + e] = acc;
+        }
+}
+
 /* ------------------------------------------------------- TopKRouter */
 /* [MegaDLMs] "Routing Mechanisms": softmax over the expert logits, then the
  * top-k experts of each token; returns the probability weights (gates) and

@@ -39,6 +39,7 @@ def _load():
     lib = ctypes.CDLL(build())
     vp, i64, i32, dbl = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_double
     sig = {
+        "oracle_router_logits": (None, [vp, i32, i64, i32, vp, i32, vp]),
         "oracle_route_topk": (i32, [vp, i64, i32, i32, i32, vp, vp]),
         "oracle_capacity": (i64, [dbl, i64, i32, i32]),
         "oracle_permute": (i64, [vp, i64, i32, i32, i64, vp, i32, vp, vp, vp, vp, vp, vp]),
@@ -78,6 +79,20 @@ def _dt(a: np.ndarray) -> int:
     if a.dtype == np.uint16:
         return BF16
     raise TypeError("activations must be float32 or bf16 bit patterns (uint16), got %s" % a.dtype)
+
+
+
+def router_logits(x: np.ndarray, W_r: np.ndarray) -> np.ndarray:
+    """The router's linear gate x W_r^T, float64 [T, E]."""
+    x = np.ascontiguousarray(x)
+    W_r = np.ascontiguousarray(W_r)
+    dt = _dt(x)
+    assert W_r.dtype == x.dtype and W_r.shape[1] == x.shape[1]
+    T, d = x.shape
+    E = W_r.shape[0]
+    out = np.empty((T, E), np.float64)
+    _load().oracle_router_logits(x.ctypes.data, dt, T, d, W_r.ctypes.data, E, out.ctypes.data)
+    return out
 
 
 def route_topk(logits: np.ndarray, k: int, norm_topk: bool = False):

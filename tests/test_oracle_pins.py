@@ -327,6 +327,28 @@ def test_ffn_bf16_rounds_hidden_and_output():
         assert np.array_equal(y[i], synth.bf16_to_f32(synth.f32_to_bf16(y[i].astype(np.float32))))
 
 
+# ------------------------------------------------------- router linear gate
+def test_router_logits_match_float64_matmul():
+    x = synth.normal_bf16(3, 1, (37, 128))
+    Wr = synth.normal_bf16(3, 2, (24, 128), 0.0, 0.1)
+    got = O.router_logits(x, Wr)
+    want = synth.bf16_to_f32(x).astype(np.float64) @ synth.bf16_to_f32(Wr).astype(np.float64).T
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12)
+    xf, Wf = RNG.normal(size=(9, 17)).astype(np.float32), RNG.normal(size=(5, 17)).astype(np.float32)
+    np.testing.assert_allclose(O.router_logits(xf, Wf), xf.astype(np.float64) @ Wf.astype(np.float64).T, rtol=1e-12)
+
+
+def test_router_logits_exact_on_small_integers_and_one_hot_rows():
+    xi = RNG.integers(-8, 9, size=(50, 64))
+    Wi = RNG.integers(-8, 9, size=(16, 64))
+    got = O.router_logits(xi.astype(np.float32), Wi.astype(np.float32))
+    assert np.array_equal(got, (xi @ Wi.T).astype(np.float64))
+    # one-hot hidden states pick out one column of W_r
+    W = RNG.normal(size=(6, 10)).astype(np.float32)
+    eye = np.eye(10, dtype=np.float32)
+    assert np.array_equal(O.router_logits(eye, W), W.T.astype(np.float64))
+
+
 # -------------------------------------------------------------- combine
 def test_combine_identity_experts_closed_form():
     T, E, k, d = 70, 6, 3, 5
