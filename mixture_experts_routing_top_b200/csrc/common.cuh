@@ -66,6 +66,39 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Top-KM insertion for one token's logits seen in ascending expert order:
+// bv/bi hold the KM best so far, larger logit first.  A logit enters only if
+// strictly larger than the current KM-th, and slides above strictly smaller
+// entries only, so among equal logits the lower expert ranks first.
+template <int KM>
+__device__ __forceinline__ void topk_insert(float (&bv)[KM], int (&bi)[KM], float l, int e) {
+    if (!(l > bv[KM - 1])) return;
+    bool placed = false;
+#pragma unroll
+    for (int j = KM - 1; j >= 0; --j) {
+        if (!placed) {
+            if (j > 0 && l > bv[j - 1]) {
+                bv[j] = bv[j - 1];
+                bi[j] = bi[j - 1];
+            } else {
+                bv[j] = l;
+                bi[j] = e;
+                placed = true;
+            }
+        }
+    }
+}
+
+// exp(l - m) with the rounding error of l - m carried into the result
+// (TwoSum of l and -m, then exp(hi) * (1 + lo)).
+__device__ __forceinline__ float exp_diff(float l, float m) {
+    const float hi = __fsub_rn(l, m);
+    const float bb = __fsub_rn(hi, l);
+    const float lo = __fadd_rn(__fsub_rn(l, __fsub_rn(hi, bb)), __fsub_rn(-m, bb));
+    const float e = expf(hi);
+    return __fmaf_rn(e, lo, e);
+}
+
 template <typename T>
 __device__ __forceinline__ T warp_sum(T v) {
 #pragma unroll

@@ -5,6 +5,8 @@
 // takes a softmax over the expert logits and keeps each token's k best
 // experts with their probabilities; the expert-choice router lets every
 // expert pick the tokens with the highest routing score.
+#include <cstdlib>
+
 #include "common.cuh"
 
 namespace moe {
@@ -164,6 +166,158 @@ __global__ void __launch_bounds__(256) route_topk_vec_kernel(const float* __rest
         if (lane < k) {
             expert_idx[t * k + lane] = my_idx;
             gate[t * k + lane] = (float)((double)my_e / s);
+        }
+    }
+}
+
+// Thread-per-token variant for k <= 8 and E % 4 == 0 (any E up to 1024).
+// Each warp owns 32 consecutive tokens and walks their logits in chunks of
+// 32 experts through its own shared-memory ring (cp.async, two chunks in
+// flight; lanes copy 128-byte row pieces, 8 lanes per row, rows padded to
+// 36 floats so that 128-bit reads of a lane's own row are conflict-free).
+// Warps never wait for one another.  Every lane scans its own token: one
+// uniform pass over the chunk takes its maximum and marks the experts that
+// beat the current k-th best; the softmax denominator adds the chunk's terms
+// exp(l - m_run) relative to the running maximum (compensated fp32 sums per
+// chunk, the fp64 total rescaled when the maximum grows; skipped when the
+// gates are renormalised over the k); only the marked experts go through
+// the top-k insertion, in expert order.  Ranking ties resolve as in the
+// other variants (lower expert first).
+constexpr int kRowWarps = 4;                              // warps per CTA
+constexpr int kRowChunk = 32;                             // experts per chunk
+constexpr int kRowStride = 36;                            // floats per staged row
+constexpr int kRowBufs = 3;
+constexpr int kRowWarpFloats = kRowBufs * 32 * kRowStride;
+constexpr int kRowSmem = kRowWarps * kRowWarpFloats * 4;  // 54 KB
+
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"((unsigned)__cvta_generic_to_shared(smem_dst)),
+                 "l"(gmem_src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
+
+template <int KM>
+__global__ void __launch_bounds__(32 * kRowWarps, 4) route_topk_rows_kernel(const float* __restrict__ logits, int T,
+                                                                            int E, int k, int norm_topk,
+                                                                            int32_t* __restrict__ expert_idx,
+                                                                            float* __restrict__ gate) {
+    extern __shared__ __align__(16) float row_ring[];
+    const int lane = threadIdx.x & 31;
+    float* ring = row_ring + (threadIdx.x >> 5) * kRowWarpFloats;
+    const int E4 = E >> 2;
+    const int nchunk = (E + kRowChunk - 1) / kRowChunk;
+    const int lq = lane & 7;              // float4 slot this lane copies within a row piece
+    const int lr = lane >> 3;             // first row this lane copies (then every 4th)
+    const long long nwarps = (long long)gridDim.x * kRowWarps;
+    for (long long w = (long long)blockIdx.x * kRowWarps + (threadIdx.x >> 5); w * 32 < T; w += nwarps) {
+        const long long t0 = w * 32;
+        auto issue = [&](int c) {
+            if (c < nchunk) {
+                const int f4 = c * (kRowChunk / 4) + lq;
+                float* dst = ring + (c % kRowBufs) * (32 * kRowStride);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const long long tok = t0 + lr + 4 * u;
+                    if (tok < T && f4 < E4)
+                        cp_async16(&dst[(lr + 4 * u) * kRowStride + 4 * lq], logits + tok * E + 4 * f4);
+                }
+            }
+            cp_async_commit();                 // one group per chunk slot, empty past the last chunk
+        };
+        float bv[KM];
+        int bi[KM];
+#pragma unroll
+        for (int j = 0; j < KM; ++j) { bv[j] = -INFINITY; bi[j] = -1; }
+        float m_run = -INFINITY;           // running maximum (the softmax reference)
+        double s = 0.0;                    // sum of exp(l - m_run) so far
+        const long long t = t0 + lane;
+#pragma unroll
+        for (int c = 0; c < kRowBufs - 1; ++c) issue(c);
+        for (int c = 0; c < nchunk; ++c) {
+            issue(c + kRowBufs - 1);           // into the slot scanned one iteration ago
+            cp_async_wait<kRowBufs - 1>();     // chunk c: this lane's copies have landed
+            __syncwarp();                      // ... and the other lanes' copies are visible
+            if (t < T) {
+                const float* row = ring + (c % kRowBufs) * (32 * kRowStride) + lane * kRowStride;
+                const int e0 = c * kRowChunk;
+                const int nv = min(kRowChunk, E - e0);
+                if (c == 0) {                  // seed the list with the first KM experts
+#pragma unroll
+                    for (int i = 0; i < KM; ++i)
+                        if (i < nv) topk_insert<KM>(bv, bi, row[i], i);
+                }
+                const int skip = c == 0 ? KM : 0;
+                const float tau = bv[KM - 1];
+                // four independent accumulators (one per float4 lane) keep the dependency chains short
+                float cm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+                unsigned m4[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                for (int q = 0; q < kRowChunk / 4; ++q) {
+                    const float4 v4 = *reinterpret_cast<const float4*>(row + 4 * q);
+                    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int i = 4 * q + u;
+                        if (i < nv) {
+                            cm4[u] = fmaxf(cm4[u], v[u]);
+                            if (i >= skip && v[u] > tau) m4[u] |= 1u << i;
+                        }
+                    }
+                }
+                const float cm = fmaxf(fmaxf(cm4[0], cm4[1]), fmaxf(cm4[2], cm4[3]));
+                unsigned msk = m4[0] | m4[1] | m4[2] | m4[3];
+                if (!norm_topk) {
+                    if (cm > m_run) {
+                        s *= exp((double)m_run - (double)cm);
+                        m_run = cm;
+                    }
+                    float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f}, cc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+                    for (int q = 0; q < kRowChunk / 4; ++q) {
+                        const float4 v4 = *reinterpret_cast<const float4*>(row + 4 * q);
+                        const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            if (4 * q + u < nv) {
+                                const float y = __fsub_rn(__expf(__fsub_rn(v[u], m_run)), cc[u]);
+                                const float tt = __fadd_rn(cs[u], y);
+                                cc[u] = __fsub_rn(__fsub_rn(tt, cs[u]), y);
+                                cs[u] = tt;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) s += (double)cs[u] - (double)cc[u];
+                }
+                // insert the candidates in expert order (each re-checked against the moving threshold)
+                while (msk) {
+                    const int i = __ffs(msk) - 1;
+                    msk &= msk - 1;
+                    topk_insert<KM>(bv, bi, row[i], e0 + i);
+                }
+            }
+            __syncwarp();                      // slot c % kRowBufs may be refilled
+        }
+        cp_async_wait<0>();
+        if (t < T) {
+            const float m = bv[0];
+            float ej[KM];
+#pragma unroll
+            for (int j = 0; j < KM; ++j) ej[j] = j < k ? exp_diff(bv[j], m) : 0.0f;
+            if (norm_topk) {
+                s = 0.0;
+#pragma unroll
+                for (int j = 0; j < KM; ++j) s += (double)ej[j];
+            }
+#pragma unroll
+            for (int j = 0; j < KM; ++j) {
+                if (j < k) {
+                    expert_idx[t * k + j] = bi[j];
+                    gate[t * k + j] = (float)((double)ej[j] / s);
+                }
+            }
         }
     }
 }
@@ -684,6 +838,17 @@ using namespace moe;
 
 // ------------------------------------------------------------ host side
 
+namespace {
+// Thread per token needs enough tokens to occupy the GPU (T threads in
+// all); below that the warp-per-token kernels keep more warps in flight.
+// LIBMOE_TOPK_ROWS=0/1 forces either choice.
+bool use_rows_variant(int T) {
+    const char* env = getenv("LIBMOE_TOPK_ROWS");
+    if (env && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
+    return T >= 32768;
+}
+}  // namespace
+
 extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, int norm_topk,
                                      int32_t* expert_idx, float* gate, moe_stream_t stream) {
     if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_ARG;
@@ -696,6 +861,29 @@ extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, i
     int blocks = (int)((warps_needed + 7) / 8);
     if (blocks > 148 * 16) blocks = 148 * 16;
     const int nv = (E + 31) / 32;
+    if (E % 4 == 0 && k <= 8 && ((uintptr_t)logits & 15) == 0 && use_rows_variant(T)) {
+        static bool attr_done = false;
+        if (!attr_done) {
+            for (auto fn : {route_topk_rows_kernel<1>, route_topk_rows_kernel<2>, route_topk_rows_kernel<4>,
+                            route_topk_rows_kernel<8>})
+                if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowSmem) != cudaSuccess)
+                    return MOE_ERR_CUDA;
+            attr_done = true;
+        }
+        const long long warps = ((long long)T + 31) / 32;
+        long long rb = (warps + kRowWarps - 1) / kRowWarps;
+        const int rblocks = (int)(rb < 148 * 8 ? rb : 148 * 8);
+#define MOE_TOPKR_CASE(KM)                                                                              \
+    route_topk_rows_kernel<KM><<<rblocks, 32 * kRowWarps, kRowSmem, s>>>(logits, T, E, k, norm_topk, expert_idx, \
+                                                                         gate)
+        if (k <= 1) MOE_TOPKR_CASE(1);
+        else if (k <= 2) MOE_TOPKR_CASE(2);
+        else if (k <= 4) MOE_TOPKR_CASE(4);
+        else MOE_TOPKR_CASE(8);
+#undef MOE_TOPKR_CASE
+        MOE_LAUNCH_CHECK();
+        return MOE_OK;
+    }
     if (E % 4 == 0 && ((uintptr_t)logits & 15) == 0) {
         const int nv4 = (E + 127) / 128;
 #define MOE_TOPKV_CASE(N) \

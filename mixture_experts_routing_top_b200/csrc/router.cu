@@ -42,16 +42,6 @@ struct RouterArgs {
     unsigned* err;
 };
 
-// exp(l - m) with the rounding error of l - m carried into the result
-// (TwoSum of l and -m, then exp(hi) * (1 + lo)).
-__device__ __forceinline__ float exp_diff(float l, float m) {
-    const float hi = __fsub_rn(l, m);
-    const float bb = __fsub_rn(hi, l);
-    const float lo = __fadd_rn(__fsub_rn(l, __fsub_rn(hi, bb)), __fsub_rn(-m, bb));
-    const float e = expf(hi);
-    return __fmaf_rn(e, lo, e);
-}
-
 template <int KM>
 __global__ void __launch_bounds__(THREADS, 1) router_topk_kernel(const __grid_constant__ CUtensorMap map_x,
                                                                  const __grid_constant__ CUtensorMap map_w,
@@ -181,26 +171,8 @@ __global__ void __launch_bounds__(THREADS, 1) router_topk_kernel(const __grid_co
                 tmem_ld16(taddr + c, v);
                 tmem_ld_wait();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int e = c + i;
-                    const float l = v[i];
-                    if (e < E && l > bv[KM - 1]) {      // strict: an equal logit of a later expert ranks lower
-                        bool placed = false;
-#pragma unroll
-                        for (int j = KM - 1; j >= 0; --j) {
-                            if (!placed) {
-                                if (j > 0 && l > bv[j - 1]) {
-                                    bv[j] = bv[j - 1];
-                                    bi[j] = bi[j - 1];
-                                } else {
-                                    bv[j] = l;
-                                    bi[j] = e;
-                                    placed = true;
-                                }
-                            }
-                        }
-                    }
-                }
+                for (int i = 0; i < 16; ++i)
+                    if (c + i < E) topk_insert<KM>(bv, bi, v[i], c + i);
                 if (valid && lrow) {
                     float4* dst = reinterpret_cast<float4*>(lrow + c);
                     dst[0] = make_float4(v[0], v[1], v[2], v[3]);

@@ -156,17 +156,24 @@ inline bool tma_encoder_ready() {
     return true;
 }
 
-// 2-D bf16 tensor [rows, K] (K contiguous), box = 64 x box_rows (one 128-byte
-// swizzle row of K per box row).  Rows past the tensor read as zeros.
-inline bool make_bf16_map(CUtensorMap* m, const void* base, long long rows, int K, int box_rows) {
-    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
-    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+// 2-D row-major tensor [rows, cols] of elem_bytes-sized elements, box =
+// box_cols x box_rows with box_cols * elem_bytes == 128 (one 128-byte
+// swizzle row per box row).  Elements past the tensor read as zeros.
+inline bool make_tile_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, long long rows,
+                          long long cols, int box_cols, int box_rows) {
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)cols * elem_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = tma_encoder()(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-                               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+    CUresult r = tma_encoder()(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// bf16 [rows, K] (K contiguous), box = 64 x box_rows.
+inline bool make_bf16_map(CUtensorMap* m, const void* base, long long rows, int K, int box_rows) {
+    return make_tile_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, K, 64, box_rows);
 }
 
 inline int sm_count() {

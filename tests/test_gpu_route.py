@@ -21,19 +21,37 @@ def check_topk(logits, k, norm=False):
     np.testing.assert_allclose(gg, rgate, rtol=GATE_RTOL, atol=1e-30)
 
 
+@pytest.fixture(params=["rows", "warp"])
+def topk_kind(request, monkeypatch):
+    """Run a test with the thread-per-token top-k kernel and with the
+    warp-per-token ones (the library picks by T; the tests force each)."""
+    monkeypatch.setenv("LIBMOE_TOPK_ROWS", "1" if request.param == "rows" else "0")
+    return request.param
+
+
 @pytest.mark.parametrize("T,E,k", [(1, 1, 1), (7, 3, 2), (1000, 8, 2), (333, 33, 5), (512, 64, 6), (300, 100, 7),
-                                   (1025, 256, 8), (200, 1024, 32), (64, 160, 32), (50, 5, 5)])
+                                   (1025, 256, 8), (200, 1024, 32), (64, 160, 32), (50, 5, 5), (129, 36, 4),
+                                   (300, 1020, 8), (77, 12, 1)])
 @pytest.mark.parametrize("norm", [False, True])
-def test_topk_random(T, E, k, norm):
+def test_topk_random(T, E, k, norm, topk_kind):
     check_topk(synth.normal_f32(11, 1, (T, E), 0.0, 2.0), k, norm)
 
 
-def test_topk_ties_lower_index_wins():
+def test_topk_ties_lower_index_wins(topk_kind):
     rng = np.random.default_rng(0)
     for E, k in ((8, 3), (40, 6), (256, 8)):
         logits = rng.integers(-2, 3, size=(2000, E)).astype(np.float32)
         check_topk(logits, k)
     check_topk(np.zeros((10, 70), np.float32), 7, True)
+    z = np.zeros((300, 64), np.float32)
+    z[:, ::3] = -0.0                                  # -0 and +0 are equal logits: the lower expert wins
+    check_topk(z, 8)
+
+
+@pytest.mark.parametrize("E,k,norm", [(256, 8, True), (64, 6, False), (8, 2, False), (128, 1, False)])
+def test_topk_large_T_default_choice(E, k, norm):
+    """T large enough for the thread-per-token kernel to be the default."""
+    check_topk(synth.normal_f32(12, 1, (70001, E)), k, norm)
 
 
 def test_topk_empty():
