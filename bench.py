@@ -54,6 +54,8 @@ def parse(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=24, help="expert-MLP rows in the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--routing-only", action="store_true",
+                    help="time routing and co-selection alone at the workload's shape (top-k workloads)")
     ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
                     help="override a workload field (e.g. T=4096) - for smaller profiling cases, not bench lines")
     return ap.parse_args(argv)
@@ -75,6 +77,8 @@ def workload_from_args(args):
         w = w.with_(**{key: type(getattr(w, key))(val)})
     if args.set:
         w = w.with_(name=w.name + "[" + ",".join(args.set) + "]")
+    if getattr(args, "routing_only", False):
+        w = w.with_(name=w.name + "[routing only]")
     return w
 
 
@@ -517,7 +521,89 @@ class ExpertChoiceRunner:
                           % (w.T, t_rest, len(rows), R, t_row), "cpu": _cpu_name()}
 
 
-def make_runner(w, rank, device):
+class RoutingRunner:
+    """Routing and its statistic alone (top-k, or the fused router with
+    router=1, then co-selection) at a workload's shape: the routing step
+    measured where its inputs are large enough for HBM to matter."""
+
+    def __init__(self, w, rank, device):
+        import torch
+
+        from mixture_experts_routing_top_b200 import libmoe as M, workloads as W
+
+        self.w, self.M = w, M
+        wr = rank_batch(w, rank)
+        self.idx = torch.empty((w.T, w.k), dtype=torch.int32, device=device)
+        self.gate = torch.empty((w.T, w.k), dtype=torch.float32, device=device)
+        self.cosel = torch.zeros((w.E, w.E), dtype=torch.int32, device=device)
+        if w.router:
+            self.in_np = [W.make_x(wr)]
+            self.Wr_np = W.make_router_weights(w)
+            self.Wr = _dev(self.Wr_np, device)
+            route = lambda inp: M.router_topk(inp, self.Wr, w.k, w.norm_topk, self.idx, self.gate)
+        else:
+            self.in_np = [W.make_logits(wr)]
+            route = lambda inp: M.route_topk(inp, w.k, w.norm_topk, self.idx, self.gate)
+        self.inp = _dev(self.in_np[0], device)
+        self.route = route
+        self.resident_bytes = self.inp.numel() * self.inp.element_size()
+        self.stages = [("route", lambda: route(self.inp)),
+                       ("coselect", lambda: M.coselect(self.idx, w.E, into=self.cosel))]
+
+    def after_warmup(self):
+        pass
+
+    def work(self):
+        w = self.w
+        T, E, k = w.T, w.E, w.k
+        b = 2 if w.dtype == "bf16" else 4
+        route_in = T * w.d * b + E * w.d * b if w.router else T * E * 4
+        return {"route": ("bytes", route_in + T * k * 8), "coselect": ("bytes", T * k * 4 + E * E * 4)}
+
+    def e2e_setup(self):
+        import torch
+
+        self.h_in = _pinned(self.in_np[0])
+        self.h_out = [torch.empty(self.idx.shape, dtype=torch.int32).pin_memory(),
+                      torch.empty(self.gate.shape, dtype=torch.float32).pin_memory()]
+        self.d_in = [self.inp, torch.empty_like(self.inp)]
+
+    def e2e_run(self, n):
+        for i in range(n):
+            d = self.d_in[i & 1]
+            d.copy_(self.h_in, non_blocking=True)
+            self.route(d)
+            self.h_out[0].copy_(self.idx, non_blocking=True)
+            self.h_out[1].copy_(self.gate, non_blocking=True)
+
+    def e2e_bytes(self):
+        return self.h_in.numel() * self.h_in.element_size(), sum(h.numel() * h.element_size() for h in self.h_out)
+
+    def extra(self):
+        return {"routing_only": True}
+
+    def cpu_baseline(self, n_rows):
+        from oracle import oracle as O
+
+        w = self.w
+        Ts = min(w.T, 16384)
+        t0 = time.perf_counter()
+        if w.router:
+            lg = O.router_logits(self.in_np[0][:Ts], self.Wr_np).astype(np.float32)
+        else:
+            lg = self.in_np[0][:Ts]
+        idx, _ = O.route_topk(lg, w.k, w.norm_topk)
+        O.coselect(idx, w.E)
+        t = time.perf_counter() - t0
+        return {"value": Ts / t, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                "sample": "routing and co-selection on %d of %d tokens (%.2f s)" % (Ts, w.T, t), "cpu": _cpu_name()}
+
+
+def make_runner(w, rank, device, routing_only=False):
+    if routing_only:
+        if kind_of(w) == "ec":
+            raise SystemExit("--routing-only times top-k routing; the expert-choice workload routes inside its step")
+        return RoutingRunner(w, rank, device)
     return ExpertChoiceRunner(w, rank, device) if kind_of(w) == "ec" else TopKRunner(w, rank, device)
 
 
@@ -531,7 +617,7 @@ def run_libmoe(args, w, rank, world, local_rank):
     B.build()
     device = torch.device("cuda", local_rank)
     torch.cuda.set_device(device)
-    run = make_runner(w, rank, device)
+    run = make_runner(w, rank, device, args.routing_only)
     stream = torch.cuda.current_stream(device)
     names = [n for n, _ in run.stages]
     ns = len(names)

@@ -62,17 +62,25 @@ def check_router(x, Wr, k, norm=False, tokens=None):
     return clear.mean()
 
 
+@pytest.fixture(params=["persistent", "pair"])
+def router_kind(request, monkeypatch):
+    """Run a test with the persistent router kernel and with the one that
+    splits K over a CTA pair (the library picks by T; the tests force each)."""
+    monkeypatch.setenv("LIBMOE_ROUTER_PAIR", "1" if request.param == "pair" else "0")
+    return request.param
+
+
 @pytest.mark.parametrize("T,d,E,k", [(1, 64, 8, 2), (77, 128, 16, 1), (1000, 256, 8, 2), (1000, 64, 64, 6),
                                      (4097, 512, 128, 4), (300, 1024, 256, 8), (129, 192, 24, 3),
-                                     (2500, 2048, 72, 8)])
+                                     (2500, 2048, 72, 8), (700, 192, 8, 2)])
 @pytest.mark.parametrize("norm", [False, True])
-def test_router_bf16_random(T, d, E, k, norm):
+def test_router_bf16_random(T, d, E, k, norm, router_kind):
     x = synth.normal_bf16(21, 1, (T, d))
     Wr = synth.normal_bf16(21, 2, (E, d), 0.0, d ** -0.5)
     assert check_router(x, Wr, k, norm) > 0.95
 
 
-def test_router_exact_integers_and_ties():
+def test_router_exact_integers_and_ties(router_kind):
     """Small integers: exact logits, many ties (and all-zero rows, where the
     k lowest experts win)."""
     rng = np.random.default_rng(5)
@@ -91,7 +99,7 @@ def test_router_exact_integers_and_ties():
 
 
 @pytest.mark.parametrize("w", [W.MIXTRAL, W.FINE], ids=lambda w: w.name)
-def test_router_full_size(w):
+def test_router_full_size(w, router_kind):
     x = W.make_x(w)
     Wr = W.make_router_weights(w)
     rng = np.random.default_rng(1)
