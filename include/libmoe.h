@@ -208,6 +208,7 @@ moe_status moe_gather_rows(const void* x, int dtype, int T, int d, const int32_t
  * of `buffer` go through expert e:
  *   SwiGLU: h = silu(x W1[e]^T) * (x W3[e]^T),  y = h W2[e]^T
  *   GELU:   h = gelu(x W1[e]^T) (erf form),     y = h W2[e]^T
+ *           (erf evaluated by Abramowitz & Stegun 7.1.28: |error| <= 2e-6 in fp32)
  * bf16: tensor-core GEMMs with fp32 accumulation; h is stored as bf16 in the
  * workspace, y as bf16.  fp32: fp32 FMA throughout (small layers).
  *   buffer  [R_max, d]; offsets [E + 1] int32 on the device, offsets[0] = 0,

@@ -55,6 +55,45 @@ def test_expert_ffn_bf16(counts, d, F, act, gemm_kind):
     assert_layer_close(got, ref)
 
 
+def test_gelu_epilogue_matches_exact_erf(gemm_kind):
+    """One expert whose W1 and W2 are identities: the MLP returns gelu(x)
+    itself.  fp32: within the erf approximation's bound (A&S 7.1.28, 2e-6
+    absolute in fp32) plus fp32 rounding; bf16: the exact GELU rounded to
+    bf16, up to one bf16 step where the exact value sits on a rounding
+    boundary."""
+    import math
+    d = 64
+    xs = np.concatenate([np.linspace(-8.0, 8.0, 4091), [0.0, 1e-6, -1e-6, 1e-3, -1e-3]])
+    n = xs.size
+    eye = np.eye(d)
+    for bf16 in (False, True):
+        rows = np.zeros((n, d))
+        rows[:, 0] = xs
+        if bf16:
+            x = synth.f32_to_bf16(rows.astype(np.float32))
+            W = synth.f32_to_bf16(eye.astype(np.float32))
+        else:
+            x, W = rows.astype(np.float32), eye.astype(np.float32)
+        xv = as_f64(x)[:, 0]
+        y = torch.zeros((n, d), dtype=torch.bfloat16 if bf16 else torch.float32, device="cuda")
+        M.expert_ffn(to_dev(x), to_dev(np.array([0, n], np.int32)), to_dev(W[None]), None, to_dev(W[None]), "gelu",
+                     y=y)
+        got = as_f64(to_np(y))[:, 0]
+        exact = np.array([0.5 * v * (1.0 + math.erf(v / math.sqrt(2.0))) for v in xv])
+        # absolute error of 0.5 x (1 + erf): the approximation's 2e-6 on erf (in fp32, where 1 + erf also
+        # cancels to 0 in the far negative tail) times 0.5 |x|
+        approx = 1.1e-6 * np.abs(xv)
+        if bf16:
+            want = as_f64(synth.f32_to_bf16(exact.astype(np.float32)))
+            step = np.abs(want) * 2.0 ** -7 + 1e-38
+            assert (np.abs(got - want) <= step + approx).all()
+            # where |gelu| >= 0.05 the fp32 value of 1 + erf keeps its relative precision: bf16 values agree
+            big = np.abs(exact) >= 0.05
+            assert (got[big] == want[big]).mean() > 0.99
+        else:
+            assert (np.abs(got - exact) <= approx + 1e-6 * np.abs(exact) + 1e-30).all()
+
+
 def test_expert_ffn_fp32():
     got, ref = ffn_case([70, 0, 90, 100], 64, 128, "swiglu", bf16=False)
     assert_layer_close(got, ref, rel=1e-4)
