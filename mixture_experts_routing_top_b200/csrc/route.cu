@@ -346,9 +346,10 @@ constexpr int kEcThreads = 256;
 __global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __restrict__ logits, int T, int E, int tpb,
                                                                  double* __restrict__ lse_out,
                                                                  unsigned long long* __restrict__ keysT) {
-    extern __shared__ double ex[];                 // [tpb][E+1] exps (padded rows), then [tpb] row max / lse
-    const int ld = E + 1;
+    extern __shared__ double ex[];                 // [tpb][E+1] exps (padded rows), [tpb] row max / lse, then
+    const int ld = E + 1;                          // [tpb][E+1] the logits as floats (padded rows)
     double* rowv = ex + (size_t)tpb * ld;
+    float* lg = reinterpret_cast<float*>(rowv + tpb);
     const long long t0 = (long long)blockIdx.x * tpb;
     const int rows = (int)min((long long)tpb, (long long)T - t0);
     const float* src = logits + t0 * E;
@@ -367,7 +368,9 @@ __global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __
 #pragma unroll 4
     for (int f = threadIdx.x; f < n; f += blockDim.x) {
         const int r = f / E, c = f - r * E;
-        ex[r * ld + c] = exp((double)__ldg(src + f) - rowv[r]);
+        const float l = __ldg(src + f);
+        lg[r * ld + c] = l;
+        ex[r * ld + c] = exp((double)l - rowv[r]);
     }
     __syncthreads();
     // ascending-expert sums, one thread per token
@@ -385,13 +388,13 @@ __global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __
 #pragma unroll 4
     for (int f = threadIdx.x; f < rows * E; f += blockDim.x) {
         const int c = f / rows, r = f - c * rows;
-        keysT[(long long)c * T + t0 + r] = key_bits((double)__ldg(src + (long long)r * E + c) - rowv[r]);
+        keysT[(long long)c * T + t0 + r] = key_bits((double)lg[r * ld + c] - rowv[r]);
     }
 }
 
 int ec_tokens_per_block(int E) {
     int tpb = 32;                                   // ~33 KB at E = 128: several CTAs per SM
-    while (tpb > 1 && (size_t)tpb * (E + 2) * sizeof(double) > 96 * 1024) tpb >>= 1;
+    while (tpb > 1 && (size_t)tpb * ((E + 2) * sizeof(double) + (E + 1) * sizeof(float)) > 96 * 1024) tpb >>= 1;
     return tpb;
 }
 
@@ -840,12 +843,13 @@ using namespace moe;
 
 namespace {
 // Thread per token needs enough tokens to occupy the GPU (T threads in
-// all); below that the warp-per-token kernels keep more warps in flight.
-// LIBMOE_TOPK_ROWS=0/1 forces either choice.
-bool use_rows_variant(int T) {
+// all), and pays off when the warp kernels would spend many reduction
+// rounds (k >= 4); otherwise the warp-per-token kernels keep more warps in
+// flight.  LIBMOE_TOPK_ROWS=0/1 forces either choice.
+bool use_rows_variant(int T, int k) {
     const char* env = getenv("LIBMOE_TOPK_ROWS");
     if (env && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
-    return T >= 32768;
+    return T >= 32768 && k >= 4;
 }
 }  // namespace
 
@@ -861,7 +865,7 @@ extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, i
     int blocks = (int)((warps_needed + 7) / 8);
     if (blocks > 148 * 16) blocks = 148 * 16;
     const int nv = (E + 31) / 32;
-    if (E % 4 == 0 && k <= 8 && ((uintptr_t)logits & 15) == 0 && use_rows_variant(T)) {
+    if (E % 4 == 0 && k <= 8 && ((uintptr_t)logits & 15) == 0 && use_rows_variant(T, k)) {
         static bool attr_done = false;
         if (!attr_done) {
             for (auto fn : {route_topk_rows_kernel<1>, route_topk_rows_kernel<2>, route_topk_rows_kernel<4>,
@@ -957,7 +961,7 @@ extern "C" moe_status moe_route_ec(const float* logits, int T, int E, int C, int
     if (cudaMemsetAsync(mask, 0, sizeof(unsigned) * (size_t)T * mw, s) != cudaSuccess) return MOE_ERR_CUDA;
     {
         const int tpb = ec_tokens_per_block(E);
-        const size_t smem = (size_t)tpb * (E + 2) * sizeof(double);
+        const size_t smem = (size_t)tpb * ((E + 2) * sizeof(double) + (E + 1) * sizeof(float));
         if (smem > 48 * 1024 &&
             cudaFuncSetAttribute(ec_lse_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
             return MOE_ERR_CUDA;
