@@ -26,9 +26,11 @@
 //               heads per group and gives every kept slot its head's row.
 //   5. copy:    one token per warp, x[t] read once (16-byte vectors) and
 //               written to each distinct row the token owns.
+#include <cstdlib>
 #include <mutex>
 
 #include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace moe {
 
@@ -471,6 +473,85 @@ __global__ void __launch_bounds__(256) copy_rows_csr_kernel(const uint4* __restr
     }
 }
 
+// Bulk-copy variant: a warp takes one token at a time and lane 0 moves the
+// row with the bulk-copy engine - one cp.async.bulk load of x[t] into the
+// warp's shared-memory slot, then one cp.async.bulk store per distinct
+// destination row - so a 4-16 KB row costs a handful of instructions instead
+// of a 16-byte load and k 16-byte stores per lane per vector, which at these
+// row sizes throttle the load/store queues.  Many warps per SM keep rows in
+// flight.  No multicast.  The wait for the load is bounded; on expiry the
+// warp records MOE_ERR_TIMEOUT and stops.
+constexpr int kBulkWarps = 4;
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" :: "l"(dst), "r"(src), "r"(bytes)
+                 : "memory");
+}
+
+__global__ void __launch_bounds__(32 * kBulkWarps) copy_rows_bulk_kernel(const uint8_t* __restrict__ x, int T,
+                                                                         int row_bytes, int slot_bytes,
+                                                                         const int32_t* __restrict__ row_map, int k,
+                                                                         uint8_t* __restrict__ buffer, unsigned* err) {
+    extern __shared__ __align__(128) uint8_t bulk_slots[];
+    __shared__ __align__(8) uint64_t bars[kBulkWarps];
+    __shared__ int no_abort;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const uint32_t slot = tc::smem_u32(bulk_slots + (size_t)wid * slot_bytes);
+    const uint32_t bar = tc::smem_u32(&bars[wid]);
+    if (threadIdx.x == 0) no_abort = 0;
+    if (lane == 0) tc::mbar_init(bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncthreads();
+    uint32_t phase = 0;
+    const long long nworkers = (long long)gridDim.x * kBulkWarps;
+    for (long long t = (long long)blockIdx.x * kBulkWarps + wid; t < T; t += nworkers) {
+        int r = -1;
+        if (lane < k) r = row_map[t * k + lane];
+        const unsigned valid = __ballot_sync(0xffffffffu, r >= 0);
+        unsigned uniq = 0;                     // first slot of every distinct destination row
+        for (int j = 0; j < k; ++j) {
+            const int rj = __shfl_sync(0xffffffffu, r, j);
+            if (!((valid >> j) & 1u)) continue;
+            bool dup = false;
+            for (int q = 0; q < j; ++q) dup |= (((uniq >> q) & 1u) && __shfl_sync(0xffffffffu, r, q) == rj);
+            if (!dup) uniq |= 1u << j;
+        }
+        if (!uniq) continue;
+        int ok = 1;
+        if (lane == 0) {
+            tc::mbar_expect_tx(bar, (uint32_t)row_bytes);
+            bulk_load(slot, x + t * (long long)row_bytes, (uint32_t)row_bytes, bar);
+            ok = tc::mbar_wait(bar, phase, &no_abort) ? 1 : 0;
+        }
+        phase ^= 1u;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+            if (lane == 0) {
+                raise_error(err, kErrTimeout);
+                tc::mbar_wait(bar, phase ^ 1u, &no_abort);   // the load may still land: let it, once more bounded
+            }
+            break;
+        }
+        unsigned m = uniq;
+        while (m) {
+            const int j = __ffs(m) - 1;
+            m &= m - 1;
+            const int rj = __shfl_sync(0xffffffffu, r, j);
+            if (lane == 0) bulk_store(buffer + (long long)rj * row_bytes, slot, (uint32_t)row_bytes);
+        }
+        if (lane == 0) {
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // the slot may be reloaded
+        }
+        __syncwarp();
+    }
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 int copy_grid(long long T) {
     long long warps = T;
     long long blocks = (warps + 7) / 8;
@@ -511,6 +592,13 @@ PermWs perm_layout(int T, int k, int E, int G) {
     return w;
 }
 
+// LIBMOE_BULK_COPY=0/1 forces the vectorised or the bulk-copy row copy.
+bool bulk_copy_enabled() {
+    const char* env = getenv("LIBMOE_BULK_COPY");
+    if (env && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
+    return true;
+}
+
 bool set_smem(const void* fn, size_t bytes) {
     if (bytes <= 48 * 1024) return true;
     return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
@@ -520,6 +608,19 @@ moe_status launch_copy_slots(const void* x, int T, int row_bytes, const int32_t*
                              cudaStream_t s) {
     const int vpr = row_bytes / 16;
     const int grid = copy_grid(T);
+    const int slot_bytes = (row_bytes + 127) / 128 * 128;
+    if (bulk_copy_enabled() && slot_bytes <= 32 * 1024 && ((uintptr_t)x & 15) == 0 && ((uintptr_t)buffer & 15) == 0) {
+        unsigned* err = device_error_word();
+        if (!err) return MOE_ERR_CUDA;
+        const size_t smem = (size_t)kBulkWarps * slot_bytes;
+        if (!set_smem((const void*)copy_rows_bulk_kernel, smem)) return MOE_ERR_CUDA;
+        long long nb = ((long long)T + kBulkWarps - 1) / kBulkWarps;
+        const int blocks = (int)(nb < 148 * 16 ? nb : 148 * 16);
+        copy_rows_bulk_kernel<<<blocks, 32 * kBulkWarps, smem, s>>>((const uint8_t*)x, T, row_bytes, slot_bytes, row_map,
+                                                                    k, (uint8_t*)buffer, err);
+        MOE_LAUNCH_CHECK();
+        return MOE_OK;
+    }
     if (vpr <= 32) copy_rows_slots_kernel<1><<<grid, 256, 0, s>>>((const uint4*)x, T, vpr, row_map, k, (uint4*)buffer);
     else if (vpr <= 64) copy_rows_slots_kernel<2><<<grid, 256, 0, s>>>((const uint4*)x, T, vpr, row_map, k, (uint4*)buffer);
     else copy_rows_slots_kernel<4><<<grid, 256, 0, s>>>((const uint4*)x, T, vpr, row_map, k, (uint4*)buffer);
