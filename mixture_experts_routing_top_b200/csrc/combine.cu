@@ -10,7 +10,10 @@
 // registers first (slots that share a group-major row are read once, their
 // gates summed in slot order), then each lane streams 8-element vectors of
 // every distinct row and accumulates in fp32.
+#include <cstdlib>
+
 #include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace moe {
 
@@ -135,6 +138,158 @@ __global__ void __launch_bounds__(256) unpermute_vec_kernel(const void* __restri
                 int v = v0 + u * 32 + lane;
                 if (v < nvec) Vec8<OUT_BF16>::store(out, t * d + 8LL * v, acc[u]);
             }
+        }
+    }
+}
+
+// Bulk-staged combine (k <= 8, 16-byte rows): a warp takes one token.  Lane 0
+// brings the token's kept rows and its shared-expert row into the warp's
+// shared memory 1 KB column chunk by 1 KB chunk with the bulk-copy engine,
+// the next chunk in flight while the lanes add up the current one from
+// shared memory (two 16-byte pieces per lane: rows in first-appearance slot
+// order with their summed gates, then the shared row, in fp32 - the order of
+// unpermute_vec_kernel, so the results are the same bits) and store it.  No
+// per-lane global loads and few registers, so many tokens are in flight per
+// SM.  Waits bounded; on expiry the warp records MOE_ERR_TIMEOUT and stops.
+constexpr int kCmbWarps = 4;
+constexpr int kCmbChunk = 1024;                        // bytes of a row per chunk
+constexpr int kCmbRows = 9;                            // up to 8 kept rows + the shared row
+constexpr int kCmbStage = kCmbRows * kCmbChunk;        // 9 KB
+constexpr int kCmbSmem = kCmbWarps * 2 * kCmbStage;    // 72 KB
+
+template <bool BF16>
+__device__ __forceinline__ void piece_to_f32(uint4 v, float* f) {   // 16 bytes -> 8 (bf16) or 4 (fp32) values
+    if (BF16) {
+        f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x); f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+        f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z); f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+    } else {
+        f[0] = __uint_as_float(v.x); f[1] = __uint_as_float(v.y); f[2] = __uint_as_float(v.z); f[3] = __uint_as_float(v.w);
+    }
+}
+
+template <bool OUT_BF16, int N>
+__device__ __forceinline__ void store_piece(void* out, long long e, const float* f) {   // N = 8 or 4 values
+    if (OUT_BF16) {
+        uint16_t* o = static_cast<uint16_t*>(out) + e;
+        if (N == 8) {
+            uint4 w;
+            w.x = pack_bf16x2(f[0], f[1]); w.y = pack_bf16x2(f[2], f[3]);
+            w.z = pack_bf16x2(f[4], f[5]); w.w = pack_bf16x2(f[6], f[7]);
+            *reinterpret_cast<uint4*>(o) = w;
+        } else {
+            uint2 w;
+            w.x = pack_bf16x2(f[0], f[1]); w.y = pack_bf16x2(f[2], f[3]);
+            *reinterpret_cast<uint2*>(o) = w;
+        }
+    } else {
+        float4* o = reinterpret_cast<float4*>(static_cast<float*>(out) + e);
+        o[0] = make_float4(f[0], f[1], f[2], f[3]);
+        if (N == 8) o[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
+}
+
+template <bool IN_BF16, bool OUT_BF16>
+__global__ void __launch_bounds__(32 * kCmbWarps) unpermute_bulk_kernel(const uint8_t* __restrict__ y, int R, int T,
+                                                                        int d, int k,
+                                                                        const int32_t* __restrict__ row_map,
+                                                                        const float* __restrict__ gate,
+                                                                        const uint8_t* __restrict__ shared,
+                                                                        void* __restrict__ out, unsigned* err) {
+    extern __shared__ __align__(128) uint8_t cmb_smem[];
+    __shared__ __align__(8) uint64_t bars[kCmbWarps][2];
+    __shared__ int no_abort;
+    constexpr int ESZ = IN_BF16 ? 2 : 4;
+    constexpr int N = 16 / ESZ;                        // values per 16-byte piece
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    uint8_t* ws = cmb_smem + (size_t)wid * 2 * kCmbStage;
+    const long long row_bytes = (long long)d * ESZ;
+    const int nchunk = (int)((row_bytes + kCmbChunk - 1) / kCmbChunk);
+    if (threadIdx.x == 0) no_abort = 0;
+    if (lane == 0) {
+        tc::mbar_init(tc::smem_u32(&bars[wid][0]), 1);
+        tc::mbar_init(tc::smem_u32(&bars[wid][1]), 1);
+    }
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncthreads();
+    uint32_t par = 0;                                  // bit st: parity of stage st's next completion
+    const long long nworkers = (long long)gridDim.x * kCmbWarps;
+    for (long long t = (long long)blockIdx.x * kCmbWarps + wid; t < T; t += nworkers) {
+        int my_row;
+        float my_gate;
+        const int nu = token_rows(row_map, gate, t, k, R, err, my_row, my_gate);
+        int rr[8];
+        float gg[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            rr[j] = __shfl_sync(0xffffffffu, my_row, j);
+            gg[j] = __shfl_sync(0xffffffffu, my_gate, j);
+        }
+        const int nr = nu + (shared ? 1 : 0);
+        if (nr == 0) {                                 // every slot dropped and no shared expert: zeros
+            const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+            for (long long e = (long long)lane * N; e < d; e += 32LL * N) store_piece<OUT_BF16, N>(out, t * d + e, z);
+            continue;
+        }
+        auto issue = [&](int c, int st) {              // lane 0: chunk c of every row into stage st
+            if (lane != 0) return;
+            const long long off = (long long)c * kCmbChunk;
+            const uint32_t bytes = (uint32_t)min((long long)kCmbChunk, row_bytes - off);
+            const uint32_t bar = tc::smem_u32(&bars[wid][st]);
+            const uint32_t dst = tc::smem_u32(ws + st * kCmbStage);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // earlier reads of the stage come first
+            tc::mbar_expect_tx(bar, bytes * (uint32_t)nr);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j < nu) tc::bulk_load(dst + j * kCmbChunk, y + (long long)rr[j] * row_bytes + off, bytes, bar);
+            if (shared) tc::bulk_load(dst + 8 * kCmbChunk, shared + t * row_bytes + off, bytes, bar);
+        };
+        issue(0, 0);
+        bool ok = true;
+        for (int c = 0; c < nchunk; ++c) {
+            const int st = c & 1;
+            if (c + 1 < nchunk) issue(c + 1, st ^ 1);  // that stage's previous chunk was consumed last iteration
+            const uint32_t pst = (par >> st) & 1u;
+            const bool got = tc::mbar_wait(tc::smem_u32(&bars[wid][st]), pst, &no_abort);
+            par ^= 1u << st;
+            if (!__all_sync(0xffffffffu, got)) {
+                ok = false;
+                if (lane == 0) {                       // loads still in flight may land: give them one more bounded wait
+                    tc::mbar_wait(tc::smem_u32(&bars[wid][st]), pst, &no_abort);
+                    if (c + 1 < nchunk) tc::mbar_wait(tc::smem_u32(&bars[wid][st ^ 1]), (par >> (st ^ 1)) & 1u, &no_abort);
+                }
+                break;
+            }
+            const uint8_t* stage = ws + st * kCmbStage;
+#pragma unroll
+            for (int pc = 0; pc < 2; ++pc) {
+                const int boff = pc * 512 + lane * 16;               // byte offset of this lane's piece
+                const long long e = ((long long)c * kCmbChunk + boff) / ESZ;
+                if (e >= d) continue;
+                float acc[N];
+#pragma unroll
+                for (int i = 0; i < N; ++i) acc[i] = 0.0f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (j < nu) {
+                        float f[N];
+                        piece_to_f32<IN_BF16>(*reinterpret_cast<const uint4*>(stage + j * kCmbChunk + boff), f);
+#pragma unroll
+                        for (int i = 0; i < N; ++i) acc[i] = __fmaf_rn(gg[j], f[i], acc[i]);
+                    }
+                }
+                if (shared) {
+                    float f[N];
+                    piece_to_f32<IN_BF16>(*reinterpret_cast<const uint4*>(stage + 8 * kCmbChunk + boff), f);
+#pragma unroll
+                    for (int i = 0; i < N; ++i) acc[i] += f[i];
+                }
+                store_piece<OUT_BF16, N>(out, t * d + e, acc);
+            }
+            __syncwarp();
+        }
+        if (!ok) {
+            if (lane == 0) raise_error(err, kErrTimeout);
+            return;
         }
     }
 }
@@ -398,6 +553,15 @@ __global__ void __launch_bounds__(256) unpermute_groups_kernel(const void* __res
     }
 }
 
+// The bulk-staged combine pays off when a token has several rows to gather
+// (k >= 4); with one or two rows per token its per-chunk waits are exposed
+// and the register kernel is faster.  LIBMOE_BULK_COMBINE=0/1 forces either.
+bool bulk_combine_enabled(int k) {
+    const char* env = getenv("LIBMOE_BULK_COMBINE");
+    if (env && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
+    return k >= 4;
+}
+
 int token_grid(long long T) {
     long long blocks = (T + 7) / 8;
     long long cap = 148LL * 8;
@@ -434,7 +598,28 @@ extern "C" moe_status moe_unpermute(const void* y, int dtype, int R, int T, int 
     const int in_esz = in_bf16 ? 2 : 4, out_esz = out_bf16 ? 2 : 4;
     const bool vec = (d % 8 == 0) && ((d * in_esz) % 16 == 0) && ((d * out_esz) % 16 == 0) &&
                      (y == nullptr || aligned16(y)) && aligned16(out) && (shared == nullptr || aligned16(shared));
-    if (vec) {
+    if (vec && k <= 8 && bulk_combine_enabled(k)) {
+        static bool attr_done = false;
+        if (!attr_done) {
+            for (auto fn : {unpermute_bulk_kernel<true, true>, unpermute_bulk_kernel<true, false>,
+                            unpermute_bulk_kernel<false, true>, unpermute_bulk_kernel<false, false>})
+                if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kCmbSmem) != cudaSuccess)
+                    return MOE_ERR_CUDA;
+            attr_done = true;
+        }
+        long long nb = ((long long)T + kCmbWarps - 1) / kCmbWarps;
+        const int blocks = (int)(nb < 148 * 8 ? nb : 148 * 8);
+        const uint8_t* yb = (const uint8_t*)y;
+        const uint8_t* sb = (const uint8_t*)shared;
+        if (in_bf16 && out_bf16)
+            unpermute_bulk_kernel<true, true><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
+        else if (in_bf16)
+            unpermute_bulk_kernel<true, false><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
+        else if (out_bf16)
+            unpermute_bulk_kernel<false, true><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
+        else
+            unpermute_bulk_kernel<false, false><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
+    } else if (vec) {
         const int nvec = d / 8;
         if (nvec <= 32) MOE_DISPATCH_VEC(unpermute_vec_kernel, 1, y, R, T, d, k, row_map, gate, shared, out, err);
         else if (nvec <= 64) MOE_DISPATCH_VEC(unpermute_vec_kernel, 2, y, R, T, d, k, row_map, gate, shared, out, err);

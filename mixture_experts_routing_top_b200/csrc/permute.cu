@@ -483,15 +483,6 @@ __global__ void __launch_bounds__(256) copy_rows_csr_kernel(const uint4* __restr
 // warp records MOE_ERR_TIMEOUT and stops.
 constexpr int kBulkWarps = 4;
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-                 :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
-}
-__device__ __forceinline__ void bulk_store(void* dst, uint32_t src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" :: "l"(dst), "r"(src), "r"(bytes)
-                 : "memory");
-}
-
 __global__ void __launch_bounds__(32 * kBulkWarps) copy_rows_bulk_kernel(const uint8_t* __restrict__ x, int T,
                                                                          int row_bytes, int slot_bytes,
                                                                          const int32_t* __restrict__ row_map, int k,
@@ -524,7 +515,7 @@ __global__ void __launch_bounds__(32 * kBulkWarps) copy_rows_bulk_kernel(const u
         int ok = 1;
         if (lane == 0) {
             tc::mbar_expect_tx(bar, (uint32_t)row_bytes);
-            bulk_load(slot, x + t * (long long)row_bytes, (uint32_t)row_bytes, bar);
+            tc::bulk_load(slot, x + t * (long long)row_bytes, (uint32_t)row_bytes, bar);
             ok = tc::mbar_wait(bar, phase, &no_abort) ? 1 : 0;
         }
         phase ^= 1u;
@@ -541,15 +532,61 @@ __global__ void __launch_bounds__(32 * kBulkWarps) copy_rows_bulk_kernel(const u
             const int j = __ffs(m) - 1;
             m &= m - 1;
             const int rj = __shfl_sync(0xffffffffu, r, j);
-            if (lane == 0) bulk_store(buffer + (long long)rj * row_bytes, slot, (uint32_t)row_bytes);
+            if (lane == 0) tc::bulk_store(buffer + (long long)rj * row_bytes, slot, (uint32_t)row_bytes);
         }
         if (lane == 0) {
-            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-            asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");   // the slot may be reloaded
+            tc::bulk_commit();
+            tc::bulk_wait_read0();             // the slot may be reloaded
         }
         __syncwarp();
     }
-    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    if (lane == 0) tc::bulk_wait0();
+}
+
+// Expert-choice dispatch through the bulk-copy engine: the same scheme as
+// copy_rows_bulk_kernel with the destinations taken from the token CSR
+// (rows outside [0, R) are skipped and reported).
+__global__ void __launch_bounds__(32 * kBulkWarps) copy_rows_csr_bulk_kernel(const uint8_t* __restrict__ x, int T,
+                                                                             int row_bytes, int slot_bytes,
+                                                                             const int32_t* __restrict__ tok_ptr,
+                                                                             const int32_t* __restrict__ tok_row, int R,
+                                                                             uint8_t* __restrict__ buffer,
+                                                                             unsigned* err) {
+    extern __shared__ __align__(128) uint8_t bulk_slots[];
+    __shared__ __align__(8) uint64_t bars[kBulkWarps];
+    __shared__ int no_abort;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const uint32_t slot = tc::smem_u32(bulk_slots + (size_t)wid * slot_bytes);
+    const uint32_t bar = tc::smem_u32(&bars[wid]);
+    if (threadIdx.x == 0) no_abort = 0;
+    if (lane == 0) tc::mbar_init(bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncthreads();
+    uint32_t phase = 0;
+    const long long nworkers = (long long)gridDim.x * kBulkWarps;
+    if (lane == 0) {
+        for (long long t = (long long)blockIdx.x * kBulkWarps + wid; t < T; t += nworkers) {
+            const int p0 = max(tok_ptr[t], 0), p1 = min(tok_ptr[t + 1], R);
+            if (p1 <= p0) continue;
+            tc::mbar_expect_tx(bar, (uint32_t)row_bytes);
+            tc::bulk_load(slot, x + t * (long long)row_bytes, (uint32_t)row_bytes, bar);
+            const bool ok = tc::mbar_wait(bar, phase, &no_abort);
+            phase ^= 1u;
+            if (!ok) {
+                raise_error(err, kErrTimeout);
+                tc::mbar_wait(bar, phase ^ 1u, &no_abort);
+                break;
+            }
+            for (int p = p0; p < p1; ++p) {
+                const int r = tok_row[p];
+                if (r < 0 || r >= R) { raise_error(err, kErrIndex); continue; }
+                tc::bulk_store(buffer + (long long)r * row_bytes, slot, (uint32_t)row_bytes);
+            }
+            tc::bulk_commit();
+            tc::bulk_wait_read0();
+        }
+        tc::bulk_wait0();
+    }
 }
 
 int copy_grid(long long T) {
@@ -744,6 +781,17 @@ extern "C" moe_status moe_gather_rows(const void* x, int dtype, int T, int d, co
     if (!err) return MOE_ERR_CUDA;
     const int vpr = (int)(row_bytes / 16);
     const int grid = copy_grid(T);
+    const int slot_bytes = (int)((row_bytes + 127) / 128 * 128);
+    if (bulk_copy_enabled() && slot_bytes <= 32 * 1024) {
+        const size_t smem = (size_t)kBulkWarps * slot_bytes;
+        if (!set_smem((const void*)copy_rows_csr_bulk_kernel, smem)) return MOE_ERR_CUDA;
+        long long nb = ((long long)T + kBulkWarps - 1) / kBulkWarps;
+        const int blocks = (int)(nb < 148 * 16 ? nb : 148 * 16);
+        copy_rows_csr_bulk_kernel<<<blocks, 32 * kBulkWarps, smem, s>>>((const uint8_t*)x, T, (int)row_bytes, slot_bytes,
+                                                                        tok_ptr, tok_row, R, (uint8_t*)buffer, err);
+        MOE_LAUNCH_CHECK();
+        return MOE_OK;
+    }
     if (vpr <= 32) copy_rows_csr_kernel<1><<<grid, 256, 0, s>>>((const uint4*)x, T, vpr, tok_ptr, tok_row, R, (uint4*)buffer, err);
     else if (vpr <= 64) copy_rows_csr_kernel<2><<<grid, 256, 0, s>>>((const uint4*)x, T, vpr, tok_ptr, tok_row, R, (uint4*)buffer, err);
     else copy_rows_csr_kernel<4><<<grid, 256, 0, s>>>((const uint4*)x, T, vpr, tok_ptr, tok_row, R, (uint4*)buffer, err);

@@ -40,10 +40,18 @@ def check_combine(Y, row_map, gate, shared=None, out_bf16=False):
     assert (err <= tol).all(), "max excess %.3g" % (err - tol).max()
 
 
+@pytest.fixture(params=["bulk", "register"])
+def combine_kind(request, monkeypatch):
+    """Run a test with the bulk-staged combine and with the register one (the
+    library picks by k; the tests force each)."""
+    monkeypatch.setenv("LIBMOE_BULK_COMBINE", "1" if request.param == "bulk" else "0")
+    return request.param
+
+
 @pytest.mark.parametrize("T,E,k,cf,d,bf16", [(256, 8, 2, 1.25, 64, False), (1000, 8, 2, 0.5, 40, False),
                                              (777, 64, 6, 1.5, 136, True), (300, 256, 8, 0.0, 7168, True),
                                              (50, 4, 3, 0.9, 9, False), (64, 1024, 32, 0.0, 16, False)])
-def test_combine_expert_major(T, E, k, cf, d, bf16):
+def test_combine_expert_major(T, E, k, cf, d, bf16, combine_kind):
     lg = synth.normal_f32(2, 1, (T, E))
     idx, gate = O.route_topk(lg, k)
     p = O.permute(idx, E, O.capacity(cf, T, k, E))
@@ -57,7 +65,7 @@ def test_combine_expert_major(T, E, k, cf, d, bf16):
 
 
 @pytest.mark.parametrize("G", [8, 32, 64])
-def test_combine_group_major_identity_experts(G):
+def test_combine_group_major_identity_experts(G, combine_kind):
     w = W.SWEEP.with_(T=2048)
     idx, gate = O.route_topk(W.make_logits(w), w.k, True)
     p = O.permute(idx, w.E, O.capacity(0.0, w.T, w.k, w.E), W.equal_groups(w.E, G))
@@ -81,8 +89,11 @@ def test_combine_expert_choice(T, E, C, d):
     assert (np.abs(got - ref) <= REL * scale + 1e-30).all()
 
 
-def test_gather_rows_matches_token_csr():
-    T, E, C, d = 3000, 64, 100, 64
+@pytest.mark.parametrize("bulk", ["1", "0"])
+@pytest.mark.parametrize("d", [64, 1024, 7168])
+def test_gather_rows_matches_token_csr(bulk, d, monkeypatch):
+    monkeypatch.setenv("LIBMOE_BULK_COPY", bulk)          # bulk-copy engine, then the vectorised copy
+    T, E, C = 3000, 64, 100
     lg = synth.normal_f32(4, 1, (T, E))
     ec_token, _, tok_ptr, tok_row = O.route_ec(lg, C)
     x = synth.normal_bf16(4, 2, (T, d))

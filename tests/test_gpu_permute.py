@@ -44,11 +44,19 @@ def routed(T, E, k, seed=3, skew=0.0):
     return O.route_topk(lg, k)[0]
 
 
+@pytest.fixture(params=["bulk", "vector"])
+def copy_kind(request, monkeypatch):
+    """Run a test with the bulk-copy row copy and with the vectorised one
+    (the library uses the bulk copy whenever rows fit its shared-memory slot)."""
+    monkeypatch.setenv("LIBMOE_BULK_COPY", "1" if request.param == "bulk" else "0")
+    return request.param
+
+
 @pytest.mark.parametrize("T,E,k,cf,d,bf16", [
     (1, 1, 1, 1.0, 8, False), (1, 4, 2, 0.5, 8, True), (33, 3, 1, 0.7, 4, False), (1000, 8, 2, 0.5, 40, False),
     (1000, 8, 2, 1.25, 64, True), (4099, 16, 4, 0.9, 24, True), (777, 1024, 32, 2.0, 16, True),
     (2000, 64, 6, 0.0, 8, True), (513, 5, 5, 1.0, 64, False)])
-def test_expert_major(T, E, k, cf, d, bf16):
+def test_expert_major(T, E, k, cf, d, bf16, copy_kind):
     idx = routed(T, E, k, skew=1.0)
     x = synth.normal_bf16(1, 2, (T, d)) if bf16 else synth.normal_f32(1, 2, (T, d))
     _, ref = run(x, idx, E, cf)
@@ -58,7 +66,7 @@ def test_expert_major(T, E, k, cf, d, bf16):
 
 @pytest.mark.parametrize("T,E,k,G,cf", [(1000, 8, 2, 4, 0.0), (1000, 8, 3, 2, 0.6), (3001, 64, 6, 8, 1.5),
                                         (3001, 64, 6, 64, 0.0), (500, 16, 4, 1, 0.0), (4096, 256, 8, 32, 0.0)])
-def test_group_major(T, E, k, G, cf):
+def test_group_major(T, E, k, G, cf, copy_kind):
     idx = routed(T, E, k)
     x = synth.normal_bf16(1, 2, (T, 72))
     run(x, idx, E, cf, W.equal_groups(E, G))
