@@ -66,7 +66,7 @@ __device__ __forceinline__ int token_rows(const int32_t* __restrict__ row_map, c
     float g = 0.0f;
     if (lane < k) {
         r = row_map[t * k + lane];
-        g = gate[t * k + lane];
+        g = gate ? gate[t * k + lane] : 1.0f;
         if (r >= R) { raise_error(err, kErrIndex); r = -1; }
     }
     int nu = 0;
@@ -150,7 +150,9 @@ __global__ void __launch_bounds__(256) unpermute_vec_kernel(const void* __restri
 // order with their summed gates, then the shared row, in fp32 - the order of
 // unpermute_vec_kernel, so the results are the same bits) and store it.  No
 // per-lane global loads and few registers, so many tokens are in flight per
-// SM.  Waits bounded; on expiry the warp records MOE_ERR_TIMEOUT and stops.
+// SM.  UNIT: every distinct row with weight 1 (the sum of a token's group
+// rows, same order and bits as unpermute_groups_kernel).  Waits bounded; on
+// expiry the warp records MOE_ERR_TIMEOUT and stops.
 constexpr int kCmbWarps = 4;
 constexpr int kCmbChunk = 1024;                        // bytes of a row per chunk
 constexpr int kCmbRows = 9;                            // up to 8 kept rows + the shared row
@@ -188,7 +190,7 @@ __device__ __forceinline__ void store_piece(void* out, long long e, const float*
     }
 }
 
-template <bool IN_BF16, bool OUT_BF16>
+template <bool IN_BF16, bool OUT_BF16, bool UNIT>
 __global__ void __launch_bounds__(32 * kCmbWarps) unpermute_bulk_kernel(const uint8_t* __restrict__ y, int R, int T,
                                                                         int d, int k,
                                                                         const int32_t* __restrict__ row_map,
@@ -274,7 +276,7 @@ __global__ void __launch_bounds__(32 * kCmbWarps) unpermute_bulk_kernel(const ui
                         float f[N];
                         piece_to_f32<IN_BF16>(*reinterpret_cast<const uint4*>(stage + j * kCmbChunk + boff), f);
 #pragma unroll
-                        for (int i = 0; i < N; ++i) acc[i] = __fmaf_rn(gg[j], f[i], acc[i]);
+                        for (int i = 0; i < N; ++i) acc[i] = __fmaf_rn(UNIT ? 1.0f : gg[j], f[i], acc[i]);
                     }
                 }
                 if (shared) {
@@ -553,6 +555,23 @@ __global__ void __launch_bounds__(256) unpermute_groups_kernel(const void* __res
     }
 }
 
+template <bool UNIT>
+void launch_unpermute_bulk(bool in_bf16, bool out_bf16, cudaStream_t s, const void* y, int R, int T, int d, int k,
+                           const int32_t* row_map, const float* gate, const void* shared, void* out, unsigned* err) {
+    long long nb = ((long long)T + kCmbWarps - 1) / kCmbWarps;
+    const int blocks = (int)(nb < 148 * 8 ? nb : 148 * 8);
+    const uint8_t* yb = (const uint8_t*)y;
+    const uint8_t* sb = (const uint8_t*)shared;
+    if (in_bf16 && out_bf16)
+        unpermute_bulk_kernel<true, true, UNIT><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
+    else if (in_bf16)
+        unpermute_bulk_kernel<true, false, UNIT><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
+    else if (out_bf16)
+        unpermute_bulk_kernel<false, true, UNIT><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
+    else
+        unpermute_bulk_kernel<false, false, UNIT><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
+}
+
 // The bulk-staged combine pays off when a token has several rows to gather
 // (k >= 4); with one or two rows per token its per-chunk waits are exposed
 // and the register kernel is faster.  LIBMOE_BULK_COMBINE=0/1 forces either.
@@ -601,24 +620,13 @@ extern "C" moe_status moe_unpermute(const void* y, int dtype, int R, int T, int 
     if (vec && k <= 8 && bulk_combine_enabled(k)) {
         static bool attr_done = false;
         if (!attr_done) {
-            for (auto fn : {unpermute_bulk_kernel<true, true>, unpermute_bulk_kernel<true, false>,
-                            unpermute_bulk_kernel<false, true>, unpermute_bulk_kernel<false, false>})
+            for (auto fn : {unpermute_bulk_kernel<true, true, false>, unpermute_bulk_kernel<true, false, false>,
+                            unpermute_bulk_kernel<false, true, false>, unpermute_bulk_kernel<false, false, false>})
                 if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kCmbSmem) != cudaSuccess)
                     return MOE_ERR_CUDA;
             attr_done = true;
         }
-        long long nb = ((long long)T + kCmbWarps - 1) / kCmbWarps;
-        const int blocks = (int)(nb < 148 * 8 ? nb : 148 * 8);
-        const uint8_t* yb = (const uint8_t*)y;
-        const uint8_t* sb = (const uint8_t*)shared;
-        if (in_bf16 && out_bf16)
-            unpermute_bulk_kernel<true, true><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
-        else if (in_bf16)
-            unpermute_bulk_kernel<true, false><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
-        else if (out_bf16)
-            unpermute_bulk_kernel<false, true><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
-        else
-            unpermute_bulk_kernel<false, false><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
+        launch_unpermute_bulk<false>(in_bf16, out_bf16, s, y, R, T, d, k, row_map, gate, shared, out, err);
     } else if (vec) {
         const int nvec = d / 8;
         if (nvec <= 32) MOE_DISPATCH_VEC(unpermute_vec_kernel, 1, y, R, T, d, k, row_map, gate, shared, out, err);
@@ -723,6 +731,19 @@ extern "C" moe_status moe_unpermute_groups(const void* y_g, int dtype, int R_g, 
     cudaStream_t s = (cudaStream_t)stream;
     unsigned* err = device_error_word();
     if (!err) return MOE_ERR_CUDA;
+    if (k <= 8 && bulk_combine_enabled(k)) {
+        static bool attr_done = false;
+        if (!attr_done) {
+            for (auto fn : {unpermute_bulk_kernel<true, true, true>, unpermute_bulk_kernel<true, false, true>,
+                            unpermute_bulk_kernel<false, true, true>, unpermute_bulk_kernel<false, false, true>})
+                if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kCmbSmem) != cudaSuccess)
+                    return MOE_ERR_CUDA;
+            attr_done = true;
+        }
+        launch_unpermute_bulk<true>(in_bf16, out_bf16, s, y_g, R_g, T, d, k, row_map_g, nullptr, shared, out, err);
+        MOE_LAUNCH_CHECK();
+        return MOE_OK;
+    }
     const int grid = token_grid(T);
     const int nvec = d / 8;
     if (nvec <= 32) MOE_DISPATCH_VEC(unpermute_groups_kernel, 1, y_g, R_g, T, d, k, row_map_g, shared, out, err);

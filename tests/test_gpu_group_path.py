@@ -79,8 +79,10 @@ def test_group_precombine(T, E, k, cf, G, d, bf16):
     assert (got[R_g:] == 5.0).all()
 
 
+@pytest.mark.parametrize("bulk", ["1", "0"])
 @pytest.mark.parametrize("T,E,k,cf,G,d,bf16", CASES)
-def test_unpermute_groups(T, E, k, cf, G, d, bf16):
+def test_unpermute_groups(T, E, k, cf, G, d, bf16, bulk, monkeypatch):
+    monkeypatch.setenv("LIBMOE_BULK_COMBINE", bulk)       # bulk-staged kernel (k <= 8), then the register one
     idx, gate, goe, pe, pg = routing(T, E, k, cf, G, seed=2)
     R_g = max(pg["R"], 1)
     Yg = synth.normal_bf16(2, 3, (R_g, d)) if bf16 else synth.normal_f32(2, 3, (R_g, d))
