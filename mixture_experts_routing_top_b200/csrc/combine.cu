@@ -144,9 +144,10 @@ __global__ void __launch_bounds__(256) unpermute_vec_kernel(const void* __restri
 
 // Bulk-staged combine (k <= 8, 16-byte rows): a warp takes one token.  Lane 0
 // brings the token's kept rows and its shared-expert row into the warp's
-// shared memory 1 KB column chunk by 1 KB chunk with the bulk-copy engine,
-// the next chunk in flight while the lanes add up the current one from
-// shared memory (two 16-byte pieces per lane: rows in first-appearance slot
+// shared memory column chunk by column chunk (a 9 KB stage shared by the
+// rows: 1 KB per row for 8 rows and a shared row, 4 KB for two rows) with
+// the bulk-copy engine, the next chunk in flight while the lanes add up the
+// current one from shared memory (16-byte pieces per lane: rows in first-appearance slot
 // order with their summed gates, then the shared row, in fp32 - the order of
 // unpermute_vec_kernel, so the results are the same bits) and store it.  No
 // per-lane global loads and few registers, so many tokens are in flight per
@@ -154,9 +155,8 @@ __global__ void __launch_bounds__(256) unpermute_vec_kernel(const void* __restri
 // rows, same order and bits as unpermute_groups_kernel).  Waits bounded; on
 // expiry the warp records MOE_ERR_TIMEOUT and stops.
 constexpr int kCmbWarps = 4;
-constexpr int kCmbChunk = 1024;                        // bytes of a row per chunk
-constexpr int kCmbRows = 9;                            // up to 8 kept rows + the shared row
-constexpr int kCmbStage = kCmbRows * kCmbChunk;        // 9 KB
+constexpr int kCmbStage = 9 * 1024;                    // per stage: up to 8 rows + the shared row, 1 KB each
+                                                       // (fewer rows: larger chunks)
 constexpr int kCmbSmem = kCmbWarps * 2 * kCmbStage;    // 72 KB
 
 template <bool BF16>
@@ -190,13 +190,46 @@ __device__ __forceinline__ void store_piece(void* out, long long e, const float*
     }
 }
 
-template <bool IN_BF16, bool OUT_BF16, bool UNIT>
+// Rows of a token taken from the expert-choice CSR instead of a row map:
+// tok_row[tok_ptr[t] .. tok_ptr[t+1]) with gates ec_gate[row].
+struct CsrRows {
+    const int32_t* tok_ptr;
+    const int32_t* tok_row;
+    const float* ec_gate;
+};
+
+// A token of the expert-choice combine with more than 8 rows (rare: it needs
+// more than 8 experts to pick the same token): the lanes read the rows
+// directly, in CSR order.
+template <bool IN_BF16, bool OUT_BF16>
+__device__ void ec_token_direct(const void* y, int R, int d, long long t, int p0, int p1, const CsrRows& c, void* out,
+                                unsigned* err) {
+    const int lane = threadIdx.x & 31;
+    for (int e = lane * 8; e < d; e += 256) {
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+        for (int p = p0; p < p1; ++p) {
+            const int r = c.tok_row[p];
+            if (r < 0 || r >= R) { if (e == lane * 8) raise_error(err, kErrIndex); continue; }
+            const float g = c.ec_gate[r];
+            float f[8];
+            Vec8<IN_BF16>::load(y, (long long)r * d + e, f);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) acc[i] = __fmaf_rn(g, f[i], acc[i]);
+        }
+        Vec8<OUT_BF16>::store(out, t * d + e, acc);
+    }
+}
+
+template <bool IN_BF16, bool OUT_BF16, bool UNIT, bool CSR>
 __global__ void __launch_bounds__(32 * kCmbWarps) unpermute_bulk_kernel(const uint8_t* __restrict__ y, int R, int T,
                                                                         int d, int k,
                                                                         const int32_t* __restrict__ row_map,
                                                                         const float* __restrict__ gate,
                                                                         const uint8_t* __restrict__ shared,
-                                                                        void* __restrict__ out, unsigned* err) {
+                                                                        void* __restrict__ out, unsigned* err,
+                                                                        CsrRows csr) {
     extern __shared__ __align__(128) uint8_t cmb_smem[];
     __shared__ __align__(8) uint64_t bars[kCmbWarps][2];
     __shared__ int no_abort;
@@ -205,7 +238,6 @@ __global__ void __launch_bounds__(32 * kCmbWarps) unpermute_bulk_kernel(const ui
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
     uint8_t* ws = cmb_smem + (size_t)wid * 2 * kCmbStage;
     const long long row_bytes = (long long)d * ESZ;
-    const int nchunk = (int)((row_bytes + kCmbChunk - 1) / kCmbChunk);
     if (threadIdx.x == 0) no_abort = 0;
     if (lane == 0) {
         tc::mbar_init(tc::smem_u32(&bars[wid][0]), 1);
@@ -216,9 +248,23 @@ __global__ void __launch_bounds__(32 * kCmbWarps) unpermute_bulk_kernel(const ui
     uint32_t par = 0;                                  // bit st: parity of stage st's next completion
     const long long nworkers = (long long)gridDim.x * kCmbWarps;
     for (long long t = (long long)blockIdx.x * kCmbWarps + wid; t < T; t += nworkers) {
-        int my_row;
-        float my_gate;
-        const int nu = token_rows(row_map, gate, t, k, R, err, my_row, my_gate);
+        int my_row = -1, nu;
+        float my_gate = 0.0f;
+        if (CSR) {                                     // lane j < nu: the token's j-th row (-1 if out of range)
+            const int p0 = max(csr.tok_ptr[t], 0), p1 = min(csr.tok_ptr[t + 1], R);
+            nu = max(p1 - p0, 0);
+            if (nu > 8) {
+                ec_token_direct<IN_BF16, OUT_BF16>(y, R, d, t, p0, p1, csr, out, err);
+                continue;
+            }
+            if (lane < nu) {
+                const int r = csr.tok_row[p0 + lane];
+                if (r < 0 || r >= R) raise_error(err, kErrIndex);
+                else { my_row = r; my_gate = csr.ec_gate[r]; }
+            }
+        } else {
+            nu = token_rows(row_map, gate, t, k, R, err, my_row, my_gate);
+        }
         int rr[8];
         float gg[8];
 #pragma unroll
@@ -226,24 +272,32 @@ __global__ void __launch_bounds__(32 * kCmbWarps) unpermute_bulk_kernel(const ui
             rr[j] = __shfl_sync(0xffffffffu, my_row, j);
             gg[j] = __shfl_sync(0xffffffffu, my_gate, j);
         }
-        const int nr = nu + (shared ? 1 : 0);
+        const int nr = __popc(__ballot_sync(0xffffffffu, lane < nu && my_row >= 0)) + (shared ? 1 : 0);
         if (nr == 0) {                                 // every slot dropped and no shared expert: zeros
             const float z[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
             for (long long e = (long long)lane * N; e < d; e += 32LL * N) store_piece<OUT_BF16, N>(out, t * d + e, z);
             continue;
         }
+        // chunk size for this token: the stage (9 KB) divided among its row slots, in 512-byte
+        // steps, so that a token with few rows moves a few KB per wait
+        const int slots = nu + (shared ? 1 : 0);
+        int cb = kCmbStage / slots / 512 * 512;
+        const int row_cb = (int)((row_bytes + 511) / 512 * 512);
+        if (cb > row_cb) cb = row_cb;
+        const int nchunk = (int)((row_bytes + cb - 1) / cb);
         auto issue = [&](int c, int st) {              // lane 0: chunk c of every row into stage st
             if (lane != 0) return;
-            const long long off = (long long)c * kCmbChunk;
-            const uint32_t bytes = (uint32_t)min((long long)kCmbChunk, row_bytes - off);
+            const long long off = (long long)c * cb;
+            const uint32_t bytes = (uint32_t)min((long long)cb, row_bytes - off);
             const uint32_t bar = tc::smem_u32(&bars[wid][st]);
             const uint32_t dst = tc::smem_u32(ws + st * kCmbStage);
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // earlier reads of the stage come first
             tc::mbar_expect_tx(bar, bytes * (uint32_t)nr);
 #pragma unroll
             for (int j = 0; j < 8; ++j)
-                if (j < nu) tc::bulk_load(dst + j * kCmbChunk, y + (long long)rr[j] * row_bytes + off, bytes, bar);
-            if (shared) tc::bulk_load(dst + 8 * kCmbChunk, shared + t * row_bytes + off, bytes, bar);
+                if (j < nu && rr[j] >= 0)
+                    tc::bulk_load(dst + j * cb, y + (long long)rr[j] * row_bytes + off, bytes, bar);
+            if (shared) tc::bulk_load(dst + nu * cb, shared + t * row_bytes + off, bytes, bar);
         };
         issue(0, 0);
         bool ok = true;
@@ -262,26 +316,25 @@ __global__ void __launch_bounds__(32 * kCmbWarps) unpermute_bulk_kernel(const ui
                 break;
             }
             const uint8_t* stage = ws + st * kCmbStage;
-#pragma unroll
-            for (int pc = 0; pc < 2; ++pc) {
-                const int boff = pc * 512 + lane * 16;               // byte offset of this lane's piece
-                const long long e = ((long long)c * kCmbChunk + boff) / ESZ;
-                if (e >= d) continue;
+#pragma unroll 2
+            for (int boff = lane * 16; boff < cb; boff += 512) {       // this lane's 16-byte pieces of the chunk
+                const long long e = ((long long)c * cb + boff) / ESZ;
+                if (e >= d) break;
                 float acc[N];
 #pragma unroll
                 for (int i = 0; i < N; ++i) acc[i] = 0.0f;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    if (j < nu) {
+                    if (j < nu && rr[j] >= 0) {
                         float f[N];
-                        piece_to_f32<IN_BF16>(*reinterpret_cast<const uint4*>(stage + j * kCmbChunk + boff), f);
+                        piece_to_f32<IN_BF16>(*reinterpret_cast<const uint4*>(stage + j * cb + boff), f);
 #pragma unroll
                         for (int i = 0; i < N; ++i) acc[i] = __fmaf_rn(UNIT ? 1.0f : gg[j], f[i], acc[i]);
                     }
                 }
                 if (shared) {
                     float f[N];
-                    piece_to_f32<IN_BF16>(*reinterpret_cast<const uint4*>(stage + 8 * kCmbChunk + boff), f);
+                    piece_to_f32<IN_BF16>(*reinterpret_cast<const uint4*>(stage + nu * cb + boff), f);
 #pragma unroll
                     for (int i = 0; i < N; ++i) acc[i] += f[i];
                 }
@@ -555,21 +608,41 @@ __global__ void __launch_bounds__(256) unpermute_groups_kernel(const void* __res
     }
 }
 
-template <bool UNIT>
-void launch_unpermute_bulk(bool in_bf16, bool out_bf16, cudaStream_t s, const void* y, int R, int T, int d, int k,
-                           const int32_t* row_map, const float* gate, const void* shared, void* out, unsigned* err) {
+template <bool UNIT, bool CSR>
+moe_status launch_unpermute_bulk(bool in_bf16, bool out_bf16, cudaStream_t s, const void* y, int R, int T, int d,
+                                 int k, const int32_t* row_map, const float* gate, const void* shared, void* out,
+                                 unsigned* err, CsrRows csr = CsrRows{nullptr, nullptr, nullptr}) {
+    static bool attr_done = false;
+    if (!attr_done) {
+        for (auto fn : {unpermute_bulk_kernel<true, true, UNIT, CSR>, unpermute_bulk_kernel<true, false, UNIT, CSR>,
+                        unpermute_bulk_kernel<false, true, UNIT, CSR>, unpermute_bulk_kernel<false, false, UNIT, CSR>})
+            if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kCmbSmem) != cudaSuccess)
+                return MOE_ERR_CUDA;
+        attr_done = true;
+    }
     long long nb = ((long long)T + kCmbWarps - 1) / kCmbWarps;
     const int blocks = (int)(nb < 148 * 8 ? nb : 148 * 8);
     const uint8_t* yb = (const uint8_t*)y;
     const uint8_t* sb = (const uint8_t*)shared;
     if (in_bf16 && out_bf16)
-        unpermute_bulk_kernel<true, true, UNIT><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
+        unpermute_bulk_kernel<true, true, UNIT, CSR><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err, csr);
     else if (in_bf16)
-        unpermute_bulk_kernel<true, false, UNIT><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
+        unpermute_bulk_kernel<true, false, UNIT, CSR><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err, csr);
     else if (out_bf16)
-        unpermute_bulk_kernel<false, true, UNIT><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
+        unpermute_bulk_kernel<false, true, UNIT, CSR><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err, csr);
     else
-        unpermute_bulk_kernel<false, false, UNIT><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err);
+        unpermute_bulk_kernel<false, false, UNIT, CSR><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err, csr);
+    return MOE_OK;
+}
+
+// Expert choice: a token has about E*C/T rows (2 at the expert-choice
+// workload), too few for the staging to pay (measured 95 vs 56 us there), so
+// the register kernel is the default; LIBMOE_BULK_COMBINE=1 selects the
+// bulk-staged one.
+bool bulk_combine_ec_enabled() {
+    const char* env = getenv("LIBMOE_BULK_COMBINE");
+    if (env && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
+    return false;
 }
 
 // The bulk-staged combine pays off when a token has several rows to gather
@@ -618,15 +691,9 @@ extern "C" moe_status moe_unpermute(const void* y, int dtype, int R, int T, int 
     const bool vec = (d % 8 == 0) && ((d * in_esz) % 16 == 0) && ((d * out_esz) % 16 == 0) &&
                      (y == nullptr || aligned16(y)) && aligned16(out) && (shared == nullptr || aligned16(shared));
     if (vec && k <= 8 && bulk_combine_enabled(k)) {
-        static bool attr_done = false;
-        if (!attr_done) {
-            for (auto fn : {unpermute_bulk_kernel<true, true, false>, unpermute_bulk_kernel<true, false, false>,
-                            unpermute_bulk_kernel<false, true, false>, unpermute_bulk_kernel<false, false, false>})
-                if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kCmbSmem) != cudaSuccess)
-                    return MOE_ERR_CUDA;
-            attr_done = true;
-        }
-        launch_unpermute_bulk<false>(in_bf16, out_bf16, s, y, R, T, d, k, row_map, gate, shared, out, err);
+        const moe_status st = launch_unpermute_bulk<false, false>(in_bf16, out_bf16, s, y, R, T, d, k, row_map, gate,
+                                                                  shared, out, err);
+        if (st != MOE_OK) return st;
     } else if (vec) {
         const int nvec = d / 8;
         if (nvec <= 32) MOE_DISPATCH_VEC(unpermute_vec_kernel, 1, y, R, T, d, k, row_map, gate, shared, out, err);
@@ -654,7 +721,11 @@ extern "C" moe_status moe_unpermute_ec(const void* y, int dtype, int R, int T, i
     const int in_esz = in_bf16 ? 2 : 4, out_esz = out_bf16 ? 2 : 4;
     const bool vec = (d % 8 == 0) && ((d * in_esz) % 16 == 0) && ((d * out_esz) % 16 == 0) &&
                      (y == nullptr || aligned16(y)) && aligned16(out);
-    if (vec) {
+    if (vec && bulk_combine_ec_enabled()) {
+        const moe_status st = launch_unpermute_bulk<false, true>(in_bf16, out_bf16, s, y, R, T, d, 0, nullptr, nullptr,
+                                                                 nullptr, out, err, CsrRows{tok_ptr, tok_row, ec_gate});
+        if (st != MOE_OK) return st;
+    } else if (vec) {
         const int nvec = d / 8;
         if (nvec <= 32) MOE_DISPATCH_VEC(unpermute_ec_vec_kernel, 1, y, R, T, d, tok_ptr, tok_row, ec_gate, out, err);
         else if (nvec <= 64) MOE_DISPATCH_VEC(unpermute_ec_vec_kernel, 2, y, R, T, d, tok_ptr, tok_row, ec_gate, out, err);
@@ -732,15 +803,9 @@ extern "C" moe_status moe_unpermute_groups(const void* y_g, int dtype, int R_g, 
     unsigned* err = device_error_word();
     if (!err) return MOE_ERR_CUDA;
     if (k <= 8 && bulk_combine_enabled(k)) {
-        static bool attr_done = false;
-        if (!attr_done) {
-            for (auto fn : {unpermute_bulk_kernel<true, true, true>, unpermute_bulk_kernel<true, false, true>,
-                            unpermute_bulk_kernel<false, true, true>, unpermute_bulk_kernel<false, false, true>})
-                if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kCmbSmem) != cudaSuccess)
-                    return MOE_ERR_CUDA;
-            attr_done = true;
-        }
-        launch_unpermute_bulk<true>(in_bf16, out_bf16, s, y_g, R_g, T, d, k, row_map_g, nullptr, shared, out, err);
+        const moe_status st = launch_unpermute_bulk<true, false>(in_bf16, out_bf16, s, y_g, R_g, T, d, k, row_map_g,
+                                                                 nullptr, shared, out, err);
+        if (st != MOE_OK) return st;
         MOE_LAUNCH_CHECK();
         return MOE_OK;
     }

@@ -77,8 +77,9 @@ def test_combine_group_major_identity_experts(G, combine_kind):
     np.testing.assert_allclose(got, as_f64(x), rtol=1e-5, atol=1e-6)
 
 
-@pytest.mark.parametrize("T,E,C,d", [(40, 4, 10, 8), (3000, 64, 100, 64), (5000, 128, 79, 1024)])
-def test_combine_expert_choice(T, E, C, d):
+@pytest.mark.parametrize("T,E,C,d", [(40, 4, 10, 8), (3000, 64, 100, 64), (5000, 128, 79, 1024), (300, 16, 250, 136),
+                                     (2000, 32, 1500, 2048)])
+def test_combine_expert_choice(T, E, C, d, combine_kind):
     lg = synth.normal_f32(4, 1, (T, E))
     ec_token, ec_gate, tok_ptr, tok_row = O.route_ec(lg, C)
     Y = synth.normal_bf16(4, 9, (E * C, d))
