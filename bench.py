@@ -54,6 +54,8 @@ def parse(argv=None):
     ap.add_argument("--cpu-rows", type=int, default=24, help="expert-MLP rows in the CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
+    ap.add_argument("--graph", action="store_true",
+                    help="time the step as one CUDA-graph replay (stage times from an eager pass before it)")
     ap.add_argument("--routing-only", action="store_true",
                     help="time routing and co-selection alone at the workload's shape (top-k workloads)")
     ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
@@ -643,6 +645,22 @@ def run_libmoe(args, w, rank, world, local_rank):
 
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(ns + 1)] for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    graph = None
+    if args.graph:
+        # stage times from an eager pass, then the whole step captured once and replayed
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+        stage_ms_eager = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in enumerate(names)}
+        n_cap = M.kernel_launches()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        per_step = M.kernel_launches() - n_cap
+        graph.replay()
+        torch.cuda.synchronize()
     clocks = Clocks()
     if world > 1:
         dist.barrier()
@@ -658,10 +676,16 @@ def run_libmoe(args, w, rank, world, local_rank):
     for i in range(args.steps):
         if flush is not None:
             flush.zero_()
-        step(evs[i])
+        if graph is None:
+            step(evs[i])
+        else:
+            evs[i][0].record(stream)
+            graph.replay()
+            evs[i][ns].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
-    launches = M.kernel_launches() - n0
+    # graph replays launch their kernels without the host: count them from the capture
+    launches = M.kernel_launches() - n0 if graph is None else per_step * args.steps
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
@@ -670,7 +694,10 @@ def run_libmoe(args, w, rank, world, local_rank):
         elapsed_ms = t_start.elapsed_time(t_end)
     else:
         elapsed_ms = sum(e[0].elapsed_time(e[ns]) for e in evs)
-    stage_ms = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in enumerate(names)}
+    if graph is None:
+        stage_ms = {n: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs) for j, n in enumerate(names)}
+    else:
+        stage_ms = stage_ms_eager
     if M.device_error() != 0:
         raise RuntimeError("device fault word set during the timed steps")
     elapsed_ms, launches = reduce_over_ranks(elapsed_ms, launches, device)
@@ -732,6 +759,8 @@ def run_libmoe(args, w, rank, world, local_rank):
         cfg["F_shared"] = w.F_shared
     if w.G and not w.F:
         cfg["G"] = w.G
+    if graph is not None:
+        cfg["launch"] = "step replayed as one CUDA graph; stage times from an eager pass"
     cfg.update({"global_batch": world * w.T, "parallelism": "independent replicas, one batch per GPU",
                 "l2": ("flushed between timed steps (256 MB write outside the events)" if flush is not None else
                        "inputs larger than L2: %.2f GB resident inputs read every step" % (run.resident_bytes / 1e9))})

@@ -211,3 +211,32 @@ class HostPipeline:
                 hout.copy_(self.dout[b], non_blocking=True)
                 self.ev_drained[b].record(self.s_out)
         s_c.wait_stream(self.s_out)
+
+
+class CapturedForward:
+    """A layer call captured once into a CUDA graph.
+
+    fn(*inputs, out=out) runs on the current stream with every buffer
+    preallocated (the layers here are written that way), so the whole call -
+    all its kernels, workspace clears included - can be recorded once and
+    replayed with no host launch work.  Inputs are read from, and the result
+    written to, the tensors given here: copy new inputs into them before a
+    replay.  The call is run `warmup` times on a side stream first (first
+    calls set kernel attributes and look up driver entry points, which a
+    capture must not see)."""
+
+    def __init__(self, fn, inputs, out, warmup: int = 2):
+        self.fn, self.inputs, self.out = fn, list(inputs), out
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            for _ in range(warmup):
+                fn(*self.inputs, out=out)
+        torch.cuda.current_stream().wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            fn(*self.inputs, out=out)
+
+    def replay(self):
+        self.graph.replay()
+        return self.out

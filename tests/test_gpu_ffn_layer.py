@@ -210,3 +210,25 @@ def test_host_pipeline_matches_plain_forward():
     for (lg, x), got in zip(h_in, h_out):
         want = L.forward(lg.cuda(), x.cuda()).cpu()
         assert torch.equal(got, want)
+
+
+@pytest.mark.parametrize("bf16", [False, True])
+def test_captured_forward_matches_eager(bf16):
+    """The whole top-k layer recorded as one CUDA graph: replays give exactly
+    the eager outputs, and follow new contents of the input tensors."""
+    w = W.TINY if not bf16 else W.FINE.with_(T=2048, F_shared=0)
+    dt = torch.bfloat16 if bf16 else torch.float32
+    Wt = weights_dev(W.make_weights(w))
+    L = Lyr.TopKLayer(w.T, w.d, w.E, w.k, w.F, w.capacity_factor, dt, *Wt)
+    lg0, x0 = to_dev(W.make_logits(w)), to_dev(W.make_x(w))
+    want0 = L.forward(lg0, x0).clone()
+    w1 = w.with_(seed=5)
+    lg1, x1 = to_dev(W.make_logits(w1)), to_dev(W.make_x(w1))
+    want1 = L.forward(lg1, x1).clone()
+    lg, x = lg0.clone(), x0.clone()
+    cap = Lyr.CapturedForward(lambda a, b, out: L.forward(a, b, out=out), [lg, x], torch.empty_like(L.out))
+    assert torch.equal(cap.replay(), want0)
+    lg.copy_(lg1)
+    x.copy_(x1)
+    assert torch.equal(cap.replay(), want1)
+    assert M.device_error() == 0
