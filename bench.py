@@ -805,8 +805,16 @@ def run_reference(args, w):
                             O.capacity(w.capacity_factor, Ts, w.k, w.E), None if grouped else goe)["R"]
     Y = synth.normal_bf16(99, 1, (R_probe, w.d)) if w.dtype == "bf16" else synth.normal_f32(99, 1, (R_probe, w.d))
 
+    routing_only = getattr(args, "routing_only", False) and not is_ec
+
     def step(i):
         t0 = time.perf_counter()
+        if routing_only:                       # routing and co-selection alone
+            lg = O.router_logits(x, Wr).astype(np.float32) if Wr is not None else logits
+            idx, _ = O.route_topk(lg, w.k, w.norm_topk)
+            O.coselect(idx, w.E)
+            t1 = time.perf_counter()
+            return (t1 - t0) / Ts, t1 - t0
         if is_ec:
             ec_token, ec_gate, tok_ptr, tok_row = O.route_ec(logits, C)
             buf = O.gather_rows(x, ec_token.reshape(-1))
@@ -848,6 +856,8 @@ def run_reference(args, w):
     value = len(per_token) / sum(per_token)
     sample = ("per step: routing, capacity, permutation, row copy and combine over %d of %d tokens%s, "
               "extrapolated per token" % (Ts, w.T, ", plus the expert MLP of one buffer row" if w.F else ""))
+    if routing_only:
+        sample = "per step: routing and co-selection over %d of %d tokens, extrapolated per token" % (Ts, w.T)
     return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(wall), 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
