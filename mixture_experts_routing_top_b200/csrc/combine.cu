@@ -8,8 +8,10 @@
 //
 // One warp per token.  The token's (row, gate) pairs are deduplicated in
 // registers first (slots that share a group-major row are read once, their
-// gates summed in slot order), then each lane streams 8-element vectors of
-// every distinct row and accumulates in fp32.
+// gates summed in slot order), then either each lane streams 8-element
+// vectors of every distinct row and accumulates in fp32, or (k >= 4) the
+// rows are staged chunk by chunk in shared memory by the bulk-copy engine
+// and summed from there in the same order.
 #include <cstdlib>
 
 #include "common.cuh"

@@ -24,8 +24,10 @@
 //               slots, each token's group heads and the per-block group
 //               counts (its last CTA scanning them), one kernel ranks the
 //               heads per group and gives every kept slot its head's row.
-//   5. copy:    one token per warp, x[t] read once (16-byte vectors) and
-//               written to each distinct row the token owns.
+//   5. copy:    one token per warp, x[t] read once and written to each
+//               distinct row the token owns - through the bulk-copy engine
+//               (one bulk load into shared memory, one bulk store per row)
+//               when the row fits a 32 KB slot, else in 16-byte vectors.
 #include <cstdlib>
 #include <mutex>
 
