@@ -160,6 +160,35 @@ def reduce_over_ranks(elapsed_ms, launches, device):
     return float(t.item()), int(c.item())
 
 
+def job_histogram(name, hist, world, device):
+    """The job's histogram from the ranks' accumulated ones: one int32 SUM
+    all-reduce of the E x E counts (outside the timed steps).  Every rank ran
+    the same number of passes over T tokens, so the job total must be the
+    world size times this rank's; returns the record for the JSON line."""
+    import torch
+
+    from mixture_experts_routing_top_b200 import layer as Lyr
+
+    local_total = int(hist.sum().item())
+    job = hist.clone()
+    if device.type == "cuda":
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        Lyr.reduce_histogram(job)
+        b.record()
+        torch.cuda.synchronize()
+        us = 1e3 * a.elapsed_time(b)
+    else:
+        t0 = time.perf_counter()
+        Lyr.reduce_histogram(job)
+        us = 1e6 * (time.perf_counter() - t0)
+    E = int(hist.shape[0])
+    return job, {"name": name, "E": E, "bytes": E * E * 4, "ranks": world,
+                 "collective": "all_reduce sum int32" if world > 1 else "none (one rank)",
+                 "allreduce_us": round(us, 1) if world > 1 else 0.0,
+                 "total": int(job.sum().item()), "consistent": int(job.sum().item()) == world * local_total}
+
+
 def throughput(world, tokens_per_rank, steps, max_elapsed_ms):
     """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
     return world * tokens_per_rank * steps / (max_elapsed_ms / 1e3)
@@ -265,6 +294,9 @@ class TopKRunner:
     def _combine(self):
         y = self._y if self.w.F else self.L.perm["buffer"]
         self.L.combine(y, self._sh)
+
+    def histogram(self):
+        return "coselect", self.cosel
 
     def after_warmup(self):
         self.R = int(self.L.perm["offsets"][-1].item())
@@ -444,6 +476,9 @@ class ExpertChoiceRunner:
         M.route_topk(self.logits2, 1, False, self.top1[1], self.g1[1])
         M.transition(self.top1[0], self.top1[1], self.w.E, into=self.trans)
 
+    def histogram(self):
+        return "transition", self.trans
+
     def after_warmup(self):
         tp = self.L.routing[2]
         self.chosen = int((tp[1:] > tp[:-1]).sum().item())
@@ -551,6 +586,9 @@ class RoutingRunner:
         self.resident_bytes = self.inp.numel() * self.inp.element_size()
         self.stages = [("route", lambda: route(self.inp)),
                        ("coselect", lambda: M.coselect(self.idx, w.E, into=self.cosel))]
+
+    def histogram(self):
+        return "coselect", self.cosel
 
     def after_warmup(self):
         pass
@@ -701,6 +739,7 @@ def run_libmoe(args, w, rank, world, local_rank):
     if M.device_error() != 0:
         raise RuntimeError("device fault word set during the timed steps")
     elapsed_ms, launches = reduce_over_ranks(elapsed_ms, launches, device)
+    _, hist_rec = job_histogram(*run.histogram(), world, device)
 
     # end to end through the public API: pinned host inputs -> layer -> host output
     e2e = None
@@ -772,6 +811,7 @@ def run_libmoe(args, w, rank, world, local_rank):
         "config": cfg, "roofline": roof, "stages": report, "gpu_launches": launches, "clocks": clk,
     }
     res.update(run.extra())
+    res["job_histogram"] = hist_rec
     if e2e:
         res["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:

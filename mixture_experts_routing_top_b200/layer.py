@@ -240,3 +240,21 @@ class CapturedForward:
     def replay(self):
         self.graph.replay()
         return self.out
+
+
+def reduce_histogram(hist: torch.Tensor, group=None) -> torch.Tensor:
+    """Sums an accumulated routing histogram (co-selection or layer-to-layer
+    transition counts, int32 [E,E]) over the ranks of a token-sharded job,
+    in place, and returns it.
+
+    Both histograms of "Expert Coupling in MoE Pretraining" (Abstract) are
+    sums over tokens, so when each rank routes its own tokens the sum over
+    ranks is the histogram of the whole job: the one exchange a
+    token-sharded layer has, taken once when the statistic is read (placing
+    experts by their co-selection wants the job's counts, identical on every
+    rank).  With one process, or no process group, the tensor is unchanged."""
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(hist, op=dist.ReduceOp.SUM, group=group)
+    return hist
