@@ -301,14 +301,17 @@ moe_status moe_unpermute_groups(const void* y_g, int dtype, int R_g, int T, int 
  * Abstract: pairs of experts a token selects together), on the routing
  * decisions before capacity: cosel[a][b] += 1 for every ordered pair of
  * slots (i, j) of a token with a = expert_idx[t, i], b = expert_idx[t, j].
- * The diagonal is each expert's load.  cosel [E, E] int32, accumulated. */
+ * The diagonal is each expert's load.  cosel [E, E] int32, accumulated.
+ * An index outside [0, E) is skipped with every pair it is part of, and
+ * sets MOE_ERR_DEVICE_INDEX in the fault word.  E <= 1024, k <= 32. */
 moe_status moe_coselect(const int32_t* expert_idx, int T, int k, int E, int32_t* cosel,
                         moe_stream_t stream);
 
 /* Layer-to-layer expert transitions (same Abstract: a token's expert
  * choices in one layer are predictive of its choices in the next):
  * trans[a][b] += 1 for every a among idx1[t, :k1] and b among idx2[t, :k2].
- * trans [E, E] int32, accumulated. */
+ * trans [E, E] int32, accumulated.  Out-of-range indices as for
+ * moe_coselect.  E <= 1024, k1, k2 <= 32. */
 moe_status moe_transition(const int32_t* idx1, int k1, const int32_t* idx2, int k2, int T, int E,
                           int32_t* trans, moe_stream_t stream);
 

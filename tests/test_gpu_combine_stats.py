@@ -103,9 +103,17 @@ def test_gather_rows_matches_token_csr(bulk, d, monkeypatch):
 
 
 # -------------------------------------------------------------- histograms
+@pytest.fixture(params=["sym", "ordered"])
+def cosel_kind(request, monkeypatch):
+    """Co-selection through the kernel that counts each unordered slot pair
+    once and mirrors it (the default), and through the ordered-pair kernel."""
+    monkeypatch.setenv("LIBMOE_COSEL_SYM", "1" if request.param == "sym" else "0")
+    return request.param
+
+
 @pytest.mark.parametrize("T,E,k", [(1, 1, 1), (100, 8, 2), (16384, 64, 6), (5000, 1000, 3), (20000, 256, 8),
-                                   (3000, 7, 7)])
-def test_coselect(T, E, k):
+                                   (3000, 7, 7), (70000, 256, 8), (999, 130, 5), (4096, 1024, 8)])
+def test_coselect(T, E, k, cosel_kind):
     idx, _ = O.route_topk(synth.normal_f32(6, 1, (T, E)), k)
     got = M.coselect(to_dev(idx), E)
     ref = O.coselect(idx, E)
@@ -114,7 +122,29 @@ def test_coselect(T, E, k):
     assert np.array_equal(to_np(got), 2 * ref)
 
 
-def test_coselect_workloads():
+def test_coselect_duplicates_and_bad_indices(cosel_kind):
+    """Rows that repeat an expert (every ordered slot pair still counts, so a
+    repeated expert adds 2 to its diagonal per extra pair) and entries out of
+    range (pairs that touch one are skipped and the fault word is set)."""
+    rng = np.random.default_rng(11)
+    for T, E, k in ((3000, 6, 4), (2000, 40, 7), (500, 256, 8), (1000, 3, 1)):
+        idx = rng.integers(0, E, size=(T, k)).astype(np.int32)
+        assert np.array_equal(to_np(M.coselect(to_dev(idx), E)), O.coselect(idx, E))
+        assert M.device_error() == 0
+        bad = idx.copy()
+        bad[::17, 0] = E
+        bad[5::23, -1] = -1
+        got = to_np(M.coselect(to_dev(bad), E))
+        assert M.device_error() == 8
+        ok = (bad >= 0) & (bad < E)
+        ref = np.zeros((E, E), np.int64)
+        for t in range(T):
+            v = bad[t][ok[t]]
+            np.add.at(ref, (v[:, None], v[None, :]), 1)      # every ordered pair of valid slots
+        assert np.array_equal(got, ref)
+
+
+def test_coselect_workloads(cosel_kind):
     for w in (W.FINE, W.SWEEP):
         idx, _ = O.route_topk(W.make_logits(w), w.k, w.norm_topk)
         assert np.array_equal(to_np(M.coselect(to_dev(idx), w.E)), O.coselect(idx, w.E))
