@@ -183,10 +183,11 @@ def job_histogram(name, hist, world, device):
         Lyr.reduce_histogram(job)
         us = 1e6 * (time.perf_counter() - t0)
     E = int(hist.shape[0])
+    total = int(job.sum().item())
     return job, {"name": name, "E": E, "bytes": E * E * 4, "ranks": world,
                  "collective": "all_reduce sum int32" if world > 1 else "none (one rank)",
                  "allreduce_us": round(us, 1) if world > 1 else 0.0,
-                 "total": int(job.sum().item()), "consistent": int(job.sum().item()) == world * local_total}
+                 "total": total, "consistent": total == world * local_total}
 
 
 def throughput(world, tokens_per_rank, steps, max_elapsed_ms):
