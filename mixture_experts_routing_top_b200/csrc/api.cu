@@ -1,6 +1,8 @@
 // api.cu - status strings, ABI version and the per-device fault word.
 #include <atomic>
+#include <map>
 #include <mutex>
+#include <utility>
 
 #include "common.cuh"
 
@@ -28,6 +30,23 @@ unsigned* device_error_word() {
         g_err_addr[dev] = static_cast<unsigned*>(p);
     }
     return g_err_addr[dev];
+}
+
+// The dynamic shared-memory limit is an attribute of the kernel's instance
+// on one device, so it is raised once per (kernel, device) and remembered.
+bool set_smem_limit(const void* fn, size_t bytes) {
+    if (bytes <= 48 * 1024) return true;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    static std::mutex mu;
+    static std::map<std::pair<const void*, int>, size_t> raised;
+    std::lock_guard<std::mutex> lk(mu);
+    const auto key = std::make_pair(fn, dev);
+    const auto it = raised.find(key);
+    if (it != raised.end() && it->second >= bytes) return true;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) return false;
+    raised[key] = bytes;
+    return true;
 }
 
 }  // namespace moe

@@ -614,14 +614,9 @@ template <bool UNIT, bool CSR>
 moe_status launch_unpermute_bulk(bool in_bf16, bool out_bf16, cudaStream_t s, const void* y, int R, int T, int d,
                                  int k, const int32_t* row_map, const float* gate, const void* shared, void* out,
                                  unsigned* err, CsrRows csr = CsrRows{nullptr, nullptr, nullptr}) {
-    static bool attr_done = false;
-    if (!attr_done) {
-        for (auto fn : {unpermute_bulk_kernel<true, true, UNIT, CSR>, unpermute_bulk_kernel<true, false, UNIT, CSR>,
-                        unpermute_bulk_kernel<false, true, UNIT, CSR>, unpermute_bulk_kernel<false, false, UNIT, CSR>})
-            if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kCmbSmem) != cudaSuccess)
-                return MOE_ERR_CUDA;
-        attr_done = true;
-    }
+    for (auto fn : {unpermute_bulk_kernel<true, true, UNIT, CSR>, unpermute_bulk_kernel<true, false, UNIT, CSR>,
+                    unpermute_bulk_kernel<false, true, UNIT, CSR>, unpermute_bulk_kernel<false, false, UNIT, CSR>})
+        if (!set_smem_limit((const void*)fn, kCmbSmem)) return MOE_ERR_CUDA;
     long long nb = ((long long)T + kCmbWarps - 1) / kCmbWarps;
     const int blocks = (int)(nb < 148 * 8 ? nb : 148 * 8);
     const uint8_t* yb = (const uint8_t*)y;

@@ -19,6 +19,10 @@ unsigned* device_error_word();
 // Counts kernel launches made by the library (moe_kernel_launches).
 void count_launch();
 
+// Lets kernel fn take `bytes` of dynamic shared memory on the current device
+// (no-op up to 48 KB).  False if the runtime refused.
+bool set_smem_limit(const void* fn, size_t bytes);
+
 __device__ __forceinline__ void raise_error(unsigned* err, unsigned bits) {
     if (err) atomicOr(err, bits);
 }

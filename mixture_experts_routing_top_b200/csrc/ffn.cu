@@ -641,13 +641,7 @@ namespace {
 template <int MODE>
 moe_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, const tc::GemmArgs& a,
                        cudaStream_t s) {
-    static bool attr_done = false;
-    if (!attr_done) {
-        if (cudaFuncSetAttribute(tc::grouped_gemm_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tc::SMEM_BYTES) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        attr_done = true;
-    }
+    if (!set_smem_limit((const void*)tc::grouped_gemm_kernel<MODE>, tc::SMEM_BYTES)) return MOE_ERR_CUDA;
     const int bn_out = MODE == tc::MODE_SWIGLU ? 128 : 256;
     const long long n_tiles = (a.N_out + bn_out - 1) / bn_out;
     const long long m_tiles_max = (a.R_max + tc::BM - 1) / tc::BM + a.E;
@@ -662,13 +656,7 @@ moe_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUte
 template <int MODE>
 moe_status launch_gemm2(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, const tc::GemmArgs& a,
                         cudaStream_t s) {
-    static bool attr_done = false;
-    if (!attr_done) {
-        if (cudaFuncSetAttribute(tc2::grouped_gemm2_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 tc2::SMEM_BYTES) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        attr_done = true;
-    }
+    if (!set_smem_limit((const void*)tc2::grouped_gemm2_kernel<MODE>, tc2::SMEM_BYTES)) return MOE_ERR_CUDA;
     const int bn_out = MODE == tc::MODE_SWIGLU ? 128 : 256;
     const long long n_tiles = (a.N_out + bn_out - 1) / bn_out;
     const long long m_tiles_max = (a.R_max + tc2::BM - 1) / tc2::BM + a.E;

@@ -638,11 +638,6 @@ bool bulk_copy_enabled() {
     return true;
 }
 
-bool set_smem(const void* fn, size_t bytes) {
-    if (bytes <= 48 * 1024) return true;
-    return cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) == cudaSuccess;
-}
-
 moe_status launch_copy_slots(const void* x, int T, int row_bytes, const int32_t* row_map, int k, void* buffer,
                              cudaStream_t s) {
     const int vpr = row_bytes / 16;
@@ -652,7 +647,7 @@ moe_status launch_copy_slots(const void* x, int T, int row_bytes, const int32_t*
         unsigned* err = device_error_word();
         if (!err) return MOE_ERR_CUDA;
         const size_t smem = (size_t)kBulkWarps * slot_bytes;
-        if (!set_smem((const void*)copy_rows_bulk_kernel, smem)) return MOE_ERR_CUDA;
+        if (!set_smem_limit((const void*)copy_rows_bulk_kernel, smem)) return MOE_ERR_CUDA;
         long long nb = ((long long)T + kBulkWarps - 1) / kBulkWarps;
         const int blocks = (int)(nb < 148 * 16 ? nb : 148 * 16);
         copy_rows_bulk_kernel<<<blocks, 32 * kBulkWarps, smem, s>>>((const uint8_t*)x, T, row_bytes, slot_bytes, row_map,
@@ -738,7 +733,7 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
     if (!group_of_expert) {
         // 4. ranks and rows (its block 0 writes counts, offsets and dropped when fused)
         const size_t rank_smem = sizeof(int) * ((size_t)nw * E + 2 * (size_t)E);
-        if (!set_smem((const void*)perm_rank_kernel, rank_smem)) return MOE_ERR_CUDA;
+        if (!set_smem_limit((const void*)perm_rank_kernel, rank_smem)) return MOE_ERR_CUDA;
         perm_rank_kernel<<<nblk, kIdxThreads, rank_smem, s>>>(expert_idx, T, k, E, nblk, fused_e, cnt, base, cap,
                                                               counts, offsets, dropped, row_map, row_token, err);
         MOE_LAUNCH_CHECK();
@@ -748,7 +743,7 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
         int32_t* gbase = (int32_t*)(ws + L.gbase);
         int32_t* gtotal = (int32_t*)(ws + L.gtotal);
         const size_t heads_smem = sizeof(int) * ((size_t)nw * E + 2 * (size_t)E + G) + (size_t)kTB * k;
-        if (!set_smem((const void*)perm_group_heads_kernel, heads_smem)) return MOE_ERR_CUDA;
+        if (!set_smem_limit((const void*)perm_group_heads_kernel, heads_smem)) return MOE_ERR_CUDA;
         perm_group_heads_kernel<<<nblk, kIdxThreads, heads_smem, s>>>(expert_idx, group_of_expert, T, k, E, G, nblk,
                                                                         fused_e, cnt, base, cap, counts, dropped, code,
                                                                         gcnt, err);
@@ -761,7 +756,7 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
             MOE_LAUNCH_CHECK();
         }
         const size_t rows_smem = sizeof(int) * ((size_t)nw * G + 2 * (size_t)G + (size_t)kTB * k);
-        if (!set_smem((const void*)perm_group_rows_kernel, rows_smem)) return MOE_ERR_CUDA;
+        if (!set_smem_limit((const void*)perm_group_rows_kernel, rows_smem)) return MOE_ERR_CUDA;
         perm_group_rows_kernel<<<nblk, kIdxThreads, rows_smem, s>>>(code, T, k, G, nblk, fused_g, gcnt, gbase, offsets,
                                                                       offsets, row_map, row_token);
         MOE_LAUNCH_CHECK();
@@ -786,7 +781,7 @@ extern "C" moe_status moe_gather_rows(const void* x, int dtype, int T, int d, co
     const int slot_bytes = (int)((row_bytes + 127) / 128 * 128);
     if (bulk_copy_enabled() && slot_bytes <= 32 * 1024) {
         const size_t smem = (size_t)kBulkWarps * slot_bytes;
-        if (!set_smem((const void*)copy_rows_csr_bulk_kernel, smem)) return MOE_ERR_CUDA;
+        if (!set_smem_limit((const void*)copy_rows_csr_bulk_kernel, smem)) return MOE_ERR_CUDA;
         long long nb = ((long long)T + kBulkWarps - 1) / kBulkWarps;
         const int blocks = (int)(nb < 148 * 16 ? nb : 148 * 16);
         copy_rows_csr_bulk_kernel<<<blocks, 32 * kBulkWarps, smem, s>>>((const uint8_t*)x, T, (int)row_bytes, slot_bytes,

@@ -866,14 +866,9 @@ extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, i
     if (blocks > 148 * 16) blocks = 148 * 16;
     const int nv = (E + 31) / 32;
     if (E % 4 == 0 && k <= 8 && ((uintptr_t)logits & 15) == 0 && use_rows_variant(T, k)) {
-        static bool attr_done = false;
-        if (!attr_done) {
-            for (auto fn : {route_topk_rows_kernel<1>, route_topk_rows_kernel<2>, route_topk_rows_kernel<4>,
-                            route_topk_rows_kernel<8>})
-                if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kRowSmem) != cudaSuccess)
-                    return MOE_ERR_CUDA;
-            attr_done = true;
-        }
+        for (auto fn : {route_topk_rows_kernel<1>, route_topk_rows_kernel<2>, route_topk_rows_kernel<4>,
+                        route_topk_rows_kernel<8>})
+            if (!set_smem_limit((const void*)fn, kRowSmem)) return MOE_ERR_CUDA;
         const long long warps = ((long long)T + 31) / 32;
         long long rb = (warps + kRowWarps - 1) / kRowWarps;
         const int rblocks = (int)(rb < 148 * 8 ? rb : 148 * 8);
@@ -962,18 +957,13 @@ extern "C" moe_status moe_route_ec(const float* logits, int T, int E, int C, int
     {
         const int tpb = ec_tokens_per_block(E);
         const size_t smem = (size_t)tpb * ((E + 2) * sizeof(double) + (E + 1) * sizeof(float));
-        if (smem > 48 * 1024 &&
-            cudaFuncSetAttribute(ec_lse_keys_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-            return MOE_ERR_CUDA;
+        if (!set_smem_limit((const void*)ec_lse_keys_kernel, smem)) return MOE_ERR_CUDA;
         ec_lse_keys_kernel<<<ceil_div(T, tpb), kEcThreads, smem, s>>>(logits, T, E, tpb, lse, keys);
         MOE_LAUNCH_CHECK();
     }
     if (T <= kEcSmemTokens) {
         const size_t smem = sizeof(unsigned) * (size_t)T;
-        if (smem > 48 * 1024 &&
-            cudaFuncSetAttribute(ec_select_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
-                cudaSuccess)
-            return MOE_ERR_CUDA;
+        if (!set_smem_limit((const void*)ec_select_smem_kernel, smem)) return MOE_ERR_CUDA;
         ec_select_smem_kernel<<<E, 1024, smem, s>>>(keys, logits, lse, T, E, C, ec_token, ec_gate, mask, mw);
     } else {
         ec_select_kernel<<<E, 1024, 0, s>>>(keys, logits, lse, T, E, C, ec_token, ec_gate, mask, mw);

@@ -244,13 +244,7 @@ __global__ void __launch_bounds__(256) router_logits_f32_kernel(const float* __r
 
 template <int KM>
 moe_status launch_router(const CUtensorMap& mx, const CUtensorMap& mw, const RouterArgs& a, cudaStream_t s) {
-    static bool attr_done = false;
-    if (!attr_done) {
-        if (cudaFuncSetAttribute(router_topk_kernel<KM>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES) !=
-            cudaSuccess)
-            return MOE_ERR_CUDA;
-        attr_done = true;
-    }
+    if (!set_smem_limit((const void*)router_topk_kernel<KM>, SMEM_BYTES)) return MOE_ERR_CUDA;
     const int tiles = (a.T + BM - 1) / BM;
     int grid = sm_count();
     if (tiles < grid) grid = tiles;
@@ -484,13 +478,7 @@ __global__ void __launch_bounds__(THREADS, 1) router_topk_pair_kernel(const __gr
 
 template <int KM>
 moe_status launch_router_pair(const CUtensorMap& mx, const CUtensorMap& mw, const RouterArgs& a, cudaStream_t s) {
-    static bool attr_done = false;
-    if (!attr_done) {
-        if (cudaFuncSetAttribute(router_topk_pair_kernel<KM>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 SMEM_BYTES) != cudaSuccess)
-            return MOE_ERR_CUDA;
-        attr_done = true;
-    }
+    if (!set_smem_limit((const void*)router_topk_pair_kernel<KM>, SMEM_BYTES)) return MOE_ERR_CUDA;
     const int tiles = (a.T + BM - 1) / BM;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * tiles, 1, 1);

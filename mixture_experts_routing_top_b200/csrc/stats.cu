@@ -177,9 +177,7 @@ moe_status launch_cosel_sym(const int32_t* idx, int k, int T, int E, int32_t* hi
     int tokens_per_cta = ceil_div(T, tok_ctas);
     if (tokens_per_cta < 256) tokens_per_cta = 256;
     tok_ctas = ceil_div(T, tokens_per_cta);
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(cosel_sym_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return MOE_ERR_CUDA;
+    if (!set_smem_limit((const void*)cosel_sym_kernel, smem)) return MOE_ERR_CUDA;
     cosel_sym_kernel<<<dim3(tok_ctas, nb), 512, smem, s>>>(idx, k, T, E, sb, tokens_per_cta, hist, err);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
@@ -199,9 +197,7 @@ moe_status launch_pair_hist(const int32_t* idx1, int k1, const int32_t* idx2, in
     int tokens_per_cta = ceil_div(T, tok_ctas);
     if (tokens_per_cta < 256) tokens_per_cta = 256;
     tok_ctas = ceil_div(T, tokens_per_cta);
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(pair_hist_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-        return MOE_ERR_CUDA;
+    if (!set_smem_limit((const void*)pair_hist_kernel, smem)) return MOE_ERR_CUDA;
     pair_hist_kernel<<<dim3(tok_ctas, nbands), 512, smem, s>>>(idx1, k1, idx2, k2, T, E, band, tokens_per_cta, hist, err);
     MOE_LAUNCH_CHECK();
     return MOE_OK;

@@ -9,6 +9,7 @@
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -235,15 +236,17 @@ inline bool make_bf16_map(CUtensorMap* m, const void* base, long long rows, int 
     return make_tile_map(m, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rows, K, 64, box_rows);
 }
 
+// SM count of the current device (read once per device).
 inline int sm_count() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0;
-        cudaGetDevice(&dev);
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        if (n <= 0) n = 148;
+    static std::atomic<int> n[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    int v = n[dev].load(std::memory_order_relaxed);
+    if (v <= 0) {
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0) v = 148;
+        n[dev].store(v, std::memory_order_relaxed);
     }
-    return n;
+    return v;
 }
 
 }  // namespace tc
