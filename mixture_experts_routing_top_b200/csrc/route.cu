@@ -354,10 +354,15 @@ __global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __
     const int rows = (int)min((long long)tpb, (long long)T - t0);
     const float* src = logits + t0 * E;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    // row max (exact in any order): one warp per row
+    // logits into shared memory (read from global once) and each row's max
+    // (exact in any order): one warp per row
     for (int r = wid; r < rows; r += nw) {
         float m = -INFINITY;
-        for (int c = lane; c < E; c += 32) m = fmaxf(m, __ldg(src + (long long)r * E + c));
+        for (int c = lane; c < E; c += 32) {
+            const float l = __ldg(src + (long long)r * E + c);
+            lg[r * ld + c] = l;
+            m = fmaxf(m, l);
+        }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0) rowv[r] = (double)m;
@@ -368,9 +373,7 @@ __global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __
 #pragma unroll 4
     for (int f = threadIdx.x; f < n; f += blockDim.x) {
         const int r = f / E, c = f - r * E;
-        const float l = __ldg(src + f);
-        lg[r * ld + c] = l;
-        ex[r * ld + c] = exp((double)l - rowv[r]);
+        ex[r * ld + c] = exp((double)lg[r * ld + c] - rowv[r]);
     }
     __syncthreads();
     // ascending-expert sums, one thread per token
