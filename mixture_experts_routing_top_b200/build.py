@@ -4,11 +4,16 @@ Each ``csrc/*.cu`` compiles to an object in ``_build/`` (in parallel, only
 when its source or a header changed), then nvcc links them into
 ``libmoe.so`` in ``lib/``.  The CUDA runtime is linked statically; the
 driver entry point for tensor-map encoding is looked up at run time, so the
-library needs no libcuda at link time.
+library needs no libcuda at link time.  Several processes may call build()
+at once (one per rank under torchrun): a file lock in ``_build/`` lets one
+of them compile while the others wait and then find everything up to date,
+and objects and the library are written under temporary names and renamed
+into place.
 """
 from __future__ import annotations
 
 import concurrent.futures as cf
+import fcntl
 import glob
 import os
 import subprocess
@@ -38,10 +43,12 @@ def _compile(src: str, verbose_ptxas: bool) -> str:
     newest_dep = max([os.path.getmtime(src)] + [os.path.getmtime(h) for h in _headers()])
     if os.path.exists(obj) and os.path.getmtime(obj) >= newest_dep and not verbose_ptxas:
         return obj
-    cmd = [NVCC] + ARCH + FLAGS + (["-Xptxas", "-v"] if verbose_ptxas else []) + ["-c", src, "-o", obj]
+    tmp = obj + ".tmp%d" % os.getpid()
+    cmd = [NVCC] + ARCH + FLAGS + (["-Xptxas", "-v"] if verbose_ptxas else []) + ["-c", src, "-o", tmp]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed for %s:\n%s\n%s" % (src, r.stdout, r.stderr))
+    os.replace(tmp, obj)
     if verbose_ptxas:
         sys.stderr.write(r.stderr)
     return obj
@@ -50,6 +57,12 @@ def _compile(src: str, verbose_ptxas: bool) -> str:
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     os.makedirs(BUILD, exist_ok=True)
     os.makedirs(os.path.dirname(SO), exist_ok=True)
+    with open(os.path.join(BUILD, ".lock"), "w") as lock:
+        fcntl.flock(lock, fcntl.LOCK_EX)
+        return _build_locked(force, verbose_ptxas)
+
+
+def _build_locked(force: bool, verbose_ptxas: bool) -> str:
     if force:
         for o in glob.glob(os.path.join(BUILD, "*.o")):
             os.remove(o)
