@@ -51,30 +51,40 @@ enum { MODE_SWIGLU = 0, MODE_GELU = 1, MODE_PLAIN = 2 };
 
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + expf(-z)); }
-// erf by Abramowitz & Stegun, Handbook of Mathematical Functions, 7.1.28
-// (Hastings): erf(x) = 1 - (1 + a1 x + ... + a6 x^6)^-16 for x >= 0, with
-// |error| <= 3e-7, odd in x.  Branch-free (six FMAs, four squarings, one
-// hardware reciprocal); evaluated in fp32 the error stays below 2e-6, far
-// under the bf16 rounding of the hidden activations.  The GELU epilogue of a
-// short-K GEMM is bound by instruction issue, where this form is cheaper
-// than the library erf with its range split.
-__device__ __forceinline__ float erf_as(float x) {
-    const float ax = fabsf(x);
-    float p = fmaf(ax, 4.30638e-5f, 2.765672e-4f);
-    p = fmaf(ax, p, 1.520143e-4f);
-    p = fmaf(ax, p, 9.2705272e-3f);
-    p = fmaf(ax, p, 4.22820123e-2f);
-    p = fmaf(ax, p, 7.05230784e-2f);
-    p = fmaf(ax, p, 1.0f);
-    p *= p;
-    p *= p;
-    p *= p;
-    p *= p;
-    float r;
-    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(p));
-    return copysignf(1.0f - r, x);
+// GELU with erf by Abramowitz & Stegun, Handbook of Mathematical Functions,
+// 7.1.28 (Hastings): erf(x) = 1 - (1 + a1 x + ... + a6 x^6)^-16 for x >= 0,
+// |error| <= 3e-7, odd in x.  With x = |z| / sqrt(2), the exact-erf GELU
+// 0.5 z (1 + erf(z / sqrt(2))) equals max(z, 0) - 0.5 |z| q(|z|)^-16 for
+// either sign of z, where q(y) = 1 + b1 y + ... + b6 y^6, b_i = a_i / sqrt(2)^i.
+// Branch-free: six FMAs, four squarings, one hardware reciprocal, one
+// multiply, a max and a final FMA (rounded once); evaluated in fp32 the error
+// of the erf part stays below 2e-6, far under the bf16 rounding of the hidden
+// activations.  The GELU epilogue of a short-K GEMM is bound by instruction
+// issue, where this form is cheaper than the library erf with its range split.
+constexpr double kRsqrt2 = 0.70710678118654752440;
+constexpr float kGb1 = (float)(7.05230784e-2 * kRsqrt2);
+constexpr float kGb2 = (float)(4.22820123e-2 * kRsqrt2 * kRsqrt2);
+constexpr float kGb3 = (float)(9.2705272e-3 * kRsqrt2 * kRsqrt2 * kRsqrt2);
+constexpr float kGb4 = (float)(1.520143e-4 * kRsqrt2 * kRsqrt2 * kRsqrt2 * kRsqrt2);
+constexpr float kGb5 = (float)(2.765672e-4 * kRsqrt2 * kRsqrt2 * kRsqrt2 * kRsqrt2 * kRsqrt2);
+constexpr float kGb6 = (float)(4.30638e-5 * kRsqrt2 * kRsqrt2 * kRsqrt2 * kRsqrt2 * kRsqrt2 * kRsqrt2);
+
+__device__ __forceinline__ float gelu_f(float z) {
+    const float y = fabsf(z);
+    float q = fmaf(y, kGb6, kGb5);
+    q = fmaf(y, q, kGb4);
+    q = fmaf(y, q, kGb3);
+    q = fmaf(y, q, kGb2);
+    q = fmaf(y, q, kGb1);
+    q = fmaf(y, q, 1.0f);
+    q *= q;
+    q *= q;
+    q *= q;
+    q *= q;
+    float r;                                      // q^-16 = 1 - erf(|z| / sqrt(2))
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(q));
+    return fmaf(-0.5f * y, r, fmaxf(z, 0.0f));
 }
-__device__ __forceinline__ float gelu_f(float z) { return 0.5f * z * (1.0f + erf_as(z * 0.70710678118654752f)); }
 
 // Store 32 consecutive bf16 values (64 bytes) of one output row.
 __device__ __forceinline__ void store_row32(uint16_t* dst, const float* v) {
