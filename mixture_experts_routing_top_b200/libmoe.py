@@ -106,6 +106,32 @@ def _dev(t: torch.Tensor, dtype=None, name="tensor"):
     return t
 
 
+def _buf(t: torch.Tensor, dtype, min_numel: int, name: str, device=None) -> torch.Tensor:
+    """A caller's buffer checked against what the library reads or writes
+    through its pointer: a contiguous CUDA tensor of `dtype` (None: any) with
+    at least `min_numel` elements, on `device` when given."""
+    _dev(t, dtype, name)
+    if device is not None and t.device != device:
+        raise ValueError("%s is on %s, the call's inputs on %s" % (name, t.device, device))
+    if t.numel() < min_numel:
+        raise ValueError("%s has %d elements, the call needs %d" % (name, t.numel(), min_numel))
+    return t
+
+
+def _out(t: Optional[torch.Tensor], shape, dtype, device, name: str) -> torch.Tensor:
+    """The caller's output buffer (checked as in _buf) or a new one."""
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=device)
+    n = 1
+    for v in shape:
+        n *= int(v)
+    return _buf(t, dtype, n, name, device)
+
+
+def _ws_bytes(t: torch.Tensor) -> int:
+    return t.numel() * t.element_size()
+
+
 def _act_dtype(t: torch.Tensor) -> int:
     if t.dtype == torch.float32:
         return MOE_F32
@@ -123,10 +149,8 @@ def _ws(nbytes: int, device) -> torch.Tensor:
 def route_topk(logits: torch.Tensor, k: int, norm_topk: bool = False, expert_idx=None, gate=None, stream=None):
     _dev(logits, torch.float32, "logits")
     T, E = logits.shape
-    if expert_idx is None:
-        expert_idx = torch.empty((T, k), dtype=torch.int32, device=logits.device)
-    if gate is None:
-        gate = torch.empty((T, k), dtype=torch.float32, device=logits.device)
+    expert_idx = _out(expert_idx, (T, k), torch.int32, logits.device, "expert_idx")
+    gate = _out(gate, (T, k), torch.float32, logits.device, "gate")
     _check("moe_route_topk", lib().moe_route_topk(_p(logits), T, E, k, int(bool(norm_topk)), _p(expert_idx),
                                                   _p(gate), _stream(stream)))
     return expert_idx, gate
@@ -143,12 +167,11 @@ def router_topk(x: torch.Tensor, W_r: torch.Tensor, k: int, norm_topk: bool = Fa
     if W_r.shape[1] != d:
         raise ValueError("W_r must be [E, d]")
     dev = x.device
-    if expert_idx is None:
-        expert_idx = torch.empty((T, k), dtype=torch.int32, device=dev)
-    if gate is None:
-        gate = torch.empty((T, k), dtype=torch.float32, device=dev)
-    if logits is None and (want_logits or x.dtype == torch.float32):
-        logits = torch.empty((T, E), dtype=torch.float32, device=dev)
+    _buf(W_r, x.dtype, E * d, "W_r", dev)
+    expert_idx = _out(expert_idx, (T, k), torch.int32, dev, "expert_idx")
+    gate = _out(gate, (T, k), torch.float32, dev, "gate")
+    if logits is not None or want_logits or x.dtype == torch.float32:
+        logits = _out(logits, (T, E), torch.float32, dev, "logits")
     _check("moe_router_topk", lib().moe_router_topk(
         _p(x), _act_dtype(x), T, d, _p(W_r), E, k, int(bool(norm_topk)), _p(logits), _p(expert_idx), _p(gate),
         _stream(stream)))
@@ -164,15 +187,15 @@ def route_ec(logits: torch.Tensor, C: int, workspace=None, out=None, stream=None
     _dev(logits, torch.float32, "logits")
     T, E = logits.shape
     dev = logits.device
-    if out is None:
-        out = (torch.empty((E, C), dtype=torch.int32, device=dev), torch.empty((E, C), dtype=torch.float32, device=dev),
-               torch.empty(T + 1, dtype=torch.int32, device=dev), torch.empty(E * C, dtype=torch.int32, device=dev))
-    ec_token, ec_gate, tok_ptr, tok_row = out
+    ec_token, ec_gate, tok_ptr, tok_row = out if out is not None else (None, None, None, None)
+    ec_token = _out(ec_token, (E, C), torch.int32, dev, "ec_token")
+    ec_gate = _out(ec_gate, (E, C), torch.float32, dev, "ec_gate")
+    tok_ptr = _out(tok_ptr, (T + 1,), torch.int32, dev, "tok_ptr")
+    tok_row = _out(tok_row, (E * C,), torch.int32, dev, "tok_row")
     nbytes = route_ec_workspace_bytes(T, E, C)
-    if workspace is None:
-        workspace = _ws(nbytes, dev)
+    workspace = _ws(nbytes, dev) if workspace is None else _buf(workspace, None, 0, "workspace", dev)
     _check("moe_route_ec", lib().moe_route_ec(_p(logits), T, E, C, _p(ec_token), _p(ec_gate), _p(tok_ptr),
-                                              _p(tok_row), _p(workspace), workspace.numel(), _stream(stream)))
+                                              _p(tok_row), _p(workspace), _ws_bytes(workspace), _stream(stream)))
     return ec_token, ec_gate, tok_ptr, tok_row
 
 
@@ -197,7 +220,7 @@ def permute(x: Optional[torch.Tensor], expert_idx: torch.Tensor, E: int, capacit
     T, k = expert_idx.shape
     dev = expert_idx.device
     if group_of_expert is not None:
-        _dev(group_of_expert, torch.int32, "group_of_expert")
+        _buf(group_of_expert, torch.int32, E, "group_of_expert", dev)
         if G <= 0:
             raise ValueError("G must be given with group_of_expert")
     else:
@@ -206,23 +229,30 @@ def permute(x: Optional[torch.Tensor], expert_idx: torch.Tensor, E: int, capacit
     dtype = MOE_F32
     d = 0
     if x is not None:
-        _dev(x, None, "x")
+        _buf(x, None, 0, "x", dev)
+        if x.dim() != 2 or x.shape[0] < T:
+            raise ValueError("x must be [T, d] with T = %d rows" % T)
         dtype = _act_dtype(x)
         d = x.shape[1]
     if out is None:
-        out = dict(
-            buffer=None if x is None else torch.empty((max(R_max, 1), d), dtype=x.dtype, device=dev),
-            row_map=torch.empty((T, k), dtype=torch.int32, device=dev),
-            row_token=torch.empty(max(R_max, 1), dtype=torch.int32, device=dev),
-            counts=torch.empty(E, dtype=torch.int32, device=dev),
-            offsets=torch.empty((G if G else E) + 1, dtype=torch.int32, device=dev),
-            dropped=torch.empty(1, dtype=torch.int32, device=dev))
-    if workspace is None:
-        workspace = _ws(permute_workspace_bytes(T, k, E, G), dev)
+        out = {}
+    if x is not None:
+        out["buffer"] = _out(out.get("buffer"), (max(R_max, 1), d), x.dtype, dev, "buffer")
+        if out["buffer"].shape[-1] != d:
+            raise ValueError("buffer rows must hold d = %d elements" % d)
+    else:
+        out.setdefault("buffer", None)
+    out["row_map"] = _out(out.get("row_map"), (T, k), torch.int32, dev, "row_map")
+    out["row_token"] = _out(out.get("row_token"), (max(R_max, 1),), torch.int32, dev, "row_token")
+    out["counts"] = _out(out.get("counts"), (E,), torch.int32, dev, "counts")
+    out["offsets"] = _out(out.get("offsets"), ((G if G else E) + 1,), torch.int32, dev, "offsets")
+    out["dropped"] = _out(out.get("dropped"), (1,), torch.int32, dev, "dropped")
+    workspace = (_ws(permute_workspace_bytes(T, k, E, G), dev) if workspace is None
+                 else _buf(workspace, None, 0, "workspace", dev))
     _check("moe_permute", lib().moe_permute(
         _p(x), dtype, T, d, _p(expert_idx), k, E, float(capacity_factor), _p(group_of_expert), G,
-        _p(out["buffer"]), _p(out["row_map"]), _p(out["row_token"]), _p(out["counts"]), _p(out["offsets"]),
-        _p(out["dropped"]), _p(workspace), workspace.numel(), _stream(stream)))
+        _p(out["buffer"] if x is not None else None), _p(out["row_map"]), _p(out["row_token"]), _p(out["counts"]),
+        _p(out["offsets"]), _p(out["dropped"]), _p(workspace), _ws_bytes(workspace), _stream(stream)))
     out["R_max"] = R_max
     return out
 
@@ -230,8 +260,10 @@ def permute(x: Optional[torch.Tensor], expert_idx: torch.Tensor, E: int, capacit
 def gather_rows(x: torch.Tensor, tok_ptr: torch.Tensor, tok_row: torch.Tensor, R: int, buffer=None, stream=None):
     _dev(x, None, "x")
     T, d = x.shape
-    if buffer is None:
-        buffer = torch.empty((R, d), dtype=x.dtype, device=x.device)
+    dev = x.device
+    _buf(tok_ptr, torch.int32, T + 1, "tok_ptr", dev)
+    _buf(tok_row, torch.int32, 0, "tok_row", dev)
+    buffer = _out(buffer, (R, d), x.dtype, dev, "buffer")
     _check("moe_gather_rows", lib().moe_gather_rows(_p(x), _act_dtype(x), T, d, _p(tok_ptr), _p(tok_row), R,
                                                     _p(buffer), _stream(stream)))
     return buffer
@@ -245,22 +277,26 @@ def expert_ffn_workspace_bytes(R_max: int, d: int, F: int, dtype: torch.dtype) -
 def expert_ffn(buffer: torch.Tensor, offsets: torch.Tensor, W1: torch.Tensor, W3: Optional[torch.Tensor],
                W2: torch.Tensor, act: str = "swiglu", y=None, workspace=None, stream=None):
     _dev(buffer, None, "buffer")
-    _dev(offsets, torch.int32, "offsets")
+    dev = buffer.device
     dtype = _act_dtype(buffer)
     R_max, d = buffer.shape
     E, F, d1 = W1.shape
-    if d1 != d or tuple(W2.shape) != (E, d, F):
-        raise ValueError("weight shapes: W1 [E,F,d], W2 [E,d,F]")
+    _buf(offsets, torch.int32, E + 1, "offsets", dev)
+    if d1 != d or tuple(W2.shape) != (E, d, F) or (W3 is not None and tuple(W3.shape) != (E, F, d)):
+        raise ValueError("weight shapes: W1 and W3 [E,F,d], W2 [E,d,F]")
     for name, w in (("W1", W1), ("W2", W2)) + ((("W3", W3),) if W3 is not None else ()):
-        _dev(w, buffer.dtype, name)
+        _buf(w, buffer.dtype, 0, name, dev)
+    if act not in ("swiglu", "gelu"):
+        raise ValueError("act must be 'swiglu' or 'gelu'")
     a = MOE_ACT_SWIGLU if act == "swiglu" else MOE_ACT_GELU
-    if y is None:
-        y = torch.empty_like(buffer)
-    if workspace is None:
-        workspace = _ws(expert_ffn_workspace_bytes(R_max, d, F, buffer.dtype), buffer.device)
+    y = _out(y, (R_max, d), buffer.dtype, dev, "y")
+    if y.shape[-1] != d:
+        raise ValueError("y rows must hold d = %d elements" % d)
+    workspace = (_ws(expert_ffn_workspace_bytes(R_max, d, F, buffer.dtype), dev) if workspace is None
+                 else _buf(workspace, None, 0, "workspace", dev))
     _check("moe_expert_ffn", lib().moe_expert_ffn(
         _p(buffer), dtype, R_max, d, F, E, _p(offsets), _p(W1), _p(W3), _p(W2), a, _p(y), _p(workspace),
-        workspace.numel(), _stream(stream)))
+        _ws_bytes(workspace), _stream(stream)))
     return y
 
 
@@ -268,15 +304,16 @@ def expert_ffn(buffer: torch.Tensor, offsets: torch.Tensor, W1: torch.Tensor, W3
 def unpermute(y: torch.Tensor, row_map: torch.Tensor, gate: torch.Tensor, shared: Optional[torch.Tensor] = None,
               out_dtype: Optional[torch.dtype] = None, out=None, stream=None):
     _dev(y, None, "y")
+    dev = y.device
     _dev(row_map, torch.int32, "row_map")
-    _dev(gate, torch.float32, "gate")
     T, k = row_map.shape
     d = y.shape[1]
-    out_dtype = out_dtype or y.dtype
+    _buf(row_map, torch.int32, T * k, "row_map", dev)
+    _buf(gate, torch.float32, T * k, "gate", dev)
+    out_dtype = out_dtype or (out.dtype if out is not None else y.dtype)
     if shared is not None:
-        _dev(shared, y.dtype, "shared")
-    if out is None:
-        out = torch.empty((T, d), dtype=out_dtype, device=y.device)
+        _buf(shared, y.dtype, T * d, "shared", dev)
+    out = _out(out, (T, d), out_dtype, dev, "out")
     _check("moe_unpermute", lib().moe_unpermute(
         _p(y), _act_dtype(y), y.shape[0], T, d, k, _p(row_map), _p(gate), _p(shared), _p(out), _act_dtype(out),
         _stream(stream)))
@@ -319,13 +356,13 @@ def unpermute_groups(y_g: torch.Tensor, row_map_g: torch.Tensor, shared: Optiona
                      out_dtype: Optional[torch.dtype] = None, out=None, stream=None):
     """out[t] = sum of the token's distinct group rows (+ shared[t])."""
     _dev(y_g, None, "y_g")
-    _dev(row_map_g, torch.int32, "row_map_g")
+    dev = y_g.device
+    _buf(row_map_g, torch.int32, 0, "row_map_g", dev)
     T, k = row_map_g.shape
     d = y_g.shape[1]
     if shared is not None:
-        _dev(shared, y_g.dtype, "shared")
-    if out is None:
-        out = torch.empty((T, d), dtype=out_dtype or y_g.dtype, device=y_g.device)
+        _buf(shared, y_g.dtype, T * d, "shared", dev)
+    out = _out(out, (T, d), out_dtype or (out.dtype if out is not None else y_g.dtype), dev, "out")
     _check("moe_unpermute_groups", lib().moe_unpermute_groups(
         _p(y_g), _act_dtype(y_g), y_g.shape[0], T, d, k, _p(row_map_g), _p(shared), _p(out), _act_dtype(out),
         _stream(stream)))
@@ -335,11 +372,14 @@ def unpermute_groups(y_g: torch.Tensor, row_map_g: torch.Tensor, shared: Optiona
 def unpermute_ec(y: torch.Tensor, tok_ptr: torch.Tensor, tok_row: torch.Tensor, ec_gate: torch.Tensor,
                  out_dtype: Optional[torch.dtype] = None, out=None, stream=None):
     _dev(y, None, "y")
+    dev = y.device
+    _buf(tok_ptr, torch.int32, 1, "tok_ptr", dev)
+    _buf(tok_row, torch.int32, 0, "tok_row", dev)
+    _buf(ec_gate, torch.float32, 0, "ec_gate", dev)
     T = tok_ptr.numel() - 1
     d = y.shape[1]
-    out_dtype = out_dtype or y.dtype
-    if out is None:
-        out = torch.empty((T, d), dtype=out_dtype, device=y.device)
+    out_dtype = out_dtype or (out.dtype if out is not None else y.dtype)
+    out = _out(out, (T, d), out_dtype, dev, "out")
     _check("moe_unpermute_ec", lib().moe_unpermute_ec(
         _p(y), _act_dtype(y), y.shape[0], T, d, _p(tok_ptr), _p(tok_row), _p(ec_gate), _p(out), _act_dtype(out),
         _stream(stream)))
@@ -352,6 +392,7 @@ def coselect(expert_idx: torch.Tensor, E: int, into: Optional[torch.Tensor] = No
     T, k = expert_idx.shape
     if into is None:
         into = torch.zeros((E, E), dtype=torch.int32, device=expert_idx.device)
+    _buf(into, torch.int32, E * E, "into", expert_idx.device)
     _check("moe_coselect", lib().moe_coselect(_p(expert_idx), T, k, E, _p(into), _stream(stream)))
     return into
 
@@ -365,6 +406,8 @@ def transition(idx1: torch.Tensor, idx2: torch.Tensor, E: int, into: Optional[to
         raise ValueError("idx1 and idx2 need the same token count")
     if into is None:
         into = torch.zeros((E, E), dtype=torch.int32, device=idx1.device)
+    _buf(idx2, torch.int32, 0, "idx2", idx1.device)
+    _buf(into, torch.int32, E * E, "into", idx1.device)
     _check("moe_transition", lib().moe_transition(_p(idx1), k1, _p(idx2), k2, T, E, _p(into), _stream(stream)))
     return into
 
@@ -373,18 +416,18 @@ def transition(idx1: torch.Tensor, idx2: torch.Tensor, E: int, into: Optional[to
 def place_experts(cosel: torch.Tensor, G: int, out=None, stream=None):
     _dev(cosel, torch.int32, "cosel")
     E = cosel.shape[0]
-    if out is None:
-        out = torch.empty(E, dtype=torch.int32, device=cosel.device)
+    _buf(cosel, torch.int32, E * E, "cosel")
+    out = _out(out, (E,), torch.int32, cosel.device, "out")
     _check("moe_place_experts", lib().moe_place_experts(_p(cosel), E, G, _p(out), _stream(stream)))
     return out
 
 
 def group_affinity(trans: torch.Tensor, group_of_expert: torch.Tensor, G: int, out=None, stream=None):
     _dev(trans, torch.int32, "trans")
-    _dev(group_of_expert, torch.int32, "group_of_expert")
     E = trans.shape[0]
-    if out is None:
-        out = torch.empty((E, G), dtype=torch.int64, device=trans.device)
+    _buf(trans, torch.int32, E * E, "trans")
+    _buf(group_of_expert, torch.int32, E, "group_of_expert", trans.device)
+    out = _out(out, (E, G), torch.int64, trans.device, "out")
     _check("moe_group_affinity", lib().moe_group_affinity(_p(trans), E, _p(group_of_expert), G, _p(out),
                                                           _stream(stream)))
     return out
@@ -392,11 +435,10 @@ def group_affinity(trans: torch.Tensor, group_of_expert: torch.Tensor, G: int, o
 
 def predict_home(idx1: torch.Tensor, affinity: torch.Tensor, out=None, stream=None):
     _dev(idx1, torch.int32, "idx1")
-    _dev(affinity, torch.int64, "affinity")
+    _buf(affinity, torch.int64, 0, "affinity", idx1.device)
     T, k1 = idx1.shape
     E, G = affinity.shape
-    if out is None:
-        out = torch.empty(T, dtype=torch.int32, device=idx1.device)
+    out = _out(out, (T,), torch.int32, idx1.device, "out")
     _check("moe_predict_home", lib().moe_predict_home(_p(idx1), T, k1, _p(affinity), E, G, _p(out), _stream(stream)))
     return out
 
@@ -404,11 +446,15 @@ def predict_home(idx1: torch.Tensor, affinity: torch.Tensor, out=None, stream=No
 def count_local(expert_idx: torch.Tensor, group_of_expert: torch.Tensor, G: int, home=None, into=None,
                 stream=None):
     _dev(expert_idx, torch.int32, "expert_idx")
-    _dev(group_of_expert, torch.int32, "group_of_expert")
+    dev = expert_idx.device
+    _buf(group_of_expert, torch.int32, 0, "group_of_expert", dev)
     T, k = expert_idx.shape
     E = group_of_expert.numel()
+    if home is not None:
+        _buf(home, torch.int32, T, "home", dev)
     if into is None:
-        into = torch.zeros(1, dtype=torch.int64, device=expert_idx.device)
+        into = torch.zeros(1, dtype=torch.int64, device=dev)
+    _buf(into, torch.int64, 1, "into", dev)
     _check("moe_count_local", lib().moe_count_local(_p(expert_idx), T, k, _p(group_of_expert), E, G, _p(home),
                                                     _p(into), _stream(stream)))
     return into
