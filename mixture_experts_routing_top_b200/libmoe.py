@@ -10,6 +10,7 @@ non-zero status raises.
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 from typing import Optional
 
@@ -109,7 +110,12 @@ def _dev(t: torch.Tensor, dtype=None, name="tensor"):
 def _buf(t: torch.Tensor, dtype, min_numel: int, name: str, device=None) -> torch.Tensor:
     """A caller's buffer checked against what the library reads or writes
     through its pointer: a contiguous CUDA tensor of `dtype` (None: any) with
-    at least `min_numel` elements, on `device` when given."""
+    at least `min_numel` elements, on `device` when given.  One combined test
+    on the common path (it runs on every call of a layer); the specific
+    message only on failure."""
+    if (t.is_cuda and t.is_contiguous() and (dtype is None or t.dtype == dtype)
+            and (device is None or t.device == device) and t.numel() >= min_numel):
+        return t
     _dev(t, dtype, name)
     if device is not None and t.device != device:
         raise ValueError("%s is on %s, the call's inputs on %s" % (name, t.device, device))
@@ -122,10 +128,7 @@ def _out(t: Optional[torch.Tensor], shape, dtype, device, name: str) -> torch.Te
     """The caller's output buffer (checked as in _buf) or a new one."""
     if t is None:
         return torch.empty(shape, dtype=dtype, device=device)
-    n = 1
-    for v in shape:
-        n *= int(v)
-    return _buf(t, dtype, n, name, device)
+    return _buf(t, dtype, math.prod(shape), name, device)
 
 
 def _ws_bytes(t: torch.Tensor) -> int:

@@ -45,3 +45,27 @@ def test_out_allocates_or_checks(cpu_dev):
 def test_workspace_size_counts_bytes():
     assert M._ws_bytes(torch.empty(10, dtype=torch.float32)) == 40
     assert M._ws_bytes(torch.empty(7, dtype=torch.uint8)) == 7
+
+
+class _ReportsCuda(torch.Tensor):
+    """A host tensor that answers is_cuda = True: it takes the checks' common
+    path the way a device tensor does."""
+    @property
+    def is_cuda(self):
+        return True
+
+
+def test_common_path_and_failures_with_a_device_like_tensor():
+    t = torch.empty(15, dtype=torch.float32).as_subclass(_ReportsCuda)
+    assert M._buf(t, torch.float32, 15, "y", t.device) is t
+    assert M._out(t, (3, 5), torch.float32, t.device, "y") is t
+    assert M._buf(t, None, 0, "y") is t
+    with pytest.raises(ValueError, match="needs 16"):
+        M._buf(t, torch.float32, 16, "y", t.device)
+    with pytest.raises(ValueError, match="must be torch.int32"):
+        M._buf(t, torch.int32, 1, "y")
+    with pytest.raises(ValueError, match="is on"):
+        M._buf(t, torch.float32, 1, "y", torch.device("meta"))
+    g = torch.empty(6, 5).t().as_subclass(_ReportsCuda)
+    with pytest.raises(ValueError, match="contiguous"):
+        M._buf(g, torch.float32, 1, "g")
