@@ -190,6 +190,21 @@ def job_histogram(name, hist, world, device):
                  "total": total, "consistent": total == world * local_total}
 
 
+def workload_config(w, world):
+    """The `config` object of both arms' JSON lines: the workload's name and
+    shape, the batch over all ranks and how it is spread."""
+    cfg = {"workload": w.name, "T": w.T, "d": w.d, "E": w.E}
+    cfg.update({"k": w.k, "capacity_factor": w.capacity_factor} if w.routing == "topk" else {"C": w.C})
+    if w.F:
+        cfg.update({"F": w.F, "act": w.act})
+    if w.F_shared:
+        cfg["F_shared"] = w.F_shared
+    if w.G and not w.F:
+        cfg["G"] = w.G
+    cfg.update({"global_batch": world * w.T, "parallelism": "independent replicas, one batch per GPU"})
+    return cfg
+
+
 def throughput(world, tokens_per_rank, steps, max_elapsed_ms):
     """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
     return world * tokens_per_rank * steps / (max_elapsed_ms / 1e3)
@@ -791,19 +806,11 @@ def run_libmoe(args, w, rank, world, local_rank):
                 "frac": round(ach / peak, 4), "peak_kind": pk_kind + " HBM copy"}
     roof["traffic"] = traffic_for("%s/%s" % (w.name, dom))
     value = throughput(world, w.T, args.steps, elapsed_ms)
-    cfg = {"workload": w.name, "T": w.T, "d": w.d, "E": w.E}
-    cfg.update({"k": w.k, "capacity_factor": w.capacity_factor} if w.routing == "topk" else {"C": w.C})
-    if w.F:
-        cfg.update({"F": w.F, "act": w.act})
-    if w.F_shared:
-        cfg["F_shared"] = w.F_shared
-    if w.G and not w.F:
-        cfg["G"] = w.G
+    cfg = workload_config(w, world)
     if graph is not None:
         cfg["launch"] = "step replayed as one CUDA graph; stage times from an eager pass"
-    cfg.update({"global_batch": world * w.T, "parallelism": "independent replicas, one batch per GPU",
-                "l2": ("flushed between timed steps (256 MB write outside the events)" if flush is not None else
-                       "inputs larger than L2: %.2f GB resident inputs read every step" % (run.resident_bytes / 1e9))})
+    cfg["l2"] = ("flushed between timed steps (256 MB write outside the events)" if flush is not None else
+                 "inputs larger than L2: %.2f GB resident inputs read every step" % (run.resident_bytes / 1e9))
     res = {
         "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(elapsed_ms / args.steps, 4), "higher_is_better": True,
@@ -821,7 +828,7 @@ def run_libmoe(args, w, rank, world, local_rank):
 
 
 # --------------------------------------------------------- reference arm
-def run_reference(args, w):
+def run_reference(args, w, world=1):
     """The oracle as it stands (single-threaded C) on the host cores.  Each
     step: routing, capacity, permutation (with the row copy) and the combine
     over a token sample, plus the expert MLP of one buffer row (rotating);
@@ -903,7 +910,7 @@ def run_reference(args, w):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * statistics.mean(wall), 3),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic: seeded normals and random-init expert weights",
-            "config": {"workload": w.name, "T": w.T, "d": w.d, "E": w.E},
+            "config": dict(workload_config(w, world), l2="host run of the oracle: no GPU cache involved"),
             "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
                              "sample": sample, "cpu": _cpu_name()},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -919,7 +926,7 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         if rank == 0:
-            print(json.dumps(run_reference(args, w)), flush=True)
+            print(json.dumps(run_reference(args, w, world)), flush=True)
         return
     if world > 1:
         import torch
