@@ -17,17 +17,23 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "moe_oracle.c")
 _SO = os.path.join(_HERE, "libmoe_oracle.so")
+CC_FLAGS = ["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-fno-fast-math", "-ffp-contract=off"]
 F32, BF16 = 0, 1
 SWIGLU, GELU = 0, 1
 _lib = None
 
 
 def build(force: bool = False) -> str:
-    """Compile the oracle: plain C, one thread, no vectorising fast-math."""
+    """Compile the oracle: plain C, one thread, no vectorising fast-math.
+    MOE_ORACLE_LIB names a library built elsewhere from a variant of this
+    source (the pin tests' mutation check loads a deliberately broken copy
+    through it); unset, the oracle here is built and used."""
+    override = os.environ.get("MOE_ORACLE_LIB")
+    if override:
+        return override
     if force or not os.path.exists(_SO) or os.path.getmtime(_SO) < os.path.getmtime(_SRC):
         tmp = _SO + ".tmp%d" % os.getpid()
-        subprocess.check_call(["gcc", "-O2", "-fPIC", "-shared", "-std=c11", "-fno-fast-math",
-                               "-ffp-contract=off", _SRC, "-o", tmp, "-lm"])
+        subprocess.check_call(CC_FLAGS + [_SRC, "-o", tmp, "-lm"])
         os.replace(tmp, _SO)
     return _SO
 

@@ -99,6 +99,17 @@ def test_capacity_is_exact_ceiling(w):
     assert cap == {"tiny_fp32": 80, "mixtral_top2_bf16": 2560, "fine_top6_shared_bf16": 2304}[w.name]
 
 
+@pytest.mark.parametrize("cf,T,k,E", [(1.25, 100, 3, 7), (1.0, 10, 1, 3), (0.5, 7, 1, 2), (1.3, 1000, 6, 64),
+                                      (2.0, 1, 1, 3)])
+def test_capacity_rounds_fractional_loads_up(cf, T, k, E):
+    """Whole rows: a fractional cf * T * k / E is rounded up (the exact
+    rational ceiling of the double cf), never down."""
+    q = Fraction(cf) * T * k / E
+    assert q.denominator != 1
+    cap = O.capacity(cf, T, k, E)
+    assert cap - 1 < q <= cap
+
+
 def test_capacity_unbounded():
     assert O.capacity(0.0, 100, 3, 7) >= 300
     assert O.capacity(-1.0, 100, 3, 7) >= 300
@@ -257,6 +268,11 @@ def test_round_bf16():
     ref = torch.from_numpy(vals).to(torch.bfloat16).to(torch.float64).numpy()
     got = np.array([O.round_bf16(float(v)) for v in vals])
     assert np.array_equal(got, ref)
+    # below 2^-126 bf16 values are evenly spaced (2^-133 apart): fp32 subnormals, rounded as torch rounds them
+    sub = (RNG.random(3000) * 2.0 ** -126).astype(np.float32)
+    sub = np.concatenate([sub, -sub, np.float32([1e-45, 3 * 2.0 ** -134, 2.0 ** -126])])
+    ref = torch.from_numpy(sub).to(torch.bfloat16).to(torch.float64).numpy()
+    assert np.array_equal(np.array([O.round_bf16(float(v)) for v in sub]), ref)
 
 
 def test_ffn_scalar_closed_form():
@@ -574,6 +590,13 @@ def test_place_experts_hand_traced():
     # remaining {2, 3}: masses 2, 3 -> seed 3, then 2
     C = np.array([[5, 3, 0, 1], [3, 4, 0, 0], [0, 0, 6, 2], [1, 0, 2, 3]], np.int32)
     assert O.place_experts(C, 2).tolist() == [0, 0, 1, 1]
+    # a group grows by the co-selection summed over all its members: seed 0 (mass 18); affinities to {0}:
+    # 1 -> 10, 2 -> 8 -> add 1; summed over {0, 1}: 2 -> 8 + 0, 3 -> 0 + 5 -> add 2 (expert 3 would win on
+    # its co-selection with the newest member alone); the rest form group 1
+    C = np.zeros((6, 6), np.int32)
+    for a, b, n in ((0, 1, 10), (0, 2, 8), (1, 3, 5), (4, 5, 1)):
+        C[a, b] = C[b, a] = n
+    assert O.place_experts(C, 2).tolist() == [0, 0, 0, 1, 1, 1]
     # all ties: lowest indices first
     assert O.place_experts(np.zeros((6, 6), np.int32), 2).tolist() == [0, 0, 0, 1, 1, 1]
     with pytest.raises(ValueError):
