@@ -676,3 +676,61 @@ def test_shuffling_raises_local_share_on_correlated_layers():
     after = O.count_local(b, goe, G, home) / w.T
     assert abs(before - 1 / G) < 0.02
     assert after > 2 * before
+
+
+# ------------------------------------------ per-token layer compositions
+def _layer_case(dtype, cf, F_shared):
+    w = W.TINY.with_(dtype=dtype, capacity_factor=cf, T=300, F_shared=F_shared)
+    return w, W.make_logits(w), W.make_x(w), W.make_weights(w), W.make_shared_weights(w)
+
+
+@pytest.mark.parametrize("dtype,cf,F_shared", [("f32", 1.25, 0), ("bf16", 0.75, 96)])
+def test_layer_tokens_equal_the_whole_batch_path(dtype, cf, F_shared):
+    """The per-token layer (routing and drops over all tokens, the listed
+    tokens' expert MLPs and their gated sum) equals the whole batch through
+    the oracle's permutation, row copy, expert MLPs and unpermutation, bit
+    for bit, for tokens listed in any order."""
+    w, logits, x, Wt, Ws = _layer_case(dtype, cf, F_shared)
+    idx, gate = O.route_topk(logits, w.k)
+    p = O.permute(idx, w.E, O.capacity(w.capacity_factor, w.T, w.k, w.E))
+    assert p["dropped"] > 0 or cf > 1
+    buf = O.gather_rows(x, p["row_token"])
+    Y = O.to_dtype_bits(O.expert_ffn_rows(buf, np.repeat(np.arange(w.E, dtype=np.int32), p["counts"]), *Wt, w.act), x)
+    sh = None
+    if Ws is not None:
+        sh = O.to_dtype_bits(O.expert_ffn_rows(x, np.zeros(w.T, np.int32), *Ws, "swiglu"), x)
+    full = O.unpermute(Y, p["row_map"], gate, sh)
+    toks = RNG.permutation(w.T)[:120]
+    got, info = O.topk_layer_tokens(w, logits, x, Wt, Ws, toks)
+    if dtype == "bf16":
+        assert np.array_equal(got, full[toks])           # Y is a bf16 tensor on both paths
+    else:
+        # fp32 layers round nothing; the whole-batch path hands Y to the unpermutation as fp32,
+        # one rounding per expert output: within 2^-24 of sum_j |g_j Y_j|
+        Yabs = O.to_dtype_bits(np.abs(O.expert_ffn_rows(buf, np.repeat(np.arange(w.E, dtype=np.int32), p["counts"]),
+                                                        *Wt, w.act)), x)
+        scale = O.unpermute(Yabs, p["row_map"], np.abs(gate))
+        assert (np.abs(got - full[toks]) <= 2.0 ** -24 * scale[toks] + 1e-300).all()
+        assert not np.array_equal(got, np.zeros_like(got))
+    assert np.array_equal(info["perm"]["row_map"], p["row_map"])
+
+
+def test_group_layer_tokens_equal_the_whole_batch_group_path():
+    """The same for the group-major expert path: group rows -> each group's
+    local copy to expert rows -> expert MLPs -> per-group gated pre-combine
+    -> unit sum of the token's group rows, on scattered groups with drops."""
+    w, logits, x, Wt, _ = _layer_case("bf16", 0.75, 0)
+    G = 4
+    goe = RNG.permutation(W.equal_groups(w.E, G)).astype(np.int32)
+    idx, gate = O.route_topk(logits, w.k)
+    cap = O.capacity(w.capacity_factor, w.T, w.k, w.E)
+    pe, pg = O.permute(idx, w.E, cap), O.permute(idx, w.E, cap, group_of_expert=goe)
+    xg = O.gather_rows(x, pg["row_token"])
+    xe = np.zeros((pe["R"], w.d), x.dtype)
+    O.copy_slot_rows(xg, pg["row_map"], pe["row_map"], xe)
+    Ye = O.to_dtype_bits(O.expert_ffn_rows(xe, np.repeat(np.arange(w.E, dtype=np.int32), pe["counts"]), *Wt, w.act), x)
+    P = O.group_precombine(Ye, pe["row_map"], pg["row_map"], gate, pg["R"])
+    full = O.unpermute_groups(O.to_dtype_bits(P, x), pg["row_map"])
+    toks = RNG.permutation(w.T)[:120]
+    got, _ = O.topk_group_layer_tokens(w, logits, x, Wt, None, goe, toks)
+    assert np.array_equal(got, full[toks])
