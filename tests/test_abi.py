@@ -105,3 +105,43 @@ def test_host_validation_rejects_before_launch(L):
     assert L.moe_unpermute_ec(vp, 0, 20, 10, 8, nul, vp, vp, vp, 0, nul) == 1     # null tok_ptr
     assert L.moe_coselect(vp, 10, 2, 2000, vp, nul) == 2
     assert L.moe_transition(vp, 1, vp, 0, 10, 8, vp, nul) == 1
+
+
+def test_host_validation_of_the_later_calls(L):
+    """The fused router, the group-major expert path, placement and the
+    shuffling statistic: bad arguments rejected on the host with the status
+    the header documents, before any launch (this box has no GPU)."""
+    vp, nul = ctypes.c_void_p(0x1000), None
+    router = lambda dt=1, T=10, d=128, E=16, k=2, logits=vp, x=vp: L.moe_router_topk(
+        x, dt, T, d, vp, E, k, 0, logits, vp, vp, nul)
+    assert router(d=96) == 2                 # bf16: d % 64
+    assert router(E=12) == 2                 # bf16: E % 8
+    assert router(E=264) == 2                # bf16: E <= 256
+    assert router(k=9) == 2                  # bf16: k <= 8
+    assert router(k=17) == 1                 # k > E
+    assert router(dt=7) == 1                 # dtype
+    assert router(x=nul) == 1
+    assert router(dt=0, logits=nul) == 1     # fp32 needs the logits buffer
+    assert router(T=0) == 0
+    copy = lambda dt=1, d=64, S=10, src=vp: L.moe_copy_slot_rows(src, dt, 10, d, vp, vp, S, vp, 10, nul)
+    assert copy(S=-1) == 1 and copy(dt=9) == 1 and copy(src=nul) == 1
+    assert copy(dt=0, d=3) == 2              # 12-byte rows
+    assert copy(S=0) == 0
+    pre = lambda dt=1, T=10, d=64, k=2, gate=vp: L.moe_group_precombine(vp, dt, 20, T, d, k, vp, vp, gate, vp, 20, nul)
+    assert pre(k=0) == 1 and pre(k=33) == 2 and pre(gate=nul) == 1 and pre(d=4) == 2 and pre(T=0) == 0
+    ug = lambda od=1, T=10, d=64, k=2, yg=vp, Rg=20: L.moe_unpermute_groups(yg, 1, Rg, T, d, k, vp, nul, vp, od, nul)
+    assert ug(od=4) == 1 and ug(k=40) == 2 and ug(yg=nul) == 1 and ug(d=12) == 2 and ug(T=0) == 0
+    assert L.moe_place_experts(vp, 12, 5, vp, nul) == 1                 # G does not divide E
+    assert L.moe_place_experts(vp, 2000, 1, vp, nul) == 2
+    assert L.moe_place_experts(nul, 12, 3, vp, nul) == 1
+    assert L.moe_group_affinity(vp, 16, vp, 0, vp, nul) == 1
+    assert L.moe_group_affinity(vp, 16, vp, 2000, vp, nul) == 2
+    assert L.moe_group_affinity(vp, 16, nul, 4, vp, nul) == 1
+    assert L.moe_predict_home(vp, 10, 0, vp, 16, 4, vp, nul) == 1
+    assert L.moe_predict_home(vp, 10, 33, vp, 16, 4, vp, nul) == 2
+    assert L.moe_predict_home(vp, 10, 1, vp, 16, 4, nul, nul) == 1
+    assert L.moe_predict_home(vp, 0, 1, vp, 16, 4, vp, nul) == 0
+    assert L.moe_count_local(vp, 10, 0, vp, 16, 4, nul, vp, nul) == 1
+    assert L.moe_count_local(vp, 10, 2, vp, 16, 2000, nul, vp, nul) == 2
+    assert L.moe_count_local(vp, 10, 2, vp, 16, 4, nul, nul, nul) == 1
+    assert L.moe_count_local(vp, 0, 2, vp, 16, 4, nul, vp, nul) == 0
