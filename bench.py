@@ -51,7 +51,8 @@ def parse(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="libmoe", choices=["libmoe", "reference"])
     ap.add_argument("--workload", default="mixtral_top2_bf16")
-    ap.add_argument("--cpu-rows", type=int, default=24, help="expert-MLP rows in the CPU-baseline sample")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="CPU-baseline budget: the oracle's expert-MLP (or routing) sample takes about this long")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=50)
     ap.add_argument("--graph", action="store_true",
@@ -188,6 +189,25 @@ def job_histogram(name, hist, world, device):
                  "collective": "all_reduce sum int32" if world > 1 else "none (one rank)",
                  "allreduce_us": round(us, 1) if world > 1 else 0.0,
                  "total": total, "consistent": total == world * local_total}
+
+
+def time_mlp_rows(O, buf, row_expert_of, weights, act, budget_s):
+    """(rows timed, seconds per row) of the oracle's expert MLP on buffer
+    rows spread evenly over all experts: a 4-row probe, then as many rows as
+    fit the budget (at most all of them)."""
+    R = buf.shape[0]
+
+    def run(n):
+        rows = np.linspace(0, R - 1, num=min(n, R)).astype(np.int64)
+        t0 = time.perf_counter()
+        O.expert_ffn_rows(buf[rows], row_expert_of(rows), *weights, act)
+        return len(rows), time.perf_counter() - t0
+
+    n, t = run(4)
+    want = int(min(R, budget_s / max(t / n, 1e-9)))
+    if want > n:
+        n, t = run(want)
+    return n, t / n
 
 
 def workload_config(w, world):
@@ -401,7 +421,7 @@ class TopKRunner:
                 "assignments": w.T * w.k, "place_us": round(1e3 * a.elapsed_time(b), 1),
                 "inputs": "this batch's routing, expert ids scrambled (seed 7)"}
 
-    def cpu_baseline(self, n_rows):
+    def cpu_baseline(self, budget_s):
         """The oracle as it stands, single-threaded, on a bounded sample."""
         from oracle import oracle as O
         from mixture_experts_routing_top_b200 import synth
@@ -436,15 +456,11 @@ class TopKRunner:
         sample = "%sroute, capacity, permute, row copy and combine on %d of %d tokens (%.2f s)" % (
             "router gate, " if w.router else "", Ts, w.T, t_rp + t_comb)
         if w.F:
-            rows = np.linspace(0, R - 1, num=min(n_rows, R)).astype(np.int64)
-            row_e = np.searchsorted(pe["offsets"], rows, side="right").astype(np.int32) - 1
-            W1, W3, W2 = self.weights_np
-            t0 = time.perf_counter()
-            O.expert_ffn_rows(buf[rows], row_e, W1, W3, W2, w.act)
-            t_row = (time.perf_counter() - t0) / len(rows)
+            row_expert = lambda rows: (np.searchsorted(pe["offsets"], rows, side="right") - 1).astype(np.int32)
+            n, t_row = time_mlp_rows(O, buf, row_expert, self.weights_np, w.act, budget_s)
             per_token += t_row * R / Ts
-            sample += "; expert MLP on %d of %d rows, %.3f s per row, extrapolated to all rows" % (
-                len(rows), R, t_row)
+            sample += "; expert MLP on %d of %d rows, %.4f s per row (%.1f s), extrapolated to all rows" % (
+                n, R, t_row, n * t_row)
             if self.shared_np is not None:
                 t0 = time.perf_counter()
                 O.expert_ffn_rows(x[:2], np.zeros(2, np.int32), *self.shared_np, "swiglu")
@@ -547,7 +563,7 @@ class ExpertChoiceRunner:
                 "predict_us": round(1e3 * a.elapsed_time(b), 1),
                 "note": "transition counts accumulated over all timed steps (identical batches)"}
 
-    def cpu_baseline(self, n_rows):
+    def cpu_baseline(self, budget_s):
         from oracle import oracle as O
         from mixture_experts_routing_top_b200 import synth
 
@@ -562,16 +578,13 @@ class ExpertChoiceRunner:
         b, _ = O.route_topk(self.logits2_np, 1)
         O.transition(a, b, w.E)
         t_rest = time.perf_counter() - t0
-        rows = np.linspace(0, R - 1, num=min(n_rows, R)).astype(np.int64)
-        W1, W3, W2 = self.weights_np
-        t0 = time.perf_counter()
-        O.expert_ffn_rows(buf[rows], (rows // w.C).astype(np.int32), W1, W3, W2, w.act)
-        t_row = (time.perf_counter() - t0) / len(rows)
+        n, t_row = time_mlp_rows(O, buf, lambda rows: (rows // w.C).astype(np.int32), self.weights_np, w.act,
+                                 budget_s)
         per_token = t_rest / w.T + t_row * R / w.T
         return {"value": 1.0 / per_token, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                 "sample": "expert-choice routing, dispatch, combine and both top-1 routings + transitions on all "
-                          "%d tokens (%.2f s); expert MLP on %d of %d rows, %.3f s per row, extrapolated"
-                          % (w.T, t_rest, len(rows), R, t_row), "cpu": _cpu_name()}
+                          "%d tokens (%.2f s); expert MLP on %d of %d rows, %.4f s per row (%.1f s), extrapolated"
+                          % (w.T, t_rest, n, R, t_row, n * t_row), "cpu": _cpu_name()}
 
 
 class RoutingRunner:
@@ -638,19 +651,27 @@ class RoutingRunner:
     def extra(self):
         return {"routing_only": True}
 
-    def cpu_baseline(self, n_rows):
+    def cpu_baseline(self, budget_s):
         from oracle import oracle as O
 
         w = self.w
-        Ts = min(w.T, 16384)
-        t0 = time.perf_counter()
-        if w.router:
-            lg = O.router_logits(self.in_np[0][:Ts], self.Wr_np).astype(np.float32)
-        else:
-            lg = self.in_np[0][:Ts]
-        idx, _ = O.route_topk(lg, w.k, w.norm_topk)
-        O.coselect(idx, w.E)
-        t = time.perf_counter() - t0
+
+        def run(n):
+            t0 = time.perf_counter()
+            if w.router:
+                lg = O.router_logits(self.in_np[0][:n], self.Wr_np).astype(np.float32)
+            else:
+                lg = self.in_np[0][:n]
+            idx, _ = O.route_topk(lg, w.k, w.norm_topk)
+            O.coselect(idx, w.E)
+            return time.perf_counter() - t0
+
+        Ts = min(w.T, 256)
+        t = run(Ts)
+        want = int(min(w.T, budget_s * Ts / max(t, 1e-9)))       # as many tokens as fit the budget
+        if want > Ts:
+            Ts = want
+            t = run(Ts)
         return {"value": Ts / t, "unit": "tokens/s", "cores": 1, "kind": "oracle",
                 "sample": "routing and co-selection on %d of %d tokens (%.2f s)" % (Ts, w.T, t), "cpu": _cpu_name()}
 
@@ -823,7 +844,7 @@ def run_libmoe(args, w, rank, world, local_rank):
     if e2e:
         res["e2e"] = e2e
     if world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = run.cpu_baseline(args.cpu_rows)
+        res["cpu_baseline"] = run.cpu_baseline(args.cpu_seconds)
     return res
 
 
