@@ -581,6 +581,9 @@ def test_generator_deterministic_and_distribution():
     assert c.tobytes() == a[:500].tobytes()
     h = synth.normal_bf16(0, 1, (1000, 37))
     assert np.array_equal(h, synth.f32_to_bf16(a))
+    # the generator's bf16 is round-to-nearest-even of the fp32 draw, as torch converts it
+    tb = torch.from_numpy(a).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(h, tb)
     assert not np.array_equal(synth.u64(0, 1, 10), synth.u64(0, 2, 10))
 
 
