@@ -46,7 +46,8 @@ L2_BYTES = 126 * 1024 * 1024
 
 def parse(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=1,
+                    help="GPUs of the run: N > 1 needs one process per GPU (torch.distributed.run)")
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="libmoe", choices=["libmoe", "reference"])
@@ -944,6 +945,9 @@ def main():
     w = workload_from_args(args)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
+    if args.gpus > 1 and world == 1:
+        raise SystemExit("--gpus %d needs one process per GPU: launch with python -m torch.distributed.run "
+                         "--nproc-per-node %d" % (args.gpus, args.gpus))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         if rank == 0:

@@ -62,3 +62,11 @@ def test_other_ranks_print_nothing():
 def test_too_few_warmup_steps_refused():
     r = run(["--impl", "reference", "--workload", "tiny_fp32", "--steps", "3", "--warmup", "2"])
     assert r.returncode != 0 and "warmup" in r.stderr
+
+
+def test_several_gpus_need_one_process_each():
+    r = run(["--impl", "reference", "--workload", "tiny_fp32", "--gpus", "2", "--steps", "3", "--warmup", "3"])
+    assert r.returncode != 0 and "one process per GPU" in r.stderr
+    r = run(["--impl", "reference", "--workload", "tiny_fp32", "--gpus", "2", "--steps", "3", "--warmup", "3"],
+            {"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
+    assert r.returncode == 0 and r.stdout.strip() == ""
