@@ -94,6 +94,27 @@ MUTANTS = [
 ]
 
 
+# mistakes in the oracle's Python layer (argument marshalling and the per-token layer compositions)
+PY_MUTANTS = [
+    ("py_norm_topk_flag_inverted", "k, int(norm_topk), idx.ctypes.data", "k, int(not norm_topk), idx.ctypes.data"),
+    ("py_capacity_k_and_E_swapped", "oracle_capacity(float(capacity_factor), T, k, E)",
+     "oracle_capacity(float(capacity_factor), T, E, k)"),
+    ("py_layer_gate_of_slot_0", "np.float64(gate[tokens[owner[n]], slot[n]])", "np.float64(gate[tokens[owner[n]], 0])"),
+    ("py_layer_shared_subtracted", "        out += ys\n", "        out -= ys\n"),
+    ("py_group_layer_row_per_slot", "            if g not in seen:\n", "            if True:\n"),
+    ("py_expert_choice_gates_reversed", "g = _c(ec_gate, np.float32).reshape(-1)",
+     "g = _c(ec_gate, np.float32).reshape(-1)[::-1].copy()"),
+    ("py_local_count_ignores_home", "        hp = home.ctypes.data\n", "        hp = None\n"),
+    ("py_local_fraction_one_group_more", "goe.ctypes.data, G))", "goe.ctypes.data, G + 1))"),
+    ("py_expert_choice_on_negated_logits",
+     "def route_ec(logits: np.ndarray, C: int):\n    \"\"\"ExpertChoiceRouter: (ec_token [E,C], ec_gate [E,C], tok_ptr [T+1], "
+     "tok_row [E*C]).\"\"\"\n    lg = _c(logits, np.float32)",
+     "def route_ec(logits: np.ndarray, C: int):\n    \"\"\"ExpertChoiceRouter: (ec_token [E,C], ec_gate [E,C], tok_ptr [T+1], "
+     "tok_row [E*C]).\"\"\"\n    lg = _c(-np.asarray(logits), np.float32)"),
+]
+PY_SRC = os.path.join(ROOT, "oracle", "oracle.py")
+
+
 def _build(name, text):
     os.makedirs(OUT, exist_ok=True)
     c = os.path.join(OUT, name + ".c")
@@ -110,6 +131,48 @@ def _pins(so):
                         "-x", "-p", "no:cacheprovider", "-m", "not gpu"], capture_output=True, text=True, cwd=ROOT,
                        env=env, timeout=900)
     return r.returncode, r.stdout[-600:]
+
+
+def _py_package(name, text):
+    """A copy of the oracle package whose oracle.py is `text`; it builds its
+    own C library next to it on first use."""
+    root = os.path.join(OUT, name)
+    pkg = os.path.join(root, "oracle")
+    os.makedirs(pkg, exist_ok=True)
+    for f in ("__init__.py", "moe_oracle.c"):
+        with open(os.path.join(ROOT, "oracle", f)) as a, open(os.path.join(pkg, f), "w") as b:
+            b.write(a.read())
+    with open(os.path.join(pkg, "oracle.py"), "w") as b:
+        b.write(text)
+    return root
+
+
+def _py_pins(root):
+    """The pin tests with the copied package first on the import path."""
+    env = dict(os.environ, PYTHONPATH=ROOT)
+    env.pop("MOE_ORACLE_LIB", None)
+    which = subprocess.run([sys.executable, "-c", "import oracle; print(oracle.__file__)"], capture_output=True,
+                           text=True, cwd=root, env=env, timeout=300)
+    assert which.stdout.strip().startswith(root), which.stdout + which.stderr
+    r = subprocess.run([sys.executable, "-m", "pytest", os.path.join(ROOT, "tests", "test_oracle_pins.py"), "-q",
+                        "-x", "-p", "no:cacheprovider", "-m", "not gpu"], capture_output=True, text=True, cwd=root,
+                       env=env, timeout=900)
+    return r.returncode, r.stdout[-600:]
+
+
+def test_every_planted_mistake_in_the_python_layer_fails_a_pin():
+    src = open(PY_SRC).read()
+    jobs = {"py_unmutated": src}
+    for name, old, new in PY_MUTANTS:
+        assert src.count(old) == 1, "mutation site of %s is not unique in oracle.py" % name
+        jobs[name] = src.replace(old, new)
+    roots = {n: _py_package(n, t) for n, t in jobs.items()}
+    with cf.ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+        results = dict(zip(roots, ex.map(_py_pins, roots.values())))
+    rc, tail = results.pop("py_unmutated")
+    assert rc == 0, "the unmutated copy fails its pins:\n" + tail
+    survivors = {n: rc for n, (rc, _) in results.items() if rc != 1}
+    assert not survivors, "mutants not caught by a failing pin: %s" % survivors
 
 
 def test_every_planted_mistake_fails_a_pin():
