@@ -817,10 +817,14 @@ def run_libmoe(args, w, rank, world, local_rank):
     dom = max(names, key=lambda n: stage_ms[n])
     kind, amount = work[dom]
     if kind == "flops":
-        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+        # the stage runs inside a step of a few ms, in a timed region of well under a second: the burst
+        # figure (cuBLAS timed alone) is its peak; the seconds-long sustained figure is kept beside it
+        peak = pk["bf16_tflops"]
         ach = report[dom]["TFLOP/s"]
         roof = {"bound": "tensor", "stage": dom, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-                "frac": round(ach / peak, 4), "peak_kind": pk_kind + " sustained bf16 (cuBLAS, 4 s loop)"}
+                "frac": round(ach / peak, 4), "peak_kind": pk_kind + " burst bf16 (cuBLAS timed alone)"}
+        if "bf16_tflops_sustained" in pk:
+            roof["frac_sustained"] = round(ach / pk["bf16_tflops_sustained"], 4)
     else:
         peak = pk["hbm_gbs"]
         ach = report[dom]["GB/s"]

@@ -64,6 +64,8 @@ typedef enum { MOE_ACT_SWIGLU = 0, MOE_ACT_GELU = 1 } moe_act;
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* moe_status_string(int status);
+/* The same, under the name the boundary's specification uses. */
+const char* moe_status_str(moe_status status);
 
 /* ABI revision of this header; bumps on any incompatible change. */
 #define MOE_ABI_VERSION 1
@@ -77,6 +79,19 @@ moe_status moe_device_error(int clear);
 /* Number of CUDA kernels this library has launched in this process (all
  * devices, all streams).  Lets a caller count the kernels a region ran. */
 uint64_t moe_kernel_launches(void);
+
+/* Device check of the failure-detection contract above (the pages have no
+ * counterpart).  One warp waits on an mbarrier through the same bounded
+ * wait the tensor-core kernels use, with a limit of limit_ns of
+ * %globaltimer (1 us .. 1 s).  With arrive == 0 nothing ever arrives: the
+ * wait gives up, the kernel records MOE_ERR_TIMEOUT in the fault word
+ * (moe_device_error) and returns; with arrive != 0 the barrier is
+ * completed first and no fault is recorded.  No copy or MMA is in flight,
+ * so the context stays usable either way.
+ *   result  [2] int32 device out: [0] = 1 if the wait completed, 0 if it
+ *           gave up; [1] = microseconds spent waiting.
+ * Returns MOE_ERR_ARG for a limit outside the range or a NULL result. */
+moe_status moe_selftest_bounded_wait(int arrive, long long limit_ns, int32_t* result, moe_stream_t stream);
 
 /* ------------------------------------------------------------ routing */
 

@@ -4,6 +4,8 @@
 #include <mutex>
 #include <utility>
 
+#include <cuda.h>
+
 #include "common.cuh"
 
 namespace moe {
@@ -15,37 +17,76 @@ __device__ unsigned g_device_error;
 namespace {
 std::atomic<unsigned long long> g_launches{0};
 std::mutex g_mu;
-unsigned* g_err_addr[64] = {nullptr};
+
+using CtxGetCurrent = CUresult (*)(CUcontext*);
+using CtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_entry(const char* name) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint(name, &fn, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+        return nullptr;
+    return reinterpret_cast<Fn>(fn);
+}
+
+// Unique id of the context current on this thread (0 when there is none):
+// a context torn down and created again (cudaDeviceReset) gets a new id, so
+// a device address cached under the old one is never used again.
+unsigned long long current_context_id() {
+    static const CtxGetCurrent get = driver_entry<CtxGetCurrent>("cuCtxGetCurrent");
+    static const CtxGetId get_id = driver_entry<CtxGetId>("cuCtxGetId");
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (!get || !get_id || get(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+}  // namespace
+
+unsigned long long context_id() { return current_context_id(); }
+
+namespace {
+CachedAddress g_err_addr[kMaxDevices];
 }  // namespace
 
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
-unsigned* device_error_word() {
+void* symbol_address(const void* symbol, CachedAddress* cache) {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_err_addr[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-        g_err_addr[dev] = static_cast<unsigned*>(p);
-    }
-    return g_err_addr[dev];
+    CachedAddress& c = cache[dev];
+    const unsigned long long ctx = current_context_id();
+    if (c.addr && ctx != 0 && c.ctx == ctx) return c.addr;
+    // first use on this device, or its context changed: look the symbol up
+    // with the device current (this also creates the primary context)
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, symbol) != cudaSuccess) return nullptr;
+    c.addr = p;
+    c.ctx = current_context_id();
+    return p;
+}
+
+unsigned* device_error_word() {
+    return static_cast<unsigned*>(symbol_address((const void*)&g_device_error, g_err_addr));
 }
 
 // The dynamic shared-memory limit is an attribute of the kernel's instance
-// on one device, so it is raised once per (kernel, device) and remembered.
+// in one context, so it is raised once per (kernel, device, context) and
+// remembered.
 bool set_smem_limit(const void* fn, size_t bytes) {
     if (bytes <= 48 * 1024) return true;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
     static std::mutex mu;
-    static std::map<std::pair<const void*, int>, size_t> raised;
+    static std::map<std::pair<const void*, std::pair<int, unsigned long long>>, size_t> raised;
     std::lock_guard<std::mutex> lk(mu);
-    const auto key = std::make_pair(fn, dev);
+    const auto key = std::make_pair(fn, std::make_pair(dev, current_context_id()));
     const auto it = raised.find(key);
-    if (it != raised.end() && it->second >= bytes) return true;
+    if (key.second.second != 0 && it != raised.end() && it->second >= bytes) return true;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) return false;
-    raised[key] = bytes;
+    raised[std::make_pair(fn, std::make_pair(dev, current_context_id()))] = bytes;
     return true;
 }
 
@@ -65,6 +106,8 @@ extern "C" const char* moe_status_string(int status) {
         default: return "unknown status";
     }
 }
+
+extern "C" const char* moe_status_str(moe_status status) { return moe_status_string((int)status); }
 
 extern "C" int moe_abi_version(void) { return MOE_ABI_VERSION; }
 

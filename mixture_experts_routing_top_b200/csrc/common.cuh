@@ -13,6 +13,23 @@ namespace moe {
 constexpr unsigned kErrTimeout = 1u;
 constexpr unsigned kErrIndex = 2u;
 
+constexpr int kMaxDevices = 64;
+
+// Device address of a __device__ variable on the current device.  In host
+// code a __device__ variable's name is only a host-side stand-in, so the
+// address is looked up (cudaGetSymbolAddress, with the device current) on
+// first use and cached per device under the current context's unique id: a
+// context created again after cudaDeviceReset gets a fresh lookup.  `cache`
+// has kMaxDevices entries.  Null on a runtime error.
+struct CachedAddress {
+    unsigned long long ctx = 0;
+    void* addr = nullptr;
+};
+void* symbol_address(const void* symbol, CachedAddress* cache);
+
+// Unique id of the CUDA context current on this thread, 0 if none.
+unsigned long long context_id();
+
 // Address of the current device's fault word (defined in api.cu).
 unsigned* device_error_word();
 

@@ -681,15 +681,33 @@ extern "C" size_t moe_permute_workspace_bytes(int T, int k, int E, int G) {
     return perm_layout(T, k, E, G).bytes;
 }
 
-extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const int32_t* expert_idx, int k, int E,
-                                  double capacity_factor, const int32_t* group_of_expert, int G, void* buffer,
-                                  int32_t* row_map, int32_t* row_token, int32_t* counts, int32_t* offsets,
-                                  int32_t* dropped, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+// The argument checks of a permutation, shared by moe_permute and
+// moe_permute_noalloc so that both return the same status for the same
+// arguments, before any workspace question.
+static moe_status permute_check_args(const void* x, int dtype, int T, int d, const int32_t* expert_idx, int k, int E,
+                                     const int32_t* group_of_expert, int G, const void* buffer, const int32_t* row_map,
+                                     const int32_t* row_token, const int32_t* counts, const int32_t* offsets,
+                                     const int32_t* dropped) {
     if (T < 0 || k < 1 || E < 1 || k > E || d < 0) return MOE_ERR_ARG;
     if (dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_ARG;
     if (k > 32 || E > 1024) return MOE_ERR_SHAPE;
     if (group_of_expert && (G < 1 || G > 1024)) return (G < 1) ? MOE_ERR_ARG : MOE_ERR_SHAPE;
     if (!counts || !offsets || !dropped) return MOE_ERR_ARG;
+    if (T == 0) return MOE_OK;
+    if (!expert_idx || !row_map || !row_token) return MOE_ERR_ARG;
+    if ((x == nullptr) != (buffer == nullptr)) return MOE_ERR_ARG;
+    const long long row_bytes = (long long)d * (dtype == MOE_BF16 ? 2 : 4);
+    if (x && (row_bytes % 16 != 0 || ((uintptr_t)x & 15) || ((uintptr_t)buffer & 15))) return MOE_ERR_SHAPE;
+    return MOE_OK;
+}
+
+extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const int32_t* expert_idx, int k, int E,
+                                  double capacity_factor, const int32_t* group_of_expert, int G, void* buffer,
+                                  int32_t* row_map, int32_t* row_token, int32_t* counts, int32_t* offsets,
+                                  int32_t* dropped, void* workspace, size_t workspace_bytes, moe_stream_t stream) {
+    const moe_status bad = permute_check_args(x, dtype, T, d, expert_idx, k, E, group_of_expert, G, buffer, row_map,
+                                              row_token, counts, offsets, dropped);
+    if (bad != MOE_OK) return bad;
     if (T == 0) {
         // nothing routed: zero counts, offsets, dropped
         cudaStream_t s0 = (cudaStream_t)stream;
@@ -699,11 +717,8 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
         if (cudaMemsetAsync(dropped, 0, sizeof(int32_t), s0) != cudaSuccess) return MOE_ERR_CUDA;
         return MOE_OK;
     }
-    if (!expert_idx || !row_map || !row_token) return MOE_ERR_ARG;
-    if ((x == nullptr) != (buffer == nullptr)) return MOE_ERR_ARG;
     const int esz = dtype == MOE_BF16 ? 2 : 4;
     const long long row_bytes = (long long)d * esz;
-    if (x && (row_bytes % 16 != 0 || ((uintptr_t)x & 15) || ((uintptr_t)buffer & 15))) return MOE_ERR_SHAPE;
     const int Gk = group_of_expert ? G : 0;
     PermWs L = perm_layout(T, k, E, Gk);
     if (!workspace || workspace_bytes < L.bytes || ((uintptr_t)workspace & 255)) return MOE_ERR_WORKSPACE;
@@ -809,21 +824,25 @@ static __device__ __align__(256) unsigned char g_permute_noalloc_scratch[MOE_PER
 
 namespace {
 std::mutex g_noalloc_mu;
-void* g_noalloc_scratch[64] = {nullptr};
+CachedAddress g_noalloc_scratch[kMaxDevices];
 
 // Device address of this device's scratch array.  In host code the
 // array's name is only a host-side stand-in, so the address is looked up
-// once per device (with that device current) and cached.
+// with the device current on the first call on each device and cached; the
+// cache is keyed on the context's unique id, so a context created again
+// (after cudaDeviceReset) gets a fresh lookup instead of a stale address.
 void* noalloc_scratch_address() {
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_scratch[dev]) {
-        void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_permute_noalloc_scratch) != cudaSuccess) return nullptr;
-        g_noalloc_scratch[dev] = p;
-    }
-    return g_noalloc_scratch[dev];
+    CachedAddress& c = g_noalloc_scratch[dev];
+    const unsigned long long ctx = context_id();
+    if (c.addr && ctx != 0 && c.ctx == ctx) return c.addr;
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_permute_noalloc_scratch) != cudaSuccess) return nullptr;
+    c.addr = p;
+    c.ctx = context_id();
+    return p;
 }
 }  // namespace
 
@@ -831,7 +850,9 @@ extern "C" moe_status moe_permute_noalloc(const void* x, int dtype, int T, int d
                                           int E, double capacity_factor, const int32_t* group_of_expert, int G,
                                           void* buffer, int32_t* row_map, int32_t* row_token, int32_t* counts,
                                           int32_t* offsets, int32_t* dropped, moe_stream_t stream) {
-    if (T < 0 || k < 1 || E < 1 || G < 0) return MOE_ERR_ARG;
+    const moe_status bad = permute_check_args(x, dtype, T, d, expert_idx, k, E, group_of_expert, G, buffer, row_map,
+                                              row_token, counts, offsets, dropped);
+    if (bad != MOE_OK) return bad;
     const size_t need = moe_permute_workspace_bytes(T, k, E, group_of_expert ? G : 0);
     if (need > (size_t)MOE_PERMUTE_NOALLOC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
     void* scratch = noalloc_scratch_address();

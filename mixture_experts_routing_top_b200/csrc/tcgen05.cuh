@@ -41,9 +41,10 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
 }
 
-// Bounded parity wait.  Returns false on timeout or when another role of
-// this CTA has already given up.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag) {
+// Bounded parity wait.  Returns false after limit_ns of %globaltimer or
+// when another role of this CTA has already given up.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort_flag,
+                                          long long limit_ns = WAIT_NS) {
     long long t0 = 0;
     for (uint32_t i = 1;; ++i) {
         uint32_t done;
@@ -57,7 +58,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const v
             if (*abort_flag) return false;
             const long long now = globaltimer();
             if (t0 == 0) t0 = now;
-            else if (now - t0 > WAIT_NS) return false;
+            else if (now - t0 > limit_ns) return false;
         }
     }
 }

@@ -28,9 +28,11 @@ STATUS = {0: "MOE_OK", 1: "MOE_ERR_ARG", 2: "MOE_ERR_SHAPE", 3: "MOE_ERR_DTYPE",
 _vp, _i32, _i64, _dbl, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double, ctypes.c_size_t
 SIGNATURES = {
     "moe_status_string": (ctypes.c_char_p, [_i32]),
+    "moe_status_str": (ctypes.c_char_p, [_i32]),
     "moe_abi_version": (_i32, []),
     "moe_device_error": (_i32, [_i32]),
     "moe_kernel_launches": (ctypes.c_uint64, []),
+    "moe_selftest_bounded_wait": (_i32, [_i32, ctypes.c_longlong, _vp, _vp]),
     "moe_route_topk": (_i32, [_vp, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "moe_router_topk": (_i32, [_vp, _i32, _i32, _i32, _vp, _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
     "moe_route_ec_workspace_bytes": (_sz, [_i32, _i32, _i32]),
@@ -466,6 +468,14 @@ def count_local(expert_idx: torch.Tensor, group_of_expert: torch.Tensor, G: int,
 def device_error(clear: bool = True) -> int:
     """Device fault word of the current device (synchronises): 0 if clean."""
     return int(lib().moe_device_error(int(bool(clear))))
+
+
+def selftest_bounded_wait(arrive: bool, limit_ns: int, stream=None) -> torch.Tensor:
+    """Runs the bounded-wait check kernel: [completed (1/0), microseconds waited]."""
+    out = torch.full((2,), -1, dtype=torch.int32, device="cuda")
+    _check("moe_selftest_bounded_wait", lib().moe_selftest_bounded_wait(int(bool(arrive)), int(limit_ns), _p(out),
+                                                                        _stream(stream)))
+    return out
 
 
 def kernel_launches() -> int:

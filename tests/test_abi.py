@@ -44,6 +44,8 @@ def test_status_strings(L):
     for s in range(1, 9):
         assert L.moe_status_string(s) not in (b"ok", b"unknown status")
     assert L.moe_status_string(99) == b"unknown status"
+    for s in range(0, 9):
+        assert L.moe_status_str(s) == L.moe_status_string(s)
     assert L.moe_abi_version() == 1
 
 
@@ -105,6 +107,9 @@ def test_host_validation_rejects_before_launch(L):
     assert L.moe_unpermute_ec(vp, 0, 20, 10, 8, nul, vp, vp, vp, 0, nul) == 1     # null tok_ptr
     assert L.moe_coselect(vp, 10, 2, 2000, vp, nul) == 2
     assert L.moe_transition(vp, 1, vp, 0, 10, 8, vp, nul) == 1
+    assert L.moe_selftest_bounded_wait(0, 999, vp, nul) == 1                     # limit below 1 us
+    assert L.moe_selftest_bounded_wait(0, 2 * 10 ** 9, vp, nul) == 1             # above 1 s
+    assert L.moe_selftest_bounded_wait(0, 10 ** 6, nul, nul) == 1                # no result buffer
 
 
 def test_host_validation_of_the_later_calls(L):
@@ -145,3 +150,24 @@ def test_host_validation_of_the_later_calls(L):
     assert L.moe_count_local(vp, 10, 2, vp, 16, 2000, nul, vp, nul) == 2
     assert L.moe_count_local(vp, 10, 2, vp, 16, 4, nul, nul, nul) == 1
     assert L.moe_count_local(vp, 0, 2, vp, 16, 4, nul, vp, nul) == 0
+
+
+def test_noalloc_checks_arguments_before_its_scratch_size(L):
+    """moe_permute_noalloc returns moe_permute's status for bad arguments,
+    whatever the problem size; only valid problems too large for its fixed
+    scratch get MOE_ERR_WORKSPACE.  Nothing is launched in any case."""
+    vp, nul = ctypes.c_void_p(0x1000), None
+    na = lambda T=10, k=2, E=4, G=0, goe=nul, dt=1, d=8, cnt=vp: L.moe_permute_noalloc(
+        vp, dt, T, d, vp, k, E, 1.0, goe, G, vp, vp, vp, cnt, vp, vp, nul)
+    big = 1 << 22                            # needs far more scratch than the 4 MiB array holds
+    assert M.permute_workspace_bytes(big, 8, 256, 0) > 4 << 20
+    assert na(k=5) == 1                      # k > E
+    assert na(T=big, k=300, E=256) == 1      # k > E on a large problem: the argument error
+    assert na(T=big, k=33, E=256) == 2       # k > 32
+    assert na(T=big, k=8, E=2000) == 2       # E > 1024
+    assert na(T=big, k=8, E=256, dt=7) == 1  # dtype
+    assert na(T=big, k=8, E=256, d=7) == 2   # 14-byte bf16 rows
+    assert na(T=big, k=8, E=256, cnt=nul) == 1
+    assert na(T=big, k=8, E=256, goe=vp, G=0) == 1
+    assert na(T=big, k=8, E=256) == 4        # valid but beyond the scratch
+    assert na(T=262144, k=8, E=256, goe=vp, G=64) == 4

@@ -8,7 +8,8 @@ import torch
 
 from mixture_experts_routing_top_b200 import libmoe as M, layer as Lyr, synth, workloads as W
 from oracle import oracle as O
-from tests.helpers import as_f64, assert_layer_close, needs_gpu, to_dev, to_np
+from tests.helpers import (as_f64, assert_blocks_covered, assert_layer_close, needs_gpu, one_row_per_block, oracle_map,
+                           to_dev, to_np, token_chunks)
 
 pytestmark = [pytest.mark.gpu, needs_gpu]
 
@@ -130,53 +131,56 @@ def test_layer_tiny_forced_drops():
     assert all_dropped.any() and (got[all_dropped] == 0).all()
 
 
-def sampled_tokens(info, T, n, seed=0):
-    """n tokens: some with dropped slots first, the rest uniform."""
-    rng = np.random.default_rng(seed)
-    dropped = np.nonzero((info["perm"]["row_map"] < 0).any(1))[0]
-    pick = list(rng.choice(dropped, size=min(n // 2, dropped.size), replace=False)) if dropped.size else []
-    rest = rng.choice(T, size=n - len(pick), replace=False)
-    return np.unique(np.concatenate([np.asarray(pick, np.int64), rest, [0, T - 1]]))
+FULL_UNIFORM = 1024      # seeded uniform tokens per full-size layer
 
 
-def boundary_tokens(perm, E, inner_tiles):
-    """Tokens owning the buffer rows at each expert's first and last row, at
-    the first row of its last (ragged) 128-row tile and on both sides of its
-    first `inner_tiles` 128-row tile boundaries: the rows where the grouped
-    GEMMs' tiles start, end and straddle experts."""
+def boundary_tokens(perm, E):
+    """Tokens owning each expert's first and last buffer rows and the first
+    row of its last (ragged) 128-row tile: where the grouped GEMMs' tiles
+    start, end and straddle experts."""
     off, rt = perm["offsets"], perm["row_token"]
     rows = []
     for e in range(E):
         a, b = int(off[e]), int(off[e + 1])
-        if b <= a:
-            continue
-        rows += [a, b - 1, a + ((b - 1 - a) // 128) * 128]
-        for j in range(1, inner_tiles + 1):
-            if a + 128 * j < b:
-                rows += [a + 128 * j - 1, a + 128 * j]
-    return np.unique(rt[np.asarray(rows)])
+        if b > a:
+            rows += [a, b - 1, a + ((b - 1 - a) // 128) * 128]
+    return np.unique(rt[np.asarray(rows, np.int64)]) if rows else np.zeros(0, np.int64)
+
+
+def full_size_tokens(info, w, seed=0):
+    """The tokens a full-size layer is checked on: every token with a
+    dropped slot, 1024 seeded uniform tokens, the owner of one seeded row in
+    every 128-row block of every expert, the tile-boundary owners, and the
+    first and last tokens."""
+    rng = np.random.default_rng(seed)
+    perm = info["perm"]
+    dropped = np.nonzero((perm["row_map"] < 0).any(1))[0]
+    uniform = rng.choice(w.T, size=min(FULL_UNIFORM, w.T), replace=False)
+    blocks = perm["row_token"][one_row_per_block(perm["offsets"], rng)]
+    return np.unique(np.concatenate([dropped, uniform, blocks, boundary_tokens(perm, w.E), [0, w.T - 1]])), dropped
 
 
 _FULL_REF = {}
 
 
 def full_size_reference(w, logits, x, Wt, Ws):
-    """The oracle's outputs on the sampled tokens of a full-size layer,
-    computed once per workload (the test runs once per GEMM kernel)."""
+    """The oracle's outputs on the checked tokens of a full-size layer,
+    computed once per workload (the test runs once per GEMM kernel family),
+    token chunks spread over the host cores."""
     if w.name not in _FULL_REF:
         _, info = O.topk_layer_tokens(w, logits, x, Wt, Ws, [])
-        toks = np.union1d(sampled_tokens(info, w.T, 12), boundary_tokens(info["perm"], w.E, 1 if w.E <= 8 else 0))
-        ref, _ = O.topk_layer_tokens(w, logits, x, Wt, Ws, toks)
-        _FULL_REF[w.name] = (toks, ref, info["idx"])
+        toks, dropped = full_size_tokens(info, w)
+        parts = oracle_map(lambda c: O.topk_layer_tokens(w, logits, x, Wt, Ws, c)[0], token_chunks(toks))
+        _FULL_REF[w.name] = (toks, np.concatenate(parts), info, dropped)
     return _FULL_REF[w.name]
 
 
 @pytest.mark.parametrize("w", [W.MIXTRAL, W.FINE], ids=lambda w: w.name)
-def test_layer_full_size_sampled(w, gemm_kind):
+def test_layer_full_size(w, gemm_kind):
     """Full-size layer in the bench's launch configuration against the
-    oracle on sampled tokens: some with dropped slots, some uniform, and
-    those owning each expert's first and last rows and rows at 128-row tile
-    boundaries."""
+    oracle on every token with a dropped slot, 1024 seeded tokens and one
+    row of every 128-row block of every expert (so each half of every
+    256-row CTA-pair tile of the persistent schedule is compared)."""
     logits, x = W.make_logits(w), W.make_x(w)
     Wt = W.make_weights(w)
     Ws = W.make_shared_weights(w)
@@ -184,11 +188,21 @@ def test_layer_full_size_sampled(w, gemm_kind):
                       shared_weights=None if Ws is None else weights_dev(Ws))
     got = to_np(L.forward(to_dev(logits), to_dev(x)))
     assert M.device_error() == 0
-    toks, ref, idx = full_size_reference(w, logits, x, Wt, Ws)
-    assert toks.size > 30
+    toks, ref, info, dropped = full_size_reference(w, logits, x, Wt, Ws)
+    perm = info["perm"]
+    # the sample's contract: all dropped-slot tokens, >= 1024 tokens, every block covered
+    assert np.isin(dropped, toks).all() and toks.size >= FULL_UNIFORM
+    assert assert_blocks_covered(perm["offsets"], perm["row_token"], toks) >= (perm["R"] + 127) // 128
+    # the layer's own routing and permutation are those of the oracle, on all tokens
+    assert np.array_equal(to_np(L.perm["offsets"]), perm["offsets"])
+    assert np.array_equal(to_np(L.perm["row_map"]).reshape(w.T, w.k), perm["row_map"])
     assert_layer_close(got[toks], ref)
+    # tokens whose every slot dropped (and no shared expert) output exactly zero
+    if Ws is None:
+        gone = np.nonzero((perm["row_map"] < 0).all(1))[0]
+        assert (as_f64(got[gone]) == 0).all()
     # co-selection of this layer's routing, bit-exact
-    assert np.array_equal(to_np(M.coselect(L.idx, w.E)), O.coselect(idx, w.E))
+    assert np.array_equal(to_np(M.coselect(L.idx, w.E)), O.coselect(info["idx"], w.E))
 
 
 @pytest.mark.parametrize("G", W.SWEEP_G)
@@ -206,25 +220,58 @@ def test_layer_dispatch_combine_identity(G):
     np.testing.assert_allclose(got, as_f64(x), rtol=1e-5, atol=1e-6)   # renormalised gates: y == x
 
 
-def test_layer_expert_choice_sampled(gemm_kind):
+_EC_REF = {}
+
+
+def ec_reference(w, x, W1, W2):
+    """The oracle's expert-choice layer on the checked tokens: 1024 seeded
+    chosen tokens and the owner of one seeded row in every 128-row block of
+    every expert's C rows; each token's expert outputs gate-summed in the
+    token CSR's order (ascending expert).  Computed once, token chunks
+    spread over the host cores."""
+    if w.name in _EC_REF:
+        return _EC_REF[w.name]
+    logits = W.make_logits(w)
+    ec_token, ec_gate, tok_ptr, tok_row = O.route_ec(logits, w.C)
+    rng = np.random.default_rng(0)
+    chosen = np.nonzero(np.diff(tok_ptr) > 0)[0]
+    offsets = np.arange(w.E + 1, dtype=np.int64) * w.C
+    blocks = ec_token.reshape(-1)[one_row_per_block(offsets, rng)]
+    toks = np.unique(np.concatenate([rng.choice(chosen, min(FULL_UNIFORM, chosen.size), replace=False), blocks]))
+    g = ec_gate.reshape(-1).astype(np.float64)
+
+    def chunk(ts):
+        rows = [tok_row[tok_ptr[t]:tok_ptr[t + 1]] for t in ts]
+        y = O.expert_ffn_rows(x[np.repeat(ts, [r.size for r in rows])],
+                              (np.concatenate(rows) // w.C).astype(np.int32), W1, None, W2, "gelu")
+        out = np.zeros((len(ts), w.d))
+        n = 0
+        for i, r in enumerate(rows):
+            for q in r:
+                out[i] += g[q] * y[n]
+                n += 1
+        return out
+
+    ref = np.concatenate(oracle_map(chunk, token_chunks(toks)))
+    _EC_REF[w.name] = (toks, ref, (ec_token, tok_ptr), offsets)
+    return _EC_REF[w.name]
+
+
+def test_layer_expert_choice_full_size(gemm_kind):
+    """The expert-choice GELU layer at full size (T=32768, E=128, C=512):
+    1024 seeded tokens plus one row of every 128-row block of every
+    expert against the oracle; every unchosen token outputs exactly 0."""
     w = W.EXPERT_CHOICE
     logits, x = W.make_logits(w), W.make_x(w)
     W1, _, W2 = W.make_weights(w)
     L = Lyr.ExpertChoiceLayer(w.T, w.d, w.E, w.C, w.F, torch.bfloat16, to_dev(W1), None, to_dev(W2), "gelu")
     got = to_np(L.forward(to_dev(logits), to_dev(x)))
     assert M.device_error() == 0
-    ec_token, ec_gate, tok_ptr, tok_row = O.route_ec(logits, w.C)
-    rng = np.random.default_rng(0)
-    chosen = np.nonzero(np.diff(tok_ptr) > 0)[0]
-    unchosen = np.nonzero(np.diff(tok_ptr) == 0)[0]
-    toks = np.unique(np.concatenate([rng.choice(chosen, 10, replace=False), unchosen[:3]]))
-    ref = np.zeros((toks.size, w.d))
-    for i, t in enumerate(toks):
-        rows = tok_row[tok_ptr[t]:tok_ptr[t + 1]]
-        if rows.size:
-            y = O.expert_ffn_rows(x[[t] * rows.size], (rows // w.C).astype(np.int32), W1, None, W2, "gelu")
-            ref[i] = (ec_gate.reshape(-1)[rows].astype(np.float64)[:, None] * y).sum(0)
+    toks, ref, (ec_token, tok_ptr), offsets = ec_reference(w, x, W1, W2)
+    assert toks.size >= FULL_UNIFORM
+    assert assert_blocks_covered(offsets, ec_token.reshape(-1), toks) == w.E * ((w.C + 127) // 128)
     assert_layer_close(got[toks], ref)
+    unchosen = np.nonzero(np.diff(tok_ptr) == 0)[0]
     assert (as_f64(got[unchosen]) == 0).all()
 
 

@@ -8,7 +8,8 @@ import torch
 
 from mixture_experts_routing_top_b200 import layer as Lyr, libmoe as M, synth, workloads as W
 from oracle import oracle as O
-from tests.helpers import as_f64, assert_layer_close, needs_gpu, to_dev, to_np
+from tests.helpers import (as_f64, assert_blocks_covered, assert_layer_close, needs_gpu, one_row_per_block, oracle_map,
+                           to_dev, to_np, token_chunks)
 
 pytestmark = [pytest.mark.gpu, needs_gpu]
 REL = 1e-5
@@ -149,9 +150,11 @@ def test_group_layer_tiny_fp32_all_tokens(G, cf):
 
 
 @pytest.mark.parametrize("G", [4, 16])
-def test_group_layer_fine_full_size_sampled(G):
+def test_group_layer_fine_full_size(G):
     """Fine-grained layer (64 experts, top-6, shared expert) with placed
-    (non-contiguous) groups, at full size; sampled tokens vs the oracle."""
+    (non-contiguous) groups, at full size, against the oracle on 1024
+    seeded tokens, every token with a dropped slot, and one row of every
+    128-row block of every expert's rows (the rows the grouped GEMMs tile)."""
     w = W.FINE
     logits, x = W.make_logits(w), W.make_x(w)
     Wt, Ws = W.make_weights(w), W.make_shared_weights(w)
@@ -162,10 +165,15 @@ def test_group_layer_fine_full_size_sampled(G):
     got = to_np(L.forward(to_dev(logits), to_dev(x)))
     assert M.device_error() == 0
     _, info = O.topk_group_layer_tokens(w, logits, x, Wt, Ws, goe, [])
+    pe = info["perm"]                                   # expert-major rows: what the GEMMs run on
     rng = np.random.default_rng(G)
-    toks = np.unique(np.concatenate([rng.choice(w.T, 10, replace=False), [0, w.T - 1]]))
-    ref, _ = O.topk_group_layer_tokens(w, logits, x, Wt, Ws, goe, toks)
-    assert_layer_close(got[toks], ref)
+    dropped = np.nonzero((pe["row_map"] < 0).any(1))[0]
+    toks = np.unique(np.concatenate([rng.choice(w.T, 1024, replace=False), dropped,
+                                     pe["row_token"][one_row_per_block(pe["offsets"], rng)], [0, w.T - 1]]))
+    assert assert_blocks_covered(pe["offsets"], pe["row_token"], toks) >= (pe["R"] + 127) // 128
+    assert np.array_equal(to_np(L.perm_e["offsets"]), pe["offsets"])
+    parts = oracle_map(lambda c: O.topk_group_layer_tokens(w, logits, x, Wt, Ws, goe, c)[0], token_chunks(toks))
+    assert_layer_close(got[toks], np.concatenate(parts))
     # fewer rows cross to the groups than there are kept assignments
     R_g = int(L.perm["offsets"][-1].item())
     R_e = int(L.perm_e["offsets"][-1].item())

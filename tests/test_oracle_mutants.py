@@ -8,10 +8,13 @@ least one pin fail, so none of these mistakes could sit in the oracle
 unnoticed.  The unmutated copy, built the same way, must pass: the harness
 itself is sound.  The mistakes are planted in copies on the CPU only; the
 committed oracle is never changed."""
+import atexit
 import concurrent.futures as cf
 import os
+import shutil
 import subprocess
 import sys
+import tempfile
 
 import pytest
 
@@ -19,7 +22,17 @@ from oracle import oracle as O
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "moe_oracle.c")
-OUT = os.path.join(ROOT, "oracle", "_mutants")
+_OUT = []
+
+
+def _out():
+    """A temporary directory, outside the source tree, for the mutated copies
+    and their libraries; removed when the test process exits."""
+    if not _OUT:
+        d = tempfile.mkdtemp(prefix="moe_oracle_mutants_")
+        atexit.register(shutil.rmtree, d, True)
+        _OUT.append(d)
+    return _OUT[0]
 
 # (name, exact text in the oracle, its replacement)
 MUTANTS = [
@@ -116,9 +129,8 @@ PY_SRC = os.path.join(ROOT, "oracle", "oracle.py")
 
 
 def _build(name, text):
-    os.makedirs(OUT, exist_ok=True)
-    c = os.path.join(OUT, name + ".c")
-    so = os.path.join(OUT, "lib" + name + ".so")
+    c = os.path.join(_out(), name + ".c")
+    so = os.path.join(_out(), "lib" + name + ".so")
     with open(c, "w") as f:
         f.write(text)
     subprocess.run(O.CC_FLAGS + [c, "-o", so, "-lm"], check=True, capture_output=True)
@@ -136,7 +148,7 @@ def _pins(so):
 def _py_package(name, text):
     """A copy of the oracle package whose oracle.py is `text`; it builds its
     own C library next to it on first use."""
-    root = os.path.join(OUT, name)
+    root = os.path.join(_out(), name)
     pkg = os.path.join(root, "oracle")
     os.makedirs(pkg, exist_ok=True)
     for f in ("__init__.py", "moe_oracle.c"):

@@ -82,9 +82,23 @@ def test_noalloc_matches_workspace_path_on_two_calls_in_a_row():
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
-    T, k, E, G = 262144, 8, 256, 64
+    """A valid problem whose scratch exceeds the fixed array is refused with
+    MOE_ERR_WORKSPACE before anything is launched.  Real device buffers of
+    the refused problem's shape are passed (rows of d = 8, about 60 MB), so
+    the call could not touch an invalid address even if it did launch; the
+    outputs must be left exactly as they were."""
+    T, k, E, G, d = 262144, 8, 256, 64, 8
     assert M.permute_workspace_bytes(T, k, E, G) > SCRATCH_LIMIT
-    vp = ctypes.c_void_p(0x1000)                                  # never dereferenced
-    st = M.lib().moe_permute_noalloc(vp, 1, T, 8, vp, k, E, ctypes.c_double(0.0), vp, G, vp, vp, vp, vp, vp, vp,
-                                     None)
-    assert st == 4                                                # MOE_ERR_WORKSPACE, nothing launched
+    x = torch.zeros((T, d), dtype=torch.bfloat16, device="cuda")
+    idx = (torch.arange(T * k, device="cuda", dtype=torch.int32) % E).view(T, k)
+    goe = to_dev(W.equal_groups(E, G))
+    out = outputs(x, idx, E, 0.0, goe, G)
+    for t in out.values():
+        t.fill_(-7) if t.dtype == torch.int32 else t.view(torch.int16).fill_(-7)
+    torch.cuda.synchronize()
+    launches = M.kernel_launches()
+    assert call_noalloc(x, idx, E, 0.0, goe, G, out) == 4               # MOE_ERR_WORKSPACE
+    torch.cuda.synchronize()
+    assert M.kernel_launches() == launches
+    for t in out.values():
+        assert bool(((t if t.dtype == torch.int32 else t.view(torch.int16)) == -7).all())
