@@ -196,9 +196,12 @@ moe_status moe_permute(const void* x, int dtype, int T, int d,
  * held by every GPU that loads the library until the process exits.
  * Limit: moe_permute_workspace_bytes(T, k, E, G) must not exceed it
  * (e.g. T = 131072, k = 8, E = 256, G = 64 needs 3.25 MiB); larger problems
- * return MOE_ERR_WORKSPACE and launch nothing.  The first call on a device
- * looks up the array's device address (cudaGetSymbolAddress) and caches it;
- * make that first call before any stream capture.  All calls share the one
+ * return MOE_ERR_WORKSPACE and launch nothing; invalid arguments are
+ * checked first and return what moe_permute returns for them.  The first
+ * call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) and caches it for that device's context (a context
+ * created again after cudaDeviceReset gets a new lookup); make that first
+ * call before any stream capture.  All calls share the one
  * array, so calls whose kernels overlap on the GPU (different streams, no
  * ordering between them) race and give wrong results; serialise them. */
 #define MOE_PERMUTE_NOALLOC_SCRATCH_BYTES (4u << 20)

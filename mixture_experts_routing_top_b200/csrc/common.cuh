@@ -40,6 +40,15 @@ void count_launch();
 // (no-op up to 48 KB).  False if the runtime refused.
 bool set_smem_limit(const void* fn, size_t bytes);
 
+// Programmatic dependent launch.  A kernel launched with programmatic
+// stream serialization may start while the kernel before it in the stream
+// is still running; it must call pdl_wait() before its first global memory
+// access (read or write), which returns once that kernel has completed and
+// its writes are visible.  Without the launch attribute pdl_wait() returns
+// at once.  pdl_trigger() lets the next such kernel be scheduled now.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void raise_error(unsigned* err, unsigned bits) {
     if (err) atomicOr(err, bits);
 }
@@ -128,6 +137,24 @@ __device__ __forceinline__ T warp_sum(T v) {
 }
 
 inline int ceil_div(long long a, long long b) { return (int)((a + b - 1) / b); }
+
+// A kernel launch that may begin while the kernel before it in the stream
+// is finishing (programmatic stream serialization); the kernel calls
+// pdl_wait() before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int block, size_t smem, cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
 
 }  // namespace moe
 

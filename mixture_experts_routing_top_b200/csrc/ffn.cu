@@ -45,7 +45,10 @@ constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int EPI_WARPS = 4;                 // one warp per TMEM lane quarter (EPI_WARPS = 8 splits the columns in half)
 constexpr int THREADS = 64 + 32 * EPI_WARPS;  // warp 0 TMA, warp 1 MMA, then the epilogue warps
 constexpr int MAX_E = 1024;
-constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + 256 /*barriers*/ + 4 * (MAX_E + 1);
+constexpr int OUT_CHUNK_BYTES = 32 * 64;                     // one warp's 32 rows x 32 bf16 columns
+constexpr int OUT_STAGE_BYTES = EPI_WARPS * 2 * OUT_CHUNK_BYTES;   // two staging buffers per epilogue warp
+constexpr int SMEM_BYTES = 1024 /*align slack*/ + STAGES * STAGE_BYTES + OUT_STAGE_BYTES + 256 /*barriers*/ +
+                           4 * (MAX_E + 1);
 
 enum { MODE_SWIGLU = 0, MODE_GELU = 1, MODE_PLAIN = 2 };
 
@@ -100,6 +103,52 @@ __device__ __forceinline__ void store_row32(uint16_t* dst, const float* v) {
     }
 }
 
+// Output of one epilogue warp: its 32 rows x 32 columns per chunk.  When
+// all 32 rows lie inside the expert, the chunk is packed to bf16 into one of
+// the warp's two shared-memory buffers (64-byte swizzle: bank-conflict-free
+// 16-byte writes) and written by one TMA store, so the stores leave the
+// issue slots and the LSU; a buffer is rewritten only after the store issued
+// two chunks earlier has read it.  A warp whose rows straddle the expert's
+// end stores its valid rows directly: a box would overwrite the next
+// expert's rows.
+struct EpiOut {
+    uint32_t buf;   // shared address of this warp's two buffers
+    int n = 0;      // chunks staged so far
+
+    __device__ __forceinline__ void chunk(const CUtensorMap* map, uint16_t* orow, bool valid, bool full, int grow0,
+                                          int col, const float* v) {
+        const int lane = threadIdx.x & 31;
+        if (full) {
+            if (lane == 0) bulk_wait_read1();
+            __syncwarp();
+            const uint32_t b = buf + (uint32_t)(n & 1) * OUT_CHUNK_BYTES + (uint32_t)lane * 64;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint4 w;
+                w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+                w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+                w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+                w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+                st_shared_v4(b + (uint32_t)((q ^ ((lane >> 1) & 3)) << 4), w);
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(map, buf + (uint32_t)(n & 1) * OUT_CHUNK_BYTES, col, grow0);
+                bulk_commit();
+            }
+            ++n;
+        } else if (valid) {
+            store_row32(orow + col, v);
+        }
+    }
+    // every store issued by this warp has completed (before the CTA exits)
+    __device__ __forceinline__ void drain() {
+        if ((threadIdx.x & 31) == 0) bulk_wait0();
+        __syncwarp();
+    }
+};
+
 struct GemmArgs {
     const int32_t* offsets;   // [E+1] device
     int E;
@@ -115,12 +164,14 @@ template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_constant__ CUtensorMap map_a,
                                                                   const __grid_constant__ CUtensorMap map_b0,
                                                                   const __grid_constant__ CUtensorMap map_b1,
+                                                                  const __grid_constant__ CUtensorMap map_out,
                                                                   GemmArgs args) {
     constexpr int BN_OUT = (MODE == MODE_SWIGLU) ? 128 : 256;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t* stage_base = smem;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint8_t* out_stage = smem + STAGES * STAGE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + OUT_STAGE_BYTES);
     uint64_t* full = bars;                     // [STAGES]
     uint64_t* empty = bars + STAGES;           // [STAGES]
     uint64_t* tfull = bars + 2 * STAGES;       // [2]
@@ -128,7 +179,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
     uint64_t* drain = bars + 2 * STAGES + 4;   // [1] MMA completion before TMEM is freed
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* tile_prefix = reinterpret_cast<int*>(smem + STAGES * STAGE_BYTES + 256);   // [E+1]
+    int* tile_prefix = reinterpret_cast<int*>(out_stage + OUT_STAGE_BYTES + 256);   // [E+1]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int E = args.E;
@@ -153,6 +204,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         tma_prefetch_desc(&map_a);
         tma_prefetch_desc(&map_b0);
         if (MODE == MODE_SWIGLU) tma_prefetch_desc(&map_b1);
+        tma_prefetch_desc(&map_out);
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -269,6 +321,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
         const int q = warp & 3;
         const int half = (EPI_WARPS == 8) ? ((warp - 2) >> 2) : 0;
         const int r = q * 32 + lane;
+        EpiOut eo{smem_u32(out_stage + (warp - 2) * 2 * OUT_CHUNK_BYTES)};
         int it = 0;
         for (int t = blockIdx.x; t < total; t += gridDim.x, ++it) {
             int row0, row_end, brow, n0;
@@ -279,6 +332,8 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
             tc_fence_after();
             const int grow = row0 + r;
             const bool valid = grow < row_end;
+            const int grow0 = row0 + q * 32;
+            const bool full = grow0 + 31 < row_end;
             const uint32_t taddr = tmem_base + acc * ACC_N + ((uint32_t)(q * 32) << 16);
             uint16_t* orow = args.out + (long long)grow * args.N_out;
             if (MODE == MODE_SWIGLU) {
@@ -289,10 +344,10 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                     tmem_ld32(taddr + 128 + c * 32, b);
                     tmem_ld_wait();
                     const int col = n0 + c * 32;
-                    if (valid && col < args.N_out) {
+                    if (col < args.N_out) {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) a[i] = silu_f(a[i]) * b[i];
-                        store_row32(orow + col, a);
+                        eo.chunk(&map_out, orow, valid, full, grow0, col, a);
                     }
                 }
             } else {
@@ -302,18 +357,19 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                     tmem_ld32(taddr + c * 32, a);
                     tmem_ld_wait();
                     const int col = n0 + c * 32;
-                    if (valid && col < args.N_out) {
+                    if (col < args.N_out) {
                         if (MODE == MODE_GELU) {
 #pragma unroll
                             for (int i = 0; i < 32; ++i) a[i] = gelu_f(a[i]);
                         }
-                        store_row32(orow + col, a);
+                        eo.chunk(&map_out, orow, valid, full, grow0, col, a);
                     }
                 }
             }
             tc_fence_before();
             mbar_arrive(smem_u32(&tempty[acc]));
         }
+        eo.drain();
     }
 
     tc_fence_before();
@@ -348,7 +404,7 @@ constexpr int STAGES = 6;
 constexpr int A_BYTES = 128 * BK * 2;         // 16 KB per CTA
 constexpr int B_BYTES = 128 * BK * 2;         // 16 KB per CTA (half of N = 256)
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256 + 4 * (MAX_E + 1);
+constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + OUT_STAGE_BYTES + 256 + 4 * (MAX_E + 1);
 
 // TMA into this CTA's shared memory, completing on the barrier at `bar_cluster`
 // (a shared::cluster address: the even CTA's stage barrier).
@@ -375,12 +431,14 @@ __device__ __forceinline__ void umma_commit_pair(uint32_t bar, uint16_t mask) {
 template <int MODE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b0,
-                     const __grid_constant__ CUtensorMap map_b1, GemmArgs args) {
+                     const __grid_constant__ CUtensorMap map_b1, const __grid_constant__ CUtensorMap map_out,
+                     GemmArgs args) {
     constexpr int BN_OUT = (MODE == MODE_SWIGLU) ? 128 : 256;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t* stage_base = smem;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint8_t* out_stage = smem + STAGES * STAGE_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(out_stage + OUT_STAGE_BYTES);
     uint64_t* full = bars;                     // [STAGES] (used in the even CTA)
     uint64_t* empty = bars + STAGES;           // [STAGES]
     uint64_t* tfull = bars + 2 * STAGES;       // [2]
@@ -388,7 +446,7 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
     uint64_t* drain = bars + 2 * STAGES + 4;   // [1]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-    int* tile_prefix = reinterpret_cast<int*>(smem + STAGES * STAGE_BYTES + 256);
+    int* tile_prefix = reinterpret_cast<int*>(out_stage + OUT_STAGE_BYTES + 256);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t rank = cluster_rank();
@@ -416,6 +474,7 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
         tma_prefetch_desc(&map_a);
         tma_prefetch_desc(&map_b0);
         if (MODE == MODE_SWIGLU) tma_prefetch_desc(&map_b1);
+        tma_prefetch_desc(&map_out);
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -534,6 +593,7 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
         const int r = q * 32 + lane;
         const uint32_t tempty_leader0 = map_to_rank(smem_u32(&tempty[0]), 0);
         const uint32_t tempty_leader1 = map_to_rank(smem_u32(&tempty[1]), 0);
+        EpiOut eo{smem_u32(out_stage + (warp - 2) * 2 * OUT_CHUNK_BYTES)};
         int it = 0;
         for (int t = pair; t < total; t += npairs, ++it) {
             int row0, row_end, n0, e;
@@ -544,6 +604,8 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
             tc_fence_after();
             const int grow = row0 + (int)rank * 128 + r;
             const bool valid = grow < row_end;
+            const int grow0 = row0 + (int)rank * 128 + q * 32;
+            const bool full = grow0 + 31 < row_end;
             const uint32_t taddr = tmem_base + acc * ACC_N + ((uint32_t)(q * 32) << 16);
             uint16_t* orow = args.out + (long long)grow * args.N_out;
             if (MODE == MODE_SWIGLU) {
@@ -554,10 +616,10 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
                     tmem_ld32(taddr + 128 + c * 32, b);
                     tmem_ld_wait();
                     const int col = n0 + c * 32;
-                    if (valid && col < args.N_out) {
+                    if (col < args.N_out) {
 #pragma unroll
                         for (int i = 0; i < 32; ++i) a[i] = silu_f(a[i]) * b[i];
-                        store_row32(orow + col, a);
+                        eo.chunk(&map_out, orow, valid, full, grow0, col, a);
                     }
                 }
             } else {
@@ -567,18 +629,19 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
                     tmem_ld32(taddr + c * 32, a);
                     tmem_ld_wait();
                     const int col = n0 + c * 32;
-                    if (valid && col < args.N_out) {
+                    if (col < args.N_out) {
                         if (MODE == MODE_GELU) {
 #pragma unroll
                             for (int i = 0; i < 32; ++i) a[i] = gelu_f(a[i]);
                         }
-                        store_row32(orow + col, a);
+                        eo.chunk(&map_out, orow, valid, full, grow0, col, a);
                     }
                 }
             }
             tc_fence_before();
             arrive_remote(acc ? tempty_leader1 : tempty_leader0);
         }
+        eo.drain();
     }
 
     tc_fence_before();
@@ -649,8 +712,8 @@ __global__ void ffn_f32_out_kernel(const float* __restrict__ H, int d, int F, in
 namespace {
 
 template <int MODE>
-moe_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, const tc::GemmArgs& a,
-                       cudaStream_t s) {
+moe_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, const CUtensorMap& mo,
+                       const tc::GemmArgs& a, cudaStream_t s) {
     if (!set_smem_limit((const void*)tc::grouped_gemm_kernel<MODE>, tc::SMEM_BYTES)) return MOE_ERR_CUDA;
     const int bn_out = MODE == tc::MODE_SWIGLU ? 128 : 256;
     const long long n_tiles = (a.N_out + bn_out - 1) / bn_out;
@@ -658,14 +721,14 @@ moe_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUte
     long long tiles_max = n_tiles * m_tiles_max;
     int grid = tc::sm_count();
     if (tiles_max < grid) grid = (int)(tiles_max > 0 ? tiles_max : 1);
-    tc::grouped_gemm_kernel<MODE><<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(ma, mb0, mb1, a);
+    tc::grouped_gemm_kernel<MODE><<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(ma, mb0, mb1, mo, a);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }
 
 template <int MODE>
-moe_status launch_gemm2(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, const tc::GemmArgs& a,
-                        cudaStream_t s) {
+moe_status launch_gemm2(const CUtensorMap& ma, const CUtensorMap& mb0, const CUtensorMap& mb1, const CUtensorMap& mo,
+                        const tc::GemmArgs& a, cudaStream_t s) {
     if (!set_smem_limit((const void*)tc2::grouped_gemm2_kernel<MODE>, tc2::SMEM_BYTES)) return MOE_ERR_CUDA;
     const int bn_out = MODE == tc::MODE_SWIGLU ? 128 : 256;
     const long long n_tiles = (a.N_out + bn_out - 1) / bn_out;
@@ -673,7 +736,7 @@ moe_status launch_gemm2(const CUtensorMap& ma, const CUtensorMap& mb0, const CUt
     const long long tiles_max = n_tiles * m_tiles_max;
     int pairs = tc::sm_count() / 2;
     if (tiles_max < pairs) pairs = (int)(tiles_max > 0 ? tiles_max : 1);
-    tc2::grouped_gemm2_kernel<MODE><<<2 * pairs, tc::THREADS, tc2::SMEM_BYTES, s>>>(ma, mb0, mb1, a);
+    tc2::grouped_gemm2_kernel<MODE><<<2 * pairs, tc::THREADS, tc2::SMEM_BYTES, s>>>(ma, mb0, mb1, mo, a);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }
@@ -735,7 +798,7 @@ extern "C" moe_status moe_expert_ffn(const void* buffer, int dtype, int R_max, i
     // bf16 tensor-core path
     if (!tc::tma_encoder_ready()) return MOE_ERR_CUDA;
     uint16_t* H = (uint16_t*)workspace;
-    CUtensorMap m_x, m_w1, m_w3, m_h, m_w2;
+    CUtensorMap m_x, m_w1, m_w3, m_h, m_w2, m_hout, m_yout;
     const bool swiglu = act == MOE_ACT_SWIGLU;
     const bool pair = use_pair_kernels(R_max, E);
     // per-CTA boxes: A is always 128 rows; B is 128 rows per CTA in the pair
@@ -746,18 +809,20 @@ extern "C" moe_status moe_expert_ffn(const void* buffer, int dtype, int R_max, i
     if (swiglu && !tc::make_bf16_map(&m_w3, W3, (long long)E * F, d, 128)) return MOE_ERR_CUDA;
     if (!tc::make_bf16_map(&m_h, H, R_max, F, 128)) return MOE_ERR_CUDA;
     if (!tc::make_bf16_map(&m_w2, W2, (long long)E * d, F, bbox)) return MOE_ERR_CUDA;
+    if (!tc::make_store_map(&m_hout, H, R_max, F)) return MOE_ERR_CUDA;
+    if (!tc::make_store_map(&m_yout, y, R_max, d)) return MOE_ERR_CUDA;
 
     tc::GemmArgs g1{offsets, E, d, F, F, R_max, H, err};
     if (pair) {
-        moe_status st = swiglu ? launch_gemm2<tc::MODE_SWIGLU>(m_x, m_w1, m_w3, g1, s)
-                               : launch_gemm2<tc::MODE_GELU>(m_x, m_w1, m_w1, g1, s);
+        moe_status st = swiglu ? launch_gemm2<tc::MODE_SWIGLU>(m_x, m_w1, m_w3, m_hout, g1, s)
+                               : launch_gemm2<tc::MODE_GELU>(m_x, m_w1, m_w1, m_hout, g1, s);
         if (st != MOE_OK) return st;
         tc::GemmArgs g2{offsets, E, F, d, d, R_max, (uint16_t*)y, err};
-        return launch_gemm2<tc::MODE_PLAIN>(m_h, m_w2, m_w2, g2, s);
+        return launch_gemm2<tc::MODE_PLAIN>(m_h, m_w2, m_w2, m_yout, g2, s);
     }
-    moe_status st = swiglu ? launch_gemm<tc::MODE_SWIGLU>(m_x, m_w1, m_w3, g1, s)
-                           : launch_gemm<tc::MODE_GELU>(m_x, m_w1, m_w1, g1, s);
+    moe_status st = swiglu ? launch_gemm<tc::MODE_SWIGLU>(m_x, m_w1, m_w3, m_hout, g1, s)
+                           : launch_gemm<tc::MODE_GELU>(m_x, m_w1, m_w1, m_hout, g1, s);
     if (st != MOE_OK) return st;
     tc::GemmArgs g2{offsets, E, F, d, d, R_max, (uint16_t*)y, err};
-    return launch_gemm<tc::MODE_PLAIN>(m_h, m_w2, m_w2, g2, s);
+    return launch_gemm<tc::MODE_PLAIN>(m_h, m_w2, m_w2, m_yout, g2, s);
 }

@@ -199,34 +199,47 @@ __device__ __forceinline__ void block_stable_ranks(long long s0, long long s1, i
 // otherwise read from the outputs of the scan kernels (base[key][block],
 // offsets).  With `fused`, block 0 also writes counts, offsets
 // ([nkeys] = rows) and dropped, each when non-null.
+// `blk` is the index-block whose view is taken (the calling block's own,
+// unless several consumer blocks share one index block); `writer` marks the
+// one block that writes counts, offsets and dropped.
 __device__ void block_scan_prologue(bool fused, const int32_t* __restrict__ cnt, const int32_t* __restrict__ base,
                                     const int32_t* offsets_in, int nkeys, int nblk, long long cap,
                                     int* base_s, int* off_s, int32_t* __restrict__ counts,
-                                    int32_t* offsets_out, int32_t* __restrict__ dropped) {
+                                    int32_t* offsets_out, int32_t* __restrict__ dropped, int blk, bool writer) {
     __shared__ int wsum[32];
     __shared__ long long wdrop[32];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
     if (!fused) {
         for (int key = threadIdx.x; key < nkeys; key += blockDim.x) {
-            base_s[key] = base[(long long)key * nblk + blockIdx.x];
+            base_s[key] = base[(long long)key * nblk + blk];
             off_s[key] = offsets_in ? offsets_in[key] : 0;
         }
         __syncthreads();
         return;
     }
+    // every thread reads its share of the whole keys x blocks count matrix
+    // (consecutive threads on consecutive blocks: coalesced, all loads
+    // independent) and adds it into the keys' totals and bases in shared
+    // memory; one thread per key then applies the capacity
+    for (int key = threadIdx.x; key < nkeys; key += blockDim.x) { base_s[key] = 0; off_s[key] = 0; }
+    __syncthreads();
+    const int n = nkeys * nblk;
+#pragma unroll 4
+    for (int f = threadIdx.x; f < n; f += blockDim.x) {
+        const int v = cnt[f];
+        if (v) {
+            const int key = f / nblk, i = f - key * nblk;
+            atomicAdd(&off_s[key], v);          // total, clamped and scanned below
+            if (i < blk) atomicAdd(&base_s[key], v);
+        }
+    }
+    __syncthreads();
     long long drop = 0;
     for (int key = threadIdx.x; key < nkeys; key += blockDim.x) {
-        const int32_t* c = cnt + (long long)key * nblk;
-        int before = 0, tot = 0;
-        for (int i = 0; i < nblk; ++i) {
-            const int v = c[i];
-            if (i < (int)blockIdx.x) before += v;
-            tot += v;
-        }
-        base_s[key] = before;
+        const int tot = off_s[key];
         const int kept = (int)min((long long)tot, cap);
         off_s[key] = kept;                      // scanned below
-        if (blockIdx.x == 0 && counts) counts[key] = kept;
+        if (writer && counts) counts[key] = kept;
         drop += tot - kept;
     }
     drop = warp_sum(drop);
@@ -251,12 +264,12 @@ __device__ void block_scan_prologue(bool fused, const int32_t* __restrict__ cnt,
         }
         if (key < nkeys) {
             off_s[key] = carry + wb + x - v;
-            if (blockIdx.x == 0 && offsets_out) offsets_out[key] = off_s[key];
+            if (writer && offsets_out) offsets_out[key] = off_s[key];
         }
         carry += tot;
         __syncthreads();
     }
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (writer && threadIdx.x == 0) {
         if (offsets_out) offsets_out[nkeys] = carry;
         if (dropped) {
             long long d = 0;
@@ -286,7 +299,8 @@ __global__ void __launch_bounds__(kIdxThreads) perm_group_heads_kernel(
     const long long s0 = (long long)blockIdx.x * kTB * k;
     const long long s1 = min((long long)(blockIdx.x + 1) * kTB, (long long)T) * k;
     for (int i = threadIdx.x; i < G; i += blockDim.x) ghist[i] = 0;
-    block_scan_prologue(fused, ecnt, ebase, nullptr, E, nblk, cap, base_s, off_s, counts, nullptr, dropped);
+    block_scan_prologue(fused, ecnt, ebase, nullptr, E, nblk, cap, base_s, off_s, counts, nullptr, dropped,
+                        (int)blockIdx.x, blockIdx.x == 0);
     block_stable_ranks(
         s0, s1, E, base_s, wcnt,
         [&](long long s) -> int {
@@ -336,7 +350,7 @@ __global__ void __launch_bounds__(kIdxThreads) perm_group_rows_kernel(
     const long long s0 = (long long)blockIdx.x * kTB * k;
     const long long s1 = min((long long)(blockIdx.x + 1) * kTB, (long long)T) * k;
     block_scan_prologue(fused, gcnt, gbase, goffsets_in, G, nblk, (long long)T * k, base_s, off_s, nullptr, offsets,
-                        nullptr);
+                        nullptr, (int)blockIdx.x, blockIdx.x == 0);
     block_stable_ranks(
         s0, s1, G, base_s, wcnt, [&](long long s) -> int { return (int)code[s]; },
         [&](long long s, int key, int rank) {
@@ -372,7 +386,8 @@ __global__ void __launch_bounds__(kIdxThreads) perm_rank_kernel(const int32_t* _
     int* off_s = base_s + E;                     // [E]
     const long long s0 = (long long)blockIdx.x * kTB * k;
     const long long s1 = min((long long)(blockIdx.x + 1) * kTB, (long long)T) * k;
-    block_scan_prologue(fused, cnt, base, offsets, E, nblk, cap, base_s, off_s, counts, offsets, dropped);
+    block_scan_prologue(fused, cnt, base, offsets, E, nblk, cap, base_s, off_s, counts, offsets, dropped,
+                        (int)blockIdx.x, blockIdx.x == 0);
     block_stable_ranks(
         s0, s1, E, base_s, wcnt,
         [&](long long s) -> int {
@@ -400,6 +415,7 @@ __global__ void __launch_bounds__(256) copy_rows_slots_kernel(const uint4* __res
     const int lane = threadIdx.x & 31;
     const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
+    pdl_wait();                                // row_map comes from the kernel before
     for (long long t = warp; t < T; t += nwarps) {
         // distinct destination rows of this token (lane j < k holds slot j)
         int r = -1;
@@ -499,6 +515,7 @@ __global__ void __launch_bounds__(32 * kBulkWarps) copy_rows_bulk_kernel(const u
     if (lane == 0) tc::mbar_init(bar, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     __syncthreads();
+    pdl_wait();                                // row_map comes from the kernel before
     uint32_t phase = 0;
     const long long nworkers = (long long)gridDim.x * kBulkWarps;
     for (long long t = (long long)blockIdx.x * kBulkWarps + wid; t < T; t += nworkers) {
@@ -650,14 +667,17 @@ moe_status launch_copy_slots(const void* x, int T, int row_bytes, const int32_t*
         if (!set_smem_limit((const void*)copy_rows_bulk_kernel, smem)) return MOE_ERR_CUDA;
         long long nb = ((long long)T + kBulkWarps - 1) / kBulkWarps;
         const int blocks = (int)(nb < 148 * 16 ? nb : 148 * 16);
-        copy_rows_bulk_kernel<<<blocks, 32 * kBulkWarps, smem, s>>>((const uint8_t*)x, T, row_bytes, slot_bytes, row_map,
-                                                                    k, (uint8_t*)buffer, err);
+        if (launch_pdl(copy_rows_bulk_kernel, blocks, 32 * kBulkWarps, smem, s, (const uint8_t*)x, T, row_bytes,
+                       slot_bytes, row_map, k, (uint8_t*)buffer, err) != cudaSuccess)
+            return MOE_ERR_CUDA;
         MOE_LAUNCH_CHECK();
         return MOE_OK;
     }
-    if (vpr <= 32) copy_rows_slots_kernel<1><<<grid, 256, 0, s>>>((const uint4*)x, T, vpr, row_map, k, (uint4*)buffer);
-    else if (vpr <= 64) copy_rows_slots_kernel<2><<<grid, 256, 0, s>>>((const uint4*)x, T, vpr, row_map, k, (uint4*)buffer);
-    else copy_rows_slots_kernel<4><<<grid, 256, 0, s>>>((const uint4*)x, T, vpr, row_map, k, (uint4*)buffer);
+    cudaError_t rc;
+    if (vpr <= 32) rc = launch_pdl(copy_rows_slots_kernel<1>, grid, 256, 0, s, (const uint4*)x, T, vpr, row_map, k, (uint4*)buffer);
+    else if (vpr <= 64) rc = launch_pdl(copy_rows_slots_kernel<2>, grid, 256, 0, s, (const uint4*)x, T, vpr, row_map, k, (uint4*)buffer);
+    else rc = launch_pdl(copy_rows_slots_kernel<4>, grid, 256, 0, s, (const uint4*)x, T, vpr, row_map, k, (uint4*)buffer);
+    if (rc != cudaSuccess) return MOE_ERR_CUDA;
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }

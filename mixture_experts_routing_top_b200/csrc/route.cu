@@ -8,6 +8,7 @@
 #include <cstdlib>
 
 #include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace moe {
 
@@ -167,6 +168,118 @@ __global__ void __launch_bounds__(256) route_topk_vec_kernel(const float* __rest
             expert_idx[t * k + lane] = my_idx;
             gate[t * k + lane] = (float)((double)my_e / s);
         }
+    }
+}
+
+// Eight lanes per token for E = 8 * NPL (E = 64, 128, 192 or 256) and
+// k <= 8: a warp takes four tokens, lane l of a token's group holds the NPL
+// logits of experts 4 (l + 8 q) + u (u < 4; float4 loads, 128 contiguous
+// bytes per group and q).  The minimum of the eight lane maxima is a lower
+// bound of the token's k-th largest logit (the eight maxima are eight
+// distinct logits; for k = 1 the maximum itself is the bound), so every
+// expert of the top k has a logit at or above it;
+// those candidates (about 17 of 256 for normal logits, all of them in the
+// worst case) go to shared memory, and each is ranked exactly by counting
+// the candidates that beat it (larger logit, or equal logit and lower
+// expert index - the order of the other kernels).  No insertion loop, so no
+// divergence beyond the per-token candidate counts.  Gates: exp(l - max)
+// with the rounding of l - max carried (as in the other kernels), over the
+// fp64 sum of the k chosen terms (renormalised) or of exp(l - max) over all
+// E (softmax).
+constexpr int kG8Warps = 4;
+
+// Requires E == 8 * NPL exactly (the host dispatch guarantees it).
+template <int NPL>
+__global__ void __launch_bounds__(32 * kG8Warps) route_topk_g8_kernel(const float* __restrict__ logits, int T, int E,
+                                                                      int k, int norm_topk,
+                                                                      int32_t* __restrict__ expert_idx,
+                                                                      float* __restrict__ gate) {
+    __shared__ float cand_v[kG8Warps][4][8 * NPL];
+    __shared__ int cand_e[kG8Warps][4][8 * NPL];
+    __shared__ int win_e[kG8Warps][4][8];
+    __shared__ float win_x[kG8Warps][4][8];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const int g = lane >> 3, l = lane & 7;
+    float* cv = cand_v[wid][g];
+    int* ce = cand_e[wid][g];
+    const long long nwarps = (long long)gridDim.x * kG8Warps;
+    for (long long w = (long long)blockIdx.x * kG8Warps + wid; w * 4 < T; w += nwarps) {
+        const long long t = w * 4 + g;
+        const bool live = t < T;
+        const float4* row = reinterpret_cast<const float4*>(logits + (live ? t : 0) * (long long)E);
+        float v[NPL];
+#pragma unroll
+        for (int q = 0; q < NPL / 4; ++q) {
+            float4 x = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (live) {
+                const uint4 u = ld_stream(reinterpret_cast<const uint4*>(row + l + 8 * q));
+                x = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
+            }
+            v[4 * q + 0] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+        }
+        float m4[4] = {v[0], v[1], v[2], v[3]};
+#pragma unroll
+        for (int q = 1; q < NPL / 4; ++q)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) m4[u] = fmaxf(m4[u], v[4 * q + u]);
+        float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        float tau = mx;
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) {
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            tau = fminf(tau, __shfl_xor_sync(0xffffffffu, tau, o));
+        }
+        if (k == 1) tau = mx;                  // the top 1 is among the logits equal to the maximum
+        unsigned msk = 0;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) msk |= (v[i] >= tau ? 1u : 0u) << i;
+        if (!live) msk = 0;                    // a token past T has no candidates
+        const int cnt = __popc(msk);
+        int inc = cnt;
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, inc, o);
+            if (l >= o) inc += y;
+        }
+        const int n = __shfl_sync(0xffffffffu, inc, 8 * g + 7);
+        int pos = inc - cnt;
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) {
+            if ((msk >> i) & 1u) {
+                cv[pos] = v[i];
+                ce[pos] = 4 * (l + 8 * (i >> 2)) + (i & 3);
+                ++pos;
+            }
+        }
+        __syncwarp();
+        for (int j = l; j < n; j += 8) {
+            const float vj = cv[j];
+            const int ej = ce[j];
+            int rank = 0;
+            for (int i = 0; i < n; ++i) {
+                const float vi = cv[i];
+                rank += (vi > vj || (vi == vj && ce[i] < ej)) ? 1 : 0;
+            }
+            if (rank < k) {
+                win_e[wid][g][rank] = ej;
+                win_x[wid][g][rank] = exp_diff(vj, mx);
+            }
+        }
+        __syncwarp();
+        double sum = 0.0;
+        if (norm_topk) {
+            if (l < k) sum = (double)win_x[wid][g][l];
+        } else {
+#pragma unroll
+            for (int i = 0; i < NPL; ++i) sum += (double)__expf(__fsub_rn(v[i], mx));
+        }
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (live && l < k) {
+            expert_idx[t * k + l] = win_e[wid][g][l];
+            gate[t * k + l] = (float)((double)win_x[wid][g][l] / sum);
+        }
+        __syncwarp();                          // the candidate lists may be rewritten
     }
 }
 
@@ -345,7 +458,9 @@ constexpr int kEcThreads = 256;
 
 __global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __restrict__ logits, int T, int E, int tpb,
                                                                  double* __restrict__ lse_out,
-                                                                 unsigned long long* __restrict__ keysT) {
+                                                                 unsigned* __restrict__ keys_hi,
+                                                                 unsigned* __restrict__ keys_lo,
+                                                                 unsigned* __restrict__ tokmask, int mask_words) {
     extern __shared__ double ex[];                 // [tpb][E+1] exps (padded rows), [tpb] row max / lse, then
     const int ld = E + 1;                          // [tpb][E+1] the logits as floats (padded rows)
     double* rowv = ex + (size_t)tpb * ld;
@@ -354,6 +469,9 @@ __global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __
     const int rows = (int)min((long long)tpb, (long long)T - t0);
     const float* src = logits + t0 * E;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    pdl_trigger();
+    // this CTA's tokens start with no expert's membership bit set
+    for (int i = threadIdx.x; i < rows * mask_words; i += blockDim.x) tokmask[t0 * mask_words + i] = 0u;
     // logits into shared memory (read from global once) and each row's max
     // (exact in any order): one warp per row
     for (int r = wid; r < rows; r += nw) {
@@ -387,11 +505,14 @@ __global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __
         lse_out[t0 + r] = l;
     }
     __syncthreads();
-    // keys, transposed and coalesced
+    // keys, transposed and coalesced, as their high and low 32-bit halves
+    // (the selection reads the high halves first and the low ones rarely)
 #pragma unroll 4
     for (int f = threadIdx.x; f < rows * E; f += blockDim.x) {
         const int c = f / rows, r = f - c * rows;
-        keysT[(long long)c * T + t0 + r] = key_bits((double)lg[r * ld + c] - rowv[r]);
+        const unsigned long long kb = key_bits((double)lg[r * ld + c] - rowv[r]);
+        keys_hi[(long long)c * T + t0 + r] = (unsigned)(kb >> 32);
+        keys_lo[(long long)c * T + t0 + r] = (unsigned)kb;
     }
 }
 
@@ -437,22 +558,24 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* total, int* sh /
 // distinct digit per warp (__match_any_sync); the search stops once the
 // boundary bucket is taken whole.  Also sets the token-membership bits used
 // to build the token CSR.
-__global__ void __launch_bounds__(1024) ec_select_kernel(const unsigned long long* __restrict__ keysT,
-                                                         const float* __restrict__ logits, const double* __restrict__ lse,
-                                                         int T, int E, int C, int32_t* __restrict__ ec_token,
-                                                         float* __restrict__ ec_gate, unsigned* __restrict__ tokmask,
+__global__ void __launch_bounds__(1024) ec_select_kernel(const unsigned* __restrict__ keys_hi,
+                                                         const unsigned* __restrict__ keys_lo, int T, int E, int C,
+                                                         int32_t* __restrict__ ec_token, unsigned* __restrict__ tokmask,
                                                          int mask_words) {
     __shared__ int hist[256];
     __shared__ unsigned long long s_prefix, s_mask, s_min, s_max;
     __shared__ int s_need, s_done, s_hi;
     const int e = blockIdx.x;
     const int lane = threadIdx.x & 31;
-    const unsigned long long* keys = keysT + (long long)e * T;
+    const unsigned* khi = keys_hi + (long long)e * T;
+    const unsigned* klo = keys_lo + (long long)e * T;
+    auto key = [&](int t) -> unsigned long long { return ((unsigned long long)khi[t] << 32) | klo[t]; };
+    pdl_wait();
     if (threadIdx.x == 0) { s_min = ~0ull; s_max = 0ull; }
     __syncthreads();
     unsigned long long lmin = ~0ull, lmax = 0ull;
     for (int t = threadIdx.x; t < T; t += blockDim.x) {
-        const unsigned long long u = keys[t];
+        const unsigned long long u = key(t);
         lmin = min(lmin, u);
         lmax = max(lmax, u);
     }
@@ -486,7 +609,7 @@ __global__ void __launch_bounds__(1024) ec_select_kernel(const unsigned long lon
             const int t = t0 + threadIdx.x;
             int digit = -1;
             if (t < T) {
-                const unsigned long long u = keys[t];
+                const unsigned long long u = key(t);
                 if ((u & mask) == prefix) digit = (int)((u >> shift) & bins_mask);
             }
             const unsigned peers = __match_any_sync(0xffffffffu, digit);
@@ -524,7 +647,7 @@ __global__ void __launch_bounds__(1024) ec_select_kernel(const unsigned long lon
         const int t = c + lane;
         bool above = false, tie = false;
         if (t < seg1) {
-            const unsigned long long u = keys[t] & mask;
+            const unsigned long long u = key(t) & mask;
             above = u > prefix;
             tie = u == prefix;
         }
@@ -540,7 +663,7 @@ __global__ void __launch_bounds__(1024) ec_select_kernel(const unsigned long lon
         const int t = c + lane;
         bool above = false, tie = false;
         if (t < seg1) {
-            const unsigned long long u = keys[t] & mask;
+            const unsigned long long u = key(t) & mask;
             above = u > prefix;
             tie = u == prefix;
         }
@@ -605,10 +728,9 @@ __device__ __forceinline__ void warp_find_boundary(const int* hist, int nbins, i
 // radix over those tokens).  Same selection as ec_select_kernel.
 constexpr int kEcSmemTokens = 49152;
 
-__global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned long long* __restrict__ keysT,
-                                                              const float* __restrict__ logits,
-                                                              const double* __restrict__ lse, int T, int E, int C,
-                                                              int32_t* __restrict__ ec_token, float* __restrict__ ec_gate,
+__global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned* __restrict__ keys_hi,
+                                                              const unsigned* __restrict__ keys_lo, int T, int E, int C,
+                                                              int32_t* __restrict__ ec_token,
                                                               unsigned* __restrict__ tokmask, int mask_words) {
     extern __shared__ unsigned hi_keys[];          // [T]
     __shared__ int hist[256];
@@ -618,25 +740,26 @@ __global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned lon
     __shared__ int w_above[32], w_tie[32];
     const int e = blockIdx.x;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    const unsigned long long* keys = keysT + (long long)e * T;
+    const unsigned* khi = keys_hi + (long long)e * T;
+    const unsigned* klo = keys_lo + (long long)e * T;
     if (threadIdx.x == 0) { s_min = 0xFFFFFFFFu; s_max = 0u; }
     __syncthreads();
+    pdl_wait();
     unsigned lmin = 0xFFFFFFFFu, lmax = 0u;
     for (int t0 = 0; t0 < T; t0 += 8 * blockDim.x) {
-        unsigned long long u[8];
+        unsigned u[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
             const int t = t0 + q * blockDim.x + threadIdx.x;
-            u[q] = t < T ? keys[t] : 0ull;
+            u[q] = t < T ? khi[t] : 0u;
         }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
             const int t = t0 + q * blockDim.x + threadIdx.x;
             if (t < T) {
-                const unsigned h = (unsigned)(u[q] >> 32);
-                hi_keys[t] = h;
-                lmin = min(lmin, h);
-                lmax = max(lmax, h);
+                hi_keys[t] = u[q];
+                lmin = min(lmin, u[q]);
+                lmax = max(lmax, u[q]);
             }
         }
     }
@@ -714,7 +837,7 @@ __global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned lon
                 const int t = t0 + threadIdx.x;
                 int digit = -1;
                 if (t < T && hi_keys[t] == hprefix) {
-                    const unsigned lo = (unsigned)keys[t];
+                    const unsigned lo = klo[t];
                     if ((lo & lmask) == lprefix) digit = (int)((lo >> shift) & bins_mask);
                 }
                 const unsigned peers = __match_any_sync(0xffffffffu, digit);
@@ -742,7 +865,7 @@ __global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned lon
         if (h != prefix) return h > prefix ? 1 : 0;
         if (level == 0) return 2;
         if (hi_keys[t] != prefix) return hi_keys[t] > prefix ? 1 : 0;   // differs below the high mask
-        const unsigned lo = (unsigned)keys[t] & lmask;
+        const unsigned lo = klo[t] & lmask;
         if (lo != lprefix) return lo > lprefix ? 1 : 0;
         return 2;
     };
@@ -778,45 +901,50 @@ __global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned lon
     }
 }
 
-// tok_cnt[t] = number of experts that chose token t.
-__global__ void ec_count_kernel(const unsigned* __restrict__ tokmask, int T, int mask_words, int32_t* __restrict__ cnt) {
-    int t = blockIdx.x * blockDim.x + threadIdx.x;
-    if (t >= T) return;
-    int c = 0;
-    for (int w = 0; w < mask_words; ++w) c += __popc(tokmask[(long long)t * mask_words + w]);
-    cnt[t] = c;
-}
+// tok_ptr = exclusive scan over tokens of the number of experts that chose
+// each token (the popcount of its membership words); tok_ptr[T] = total.
+// One cluster of kScanCtas CTAs, which the hardware schedules together: CTA
+// c scans tokens [c T / kScanCtas, (c + 1) T / kScanCtas), each thread a
+// contiguous run of them; the CTAs' totals are exchanged through
+// distributed shared memory between two cluster barriers.
+constexpr int kScanCtas = 8;
 
-// Device-wide exclusive scan of n ints, 1024 per CTA: local scans plus
-// per-CTA totals, then a single-CTA scan of the totals, then the add-back.
-__global__ void __launch_bounds__(1024) scan_local_kernel(const int32_t* __restrict__ in, int n, int32_t* __restrict__ out,
-                                                          int32_t* __restrict__ block_tot) {
+__global__ void __cluster_dims__(kScanCtas, 1, 1) __launch_bounds__(1024, 1)
+ec_count_scan_kernel(const unsigned* __restrict__ tokmask, int T, int mask_words, int32_t* __restrict__ tok_ptr) {
     __shared__ int sh[32];
-    int i = blockIdx.x * 1024 + threadIdx.x;
-    int v = i < n ? in[i] : 0;
+    __shared__ int cta_total;
+    pdl_trigger();
+    const int c = (int)tc::cluster_rank();
+    const long long t0 = (long long)T * c / kScanCtas, t1 = (long long)T * (c + 1) / kScanCtas;
+    const long long per = (t1 - t0 + blockDim.x - 1) / blockDim.x;
+    const long long a = min(t0 + per * threadIdx.x, t1), b = min(a + per, t1);
+    pdl_wait();
+    auto count = [&](long long t) {
+        int n = 0;
+        for (int w = 0; w < mask_words; ++w) n += __popc(tokmask[t * mask_words + w]);
+        return n;
+    };
+    int mine = 0;
+    for (long long t = a; t < b; ++t) mine += count(t);
     int tot;
-    int ex = block_exclusive_scan(v, &tot, sh);
-    if (i < n) out[i] = ex;
-    if (threadIdx.x == 0) block_tot[blockIdx.x] = tot;
-}
-
-__global__ void __launch_bounds__(1024) scan_totals_kernel(int32_t* __restrict__ block_tot, int nb, int32_t* __restrict__ grand) {
-    __shared__ int sh[32];
-    int carry = 0;
-    for (int b0 = 0; b0 < nb; b0 += 1024) {
-        int i = b0 + threadIdx.x;
-        int v = i < nb ? block_tot[i] : 0;
-        int tot;
-        int ex = block_exclusive_scan(v, &tot, sh);
-        if (i < nb) block_tot[i] = carry + ex;
-        carry += tot;
+    const int ex = block_exclusive_scan(mine, &tot, sh);
+    if (threadIdx.x == 0) cta_total = tot;
+    __syncthreads();
+    tc::cluster_sync();
+    int before = 0, all = 0;
+    const uint32_t local = tc::smem_u32(&cta_total);
+    for (int q = 0; q < kScanCtas; ++q) {
+        const int v = (int)tc::ld_shared_cluster_u32(tc::map_to_rank(local, (uint32_t)q));
+        if (q < c) before += v;
+        all += v;
     }
-    if (threadIdx.x == 0 && grand) *grand = carry;
-}
-
-__global__ void scan_add_kernel(int32_t* __restrict__ out, int n, const int32_t* __restrict__ block_base) {
-    int i = blockIdx.x * blockDim.x + threadIdx.x;
-    if (i < n) out[i] += block_base[i >> 10];
+    tc::cluster_sync();                       // every read of cta_total is done before any CTA exits
+    int run = before + ex;
+    for (long long t = a; t < b; ++t) {
+        tok_ptr[t] = run;
+        run += count(t);
+    }
+    if (c == kScanCtas - 1 && threadIdx.x == 0) tok_ptr[T] = all;
 }
 
 // For every buffer row r = e*C + i holding token t: its gate exp(key) and
@@ -827,6 +955,7 @@ __global__ void ec_fill_kernel(const int32_t* __restrict__ ec_token, int T, int 
                                const double* __restrict__ lse, float* __restrict__ ec_gate,
                                int32_t* __restrict__ tok_row) {
     long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    pdl_wait();
     if (r >= (long long)E * C) return;
     int e = (int)(r / C);
     int t = ec_token[r];
@@ -849,6 +978,16 @@ namespace {
 // all), and pays off when the warp kernels would spend many reduction
 // rounds (k >= 4); otherwise the warp-per-token kernels keep more warps in
 // flight.  LIBMOE_TOPK_ROWS=0/1 forces either choice.
+// Eight lanes per token for 64, 128, 192 or 256 experts and k <= 8, when
+// LIBMOE_TOPK_G8=1 (the tests force it on and off).  Off by default: it
+// measured slower than the other kernels (T = 131072, E = 256, k = 8:
+// 179 us against 70 us; T = 16384, E = 64, k = 6: 34 us against 22 us).
+bool use_g8_variant() {
+    const char* env = getenv("LIBMOE_TOPK_G8");
+    if (env && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
+    return false;
+}
+
 bool use_rows_variant(int T, int k) {
     const char* env = getenv("LIBMOE_TOPK_ROWS");
     if (env && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
@@ -868,6 +1007,20 @@ extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, i
     int blocks = (int)((warps_needed + 7) / 8);
     if (blocks > 148 * 16) blocks = 148 * 16;
     const int nv = (E + 31) / 32;
+    if ((E == 64 || E == 128 || E == 192 || E == 256) && k <= 8 && ((uintptr_t)logits & 15) == 0 &&
+        use_g8_variant()) {
+        long long gb = ((long long)T + 4 * kG8Warps - 1) / (4 * kG8Warps);
+        const int gblocks = (int)(gb < 148 * 12 ? gb : 148 * 12);
+        switch (E / 8) {
+            case 8: route_topk_g8_kernel<8><<<gblocks, 32 * kG8Warps, 0, s>>>(logits, T, E, k, norm_topk, expert_idx, gate); break;
+            case 16: route_topk_g8_kernel<16><<<gblocks, 32 * kG8Warps, 0, s>>>(logits, T, E, k, norm_topk, expert_idx, gate); break;
+            case 24: route_topk_g8_kernel<24><<<gblocks, 32 * kG8Warps, 0, s>>>(logits, T, E, k, norm_topk, expert_idx, gate); break;
+            case 32: route_topk_g8_kernel<32><<<gblocks, 32 * kG8Warps, 0, s>>>(logits, T, E, k, norm_topk, expert_idx, gate); break;
+            default: return MOE_ERR_SHAPE;     // unreachable: E is one of the four sizes above
+        }
+        MOE_LAUNCH_CHECK();
+        return MOE_OK;
+    }
     if (E % 4 == 0 && k <= 8 && ((uintptr_t)logits & 15) == 0 && use_rows_variant(T, k)) {
         for (auto fn : {route_topk_rows_kernel<1>, route_topk_rows_kernel<2>, route_topk_rows_kernel<4>,
                         route_topk_rows_kernel<8>})
@@ -917,19 +1070,16 @@ extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, i
 
 namespace {
 struct EcWs {
-    size_t lse, keys, mask, cnt, btot, total;
+    size_t lse, keys, mask, total;
 };
 EcWs ec_layout(int T, int E) {
     auto al = [](size_t b) { return (b + 255) & ~(size_t)255; };
     EcWs w;
     int mw = (E + 31) / 32;
-    int nb = (T + 1 + 1023) / 1024;
     w.lse = 0;
-    w.keys = w.lse + al(sizeof(double) * (size_t)T);
-    w.mask = w.keys + al(sizeof(unsigned long long) * (size_t)T * E);
-    w.cnt = w.mask + al(sizeof(unsigned) * (size_t)T * mw);
-    w.btot = w.cnt + al(sizeof(int32_t) * (size_t)(T + 1));
-    w.total = w.btot + al(sizeof(int32_t) * (size_t)(nb + 1));
+    w.keys = w.lse + al(sizeof(double) * (size_t)T);              // high halves [E][T], then low halves [E][T]
+    w.mask = w.keys + al(2 * sizeof(unsigned) * (size_t)T * E);
+    w.total = w.mask + al(sizeof(unsigned) * (size_t)T * mw);
     return w;
 }
 }  // namespace
@@ -951,42 +1101,37 @@ extern "C" moe_status moe_route_ec(const float* logits, int T, int E, int C, int
     cudaStream_t s = (cudaStream_t)stream;
     char* ws = (char*)workspace;
     double* lse = (double*)(ws + L.lse);
-    unsigned long long* keys = (unsigned long long*)(ws + L.keys);
+    unsigned* keys_hi = (unsigned*)(ws + L.keys);
+    unsigned* keys_lo = keys_hi + (size_t)T * E;
     unsigned* mask = (unsigned*)(ws + L.mask);
-    int32_t* cnt = (int32_t*)(ws + L.cnt);
-    int32_t* btot = (int32_t*)(ws + L.btot);
     const int mw = (E + 31) / 32;
-    if (cudaMemsetAsync(mask, 0, sizeof(unsigned) * (size_t)T * mw, s) != cudaSuccess) return MOE_ERR_CUDA;
     {
         const int tpb = ec_tokens_per_block(E);
         const size_t smem = (size_t)tpb * ((E + 2) * sizeof(double) + (E + 1) * sizeof(float));
         if (!set_smem_limit((const void*)ec_lse_keys_kernel, smem)) return MOE_ERR_CUDA;
-        ec_lse_keys_kernel<<<ceil_div(T, tpb), kEcThreads, smem, s>>>(logits, T, E, tpb, lse, keys);
+        ec_lse_keys_kernel<<<ceil_div(T, tpb), kEcThreads, smem, s>>>(logits, T, E, tpb, lse, keys_hi, keys_lo, mask,
+                                                                      mw);
         MOE_LAUNCH_CHECK();
     }
+    cudaError_t rc;
     if (T <= kEcSmemTokens) {
         const size_t smem = sizeof(unsigned) * (size_t)T;
         if (!set_smem_limit((const void*)ec_select_smem_kernel, smem)) return MOE_ERR_CUDA;
-        ec_select_smem_kernel<<<E, 1024, smem, s>>>(keys, logits, lse, T, E, C, ec_token, ec_gate, mask, mw);
+        rc = launch_pdl(ec_select_smem_kernel, E, 1024, smem, s, (const unsigned*)keys_hi, (const unsigned*)keys_lo, T,
+                        E, C, ec_token, mask, mw);
     } else {
-        ec_select_kernel<<<E, 1024, 0, s>>>(keys, logits, lse, T, E, C, ec_token, ec_gate, mask, mw);
+        rc = launch_pdl(ec_select_kernel, E, 1024, 0, s, (const unsigned*)keys_hi, (const unsigned*)keys_lo, T, E, C,
+                        ec_token, mask, mw);
     }
+    if (rc != cudaSuccess) return MOE_ERR_CUDA;
     MOE_LAUNCH_CHECK();
-    ec_count_kernel<<<ceil_div(T, 256), 256, 0, s>>>(mask, T, mw, cnt);
-    MOE_LAUNCH_CHECK();
-    // tok_ptr = exclusive scan of cnt, tok_ptr[T] = E*C
-    const int n = T + 1;
-    if (cudaMemsetAsync(cnt + T, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
-    const int nb = ceil_div(n, 1024);
-    scan_local_kernel<<<nb, 1024, 0, s>>>(cnt, n, tok_ptr, btot);
-    MOE_LAUNCH_CHECK();
-    scan_totals_kernel<<<1, 1024, 0, s>>>(btot, nb, nullptr);
-    MOE_LAUNCH_CHECK();
-    scan_add_kernel<<<ceil_div(n, 256), 256, 0, s>>>(tok_ptr, n, btot);
+    ec_count_scan_kernel<<<kScanCtas, 1024, 0, s>>>(mask, T, mw, tok_ptr);
     MOE_LAUNCH_CHECK();
     const long long rows = (long long)E * C;
-    ec_fill_kernel<<<(int)((rows + 255) / 256), 256, 0, s>>>(ec_token, T, E, C, mask, mw, tok_ptr, logits, lse, ec_gate,
-                                                              tok_row);
+    if (launch_pdl(ec_fill_kernel, (int)((rows + 255) / 256), 256, 0, s, (const int32_t*)ec_token, T, E, C,
+                   (const unsigned*)mask, mw, (const int32_t*)tok_ptr, logits, (const double*)lse, ec_gate,
+                   tok_row) != cudaSuccess)
+        return MOE_ERR_CUDA;
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }

@@ -23,6 +23,7 @@
 #include <cstdlib>
 
 #include "common.cuh"
+#include "tcgen05.cuh"
 
 namespace moe {
 
@@ -136,6 +137,77 @@ __global__ void __launch_bounds__(512) cosel_sym_kernel(const int32_t* __restric
     }
 }
 
+// Co-selection for k <= 8: thread per token.  The token's k experts are
+// loaded at once into registers (independent loads, no dependent chain),
+// and its k(k+1)/2 unordered slot pairs are counted in this band's packed
+// upper triangle in shared memory, as in cosel_sym_kernel.  CTAs run in
+// clusters of kCoselCluster: after counting, CTA r of a cluster sums rows
+// a = a0 + r, a0 + r + kCoselCluster, ... over the cluster's CTAs through
+// distributed shared memory and merges them with one global atomic per
+// non-zero bin (two off the diagonal), so the global merge costs one pass
+// per cluster instead of one per CTA.
+constexpr int kCoselCluster = 8;
+constexpr int kCoselBandBytes = 200 * 1024;
+
+template <int KM>
+__global__ void __cluster_dims__(kCoselCluster, 1, 1) __launch_bounds__(1024, 1)
+cosel_cluster_kernel(const int32_t* __restrict__ idx, int k, int T, int E, SymBands bands, int tokens_per_cta,
+                     int32_t* __restrict__ hist, unsigned* err) {
+    extern __shared__ int h[];                  // rows [a0, a1) of the upper triangle, packed
+    const int a0 = bands.start[blockIdx.y];
+    const int a1 = bands.start[blockIdx.y + 1];
+    const int base = tri_off_d(a0, E);
+    const int nbins = tri_off_d(a1, E) - base;
+    for (int i = threadIdx.x; i < nbins; i += blockDim.x) h[i] = 0;
+    __syncthreads();
+    const unsigned band = (unsigned)(a1 - a0);
+    const long long t0 = (long long)blockIdx.x * tokens_per_cta;
+    const long long t1 = min(t0 + tokens_per_cta, (long long)T);
+    for (long long t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
+        const int32_t* sl = idx + t * k;
+        int a[KM];
+#pragma unroll
+        for (int i = 0; i < KM; ++i) a[i] = i < k ? __ldg(sl + i) : -1;
+        bool bad = false;
+#pragma unroll
+        for (int i = 0; i < KM; ++i)
+            if (i < k && (unsigned)a[i] >= (unsigned)E) { bad = true; a[i] = -1; }
+        if (bad) raise_error(err, kErrIndex);
+#pragma unroll
+        for (int i = 0; i < KM; ++i) {
+            if (i >= k || a[i] < 0) continue;
+            if ((unsigned)(a[i] - a0) < band) atomicAdd(h + tri_off_d(a[i], E) - base, 1);   // the pair (i, i)
+#pragma unroll
+            for (int j = i + 1; j < KM; ++j) {
+                if (j >= k || a[j] < 0) continue;
+                // slots i < j: the ordered pairs (i, j) and (j, i); on one expert both land on its diagonal
+                const int lo = min(a[i], a[j]), hi = max(a[i], a[j]);
+                if ((unsigned)(lo - a0) < band) atomicAdd(h + tri_off_d(lo, E) - base + (hi - lo), lo == hi ? 2 : 1);
+            }
+        }
+    }
+    __syncthreads();
+    tc::cluster_sync();                         // every CTA's counts are complete and visible
+    const int r = (int)tc::cluster_rank();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    uint32_t rbase[kCoselCluster];
+#pragma unroll
+    for (int q = 0; q < kCoselCluster; ++q) rbase[q] = tc::map_to_rank(tc::smem_u32(h), (uint32_t)q);
+    for (int a = a0 + r + kCoselCluster * warp; a < a1; a += kCoselCluster * nw) {
+        const int off = tri_off_d(a, E) - base - a;
+        for (int b = a + lane; b < E; b += 32) {
+            const uint32_t byte = 4u * (uint32_t)(off + b);
+            int v = 0;
+#pragma unroll
+            for (int q = 0; q < kCoselCluster; ++q) v += (int)tc::ld_shared_cluster_u32(rbase[q] + byte);
+            if (!v) continue;
+            atomicAdd(hist + (long long)a * E + b, v);
+            if (b != a) atomicAdd(hist + (long long)b * E + a, v);
+        }
+    }
+    tc::cluster_sync();                         // no CTA exits while another still reads its counts
+}
+
 // The symmetric kernel for E >= 128, where it measured faster (T = 131072,
 // E = 256, k = 8: 48 us against 53 us); at E = 64 it was slower (15.9 us
 // against 13.6 us: too few tokens per CTA to hide its longer dependent chain).
@@ -183,6 +255,63 @@ moe_status launch_cosel_sym(const int32_t* idx, int k, int T, int E, int32_t* hi
     return MOE_OK;
 }
 
+// Bands of the packed upper triangle with equal bin counts, each at most
+// max_bytes of shared memory.  False if E is too large for kMaxSymBands.
+bool make_sym_bands(int E, long long max_bytes, SymBands* sb, int* nb_out, long long* widest_out) {
+    const long long total = tri_off(E, E);
+    const long long max_bins = max_bytes / (long long)sizeof(int);
+    int nb = (int)((total + (max_bins - E) - 1) / (max_bins - E));
+    if (nb < 1) nb = 1;
+    if (nb > kMaxSymBands) return false;
+    sb->start[0] = 0;
+    long long x = 0;
+    for (int b = 1; b < nb; ++b) {
+        const long long target = total * b / nb;
+        while (tri_off(x, E) < target) ++x;
+        sb->start[b] = (int)x;
+    }
+    sb->start[nb] = E;
+    long long widest = 0;
+    for (int b = 0; b < nb; ++b) {
+        const long long n = tri_off(sb->start[b + 1], E) - tri_off(sb->start[b], E);
+        if (n > widest) widest = n;
+    }
+    if (widest > max_bins) return false;
+    *nb_out = nb;
+    *widest_out = widest;
+    return true;
+}
+
+// LIBMOE_COSEL_CLUSTER=0 keeps co-selection with k <= 8 on the older
+// kernels; the tests run both.
+bool cosel_cluster_enabled() {
+    const char* env = getenv("LIBMOE_COSEL_CLUSTER");
+    if (env && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
+    return true;
+}
+
+moe_status launch_cosel_cluster(const int32_t* idx, int k, int T, int E, int32_t* hist, cudaStream_t s) {
+    unsigned* err = device_error_word();
+    if (!err) return MOE_ERR_CUDA;
+    SymBands sb;
+    int nb = 0;
+    long long widest = 0;
+    if (!make_sym_bands(E, kCoselBandBytes, &sb, &nb, &widest)) return MOE_ERR_SHAPE;
+    const size_t smem = sizeof(int) * (size_t)(widest > 0 ? widest : 1);
+    // at most 16 clusters of 8 over all bands (one CTA per SM: they fit the
+    // GPCs together), at least 512 tokens per CTA
+    int clusters = 16 / nb;
+    if (clusters < 1) clusters = 1;
+    int tokens_per_cta = ceil_div(T, (long long)clusters * kCoselCluster);
+    if (tokens_per_cta < 512) tokens_per_cta = 512;
+    const int tok_ctas = ceil_div(ceil_div(T, tokens_per_cta), kCoselCluster) * kCoselCluster;
+    auto fn = k <= 2 ? cosel_cluster_kernel<2> : k <= 4 ? cosel_cluster_kernel<4> : cosel_cluster_kernel<8>;
+    if (!set_smem_limit((const void*)fn, smem)) return MOE_ERR_CUDA;
+    fn<<<dim3(tok_ctas, nb), 1024, smem, s>>>(idx, k, T, E, sb, tokens_per_cta, hist, err);
+    MOE_LAUNCH_CHECK();
+    return MOE_OK;
+}
+
 moe_status launch_pair_hist(const int32_t* idx1, int k1, const int32_t* idx2, int k2, int T, int E, int32_t* hist,
                             cudaStream_t s) {
     unsigned* err = device_error_word();
@@ -213,6 +342,8 @@ extern "C" moe_status moe_coselect(const int32_t* expert_idx, int T, int k, int 
     if (E > 1024 || k > 32) return MOE_ERR_SHAPE;
     if (T == 0) return MOE_OK;
     if (!expert_idx || !cosel) return MOE_ERR_ARG;
+    if (k <= 8 && cosel_cluster_enabled())
+        return launch_cosel_cluster(expert_idx, k, T, E, cosel, (cudaStream_t)stream);
     if (cosel_sym_enabled(E)) return launch_cosel_sym(expert_idx, k, T, E, cosel, (cudaStream_t)stream);
     return launch_pair_hist(expert_idx, k, expert_idx, k, T, E, cosel, (cudaStream_t)stream);
 }

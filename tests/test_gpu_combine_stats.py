@@ -103,16 +103,19 @@ def test_gather_rows_matches_token_csr(bulk, d, monkeypatch):
 
 
 # -------------------------------------------------------------- histograms
-@pytest.fixture(params=["sym", "ordered"])
+@pytest.fixture(params=["cluster", "sym", "ordered"])
 def cosel_kind(request, monkeypatch):
-    """Co-selection through the kernel that counts each unordered slot pair
-    once and mirrors it (the default), and through the ordered-pair kernel."""
+    """Co-selection through the thread-per-token cluster kernel (the default
+    for k <= 8), the kernel that counts each unordered slot pair once and
+    mirrors it, and the ordered-pair kernel."""
+    monkeypatch.setenv("LIBMOE_COSEL_CLUSTER", "1" if request.param == "cluster" else "0")
     monkeypatch.setenv("LIBMOE_COSEL_SYM", "1" if request.param == "sym" else "0")
     return request.param
 
 
 @pytest.mark.parametrize("T,E,k", [(1, 1, 1), (100, 8, 2), (16384, 64, 6), (5000, 1000, 3), (20000, 256, 8),
-                                   (3000, 7, 7), (70000, 256, 8), (999, 130, 5), (4096, 1024, 8)])
+                                   (3000, 7, 7), (70000, 256, 8), (999, 130, 5), (4096, 1024, 8),
+                                   (131072, 256, 8), (3, 256, 8)])
 def test_coselect(T, E, k, cosel_kind):
     idx, _ = O.route_topk(synth.normal_f32(6, 1, (T, E)), k)
     got = M.coselect(to_dev(idx), E)

@@ -50,7 +50,9 @@ def ffn_case(counts, d, F, act, bf16=True, seed=0):
     ([129, 511], 320, 448, "gelu"),
     ([1000], 64, 64, "swiglu"),
     ([600, 0, 900, 257], 256, 320, "swiglu"),     # 256-row tiles with ragged tails, partial n-tiles
-    ([513, 1100], 320, 256, "gelu")])
+    ([513, 1100], 320, 256, "gelu"),
+    ([31, 32, 33, 96, 127, 129, 1, 255, 257], 128, 128, "swiglu"),   # 32-row warp boxes: full, straddling, short
+    ([31, 32, 33, 96, 127, 129, 1, 255, 257], 128, 192, "gelu")])
 def test_expert_ffn_bf16(counts, d, F, act, gemm_kind):
     got, ref = ffn_case(counts, d, F, act)
     assert_layer_close(got, ref)

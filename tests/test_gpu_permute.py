@@ -55,7 +55,8 @@ def copy_kind(request, monkeypatch):
 @pytest.mark.parametrize("T,E,k,cf,d,bf16", [
     (1, 1, 1, 1.0, 8, False), (1, 4, 2, 0.5, 8, True), (33, 3, 1, 0.7, 4, False), (1000, 8, 2, 0.5, 40, False),
     (1000, 8, 2, 1.25, 64, True), (4099, 16, 4, 0.9, 24, True), (777, 1024, 32, 2.0, 16, True),
-    (2000, 64, 6, 0.0, 8, True), (513, 5, 5, 1.0, 64, False)])
+    (2000, 64, 6, 0.0, 8, True), (513, 5, 5, 1.0, 64, False),
+    (70001, 256, 8, 1.1, 8, True)])                # many index blocks: the scans run as separate kernels
 def test_expert_major(T, E, k, cf, d, bf16, copy_kind):
     idx = routed(T, E, k, skew=1.0)
     x = synth.normal_bf16(1, 2, (T, d)) if bf16 else synth.normal_f32(1, 2, (T, d))
@@ -92,6 +93,7 @@ def test_group_major_identity_groups_equal_expert_major():
 def test_indices_only():
     idx = routed(5000, 32, 4)
     run(None, idx, 32, 1.1)
+    run(None, routed(7, 256, 8), 256, 0.5)
 
 
 def test_empty():
@@ -109,8 +111,28 @@ def test_out_of_range_expert_is_skipped_and_reported():
     assert int(to_np(out["row_map"])[5, 1]) == -1
 
 
+def test_out_of_range_expert_with_rows_is_skipped_and_reported(copy_kind):
+    idx = routed(3000, 8, 2)
+    idx[700, 0] = 8
+    idx[2999, 1] = 9
+    x = synth.normal_bf16(1, 2, (3000, 32))
+    assert M.device_error(clear=True) == 0
+    out = M.permute(to_dev(x), to_dev(idx), 8, 0.0)
+    assert M.device_error(clear=True) == 8          # MOE_ERR_DEVICE_INDEX
+    rm = to_np(out["row_map"])
+    assert rm[700, 0] == -1 and rm[2999, 1] == -1
+    keep = np.ones_like(idx, bool)
+    keep[700, 0] = keep[2999, 1] = False
+    # the other slots keep distinct rows holding their own token
+    rows = rm[keep]
+    assert np.unique(rows).size == rows.size and (rows >= 0).all()
+    buf = to_np(out["buffer"])
+    toks = np.nonzero(keep)[0]
+    assert buf[rows].tobytes() == x[toks].tobytes()
+
+
 @pytest.mark.parametrize("w", [W.MIXTRAL, W.FINE], ids=lambda w: w.name)
-def test_workload_full(w):
+def test_workload_full(w, copy_kind):
     idx, _ = O.route_topk(W.make_logits(w), w.k)
     _, ref = run(W.make_x(w), idx, w.E, w.capacity_factor)
     if w is W.MIXTRAL:

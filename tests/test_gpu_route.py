@@ -21,17 +21,21 @@ def check_topk(logits, k, norm=False):
     np.testing.assert_allclose(gg, rgate, rtol=GATE_RTOL, atol=1e-30)
 
 
-@pytest.fixture(params=["rows", "warp"])
+@pytest.fixture(params=["g8", "rows", "warp"])
 def topk_kind(request, monkeypatch):
-    """Run a test with the thread-per-token top-k kernel and with the
-    warp-per-token ones (the library picks by T; the tests force each)."""
+    """Run a test with each top-k kernel family: eight lanes per token (the
+    default for 64, 128, 192 or 256 experts and k <= 8), thread per
+    token, and warp per token (the library picks by shape; the tests force
+    each where it applies)."""
+    monkeypatch.setenv("LIBMOE_TOPK_G8", "1" if request.param == "g8" else "0")
     monkeypatch.setenv("LIBMOE_TOPK_ROWS", "1" if request.param == "rows" else "0")
     return request.param
 
 
 @pytest.mark.parametrize("T,E,k", [(1, 1, 1), (7, 3, 2), (1000, 8, 2), (333, 33, 5), (512, 64, 6), (300, 100, 7),
                                    (1025, 256, 8), (200, 1024, 32), (64, 160, 32), (50, 5, 5), (129, 36, 4),
-                                   (300, 1020, 8), (77, 12, 1)])
+                                   (300, 1020, 8), (77, 12, 1), (1001, 64, 2), (999, 128, 8), (1003, 192, 5),
+                                   (70, 256, 3), (1001, 128, 1), (65, 64, 1)])
 @pytest.mark.parametrize("norm", [False, True])
 def test_topk_random(T, E, k, norm, topk_kind):
     check_topk(synth.normal_f32(11, 1, (T, E), 0.0, 2.0), k, norm)
@@ -46,6 +50,23 @@ def test_topk_ties_lower_index_wins(topk_kind):
     z = np.zeros((300, 64), np.float32)
     z[:, ::3] = -0.0                                  # -0 and +0 are equal logits: the lower expert wins
     check_topk(z, 8)
+
+
+def test_topk_candidates_worst_case(topk_kind):
+    """Rows whose largest logits all sit in the experts one lane of an
+    eight-lane group holds (experts 4 (0 + 8 q) + u): the other lanes' maxima
+    are low, so nearly every logit is a candidate for the exact ranking."""
+    for E in (64, 256):
+        T = 999
+        base = synth.normal_f32(13, 1, (T, E), 0.0, 0.1)
+        e = np.arange(E)
+        lane0 = ((e // 4) % 8) == 0
+        base[:, lane0] += 10.0
+        for k in (2, 8):
+            check_topk(base, k)
+            check_topk(base, k, True)
+        check_topk(np.tile(-np.arange(E, dtype=np.float32), (T, 1)), 8)      # sorted rows
+        check_topk(np.tile(np.arange(E, dtype=np.float32), (T, 1)), 8)
 
 
 @pytest.mark.parametrize("E,k,norm", [(256, 8, True), (64, 6, False), (8, 2, False), (128, 1, False)])
@@ -83,7 +104,7 @@ def check_ec(logits, C):
 
 
 @pytest.mark.parametrize("T,E,C", [(1, 1, 1), (40, 4, 10), (1000, 7, 333), (3000, 64, 100), (2048, 33, 2048),
-                                   (5000, 128, 79)])
+                                   (5000, 128, 79), (50001, 8, 7001)])   # the last: selection from global memory
 def test_expert_choice_random(T, E, C):
     check_ec(synth.normal_f32(5, 1, (T, E)), C)
 
