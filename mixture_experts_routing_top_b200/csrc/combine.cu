@@ -125,6 +125,8 @@ __global__ void __launch_bounds__(256) unpermute_vec_kernel(const void* __restri
                                                             const float* __restrict__ gate,
                                                             const void* __restrict__ shared, void* __restrict__ out,
                                                             unsigned* err) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     const int lane = threadIdx.x & 31;
     const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
@@ -278,6 +280,8 @@ __global__ void __launch_bounds__(32 * kCmbWarps) unpermute_bulk_kernel(const ui
                                                                         const uint8_t* __restrict__ shared,
                                                                         void* __restrict__ out, unsigned* err,
                                                                         CsrRows csr) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     extern __shared__ __align__(128) uint8_t cmb_smem[];
     __shared__ __align__(8) uint64_t bars[kCmbWarps][2];
     __shared__ int no_abort;
@@ -403,6 +407,8 @@ __global__ void __launch_bounds__(256) unpermute_scalar_kernel(const void* __res
                                                                const float* __restrict__ gate,
                                                                const void* __restrict__ shared, void* __restrict__ out,
                                                                bool out_bf16, unsigned* err) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     const int lane = threadIdx.x & 31;
     const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
@@ -433,6 +439,8 @@ __global__ void __launch_bounds__(256) unpermute_ec_vec_kernel(const void* __res
                                                                const int32_t* __restrict__ tok_row,
                                                                const float* __restrict__ ec_gate,
                                                                void* __restrict__ out, unsigned* err) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     const int lane = threadIdx.x & 31;
     const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
@@ -498,6 +506,8 @@ __global__ void __launch_bounds__(256) unpermute_ec_scalar_kernel(const void* __
                                                                   const int32_t* __restrict__ tok_row,
                                                                   const float* __restrict__ ec_gate,
                                                                   void* __restrict__ out, bool out_bf16, unsigned* err) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     const int lane = threadIdx.x & 31;
     const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
@@ -692,13 +702,13 @@ moe_status launch_unpermute_bulk(bool in_bf16, bool out_bf16, cudaStream_t s, co
     const uint8_t* yb = (const uint8_t*)y;
     const uint8_t* sb = (const uint8_t*)shared;
     if (in_bf16 && out_bf16)
-        unpermute_bulk_kernel<true, true, UNIT, CSR><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err, csr);
+        (void)launch_pdl(unpermute_bulk_kernel<true, true, UNIT, CSR>, blocks, 32 * kCmbWarps, kCmbSmem, s, yb, R, T, d, k, row_map, gate, sb, out, err, csr);
     else if (in_bf16)
-        unpermute_bulk_kernel<true, false, UNIT, CSR><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err, csr);
+        (void)launch_pdl(unpermute_bulk_kernel<true, false, UNIT, CSR>, blocks, 32 * kCmbWarps, kCmbSmem, s, yb, R, T, d, k, row_map, gate, sb, out, err, csr);
     else if (out_bf16)
-        unpermute_bulk_kernel<false, true, UNIT, CSR><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err, csr);
+        (void)launch_pdl(unpermute_bulk_kernel<false, true, UNIT, CSR>, blocks, 32 * kCmbWarps, kCmbSmem, s, yb, R, T, d, k, row_map, gate, sb, out, err, csr);
     else
-        unpermute_bulk_kernel<false, false, UNIT, CSR><<<blocks, 32 * kCmbWarps, kCmbSmem, s>>>(yb, R, T, d, k, row_map, gate, sb, out, err, csr);
+        (void)launch_pdl(unpermute_bulk_kernel<false, false, UNIT, CSR>, blocks, 32 * kCmbWarps, kCmbSmem, s, yb, R, T, d, k, row_map, gate, sb, out, err, csr);
     return MOE_OK;
 }
 
@@ -712,13 +722,18 @@ bool bulk_combine_ec_enabled() {
     return false;
 }
 
-// The bulk-staged combine pays off when a token has several rows to gather
-// (k >= 4); with one or two rows per token its per-chunk waits are exposed
-// and the register kernel is faster.  LIBMOE_BULK_COMBINE=0/1 forces either.
-bool bulk_combine_enabled(int k) {
+// The token combine (gate-weighted rows) runs on the register kernel, which
+// keeps two rows' loads in flight per warp: it measured faster than the
+// bulk-staged kernel at every shape timed (k = 2: 34 vs 44 us; clustered
+// top-6 with the shared row: 91 vs 116 us; top-8 group rows, T = 4096:
+// 68 vs 85 us, T = 131072: 1857 vs 1894 us).  The unit-weight sum of a
+// token's group rows (moe_unpermute_groups) stays on the bulk kernel, which
+// is faster there (83 vs 103 us at the clustered top-6 workload, G = 8).
+// LIBMOE_BULK_COMBINE=0/1 forces either kernel for both calls.
+bool bulk_combine_enabled(bool unit) {
     const char* env = getenv("LIBMOE_BULK_COMBINE");
     if (env && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
-    return k >= 4;
+    return unit;
 }
 
 int token_grid(long long T) {
@@ -735,10 +750,10 @@ using namespace moe;
 
 #define MOE_DISPATCH_VEC(KERNEL, NV, ...)                                                       \
     do {                                                                                        \
-        if (in_bf16 && out_bf16) KERNEL<true, true, NV><<<grid, 256, 0, s>>>(__VA_ARGS__);      \
-        else if (in_bf16) KERNEL<true, false, NV><<<grid, 256, 0, s>>>(__VA_ARGS__);            \
-        else if (out_bf16) KERNEL<false, true, NV><<<grid, 256, 0, s>>>(__VA_ARGS__);           \
-        else KERNEL<false, false, NV><<<grid, 256, 0, s>>>(__VA_ARGS__);                        \
+        if (in_bf16 && out_bf16) (void)launch_pdl(KERNEL<true, true, NV>, grid, 256, 0, s, __VA_ARGS__);   \
+        else if (in_bf16) (void)launch_pdl(KERNEL<true, false, NV>, grid, 256, 0, s, __VA_ARGS__);         \
+        else if (out_bf16) (void)launch_pdl(KERNEL<false, true, NV>, grid, 256, 0, s, __VA_ARGS__);        \
+        else (void)launch_pdl(KERNEL<false, false, NV>, grid, 256, 0, s, __VA_ARGS__);                     \
     } while (0)
 
 extern "C" moe_status moe_unpermute(const void* y, int dtype, int R, int T, int d, int k, const int32_t* row_map,
@@ -757,7 +772,7 @@ extern "C" moe_status moe_unpermute(const void* y, int dtype, int R, int T, int 
     const int in_esz = in_bf16 ? 2 : 4, out_esz = out_bf16 ? 2 : 4;
     const bool vec = (d % 8 == 0) && ((d * in_esz) % 16 == 0) && ((d * out_esz) % 16 == 0) &&
                      (y == nullptr || aligned16(y)) && aligned16(out) && (shared == nullptr || aligned16(shared));
-    if (vec && k <= 8 && bulk_combine_enabled(k)) {
+    if (vec && k <= 8 && bulk_combine_enabled(false)) {
         const moe_status st = launch_unpermute_bulk<false, false>(in_bf16, out_bf16, s, y, R, T, d, k, row_map, gate,
                                                                   shared, out, err);
         if (st != MOE_OK) return st;
@@ -769,7 +784,7 @@ extern "C" moe_status moe_unpermute(const void* y, int dtype, int R, int T, int 
         if (nvec <= 32) MOE_DISPATCH_VEC(unpermute_vec_kernel, 1, y, R, T, d, k, row_map, gate, shared, out, err);
         else MOE_DISPATCH_VEC(unpermute_vec_kernel, 2, y, R, T, d, k, row_map, gate, shared, out, err);
     } else {
-        unpermute_scalar_kernel<<<grid, 256, 0, s>>>(y, in_bf16, R, T, d, k, row_map, gate, shared, out, out_bf16, err);
+        (void)launch_pdl(unpermute_scalar_kernel, grid, 256, 0, s, y, in_bf16, R, T, d, k, row_map, gate, shared, out, out_bf16, err);
     }
     MOE_LAUNCH_CHECK();
     return MOE_OK;
@@ -799,7 +814,7 @@ extern "C" moe_status moe_unpermute_ec(const void* y, int dtype, int R, int T, i
         if (nvec <= 32) MOE_DISPATCH_VEC(unpermute_ec_vec_kernel, 1, y, R, T, d, tok_ptr, tok_row, ec_gate, out, err);
         else MOE_DISPATCH_VEC(unpermute_ec_vec_kernel, 2, y, R, T, d, tok_ptr, tok_row, ec_gate, out, err);
     } else {
-        unpermute_ec_scalar_kernel<<<grid, 256, 0, s>>>(y, in_bf16, R, T, d, tok_ptr, tok_row, ec_gate, out, out_bf16, err);
+        (void)launch_pdl(unpermute_ec_scalar_kernel, grid, 256, 0, s, y, in_bf16, R, T, d, tok_ptr, tok_row, ec_gate, out, out_bf16, err);
     }
     MOE_LAUNCH_CHECK();
     return MOE_OK;
@@ -870,7 +885,7 @@ extern "C" moe_status moe_unpermute_groups(const void* y_g, int dtype, int R_g, 
     cudaStream_t s = (cudaStream_t)stream;
     unsigned* err = device_error_word();
     if (!err) return MOE_ERR_CUDA;
-    if (k <= 8 && bulk_combine_enabled(k)) {
+    if (k <= 8 && bulk_combine_enabled(true)) {
         const moe_status st = launch_unpermute_bulk<true, false>(in_bf16, out_bf16, s, y_g, R_g, T, d, k, row_map_g,
                                                                  nullptr, shared, out, err);
         if (st != MOE_OK) return st;

@@ -166,6 +166,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                                                                   const __grid_constant__ CUtensorMap map_b1,
                                                                   const __grid_constant__ CUtensorMap map_out,
                                                                   GemmArgs args) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
     constexpr int BN_OUT = (MODE == MODE_SWIGLU) ? 128 : 256;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -211,6 +212,7 @@ __global__ void __launch_bounds__(THREADS, 1) grouped_gemm_kernel(const __grid_c
                      :: "r"(smem_u32(tmem_slot)), "r"(2 * ACC_N) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    pdl_wait();                       // the offsets and operands come from the kernels before
     if (warp == 2 && lane == 0) {
         int acc = 0;
         tile_prefix[0] = 0;
@@ -433,6 +435,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b0,
                      const __grid_constant__ CUtensorMap map_b1, const __grid_constant__ CUtensorMap map_out,
                      GemmArgs args) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
     constexpr int BN_OUT = (MODE == MODE_SWIGLU) ? 128 : 256;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -481,6 +484,7 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
                      :: "r"(smem_u32(tmem_slot)), "r"(2 * ACC_N) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
+    pdl_wait();                       // the offsets and operands come from the kernels before
     if (warp == 2 && lane == 0) {
         int acc = 0;
         tile_prefix[0] = 0;
@@ -721,7 +725,7 @@ moe_status launch_gemm(const CUtensorMap& ma, const CUtensorMap& mb0, const CUte
     long long tiles_max = n_tiles * m_tiles_max;
     int grid = tc::sm_count();
     if (tiles_max < grid) grid = (int)(tiles_max > 0 ? tiles_max : 1);
-    tc::grouped_gemm_kernel<MODE><<<grid, tc::THREADS, tc::SMEM_BYTES, s>>>(ma, mb0, mb1, mo, a);
+    (void)launch_pdl(tc::grouped_gemm_kernel<MODE>, grid, tc::THREADS, tc::SMEM_BYTES, s, ma, mb0, mb1, mo, a);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }
@@ -736,7 +740,7 @@ moe_status launch_gemm2(const CUtensorMap& ma, const CUtensorMap& mb0, const CUt
     const long long tiles_max = n_tiles * m_tiles_max;
     int pairs = tc::sm_count() / 2;
     if (tiles_max < pairs) pairs = (int)(tiles_max > 0 ? tiles_max : 1);
-    tc2::grouped_gemm2_kernel<MODE><<<2 * pairs, tc::THREADS, tc2::SMEM_BYTES, s>>>(ma, mb0, mb1, mo, a);
+    (void)launch_pdl(tc2::grouped_gemm2_kernel<MODE>, 2 * pairs, tc::THREADS, tc2::SMEM_BYTES, s, ma, mb0, mb1, mo, a);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }

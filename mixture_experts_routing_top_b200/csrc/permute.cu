@@ -42,6 +42,8 @@ constexpr int kIdxThreads = 256;
 // 1. per-block histogram of experts, stored expert-major: cnt[e * nblk + b]
 __global__ void __launch_bounds__(kIdxThreads) perm_count_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
                                                                  int nblk, int32_t* __restrict__ cnt, unsigned* err) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     extern __shared__ int hist[];
     for (int i = threadIdx.x; i < E; i += blockDim.x) hist[i] = 0;
     __syncthreads();
@@ -59,6 +61,8 @@ __global__ void __launch_bounds__(kIdxThreads) perm_count_kernel(const int32_t* 
 // 2. one CTA per key: exclusive scan over the blocks, total per key.
 __global__ void __launch_bounds__(1024) perm_scan_blocks_kernel(const int32_t* __restrict__ cnt, int nblk,
                                                                 int32_t* __restrict__ base, int32_t* __restrict__ total) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     __shared__ int sh[32];
     const int key = blockIdx.x;
     const int32_t* c = cnt + (long long)key * nblk;
@@ -98,6 +102,8 @@ __global__ void __launch_bounds__(1024) perm_scan_blocks_kernel(const int32_t* _
 __global__ void __launch_bounds__(1024) perm_offsets_kernel(const int32_t* __restrict__ total, int nkeys,
                                                             long long cap, int32_t* __restrict__ counts,
                                                             int32_t* __restrict__ offsets, int32_t* __restrict__ dropped) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     __shared__ int sh[32];
     __shared__ long long sdrop[32];
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -290,6 +296,8 @@ __global__ void __launch_bounds__(kIdxThreads) perm_group_heads_kernel(
     const int32_t* __restrict__ idx, const int32_t* __restrict__ goe, int T, int k, int E, int G, int nblk, int fused,
     const int32_t* __restrict__ ecnt, const int32_t* __restrict__ ebase, long long cap, int32_t* __restrict__ counts,
     int32_t* __restrict__ dropped, int16_t* __restrict__ code, int32_t* __restrict__ gcnt, unsigned* err) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     extern __shared__ int sm[];
     int* wcnt = sm;                                          // [8][E]
     int* base_s = wcnt + (kIdxThreads / 32) * E;             // [E]
@@ -342,6 +350,8 @@ __global__ void __launch_bounds__(kIdxThreads) perm_group_rows_kernel(
     const int16_t* __restrict__ code, int T, int k, int G, int nblk, int fused, const int32_t* __restrict__ gcnt,
     const int32_t* __restrict__ gbase, const int32_t* __restrict__ goffsets_in, int32_t* __restrict__ offsets,
     int32_t* __restrict__ row_map, int32_t* __restrict__ row_token) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     extern __shared__ int sm[];
     int* wcnt = sm;                                          // [8][G]
     int* base_s = wcnt + (kIdxThreads / 32) * G;             // [G]
@@ -380,6 +390,8 @@ __global__ void __launch_bounds__(kIdxThreads) perm_rank_kernel(const int32_t* _
                                                                 int32_t* __restrict__ dropped,
                                                                 int32_t* __restrict__ row_map,
                                                                 int32_t* __restrict__ row_token, unsigned* err) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     extern __shared__ int sm[];
     int* wcnt = sm;                              // [8][E]
     int* base_s = wcnt + (kIdxThreads / 32) * E; // [E]
@@ -753,24 +765,29 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
     int32_t* total = (int32_t*)(ws + L.total);
     const int nw = kIdxThreads / 32;
     // 1. per-block expert counts
-    perm_count_kernel<<<nblk, kIdxThreads, sizeof(int) * E, s>>>(expert_idx, T, k, E, nblk, cnt, err);
+    if (launch_pdl(perm_count_kernel, nblk, kIdxThreads, sizeof(int) * E, s, expert_idx, T, k, E, nblk, cnt, err) != cudaSuccess)
+        return MOE_ERR_CUDA;
     MOE_LAUNCH_CHECK();
     // 2-3. the scans: done by every consumer block itself when experts x
     // blocks is small, else by two kernels
     const int fused_e = (long long)E * nblk <= kFuseLimit;
     int32_t* eoffsets = group_of_expert ? nullptr : offsets;
     if (!fused_e) {
-        perm_scan_blocks_kernel<<<E, 1024, 0, s>>>(cnt, nblk, base, total);
+        if (launch_pdl(perm_scan_blocks_kernel, E, 1024, 0, s, (const int32_t*)cnt, nblk, base, total) != cudaSuccess)
+            return MOE_ERR_CUDA;
         MOE_LAUNCH_CHECK();
-        perm_offsets_kernel<<<1, 1024, 0, s>>>(total, E, cap, counts, eoffsets, dropped);
+        if (launch_pdl(perm_offsets_kernel, 1, 1024, 0, s, (const int32_t*)total, E, cap, counts, eoffsets, dropped) != cudaSuccess)
+            return MOE_ERR_CUDA;
         MOE_LAUNCH_CHECK();
     }
     if (!group_of_expert) {
         // 4. ranks and rows (its block 0 writes counts, offsets and dropped when fused)
         const size_t rank_smem = sizeof(int) * ((size_t)nw * E + 2 * (size_t)E);
         if (!set_smem_limit((const void*)perm_rank_kernel, rank_smem)) return MOE_ERR_CUDA;
-        perm_rank_kernel<<<nblk, kIdxThreads, rank_smem, s>>>(expert_idx, T, k, E, nblk, fused_e, cnt, base, cap,
-                                                              counts, offsets, dropped, row_map, row_token, err);
+        if (launch_pdl(perm_rank_kernel, nblk, kIdxThreads, rank_smem, s, expert_idx, T, k, E, nblk, fused_e,
+                       (const int32_t*)cnt, (const int32_t*)base, cap, counts, offsets, dropped, row_map, row_token,
+                       err) != cudaSuccess)
+            return MOE_ERR_CUDA;
         MOE_LAUNCH_CHECK();
     } else {
         int16_t* code = (int16_t*)(ws + L.code);
@@ -779,21 +796,26 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
         int32_t* gtotal = (int32_t*)(ws + L.gtotal);
         const size_t heads_smem = sizeof(int) * ((size_t)nw * E + 2 * (size_t)E + G) + (size_t)kTB * k;
         if (!set_smem_limit((const void*)perm_group_heads_kernel, heads_smem)) return MOE_ERR_CUDA;
-        perm_group_heads_kernel<<<nblk, kIdxThreads, heads_smem, s>>>(expert_idx, group_of_expert, T, k, E, G, nblk,
+        if (launch_pdl(perm_group_heads_kernel, nblk, kIdxThreads, heads_smem, s, expert_idx, group_of_expert, T, k, E, G, nblk,
                                                                         fused_e, cnt, base, cap, counts, dropped, code,
-                                                                        gcnt, err);
+                                                                        gcnt, err) != cudaSuccess)
+            return MOE_ERR_CUDA;
         MOE_LAUNCH_CHECK();
         const int fused_g = (long long)G * nblk <= kFuseLimit;
         if (!fused_g) {
-            perm_scan_blocks_kernel<<<G, 1024, 0, s>>>(gcnt, nblk, gbase, gtotal);
+            if (launch_pdl(perm_scan_blocks_kernel, G, 1024, 0, s, (const int32_t*)gcnt, nblk, gbase, gtotal) != cudaSuccess)
+                return MOE_ERR_CUDA;
             MOE_LAUNCH_CHECK();
-            perm_offsets_kernel<<<1, 1024, 0, s>>>(gtotal, G, (long long)T * k, nullptr, offsets, nullptr);
+            if (launch_pdl(perm_offsets_kernel, 1, 1024, 0, s, (const int32_t*)gtotal, G, (long long)T * k, (int32_t*)nullptr,
+                           offsets, (int32_t*)nullptr) != cudaSuccess)
+                return MOE_ERR_CUDA;
             MOE_LAUNCH_CHECK();
         }
         const size_t rows_smem = sizeof(int) * ((size_t)nw * G + 2 * (size_t)G + (size_t)kTB * k);
         if (!set_smem_limit((const void*)perm_group_rows_kernel, rows_smem)) return MOE_ERR_CUDA;
-        perm_group_rows_kernel<<<nblk, kIdxThreads, rows_smem, s>>>(code, T, k, G, nblk, fused_g, gcnt, gbase, offsets,
-                                                                      offsets, row_map, row_token);
+        if (launch_pdl(perm_group_rows_kernel, nblk, kIdxThreads, rows_smem, s, code, T, k, G, nblk, fused_g, gcnt, gbase, offsets,
+                                                                      offsets, row_map, row_token) != cudaSuccess)
+            return MOE_ERR_CUDA;
         MOE_LAUNCH_CHECK();
     }
     if (x && d > 0) return launch_copy_slots(x, T, (int)row_bytes, row_map, k, buffer, s);

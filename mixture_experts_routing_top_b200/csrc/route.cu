@@ -24,6 +24,8 @@ template <int NV>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                          int norm_topk, int32_t* __restrict__ expert_idx,
                                                          float* __restrict__ gate) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     const int lane = threadIdx.x & 31;
     const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
@@ -108,6 +110,8 @@ template <int NV4>
 __global__ void __launch_bounds__(256) route_topk_vec_kernel(const float* __restrict__ logits, int T, int E, int k,
                                                              int norm_topk, int32_t* __restrict__ expert_idx,
                                                              float* __restrict__ gate) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     constexpr int NV = 4 * NV4;
     const int lane = threadIdx.x & 31;
     const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -171,118 +175,6 @@ __global__ void __launch_bounds__(256) route_topk_vec_kernel(const float* __rest
     }
 }
 
-// Eight lanes per token for E = 8 * NPL (E = 64, 128, 192 or 256) and
-// k <= 8: a warp takes four tokens, lane l of a token's group holds the NPL
-// logits of experts 4 (l + 8 q) + u (u < 4; float4 loads, 128 contiguous
-// bytes per group and q).  The minimum of the eight lane maxima is a lower
-// bound of the token's k-th largest logit (the eight maxima are eight
-// distinct logits; for k = 1 the maximum itself is the bound), so every
-// expert of the top k has a logit at or above it;
-// those candidates (about 17 of 256 for normal logits, all of them in the
-// worst case) go to shared memory, and each is ranked exactly by counting
-// the candidates that beat it (larger logit, or equal logit and lower
-// expert index - the order of the other kernels).  No insertion loop, so no
-// divergence beyond the per-token candidate counts.  Gates: exp(l - max)
-// with the rounding of l - max carried (as in the other kernels), over the
-// fp64 sum of the k chosen terms (renormalised) or of exp(l - max) over all
-// E (softmax).
-constexpr int kG8Warps = 4;
-
-// Requires E == 8 * NPL exactly (the host dispatch guarantees it).
-template <int NPL>
-__global__ void __launch_bounds__(32 * kG8Warps) route_topk_g8_kernel(const float* __restrict__ logits, int T, int E,
-                                                                      int k, int norm_topk,
-                                                                      int32_t* __restrict__ expert_idx,
-                                                                      float* __restrict__ gate) {
-    __shared__ float cand_v[kG8Warps][4][8 * NPL];
-    __shared__ int cand_e[kG8Warps][4][8 * NPL];
-    __shared__ int win_e[kG8Warps][4][8];
-    __shared__ float win_x[kG8Warps][4][8];
-    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-    const int g = lane >> 3, l = lane & 7;
-    float* cv = cand_v[wid][g];
-    int* ce = cand_e[wid][g];
-    const long long nwarps = (long long)gridDim.x * kG8Warps;
-    for (long long w = (long long)blockIdx.x * kG8Warps + wid; w * 4 < T; w += nwarps) {
-        const long long t = w * 4 + g;
-        const bool live = t < T;
-        const float4* row = reinterpret_cast<const float4*>(logits + (live ? t : 0) * (long long)E);
-        float v[NPL];
-#pragma unroll
-        for (int q = 0; q < NPL / 4; ++q) {
-            float4 x = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-            if (live) {
-                const uint4 u = ld_stream(reinterpret_cast<const uint4*>(row + l + 8 * q));
-                x = make_float4(__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w));
-            }
-            v[4 * q + 0] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
-        }
-        float m4[4] = {v[0], v[1], v[2], v[3]};
-#pragma unroll
-        for (int q = 1; q < NPL / 4; ++q)
-#pragma unroll
-            for (int u = 0; u < 4; ++u) m4[u] = fmaxf(m4[u], v[4 * q + u]);
-        float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        float tau = mx;
-#pragma unroll
-        for (int o = 4; o > 0; o >>= 1) {
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            tau = fminf(tau, __shfl_xor_sync(0xffffffffu, tau, o));
-        }
-        if (k == 1) tau = mx;                  // the top 1 is among the logits equal to the maximum
-        unsigned msk = 0;
-#pragma unroll
-        for (int i = 0; i < NPL; ++i) msk |= (v[i] >= tau ? 1u : 0u) << i;
-        if (!live) msk = 0;                    // a token past T has no candidates
-        const int cnt = __popc(msk);
-        int inc = cnt;
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, inc, o);
-            if (l >= o) inc += y;
-        }
-        const int n = __shfl_sync(0xffffffffu, inc, 8 * g + 7);
-        int pos = inc - cnt;
-#pragma unroll
-        for (int i = 0; i < NPL; ++i) {
-            if ((msk >> i) & 1u) {
-                cv[pos] = v[i];
-                ce[pos] = 4 * (l + 8 * (i >> 2)) + (i & 3);
-                ++pos;
-            }
-        }
-        __syncwarp();
-        for (int j = l; j < n; j += 8) {
-            const float vj = cv[j];
-            const int ej = ce[j];
-            int rank = 0;
-            for (int i = 0; i < n; ++i) {
-                const float vi = cv[i];
-                rank += (vi > vj || (vi == vj && ce[i] < ej)) ? 1 : 0;
-            }
-            if (rank < k) {
-                win_e[wid][g][rank] = ej;
-                win_x[wid][g][rank] = exp_diff(vj, mx);
-            }
-        }
-        __syncwarp();
-        double sum = 0.0;
-        if (norm_topk) {
-            if (l < k) sum = (double)win_x[wid][g][l];
-        } else {
-#pragma unroll
-            for (int i = 0; i < NPL; ++i) sum += (double)__expf(__fsub_rn(v[i], mx));
-        }
-#pragma unroll
-        for (int o = 4; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        if (live && l < k) {
-            expert_idx[t * k + l] = win_e[wid][g][l];
-            gate[t * k + l] = (float)((double)win_x[wid][g][l] / sum);
-        }
-        __syncwarp();                          // the candidate lists may be rewritten
-    }
-}
-
 // Thread-per-token variant for k <= 8 and E % 4 == 0 (any E up to 1024).
 // Each warp owns 32 consecutive tokens and walks their logits in chunks of
 // 32 experts through its own shared-memory ring (cp.async, two chunks in
@@ -316,6 +208,8 @@ __global__ void __launch_bounds__(32 * kRowWarps, 4) route_topk_rows_kernel(cons
                                                                             int E, int k, int norm_topk,
                                                                             int32_t* __restrict__ expert_idx,
                                                                             float* __restrict__ gate) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     extern __shared__ __align__(16) float row_ring[];
     const int lane = threadIdx.x & 31;
     float* ring = row_ring + (threadIdx.x >> 5) * kRowWarpFloats;
@@ -732,7 +626,7 @@ __global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned* __
                                                               const unsigned* __restrict__ keys_lo, int T, int E, int C,
                                                               int32_t* __restrict__ ec_token,
                                                               unsigned* __restrict__ tokmask, int mask_words) {
-    extern __shared__ unsigned hi_keys[];          // [T]
+    extern __shared__ unsigned hi_keys[];          // [T], then 32 per-warp histograms of 256 bins
     __shared__ int hist[256];
     __shared__ unsigned s_min, s_max, s_prefix, s_mask;
     __shared__ unsigned s_lprefix, s_lmask;
@@ -782,30 +676,37 @@ __global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned* __
         s_lprefix = 0; s_lmask = 0;
     }
     __syncthreads();
-    // level 0: radix on the high halves (shared memory only)
+    // level 0: radix on the high halves (shared memory only), each warp
+    // counting into its own 256-bin histogram (no cross-warp contention,
+    // no per-key warp vote), summed bin by bin afterwards
+    int* whist = reinterpret_cast<int*>(hi_keys + ((T + 3) & ~3));   // [32][256]
     while (!s_done && s_hi >= 0) {
         const int hb = s_hi;
         const int shift = max(hb - 7, 0);
         const unsigned bins_mask = (1u << (hb - shift + 1)) - 1u;
-        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+        for (int i = threadIdx.x; i < 32 * 256; i += blockDim.x) whist[i] = 0;
         __syncthreads();
         const unsigned prefix = s_prefix, mask = s_mask;
+        int* mine = whist + wid * 256;
         for (int t0 = 0; t0 < T; t0 += 4 * blockDim.x) {
-            int digit[4];
+            unsigned h[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 const int t = t0 + q * blockDim.x + threadIdx.x;
-                digit[q] = -1;
-                if (t < T) {
-                    const unsigned h = hi_keys[t];
-                    if ((h & mask) == prefix) digit[q] = (int)((h >> shift) & bins_mask);
-                }
+                h[q] = t < T ? hi_keys[t] : 0u;
             }
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const unsigned peers = __match_any_sync(0xffffffffu, digit[q]);
-                if (digit[q] >= 0 && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[digit[q]], __popc(peers));
+                const int t = t0 + q * blockDim.x + threadIdx.x;
+                if (t < T && (h[q] & mask) == prefix) atomicAdd(&mine[(h[q] >> shift) & bins_mask], 1);
             }
+        }
+        __syncthreads();
+        for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+            int sum = 0;
+#pragma unroll 8
+            for (int w = 0; w < 32; ++w) sum += whist[w * 256 + b];
+            hist[b] = sum;
         }
         __syncthreads();
         if (wid == 0) warp_find_boundary(hist, (int)bins_mask + 1, s_need, &s_bin, &s_bneed, &s_bcount);
@@ -978,16 +879,6 @@ namespace {
 // all), and pays off when the warp kernels would spend many reduction
 // rounds (k >= 4); otherwise the warp-per-token kernels keep more warps in
 // flight.  LIBMOE_TOPK_ROWS=0/1 forces either choice.
-// Eight lanes per token for 64, 128, 192 or 256 experts and k <= 8, when
-// LIBMOE_TOPK_G8=1 (the tests force it on and off).  Off by default: it
-// measured slower than the other kernels (T = 131072, E = 256, k = 8:
-// 179 us against 70 us; T = 16384, E = 64, k = 6: 34 us against 22 us).
-bool use_g8_variant() {
-    const char* env = getenv("LIBMOE_TOPK_G8");
-    if (env && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
-    return false;
-}
-
 bool use_rows_variant(int T, int k) {
     const char* env = getenv("LIBMOE_TOPK_ROWS");
     if (env && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
@@ -1007,20 +898,6 @@ extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, i
     int blocks = (int)((warps_needed + 7) / 8);
     if (blocks > 148 * 16) blocks = 148 * 16;
     const int nv = (E + 31) / 32;
-    if ((E == 64 || E == 128 || E == 192 || E == 256) && k <= 8 && ((uintptr_t)logits & 15) == 0 &&
-        use_g8_variant()) {
-        long long gb = ((long long)T + 4 * kG8Warps - 1) / (4 * kG8Warps);
-        const int gblocks = (int)(gb < 148 * 12 ? gb : 148 * 12);
-        switch (E / 8) {
-            case 8: route_topk_g8_kernel<8><<<gblocks, 32 * kG8Warps, 0, s>>>(logits, T, E, k, norm_topk, expert_idx, gate); break;
-            case 16: route_topk_g8_kernel<16><<<gblocks, 32 * kG8Warps, 0, s>>>(logits, T, E, k, norm_topk, expert_idx, gate); break;
-            case 24: route_topk_g8_kernel<24><<<gblocks, 32 * kG8Warps, 0, s>>>(logits, T, E, k, norm_topk, expert_idx, gate); break;
-            case 32: route_topk_g8_kernel<32><<<gblocks, 32 * kG8Warps, 0, s>>>(logits, T, E, k, norm_topk, expert_idx, gate); break;
-            default: return MOE_ERR_SHAPE;     // unreachable: E is one of the four sizes above
-        }
-        MOE_LAUNCH_CHECK();
-        return MOE_OK;
-    }
     if (E % 4 == 0 && k <= 8 && ((uintptr_t)logits & 15) == 0 && use_rows_variant(T, k)) {
         for (auto fn : {route_topk_rows_kernel<1>, route_topk_rows_kernel<2>, route_topk_rows_kernel<4>,
                         route_topk_rows_kernel<8>})
@@ -1029,7 +906,7 @@ extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, i
         long long rb = (warps + kRowWarps - 1) / kRowWarps;
         const int rblocks = (int)(rb < 148 * 8 ? rb : 148 * 8);
 #define MOE_TOPKR_CASE(KM)                                                                              \
-    route_topk_rows_kernel<KM><<<rblocks, 32 * kRowWarps, kRowSmem, s>>>(logits, T, E, k, norm_topk, expert_idx, \
+    (void)launch_pdl(route_topk_rows_kernel<KM>, rblocks, 32 * kRowWarps, kRowSmem, s, logits, T, E, k, norm_topk, expert_idx, \
                                                                          gate)
         if (k <= 1) MOE_TOPKR_CASE(1);
         else if (k <= 2) MOE_TOPKR_CASE(2);
@@ -1042,7 +919,7 @@ extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, i
     if (E % 4 == 0 && ((uintptr_t)logits & 15) == 0) {
         const int nv4 = (E + 127) / 128;
 #define MOE_TOPKV_CASE(N) \
-    case N: route_topk_vec_kernel<N><<<blocks, threads, 0, s>>>(logits, T, E, k, norm_topk, expert_idx, gate); break;
+    case N: (void)launch_pdl(route_topk_vec_kernel<N>, blocks, threads, 0, s, logits, T, E, k, norm_topk, expert_idx, gate); break;
         switch (nv4 <= 1 ? 1 : nv4 <= 2 ? 2 : nv4 <= 4 ? 4 : 8) {
             MOE_TOPKV_CASE(1)
             MOE_TOPKV_CASE(2)
@@ -1054,7 +931,7 @@ extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, i
         return MOE_OK;
     }
 #define MOE_TOPK_CASE(N) \
-    case N: route_topk_kernel<N><<<blocks, threads, 0, s>>>(logits, T, E, k, norm_topk, expert_idx, gate); break;
+    case N: (void)launch_pdl(route_topk_kernel<N>, blocks, threads, 0, s, logits, T, E, k, norm_topk, expert_idx, gate); break;
     switch (nv <= 1 ? 1 : nv <= 2 ? 2 : nv <= 4 ? 4 : nv <= 8 ? 8 : nv <= 16 ? 16 : 32) {
         MOE_TOPK_CASE(1)
         MOE_TOPK_CASE(2)
@@ -1115,7 +992,7 @@ extern "C" moe_status moe_route_ec(const float* logits, int T, int E, int C, int
     }
     cudaError_t rc;
     if (T <= kEcSmemTokens) {
-        const size_t smem = sizeof(unsigned) * (size_t)T;
+        const size_t smem = sizeof(unsigned) * (size_t)((T + 3) & ~3) + sizeof(int) * 32 * 256;
         if (!set_smem_limit((const void*)ec_select_smem_kernel, smem)) return MOE_ERR_CUDA;
         rc = launch_pdl(ec_select_smem_kernel, E, 1024, smem, s, (const unsigned*)keys_hi, (const unsigned*)keys_lo, T,
                         E, C, ec_token, mask, mw);

@@ -33,6 +33,8 @@ __global__ void __launch_bounds__(512) pair_hist_kernel(const int32_t* __restric
                                                         const int32_t* __restrict__ idx2, int k2, int T, int E,
                                                         int band, int tokens_per_cta, int32_t* __restrict__ hist,
                                                         unsigned* err) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     extern __shared__ int h[];                  // [band][E]
     const int a0 = blockIdx.y * band;
     const int a1 = min(a0 + band, E);
@@ -76,6 +78,8 @@ struct SymBands {
 __global__ void __launch_bounds__(512) cosel_sym_kernel(const int32_t* __restrict__ idx, int k, int T, int E,
                                                         SymBands bands, int tokens_per_cta,
                                                         int32_t* __restrict__ hist, unsigned* err) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     extern __shared__ int h[];                  // rows [a0, a1) of the upper triangle, packed
     const int a0 = bands.start[blockIdx.y];
     const int a1 = bands.start[blockIdx.y + 1];
@@ -153,6 +157,8 @@ template <int KM>
 __global__ void __cluster_dims__(kCoselCluster, 1, 1) __launch_bounds__(1024, 1)
 cosel_cluster_kernel(const int32_t* __restrict__ idx, int k, int T, int E, SymBands bands, int tokens_per_cta,
                      int32_t* __restrict__ hist, unsigned* err) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
     extern __shared__ int h[];                  // rows [a0, a1) of the upper triangle, packed
     const int a0 = bands.start[blockIdx.y];
     const int a1 = bands.start[blockIdx.y + 1];
@@ -205,7 +211,7 @@ cosel_cluster_kernel(const int32_t* __restrict__ idx, int k, int T, int E, SymBa
             if (b != a) atomicAdd(hist + (long long)b * E + a, v);
         }
     }
-    tc::cluster_sync();                         // no CTA exits while another still reads its counts
+    tc::cluster_sync_relaxed();                 // no CTA exits while another still reads its counts
 }
 
 // The symmetric kernel for E >= 128, where it measured faster (T = 131072,
@@ -250,7 +256,7 @@ moe_status launch_cosel_sym(const int32_t* idx, int k, int T, int E, int32_t* hi
     if (tokens_per_cta < 256) tokens_per_cta = 256;
     tok_ctas = ceil_div(T, tokens_per_cta);
     if (!set_smem_limit((const void*)cosel_sym_kernel, smem)) return MOE_ERR_CUDA;
-    cosel_sym_kernel<<<dim3(tok_ctas, nb), 512, smem, s>>>(idx, k, T, E, sb, tokens_per_cta, hist, err);
+    (void)launch_pdl(cosel_sym_kernel, dim3(tok_ctas, nb), 512, smem, s, idx, k, T, E, sb, tokens_per_cta, hist, err);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }
@@ -307,7 +313,7 @@ moe_status launch_cosel_cluster(const int32_t* idx, int k, int T, int E, int32_t
     const int tok_ctas = ceil_div(ceil_div(T, tokens_per_cta), kCoselCluster) * kCoselCluster;
     auto fn = k <= 2 ? cosel_cluster_kernel<2> : k <= 4 ? cosel_cluster_kernel<4> : cosel_cluster_kernel<8>;
     if (!set_smem_limit((const void*)fn, smem)) return MOE_ERR_CUDA;
-    fn<<<dim3(tok_ctas, nb), 1024, smem, s>>>(idx, k, T, E, sb, tokens_per_cta, hist, err);
+    (void)launch_pdl(fn, dim3(tok_ctas, nb), 1024, smem, s, idx, k, T, E, sb, tokens_per_cta, hist, err);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }
@@ -327,7 +333,7 @@ moe_status launch_pair_hist(const int32_t* idx1, int k1, const int32_t* idx2, in
     if (tokens_per_cta < 256) tokens_per_cta = 256;
     tok_ctas = ceil_div(T, tokens_per_cta);
     if (!set_smem_limit((const void*)pair_hist_kernel, smem)) return MOE_ERR_CUDA;
-    pair_hist_kernel<<<dim3(tok_ctas, nbands), 512, smem, s>>>(idx1, k1, idx2, k2, T, E, band, tokens_per_cta, hist, err);
+    (void)launch_pdl(pair_hist_kernel, dim3(tok_ctas, nbands), 512, smem, s, idx1, k1, idx2, k2, T, E, band, tokens_per_cta, hist, err);
     MOE_LAUNCH_CHECK();
     return MOE_OK;
 }

@@ -173,6 +173,14 @@ __device__ __forceinline__ void cluster_sync() {
     asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// A cluster barrier that orders no memory: for waiting until every CTA of
+// the cluster is done reading the others' shared memory (loads whose values
+// it has consumed), without also waiting for its own outstanding global
+// writes and atomics to complete, as a release arrive would.
+__device__ __forceinline__ void cluster_sync_relaxed() {
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
+}
+
 // 32-bit load from a shared::cluster address (another CTA's shared memory,
 // mapped with map_to_rank).
 __device__ __forceinline__ uint32_t ld_shared_cluster_u32(uint32_t cluster_addr) {

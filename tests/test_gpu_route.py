@@ -21,13 +21,10 @@ def check_topk(logits, k, norm=False):
     np.testing.assert_allclose(gg, rgate, rtol=GATE_RTOL, atol=1e-30)
 
 
-@pytest.fixture(params=["g8", "rows", "warp"])
+@pytest.fixture(params=["rows", "warp"])
 def topk_kind(request, monkeypatch):
-    """Run a test with each top-k kernel family: eight lanes per token (the
-    default for 64, 128, 192 or 256 experts and k <= 8), thread per
-    token, and warp per token (the library picks by shape; the tests force
-    each where it applies)."""
-    monkeypatch.setenv("LIBMOE_TOPK_G8", "1" if request.param == "g8" else "0")
+    """Run a test with the thread-per-token top-k kernel and with the
+    warp-per-token ones (the library picks by T; the tests force each)."""
     monkeypatch.setenv("LIBMOE_TOPK_ROWS", "1" if request.param == "rows" else "0")
     return request.param
 
@@ -52,10 +49,10 @@ def test_topk_ties_lower_index_wins(topk_kind):
     check_topk(z, 8)
 
 
-def test_topk_candidates_worst_case(topk_kind):
-    """Rows whose largest logits all sit in the experts one lane of an
-    eight-lane group holds (experts 4 (0 + 8 q) + u): the other lanes' maxima
-    are low, so nearly every logit is a candidate for the exact ranking."""
+def test_topk_concentrated_and_sorted_rows(topk_kind):
+    """Rows whose largest logits sit in a strided subset of the experts
+    (every fourth group of four), and sorted rows: the threshold of the
+    thread-per-token kernel rises late or at once."""
     for E in (64, 256):
         T = 999
         base = synth.normal_f32(13, 1, (T, E), 0.0, 0.1)
