@@ -88,19 +88,25 @@ __device__ __forceinline__ void store1(void* base, long long e, float v, bool bf
     else static_cast<float*>(base)[e] = v;
 }
 
-// Per-token distinct (row, summed gate) list: lane j < nu holds entry j,
-// entries in order of first appearance, gates of repeated rows summed in
-// slot order.  Called by all 32 lanes.
-__device__ __forceinline__ int token_rows(const int32_t* __restrict__ row_map, const float* __restrict__ gate,
-                                          long long t, int k, int R, unsigned* err, int& my_row, float& my_gate) {
+// A token's raw (row, gate) slots: lane j < k holds slot j; a row at or
+// past R is reported and dropped.
+__device__ __forceinline__ void token_slots(const int32_t* __restrict__ row_map, const float* __restrict__ gate,
+                                           long long t, int k, int R, unsigned* err, int& r, float& g) {
     const int lane = threadIdx.x & 31;
-    int r = -1;
-    float g = 0.0f;
+    r = -1;
+    g = 0.0f;
     if (lane < k) {
         r = row_map[t * k + lane];
         g = gate ? gate[t * k + lane] : 1.0f;
         if (r >= R) { raise_error(err, kErrIndex); r = -1; }
     }
+}
+
+// Per-token distinct (row, summed gate) list from the raw slots: lane j < nu
+// holds entry j, entries in order of first appearance, gates of repeated
+// rows summed in slot order.  Called by all 32 lanes.
+__device__ __forceinline__ int dedupe_rows(int r, float g, int k, int& my_row, float& my_gate) {
+    const int lane = threadIdx.x & 31;
     int nu = 0;
     my_row = -1;
     my_gate = 0.0f;
@@ -119,6 +125,14 @@ __device__ __forceinline__ int token_rows(const int32_t* __restrict__ row_map, c
     return nu;
 }
 
+__device__ __forceinline__ int token_rows(const int32_t* __restrict__ row_map, const float* __restrict__ gate,
+                                          long long t, int k, int R, unsigned* err, int& my_row, float& my_gate) {
+    int r;
+    float g;
+    token_slots(row_map, gate, t, k, R, err, r, g);
+    return dedupe_rows(r, g, k, my_row, my_gate);
+}
+
 template <bool IN_BF16, bool OUT_BF16, int NV>
 __global__ void __launch_bounds__(256) unpermute_vec_kernel(const void* __restrict__ y, int R, int T, int d, int k,
                                                             const int32_t* __restrict__ row_map,
@@ -131,10 +145,15 @@ __global__ void __launch_bounds__(256) unpermute_vec_kernel(const void* __restri
     const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
     const int nvec = d >> 3;
+    // the next token's slots are loaded while the current token's rows are summed
+    int nr = -1;
+    float ng = 0.0f;
+    if (warp < T) token_slots(row_map, gate, warp, k, R, err, nr, ng);
     for (long long t = warp; t < T; t += nwarps) {
         int my_row;
         float my_gate;
-        const int nu = token_rows(row_map, gate, t, k, R, err, my_row, my_gate);
+        const int nu = dedupe_rows(nr, ng, k, my_row, my_gate);
+        if (t + nwarps < T) token_slots(row_map, gate, t + nwarps, k, R, err, nr, ng);
         for (int v0 = 0; v0 < nvec; v0 += 32 * NV) {
             float acc[NV][8];
 #pragma unroll
@@ -445,59 +464,111 @@ __global__ void __launch_bounds__(256) unpermute_ec_vec_kernel(const void* __res
     const long long warp = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const long long nwarps = (long long)gridDim.x * (blockDim.x >> 5);
     const int nvec = d >> 3;
-    for (long long t = warp; t < T; t += nwarps) {
-        const int p0 = max(tok_ptr[t], 0), p1 = min(tok_ptr[t + 1], R);
-        for (int v0 = 0; v0 < nvec; v0 += 32 * NV) {
-            float acc[NV][8];
+    // A token's rows sit one per lane (CSR position p0 + lane), with their
+    // gates.  The metadata of the warp's next token is fetched while the
+    // current token's rows are summed: its CSR rows and the pointers of the
+    // token after it before, its gates after (each load one step ahead of
+    // its use), so the dependent pointer -> row -> gate loads stay off the
+    // critical path.  Tokens with more than 32 rows take the direct loop.
+    auto ptrs = [&](long long tt, int& a, int& b) {
+        a = b = 0;
+        if (tt < T) { a = max(tok_ptr[tt], 0); b = min(tok_ptr[tt + 1], R); }
+    };
+    auto row_at = [&](int a, int b) -> int { return lane < b - a ? tok_row[a + lane] : -1; };
+    auto gate_of = [&](int r) -> float { return (r >= 0 && r < R) ? ec_gate[r] : 0.0f; };
+    long long t = warp;
+    int c0, c1, n0, n1;
+    ptrs(t, c0, c1);
+    int cr = row_at(c0, c1);
+    ptrs(t + nwarps, n0, n1);
+    float cg = gate_of(cr);
+    for (; t < T; t += nwarps) {
+        const int nr = row_at(n0, n1);
+        int m0, m1;
+        ptrs(t + 2 * nwarps, m0, m1);
+        const int cnt = c1 - c0;
+        if (cnt <= 32) {
+            const bool in = lane < cnt;
+            const bool ok = in && cr >= 0 && cr < R;
+            if (in && !ok) raise_error(err, kErrIndex);
+            const unsigned valid = __ballot_sync(0xffffffffu, ok);
+            for (int v0 = 0; v0 < nvec; v0 += 32 * NV) {
+                float acc[NV][8];
 #pragma unroll
-            for (int u = 0; u < NV; ++u)
+                for (int u = 0; u < NV; ++u)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
-            // the token's rows two at a time (both in flight), added in CSR order
-            int p = p0;
-            while (p < p1) {
-                int r0 = -1, r1 = -1;
-                for (; p < p1 && r0 < 0; ++p) {
-                    const int r = tok_row[p];
-                    if (r < 0 || r >= R) raise_error(err, kErrIndex);
-                    else r0 = r;
-                }
-                for (; p < p1 && r1 < 0; ++p) {
-                    const int r = tok_row[p];
-                    if (r < 0 || r >= R) raise_error(err, kErrIndex);
-                    else r1 = r;
-                }
-                if (r0 < 0) break;
-                const float g0 = ec_gate[r0];
-                const float g1 = r1 >= 0 ? ec_gate[r1] : 0.0f;
-                Raw8<IN_BF16> a[NV], b[NV];
-#pragma unroll
-                for (int u = 0; u < NV; ++u) {
-                    const int v = v0 + u * 32 + lane;
-                    if (v < nvec) a[u].load(y, (long long)r0 * d + 8LL * v);
-                }
-                if (r1 >= 0) {
+                    for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+                // the valid rows two at a time (both in flight), added in CSR order
+                unsigned m = valid;
+                while (m) {
+                    const int j0 = __ffs(m) - 1;
+                    m &= m - 1;
+                    const bool two = m != 0;
+                    const int j1 = two ? __ffs(m) - 1 : j0;
+                    if (two) m &= m - 1;
+                    const int r0 = __shfl_sync(0xffffffffu, cr, j0);
+                    const float g0 = __shfl_sync(0xffffffffu, cg, j0);
+                    const int r1 = __shfl_sync(0xffffffffu, cr, j1);
+                    const float g1 = __shfl_sync(0xffffffffu, cg, j1);
+                    Raw8<IN_BF16> a[NV], b[NV];
 #pragma unroll
                     for (int u = 0; u < NV; ++u) {
                         const int v = v0 + u * 32 + lane;
-                        if (v < nvec) b[u].load(y, (long long)r1 * d + 8LL * v);
+                        if (v < nvec) a[u].load(y, (long long)r0 * d + 8LL * v);
+                    }
+                    if (two) {
+#pragma unroll
+                        for (int u = 0; u < NV; ++u) {
+                            const int v = v0 + u * 32 + lane;
+                            if (v < nvec) b[u].load(y, (long long)r1 * d + 8LL * v);
+                        }
+                    }
+#pragma unroll
+                    for (int u = 0; u < NV; ++u)
+                        if (v0 + u * 32 + lane < nvec) a[u].fma_into(g0, acc[u]);
+                    if (two) {
+#pragma unroll
+                        for (int u = 0; u < NV; ++u)
+                            if (v0 + u * 32 + lane < nvec) b[u].fma_into(g1, acc[u]);
                     }
                 }
 #pragma unroll
-                for (int u = 0; u < NV; ++u)
-                    if (v0 + u * 32 + lane < nvec) a[u].fma_into(g0, acc[u]);
-                if (r1 >= 0) {
-#pragma unroll
-                    for (int u = 0; u < NV; ++u)
-                        if (v0 + u * 32 + lane < nvec) b[u].fma_into(g1, acc[u]);
+                for (int u = 0; u < NV; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec) Vec8<OUT_BF16>::store(out, t * d + 8LL * v, acc[u]);
                 }
             }
+        } else {
+            for (int v0 = 0; v0 < nvec; v0 += 32 * NV) {
+                float acc[NV][8];
 #pragma unroll
-            for (int u = 0; u < NV; ++u) {
-                int v = v0 + u * 32 + lane;
-                if (v < nvec) Vec8<OUT_BF16>::store(out, t * d + 8LL * v, acc[u]);
+                for (int u = 0; u < NV; ++u)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[u][i] = 0.0f;
+                for (int p = c0; p < c1; ++p) {
+                    const int r = tok_row[p];
+                    if (r < 0 || r >= R) { raise_error(err, kErrIndex); continue; }
+                    const float g = ec_gate[r];
+#pragma unroll
+                    for (int u = 0; u < NV; ++u) {
+                        const int v = v0 + u * 32 + lane;
+                        if (v < nvec) {
+                            Raw8<IN_BF16> a;
+                            a.load(y, (long long)r * d + 8LL * v);
+                            a.fma_into(g, acc[u]);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < NV; ++u) {
+                    const int v = v0 + u * 32 + lane;
+                    if (v < nvec) Vec8<OUT_BF16>::store(out, t * d + 8LL * v, acc[u]);
+                }
             }
         }
+        const float ng = gate_of(nr);
+        c0 = n0; c1 = n1; cr = nr; cg = ng;
+        n0 = m0; n1 = m1;
     }
 }
 

@@ -501,8 +501,26 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
     const int total = tile_prefix[E];
+    // The last partial round of the plain (down) GEMM: its tiles are split
+    // into `split` column slices of 256 / split columns (MMA N = 128 or 64),
+    // so that round takes a fraction of a tile's time on more CTA pairs
+    // instead of a whole tile's time on a few (896 tiles on 74 pairs: 12.1
+    // rounds would run as 13).  Units [0, full_units) are whole tiles.
+    int full_units = total, split = 1;
+    if (MODE == MODE_PLAIN && total > 0) {
+        full_units = ((total + npairs - 1) / npairs - 1) * npairs;
+        const int tail = total - full_units;
+        while (split < 4 && tail * split * 2 <= npairs) split *= 2;
+    }
+    const int units = full_units + (total - full_units) * split;
 
-    auto decode = [&](int t, int& row0, int& row_end, int& n0, int& e_out) {
+    auto decode = [&](int u, int& row0, int& row_end, int& n0, int& e_out, int& ncols) {
+        int t = u, sub = 0, parts = 1;
+        if (u >= full_units) {
+            t = full_units + (u - full_units) / split;
+            sub = (u - full_units) % split;
+            parts = split;
+        }
         int lo = 0, hi = E;
         while (lo < hi) {
             int mid = (lo + hi + 1) >> 1;
@@ -516,7 +534,8 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
         const int n_idx = local / mt, m_idx = local - n_idx * mt;
         row0 = b + m_idx * BM;
         row_end = en;
-        n0 = n_idx * BN_OUT;
+        ncols = BN_OUT / parts;
+        n0 = n_idx * BN_OUT + sub * ncols;
         e_out = e;
     };
 
@@ -525,9 +544,9 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
             int stage = 0;
             uint32_t phase = 0;
             uint32_t issued = 0, fill_parity = 0;
-            for (int t = pair; t < total && !*abort_flag; t += npairs) {
-                int row0, row_end, n0, e;
-                decode(t, row0, row_end, n0, e);
+            for (int t = pair; t < units && !*abort_flag; t += npairs) {
+                int row0, row_end, n0, e, ncols;
+                decode(t, row0, row_end, n0, e, ncols);
                 const int arow = row0 + (int)rank * 128;
                 int brow;
                 const CUtensorMap* bmap = &map_b0;
@@ -535,7 +554,9 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
                     brow = e * args.w_rows + n0;
                     if (!leader) bmap = &map_b1;
                 } else {
-                    brow = e * args.w_rows + n0 + (int)rank * 128;
+                    // each CTA holds half of the unit's columns (the 128-row box
+                    // also brings rows the narrower MMAs of the last round skip)
+                    brow = e * args.w_rows + n0 + (int)rank * (ncols / 2);
                 }
                 for (int kb = 0; kb < nk; ++kb) {
                     if (!mbar_wait(smem_u32(&empty[stage]), phase ^ 1u, abort_flag)) { *abort_flag = 1; break; }
@@ -561,11 +582,11 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
         }
     } else if (warp == 1) {
         if (lane == 0 && leader) {
-            constexpr uint32_t idesc = umma_idesc_bf16(BM, ACC_N);
             int stage = 0;
             uint32_t phase = 0;
             int it = 0;
-            for (int t = pair; t < total && !*abort_flag; t += npairs, ++it) {
+            for (int t = pair; t < units && !*abort_flag; t += npairs, ++it) {
+                const uint32_t idesc = umma_idesc_bf16(BM, t < full_units ? ACC_N : ACC_N / split);
                 const int acc = it & 1;
                 const uint32_t acc_phase = (it >> 1) & 1;
                 if (!mbar_wait_cluster(smem_u32(&tempty[acc]), acc_phase ^ 1u, abort_flag)) { *abort_flag = 1; break; }
@@ -599,9 +620,9 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
         const uint32_t tempty_leader1 = map_to_rank(smem_u32(&tempty[1]), 0);
         EpiOut eo{smem_u32(out_stage + (warp - 2) * 2 * OUT_CHUNK_BYTES)};
         int it = 0;
-        for (int t = pair; t < total; t += npairs, ++it) {
-            int row0, row_end, n0, e;
-            decode(t, row0, row_end, n0, e);
+        for (int t = pair; t < units; t += npairs, ++it) {
+            int row0, row_end, n0, e, ncols;
+            decode(t, row0, row_end, n0, e, ncols);
             const int acc = it & 1;
             const uint32_t acc_phase = (it >> 1) & 1;
             if (!mbar_wait(smem_u32(&tfull[acc]), acc_phase, abort_flag)) { *abort_flag = 1; break; }
@@ -627,8 +648,9 @@ grouped_gemm2_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_con
                     }
                 }
             } else {
+                const int per = (ncols / 32) / (EPI_WARPS / 4);   // 32-column chunks per epilogue warp
 #pragma unroll 1
-                for (int c = (32 / EPI_WARPS) * half; c < (32 / EPI_WARPS) * half + 32 / EPI_WARPS; ++c) {
+                for (int c = per * half; c < per * (half + 1); ++c) {
                     float a[32];
                     tmem_ld32(taddr + c * 32, a);
                     tmem_ld_wait();

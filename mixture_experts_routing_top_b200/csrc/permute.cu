@@ -41,14 +41,15 @@ constexpr int kIdxThreads = 256;
 
 // 1. per-block histogram of experts, stored expert-major: cnt[e * nblk + b]
 __global__ void __launch_bounds__(kIdxThreads) perm_count_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
-                                                                 int nblk, int32_t* __restrict__ cnt, unsigned* err) {
+                                                                 int nblk, int tb, int32_t* __restrict__ cnt,
+                                                                 unsigned* err) {
     pdl_trigger();                // the next kernel may be scheduled; it waits for this one
     pdl_wait();                   // inputs come from the kernel before
     extern __shared__ int hist[];
     for (int i = threadIdx.x; i < E; i += blockDim.x) hist[i] = 0;
     __syncthreads();
-    const long long s0 = (long long)blockIdx.x * kTB * k;
-    const long long s1 = min((long long)(blockIdx.x + 1) * kTB, (long long)T) * k;
+    const long long s0 = (long long)blockIdx.x * tb * k;
+    const long long s1 = min((long long)(blockIdx.x + 1) * tb, (long long)T) * k;
     for (long long s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
         const int e = idx[s];
         if (e < 0 || e >= E) { raise_error(err, kErrIndex); continue; }
@@ -286,14 +287,14 @@ __device__ void block_scan_prologue(bool fused, const int32_t* __restrict__ cnt,
     __syncthreads();
 }
 
-// Group-major, part 1 (one CTA per kTB tokens): expert ranks -> kept slots;
+// Group-major, part 1 (one CTA per tb tokens): expert ranks -> kept slots;
 // then, one thread per token, each kept slot's group, whether it is the
 // first kept slot of its token in that group (the row's "head"), and the
 // per-block head count of every group.  code[s]: group id for a head,
 // -2 - j for a kept slot whose head is slot j of the same token, -1 for a
 // dropped slot.
 __global__ void __launch_bounds__(kIdxThreads) perm_group_heads_kernel(
-    const int32_t* __restrict__ idx, const int32_t* __restrict__ goe, int T, int k, int E, int G, int nblk, int fused,
+    const int32_t* __restrict__ idx, const int32_t* __restrict__ goe, int T, int k, int E, int G, int nblk, int tb, int fused,
     const int32_t* __restrict__ ecnt, const int32_t* __restrict__ ebase, long long cap, int32_t* __restrict__ counts,
     int32_t* __restrict__ dropped, int16_t* __restrict__ code, int32_t* __restrict__ gcnt, unsigned* err) {
     pdl_trigger();                // the next kernel may be scheduled; it waits for this one
@@ -303,22 +304,27 @@ __global__ void __launch_bounds__(kIdxThreads) perm_group_heads_kernel(
     int* base_s = wcnt + (kIdxThreads / 32) * E;             // [E]
     int* off_s = base_s + E;                                 // [E]
     int* ghist = off_s + E;                                  // [G]
-    uint8_t* kept_s = reinterpret_cast<uint8_t*>(ghist + G); // [kTB * k]
-    const long long s0 = (long long)blockIdx.x * kTB * k;
-    const long long s1 = min((long long)(blockIdx.x + 1) * kTB, (long long)T) * k;
+    int* goe_s = ghist + G;                                  // [E]
+    int* keys_s = goe_s + E;                                 // [tb * k]
+    uint8_t* kept_s = reinterpret_cast<uint8_t*>(keys_s + tb * k); // [tb * k]
+    const long long s0 = (long long)blockIdx.x * tb * k;
+    const long long s1 = min((long long)(blockIdx.x + 1) * tb, (long long)T) * k;
     for (int i = threadIdx.x; i < G; i += blockDim.x) ghist[i] = 0;
+    // the block's experts and the group map into shared memory at once
+    for (long long sl = s0 + threadIdx.x; sl < s1; sl += blockDim.x) keys_s[sl - s0] = idx[sl];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) goe_s[e] = goe[e];
     block_scan_prologue(fused, ecnt, ebase, nullptr, E, nblk, cap, base_s, off_s, counts, nullptr, dropped,
                         (int)blockIdx.x, blockIdx.x == 0);
     block_stable_ranks(
         s0, s1, E, base_s, wcnt,
         [&](long long s) -> int {
-            const int e = idx[s];
+            const int e = keys_s[s - s0];
             if (e < 0 || e >= E) { raise_error(err, kErrIndex); return -1; }
             return e;
         },
         [&](long long s, int key, int rank) { kept_s[s - s0] = (key >= 0 && rank < cap) ? 1 : 0; });
     __syncthreads();
-    const long long t0 = (long long)blockIdx.x * kTB;
+    const long long t0 = (long long)blockIdx.x * tb;
     const int ntok = (int)((s1 - s0) / k);
     for (int tl = threadIdx.x; tl < ntok; tl += blockDim.x) {
         const long long sb = (t0 + tl) * k;
@@ -326,13 +332,13 @@ __global__ void __launch_bounds__(kIdxThreads) perm_group_heads_kernel(
             const long long s = sb + j;
             int c = -1;
             if (kept_s[s - s0]) {
-                const int g = goe[idx[s]];
+                const int g = goe_s[keys_s[s - s0]];
                 if (g < 0 || g >= G) {
                     raise_error(err, kErrIndex);
                 } else {
                     int jh = -1;
                     for (int q = 0; q < j; ++q)
-                        if (kept_s[sb + q - s0] && goe[idx[sb + q]] == g) { jh = q; break; }
+                        if (kept_s[sb + q - s0] && goe_s[keys_s[sb + q - s0]] == g) { jh = q; break; }
                     if (jh < 0) { c = g; atomicAdd(&ghist[g], 1); }
                     else c = -2 - jh;
                 }
@@ -347,7 +353,7 @@ __global__ void __launch_bounds__(kIdxThreads) perm_group_heads_kernel(
 // Group-major, part 2: head slots get stable per-group ranks (token order)
 // and their rows; every other kept slot takes its head's row.
 __global__ void __launch_bounds__(kIdxThreads) perm_group_rows_kernel(
-    const int16_t* __restrict__ code, int T, int k, int G, int nblk, int fused, const int32_t* __restrict__ gcnt,
+    const int16_t* __restrict__ code, int T, int k, int G, int nblk, int tb, int fused, const int32_t* __restrict__ gcnt,
     const int32_t* __restrict__ gbase, const int32_t* __restrict__ goffsets_in, int32_t* __restrict__ offsets,
     int32_t* __restrict__ row_map, int32_t* __restrict__ row_token) {
     pdl_trigger();                // the next kernel may be scheduled; it waits for this one
@@ -356,13 +362,15 @@ __global__ void __launch_bounds__(kIdxThreads) perm_group_rows_kernel(
     int* wcnt = sm;                                          // [8][G]
     int* base_s = wcnt + (kIdxThreads / 32) * G;             // [G]
     int* off_s = base_s + G;                                 // [G]
-    int* rows_s = off_s + G;                                 // [kTB * k]
-    const long long s0 = (long long)blockIdx.x * kTB * k;
-    const long long s1 = min((long long)(blockIdx.x + 1) * kTB, (long long)T) * k;
+    int* rows_s = off_s + G;                                 // [tb * k]
+    int* codes_s = rows_s + tb * k;                          // [tb * k]
+    const long long s0 = (long long)blockIdx.x * tb * k;
+    const long long s1 = min((long long)(blockIdx.x + 1) * tb, (long long)T) * k;
+    for (long long sl = s0 + threadIdx.x; sl < s1; sl += blockDim.x) codes_s[sl - s0] = code[sl];
     block_scan_prologue(fused, gcnt, gbase, goffsets_in, G, nblk, (long long)T * k, base_s, off_s, nullptr, offsets,
                         nullptr, (int)blockIdx.x, blockIdx.x == 0);
     block_stable_ranks(
-        s0, s1, G, base_s, wcnt, [&](long long s) -> int { return (int)code[s]; },
+        s0, s1, G, base_s, wcnt, [&](long long s) -> int { return codes_s[s - s0]; },
         [&](long long s, int key, int rank) {
             int r = -1;
             if (key >= 0) {
@@ -373,7 +381,7 @@ __global__ void __launch_bounds__(kIdxThreads) perm_group_rows_kernel(
         });
     __syncthreads();
     for (long long s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
-        const int c = code[s];
+        const int c = codes_s[s - s0];
         int r = -1;
         if (c >= 0) r = rows_s[s - s0];
         else if (c <= -2) r = rows_s[(s / k) * k + (-2 - c) - s0];
@@ -384,7 +392,7 @@ __global__ void __launch_bounds__(kIdxThreads) perm_group_rows_kernel(
 // 4. expert-major rows: stable ranks per expert (token order); a slot is
 // kept if its rank is below the capacity, at row offsets[e] + rank.
 __global__ void __launch_bounds__(kIdxThreads) perm_rank_kernel(const int32_t* __restrict__ idx, int T, int k, int E,
-                                                                int nblk, int fused, const int32_t* __restrict__ cnt,
+                                                                int nblk, int tb, int fused, const int32_t* __restrict__ cnt,
                                                                 const int32_t* __restrict__ base, long long cap,
                                                                 int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                                                 int32_t* __restrict__ dropped,
@@ -396,14 +404,18 @@ __global__ void __launch_bounds__(kIdxThreads) perm_rank_kernel(const int32_t* _
     int* wcnt = sm;                              // [8][E]
     int* base_s = wcnt + (kIdxThreads / 32) * E; // [E]
     int* off_s = base_s + E;                     // [E]
-    const long long s0 = (long long)blockIdx.x * kTB * k;
-    const long long s1 = min((long long)(blockIdx.x + 1) * kTB, (long long)T) * k;
+    int* keys_s = off_s + E;                     // [tb * k]
+    const long long s0 = (long long)blockIdx.x * tb * k;
+    const long long s1 = min((long long)(blockIdx.x + 1) * tb, (long long)T) * k;
+    // the block's experts into shared memory at once (coalesced, all loads in
+    // flight), so the ranking passes do not wait on a global load per step
+    for (long long sl = s0 + threadIdx.x; sl < s1; sl += blockDim.x) keys_s[sl - s0] = idx[sl];
     block_scan_prologue(fused, cnt, base, offsets, E, nblk, cap, base_s, off_s, counts, offsets, dropped,
                         (int)blockIdx.x, blockIdx.x == 0);
     block_stable_ranks(
         s0, s1, E, base_s, wcnt,
         [&](long long s) -> int {
-            const int e = idx[s];
+            const int e = keys_s[s - s0];
             if (e < 0 || e >= E) { raise_error(err, kErrIndex); return -1; }
             return e;
         },
@@ -640,8 +652,14 @@ struct PermWs {
 
 constexpr long long kFuseLimit = 16384;   // keys x blocks each consumer block scans itself
 
+// Tokens per block of the index kernels.  Smaller blocks (more CTAs) were
+// measured slower: every block's scan prologue then reads more block counts
+// (keys x blocks grows with the block count).
+int perm_tokens_per_block(int) { return kTB; }
+
 PermWs perm_layout(int T, int k, int E, int G) {
-    const int nblk = ceil_div(T, kTB) > 0 ? ceil_div(T, kTB) : 1;
+    const int tb = perm_tokens_per_block(T);
+    const int nblk = ceil_div(T, tb) > 0 ? ceil_div(T, tb) : 1;
     PermWs w;
     w.cnt = 0;
     w.base = w.cnt + al256(sizeof(int32_t) * (size_t)E * nblk);
@@ -758,14 +776,15 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
     unsigned* err = device_error_word();
     if (!err) return MOE_ERR_CUDA;
     const long long cap = moe_capacity(capacity_factor, T, k, E);
-    const int nblk = ceil_div(T, kTB) > 0 ? ceil_div(T, kTB) : 1;
+    const int tb = perm_tokens_per_block(T);
+    const int nblk = ceil_div(T, tb) > 0 ? ceil_div(T, tb) : 1;
     char* ws = (char*)workspace;
     int32_t* cnt = (int32_t*)(ws + L.cnt);
     int32_t* base = (int32_t*)(ws + L.base);
     int32_t* total = (int32_t*)(ws + L.total);
     const int nw = kIdxThreads / 32;
     // 1. per-block expert counts
-    if (launch_pdl(perm_count_kernel, nblk, kIdxThreads, sizeof(int) * E, s, expert_idx, T, k, E, nblk, cnt, err) != cudaSuccess)
+    if (launch_pdl(perm_count_kernel, nblk, kIdxThreads, sizeof(int) * E, s, expert_idx, T, k, E, nblk, tb, cnt, err) != cudaSuccess)
         return MOE_ERR_CUDA;
     MOE_LAUNCH_CHECK();
     // 2-3. the scans: done by every consumer block itself when experts x
@@ -782,9 +801,9 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
     }
     if (!group_of_expert) {
         // 4. ranks and rows (its block 0 writes counts, offsets and dropped when fused)
-        const size_t rank_smem = sizeof(int) * ((size_t)nw * E + 2 * (size_t)E);
+        const size_t rank_smem = sizeof(int) * ((size_t)nw * E + 2 * (size_t)E + (size_t)tb * k);
         if (!set_smem_limit((const void*)perm_rank_kernel, rank_smem)) return MOE_ERR_CUDA;
-        if (launch_pdl(perm_rank_kernel, nblk, kIdxThreads, rank_smem, s, expert_idx, T, k, E, nblk, fused_e,
+        if (launch_pdl(perm_rank_kernel, nblk, kIdxThreads, rank_smem, s, expert_idx, T, k, E, nblk, tb, fused_e,
                        (const int32_t*)cnt, (const int32_t*)base, cap, counts, offsets, dropped, row_map, row_token,
                        err) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -794,9 +813,9 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
         int32_t* gcnt = (int32_t*)(ws + L.gcnt);
         int32_t* gbase = (int32_t*)(ws + L.gbase);
         int32_t* gtotal = (int32_t*)(ws + L.gtotal);
-        const size_t heads_smem = sizeof(int) * ((size_t)nw * E + 2 * (size_t)E + G) + (size_t)kTB * k;
+        const size_t heads_smem = sizeof(int) * ((size_t)nw * E + 3 * (size_t)E + G + (size_t)tb * k) + (size_t)tb * k;
         if (!set_smem_limit((const void*)perm_group_heads_kernel, heads_smem)) return MOE_ERR_CUDA;
-        if (launch_pdl(perm_group_heads_kernel, nblk, kIdxThreads, heads_smem, s, expert_idx, group_of_expert, T, k, E, G, nblk,
+        if (launch_pdl(perm_group_heads_kernel, nblk, kIdxThreads, heads_smem, s, expert_idx, group_of_expert, T, k, E, G, nblk, tb,
                                                                         fused_e, cnt, base, cap, counts, dropped, code,
                                                                         gcnt, err) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -811,9 +830,9 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
                 return MOE_ERR_CUDA;
             MOE_LAUNCH_CHECK();
         }
-        const size_t rows_smem = sizeof(int) * ((size_t)nw * G + 2 * (size_t)G + (size_t)kTB * k);
+        const size_t rows_smem = sizeof(int) * ((size_t)nw * G + 2 * (size_t)G + 2 * (size_t)tb * k);
         if (!set_smem_limit((const void*)perm_group_rows_kernel, rows_smem)) return MOE_ERR_CUDA;
-        if (launch_pdl(perm_group_rows_kernel, nblk, kIdxThreads, rows_smem, s, code, T, k, G, nblk, fused_g, gcnt, gbase, offsets,
+        if (launch_pdl(perm_group_rows_kernel, nblk, kIdxThreads, rows_smem, s, code, T, k, G, nblk, tb, fused_g, gcnt, gbase, offsets,
                                                                       offsets, row_map, row_token) != cudaSuccess)
             return MOE_ERR_CUDA;
         MOE_LAUNCH_CHECK();

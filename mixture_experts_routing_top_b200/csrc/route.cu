@@ -812,6 +812,7 @@ constexpr int kScanCtas = 8;
 
 __global__ void __cluster_dims__(kScanCtas, 1, 1) __launch_bounds__(1024, 1)
 ec_count_scan_kernel(const unsigned* __restrict__ tokmask, int T, int mask_words, int32_t* __restrict__ tok_ptr) {
+    constexpr int kCache = 16;                 // tokens per thread whose counts stay in registers
     __shared__ int sh[32];
     __shared__ int cta_total;
     pdl_trigger();
@@ -825,23 +826,39 @@ ec_count_scan_kernel(const unsigned* __restrict__ tokmask, int T, int mask_words
         for (int w = 0; w < mask_words; ++w) n += __popc(tokmask[t * mask_words + w]);
         return n;
     };
+    int cached[kCache];
     int mine = 0;
-    for (long long t = a; t < b; ++t) mine += count(t);
+#pragma unroll
+    for (int j = 0; j < kCache; ++j) {
+        cached[j] = a + j < b ? count(a + j) : 0;
+        mine += cached[j];
+    }
+    for (long long t = a + kCache; t < b; ++t) mine += count(t);
     int tot;
     const int ex = block_exclusive_scan(mine, &tot, sh);
     if (threadIdx.x == 0) cta_total = tot;
     __syncthreads();
     tc::cluster_sync();
-    int before = 0, all = 0;
+    int v[kScanCtas];
     const uint32_t local = tc::smem_u32(&cta_total);
+#pragma unroll
+    for (int q = 0; q < kScanCtas; ++q) v[q] = (int)tc::ld_shared_cluster_u32(tc::map_to_rank(local, (uint32_t)q));
+    int before = 0, all = 0;
+#pragma unroll
     for (int q = 0; q < kScanCtas; ++q) {
-        const int v = (int)tc::ld_shared_cluster_u32(tc::map_to_rank(local, (uint32_t)q));
-        if (q < c) before += v;
-        all += v;
+        if (q < c) before += v[q];
+        all += v[q];
     }
-    tc::cluster_sync();                       // every read of cta_total is done before any CTA exits
+    tc::cluster_sync_relaxed();               // every read of cta_total is done before any CTA exits
     int run = before + ex;
-    for (long long t = a; t < b; ++t) {
+#pragma unroll
+    for (int j = 0; j < kCache; ++j) {
+        if (a + j < b) {
+            tok_ptr[a + j] = run;
+            run += cached[j];
+        }
+    }
+    for (long long t = a + kCache; t < b; ++t) {
         tok_ptr[t] = run;
         run += count(t);
     }

@@ -21,6 +21,9 @@
 // bands are cut from the triangle so that they hold equal numbers of bins.
 // Used for E >= 128 (wide histograms), where it measured faster.
 #include <cstdlib>
+#include <map>
+#include <mutex>
+#include <tuple>
 
 #include "common.cuh"
 #include "tcgen05.cuh"
@@ -296,6 +299,31 @@ bool cosel_cluster_enabled() {
     return true;
 }
 
+// How many clusters of this kernel, with this shared memory, the device runs
+// at once (cached per kernel, size, device and context).  Launching more than
+// that leaves the extra clusters for a second wave.
+int max_active_clusters(const void* fn, size_t smem, int block) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+    static std::mutex mu;
+    static std::map<std::tuple<const void*, size_t, int, unsigned long long>, int> known;
+    const auto key = std::make_tuple(fn, smem, dev, context_id());
+    std::lock_guard<std::mutex> lk(mu);
+    const auto it = known.find(key);
+    if (it != known.end()) return it->second;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kCoselCluster * 16);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, fn, &cfg) != cudaSuccess || n < 1) {
+        (void)cudaGetLastError();
+        n = 1;
+    }
+    known[key] = n;
+    return n;
+}
+
 moe_status launch_cosel_cluster(const int32_t* idx, int k, int T, int E, int32_t* hist, cudaStream_t s) {
     unsigned* err = device_error_word();
     if (!err) return MOE_ERR_CUDA;
@@ -304,15 +332,16 @@ moe_status launch_cosel_cluster(const int32_t* idx, int k, int T, int E, int32_t
     long long widest = 0;
     if (!make_sym_bands(E, kCoselBandBytes, &sb, &nb, &widest)) return MOE_ERR_SHAPE;
     const size_t smem = sizeof(int) * (size_t)(widest > 0 ? widest : 1);
-    // at most 16 clusters of 8 over all bands (one CTA per SM: they fit the
-    // GPCs together), at least 512 tokens per CTA
-    int clusters = 16 / nb;
+    auto fn = k <= 2 ? cosel_cluster_kernel<2> : k <= 4 ? cosel_cluster_kernel<4> : cosel_cluster_kernel<8>;
+    if (!set_smem_limit((const void*)fn, smem)) return MOE_ERR_CUDA;
+    // as many clusters of 8 as run at once over all bands (one wave; with one
+    // CTA per SM the GPCs hold 15 at E = 256, not 148 / 8), at least 512
+    // tokens per CTA
+    int clusters = max_active_clusters((const void*)fn, smem, 1024) / nb;
     if (clusters < 1) clusters = 1;
     int tokens_per_cta = ceil_div(T, (long long)clusters * kCoselCluster);
     if (tokens_per_cta < 512) tokens_per_cta = 512;
     const int tok_ctas = ceil_div(ceil_div(T, tokens_per_cta), kCoselCluster) * kCoselCluster;
-    auto fn = k <= 2 ? cosel_cluster_kernel<2> : k <= 4 ? cosel_cluster_kernel<4> : cosel_cluster_kernel<8>;
-    if (!set_smem_limit((const void*)fn, smem)) return MOE_ERR_CUDA;
     (void)launch_pdl(fn, dim3(tok_ctas, nb), 1024, smem, s, idx, k, T, E, sb, tokens_per_cta, hist, err);
     MOE_LAUNCH_CHECK();
     return MOE_OK;

@@ -32,7 +32,7 @@ def topk_kind(request, monkeypatch):
 @pytest.mark.parametrize("T,E,k", [(1, 1, 1), (7, 3, 2), (1000, 8, 2), (333, 33, 5), (512, 64, 6), (300, 100, 7),
                                    (1025, 256, 8), (200, 1024, 32), (64, 160, 32), (50, 5, 5), (129, 36, 4),
                                    (300, 1020, 8), (77, 12, 1), (1001, 64, 2), (999, 128, 8), (1003, 192, 5),
-                                   (70, 256, 3), (1001, 128, 1), (65, 64, 1)])
+                                   (70, 256, 3), (1001, 128, 1), (65, 64, 1), (2049, 96, 8), (33, 224, 4)])
 @pytest.mark.parametrize("norm", [False, True])
 def test_topk_random(T, E, k, norm, topk_kind):
     check_topk(synth.normal_f32(11, 1, (T, E), 0.0, 2.0), k, norm)
