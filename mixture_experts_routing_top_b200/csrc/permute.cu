@@ -632,6 +632,220 @@ __global__ void __launch_bounds__(32 * kBulkWarps) copy_rows_csr_bulk_kernel(con
     }
 }
 
+// ---------------------------------------------- expert-major, two launches
+// When the rows are copied in the same call, the expert-major permutation
+// runs as two kernels instead of count, rank and copy:
+//
+//   perm_count_cluster_kernel: one cluster of kCcCtas CTAs.  The tokens are
+//     cut into chunks of kRcTok; each CTA counts its run of chunks per
+//     expert in shared memory and scans the counts per expert over its
+//     chunks; the CTAs then read each other's per-expert totals through
+//     distributed shared memory, so every CTA knows how many slots of each
+//     expert precede its first chunk.  It writes chunk_base[c][e] = the
+//     number of slots with expert e before chunk c (token order), and its
+//     CTA 0 writes the capacity-clamped counts, the row offsets and dropped.
+//   perm_rank_copy_kernel: one CTA per chunk, one warp per token.  Each warp
+//     starts the bulk load of its token's row before anything else; the CTA
+//     then ranks the chunk's slots (chunk_base + the stable rank inside the
+//     chunk), writes row_map and row_token, and each warp stores its row to
+//     the token's kept rows.
+//
+// A chunk's ranking work is small and overlaps its own row loads, and the
+// CTAs are short (one row per warp), so no CTA waits for a separate ranking
+// kernel before moving bytes and the last wave leaves no long tail.
+constexpr int kRcTok = 8;                  // tokens per chunk = warps per rank-and-copy CTA
+constexpr int kCcCtas = 8;                 // CTAs of the counting cluster (portable size)
+constexpr int kCcThreads = 1024;
+constexpr long long kCcMaxInts = 36 * 1024;   // chunk x expert counters per counting CTA
+
+// Exclusive scan of n ints in shared memory, in place, by the whole CTA
+// (each thread scans a run of ceil(n / blockDim) elements, then the runs'
+// sums are scanned across the CTA).  Returns the total.  `wsum` holds 32.
+__device__ int block_exclusive_scan(int* a, int n, int* wsum) {
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const int m = (n + blockDim.x - 1) / blockDim.x;
+    const int b0 = min(n, (int)threadIdx.x * m), b1 = min(n, b0 + m);
+    int run = 0;
+    for (int i = b0; i < b1; ++i) run += a[i];
+    int x = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[wid] = x;
+    __syncthreads();
+    int before = 0, all = 0;
+    for (int w = 0; w < nw; ++w) {
+        const int v = wsum[w];
+        if (w < wid) before += v;
+        all += v;
+    }
+    int acc = before + x - run;
+    for (int i = b0; i < b1; ++i) {
+        const int v = a[i];
+        a[i] = acc;
+        acc += v;
+    }
+    __syncthreads();
+    return all;
+}
+
+__global__ void __cluster_dims__(kCcCtas, 1, 1) __launch_bounds__(kCcThreads, 1)
+perm_count_cluster_kernel(const int32_t* __restrict__ idx, int T, int k, int E, int nchunk, int cpc, long long cap,
+                          int32_t* __restrict__ chunk_base, int32_t* __restrict__ counts,
+                          int32_t* __restrict__ offsets, int32_t* __restrict__ dropped, unsigned* err) {
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // inputs come from the kernel before
+    extern __shared__ int cc_sm[];
+    const int r = (int)tc::cluster_rank();
+    const int c0 = min(r * cpc, nchunk);
+    const int c1 = min(c0 + cpc, nchunk);
+    const int ncc = c1 - c0;
+    // row stride of hist: the same in every CTA, so that tot[] sits at the
+    // same offset in each (the cluster reads it there); the zero entries past
+    // ncc end each row for the scan below
+    const int ld = cpc + 1;
+    int* hist = cc_sm;                         // [E][ld]: counts per expert and chunk, then scanned
+    int* tot = hist + (size_t)E * ld;          // [E] this CTA's totals, read by the whole cluster
+    int* pre = tot + E;                        // [E] slots of each expert in the lower-ranked CTAs' chunks
+    int* kept_s = pre + E;                     // [E] capacity-clamped totals
+    __shared__ int wsum[32];
+    __shared__ long long wdrop[32];
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    for (int i = threadIdx.x; i < E * ld; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const int cs = kRcTok * k;                 // slots per chunk
+    const long long s0 = (long long)c0 * cs;
+    const long long s1 = min((long long)c1 * kRcTok, (long long)T) * k;
+    for (long long s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
+        const int e = idx[s];
+        if ((unsigned)e >= (unsigned)E) { raise_error(err, kErrIndex); continue; }
+        atomicAdd(&hist[e * ld + (int)(s - s0) / cs], 1);
+    }
+    __syncthreads();
+    // one flat scan over the expert-major rows (each row ends with a zero
+    // pad): entry (e, c) then counts the slots of experts < e, plus those of
+    // expert e in chunks before c; the row's first entry is subtracted below
+    block_exclusive_scan(hist, E * ld, wsum);
+    for (int e = threadIdx.x; e < E; e += blockDim.x) tot[e] = hist[e * ld + ld - 1] - hist[e * ld];
+    tc::cluster_sync();                        // every CTA's totals are complete and visible
+    const uint32_t tot_addr = tc::smem_u32(tot);
+    uint32_t peer[kCcCtas];
+#pragma unroll
+    for (int q = 0; q < kCcCtas; ++q) peer[q] = tc::map_to_rank(tot_addr, (uint32_t)q);
+    long long drop = 0;
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        int before = 0, all = 0;
+#pragma unroll
+        for (int q = 0; q < kCcCtas; ++q) {
+            const int v = (int)tc::ld_shared_cluster_u32(peer[q] + 4u * (uint32_t)e);
+            all += v;
+            if (q < r) before += v;
+        }
+        pre[e] = before - hist[e * ld];        // the row's start, subtracted once here
+        const int kept = (int)min((long long)all, cap);
+        kept_s[e] = kept;
+        if (r == 0) counts[e] = kept;
+        drop += all - kept;
+    }
+    drop = warp_sum(drop);
+    if (lane == 0) wdrop[wid] = drop;
+    tc::cluster_sync_relaxed();                // no CTA exits while another still reads its tot[]
+    __syncthreads();                           // pre[], kept_s[] and wdrop[] are complete
+    if (r == 0) {
+        const int rows = block_exclusive_scan(kept_s, E, wsum);
+        for (int e = threadIdx.x; e < E; e += blockDim.x) offsets[e] = kept_s[e];
+        if (threadIdx.x == 0) {
+            offsets[E] = rows;
+            long long d = 0;
+            for (int w = 0; w < nw; ++w) d += wdrop[w];
+            *dropped = (int32_t)d;
+        }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < ncc * E; i += blockDim.x) {
+        const int c = i / E, e = i - c * E;
+        chunk_base[(long long)c0 * E + i] = hist[e * ld + c] + pre[e];
+    }
+}
+
+__global__ void __launch_bounds__(32 * kRcTok) perm_rank_copy_kernel(
+    const uint8_t* __restrict__ x, int T, int row_bytes, int slot_bytes, const int32_t* __restrict__ idx, int k, int E,
+    const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ offsets, long long cap,
+    int32_t* __restrict__ row_map, int32_t* __restrict__ row_token, uint8_t* __restrict__ buffer, unsigned* err) {
+    extern __shared__ __align__(128) uint8_t rc_smem[];
+    __shared__ __align__(8) uint64_t bars[kRcTok];
+    __shared__ int no_abort;
+    int* base_s = (int*)(rc_smem + (size_t)kRcTok * slot_bytes);   // [E]
+    int* off_s = base_s + E;                   // [E]
+    int* wcnt = off_s + E;                     // [kRcTok][E]
+    int* keys_s = wcnt + kRcTok * E;           // [kRcTok * k]
+    int* rows_s = keys_s + kRcTok * k;         // [kRcTok * k]
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    const uint32_t slot = tc::smem_u32(rc_smem + (size_t)wid * slot_bytes);
+    const uint32_t bar = tc::smem_u32(&bars[wid]);
+    if (threadIdx.x == 0) no_abort = 0;
+    if (lane == 0) tc::mbar_init(bar, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncthreads();
+    pdl_wait();                                // chunk_base, offsets come from the kernel before
+    const long long t0 = (long long)blockIdx.x * kRcTok;
+    const int nt = (int)min((long long)kRcTok, (long long)T - t0);
+    const bool mine = wid < nt;                // this warp's token exists
+    if (lane == 0 && mine) {
+        tc::mbar_expect_tx(bar, (uint32_t)row_bytes);
+        tc::bulk_load(slot, x + (t0 + wid) * (long long)row_bytes, (uint32_t)row_bytes, bar);
+    }
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+        base_s[e] = chunk_base[(long long)blockIdx.x * E + e];
+        off_s[e] = offsets[e];
+    }
+    const long long s0 = t0 * k, s1 = (t0 + nt) * k;
+    for (long long s = s0 + threadIdx.x; s < s1; s += blockDim.x) keys_s[s - s0] = idx[s];
+    __syncthreads();
+    block_stable_ranks(
+        s0, s1, E, base_s, wcnt,
+        [&](long long s) -> int {
+            const int e = keys_s[s - s0];
+            if ((unsigned)e >= (unsigned)E) { raise_error(err, kErrIndex); return -1; }
+            return e;
+        },
+        [&](long long s, int key, int rank) {
+            int r = -1;
+            if (key >= 0 && rank < cap) {
+                r = off_s[key] + rank;
+                row_token[r] = (int32_t)(s / k);
+            }
+            row_map[s] = r;
+            rows_s[s - s0] = r;
+        });
+    __syncthreads();
+    if (!mine) return;
+    const int rr = lane < k ? rows_s[wid * k + lane] : -1;
+    const unsigned kept = __ballot_sync(0xffffffffu, rr >= 0);
+    int ok = 1;
+    if (lane == 0) ok = tc::mbar_wait(bar, 0, &no_abort) ? 1 : 0;
+    if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        if (lane == 0) {
+            raise_error(err, kErrTimeout);
+            tc::mbar_wait(bar, 0, &no_abort);  // the load may still land: let it, once more bounded
+        }
+        return;
+    }
+    unsigned m = kept;
+    while (m) {
+        const int q = __ffs(m) - 1;
+        m &= m - 1;
+        const int rq = __shfl_sync(0xffffffffu, rr, q);
+        if (lane == 0) tc::bulk_store(buffer + (long long)rq * row_bytes, slot, (uint32_t)row_bytes);
+    }
+    if (lane == 0 && kept) {
+        tc::bulk_commit();
+        tc::bulk_wait_read0();                 // the slot is read before the CTA's shared memory goes
+    }
+}
+
 int copy_grid(long long T) {
     long long warps = T;
     long long blocks = (warps + 7) / 8;
@@ -647,8 +861,19 @@ namespace {
 size_t al256(size_t b) { return (b + 255) & ~(size_t)255; }
 
 struct PermWs {
-    size_t cnt, base, total, code, gcnt, gbase, gtotal, bytes;
+    size_t cnt, base, total, code, gcnt, gbase, gtotal, cbase, bytes;
 };
+
+// Chunks per counting CTA of the two-launch expert-major path, 0 when the
+// chunk x expert counters do not fit one CTA's shared memory.
+int rc_chunks_per_cta(int T, int E) {
+    const long long nchunk = ((long long)T + kRcTok - 1) / kRcTok;
+    const long long cpc = (nchunk + kCcCtas - 1) / kCcCtas;
+    if (cpc < 1 || (cpc + 1) * E > kCcMaxInts) return 0;
+    return (int)cpc;
+}
+
+constexpr int kRcMaxSlot = 20 * 1024;      // row bytes (rounded to 128) the rank-and-copy CTA stages
 
 constexpr long long kFuseLimit = 16384;   // keys x blocks each consumer block scans itself
 
@@ -674,8 +899,25 @@ PermWs perm_layout(int T, int k, int E, int G) {
     } else {
         w.code = w.gcnt = w.gbase = w.gtotal = end;
     }
+    w.cbase = end;
+    if (G == 0 && rc_chunks_per_cta(T, E) > 0)
+        end = w.cbase + al256(sizeof(int32_t) * (size_t)ceil_div(T, kRcTok) * E);
     w.bytes = end;
     return w;
+}
+
+// The two-launch path wins where the ranking work is heavy: the clustered
+// top-6 shape (T k = 98304) 108 -> 99 us; at the Mixtral shape (T k =
+// 16384) the count and rank kernels are cheap and the separate bulk copy
+// moves the rows faster (45-47 against 49-50 us), so small problems keep
+// the three kernels.  LIBMOE_PERM_RANKCOPY=0/1 forces either; the tests
+// run both.
+constexpr long long kRankCopyMinSlots = 32768;
+
+bool rank_copy_enabled(long long slots) {
+    const char* env = getenv("LIBMOE_PERM_RANKCOPY");
+    if (env && (env[0] == '0' || env[0] == '1')) return env[0] == '1';
+    return slots >= kRankCopyMinSlots;
 }
 
 // LIBMOE_BULK_COPY=0/1 forces the vectorised or the bulk-copy row copy.
@@ -783,6 +1025,28 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
     int32_t* base = (int32_t*)(ws + L.base);
     int32_t* total = (int32_t*)(ws + L.total);
     const int nw = kIdxThreads / 32;
+    // expert-major with rows: counting cluster, then rank and copy per chunk
+    const int cpc = (!group_of_expert && x && d > 0) ? rc_chunks_per_cta(T, E) : 0;
+    const int slot_bytes = (int)((row_bytes + 127) / 128 * 128);
+    if (cpc > 0 && slot_bytes <= kRcMaxSlot && rank_copy_enabled((long long)T * k) && bulk_copy_enabled()) {
+        const int nchunk = ceil_div(T, kRcTok);
+        int32_t* cbase = (int32_t*)(ws + L.cbase);
+        const size_t cc_smem = sizeof(int) * ((size_t)(cpc + 1) * E + 3 * (size_t)E);
+        if (!set_smem_limit((const void*)perm_count_cluster_kernel, cc_smem)) return MOE_ERR_CUDA;
+        if (launch_pdl(perm_count_cluster_kernel, kCcCtas, kCcThreads, cc_smem, s, expert_idx, T, k, E, nchunk, cpc,
+                       cap, cbase, counts, offsets, dropped, err) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        MOE_LAUNCH_CHECK();
+        const size_t rc_smem = (size_t)kRcTok * slot_bytes +
+                               sizeof(int) * ((2 + kRcTok) * (size_t)E + 2 * (size_t)kRcTok * k);
+        if (!set_smem_limit((const void*)perm_rank_copy_kernel, rc_smem)) return MOE_ERR_CUDA;
+        if (launch_pdl(perm_rank_copy_kernel, nchunk, 32 * kRcTok, rc_smem, s, (const uint8_t*)x, T, (int)row_bytes,
+                       slot_bytes, expert_idx, k, E, (const int32_t*)cbase, (const int32_t*)offsets, cap, row_map,
+                       row_token, (uint8_t*)buffer, err) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        MOE_LAUNCH_CHECK();
+        return MOE_OK;
+    }
     // 1. per-block expert counts
     if (launch_pdl(perm_count_kernel, nblk, kIdxThreads, sizeof(int) * E, s, expert_idx, T, k, E, nblk, tb, cnt, err) != cudaSuccess)
         return MOE_ERR_CUDA;

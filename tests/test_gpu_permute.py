@@ -44,11 +44,16 @@ def routed(T, E, k, seed=3, skew=0.0):
     return O.route_topk(lg, k)[0]
 
 
-@pytest.fixture(params=["bulk", "vector"])
+@pytest.fixture(params=["rankcopy", "bulk", "vector"])
 def copy_kind(request, monkeypatch):
-    """Run a test with the bulk-copy row copy and with the vectorised one
-    (the library uses the bulk copy whenever rows fit its shared-memory slot)."""
-    monkeypatch.setenv("LIBMOE_BULK_COPY", "1" if request.param == "bulk" else "0")
+    """Run a test on each way the rows can be moved: the two-launch
+    expert-major path (counting cluster, then rank and copy per chunk of
+    tokens: the library's choice for expert-major rows that fit its
+    shared-memory slots), the count / rank / bulk-copy kernels, and the
+    count / rank / vectorised-copy kernels.  Group-major calls and calls
+    without rows take the count / rank kernels under every setting."""
+    monkeypatch.setenv("LIBMOE_BULK_COPY", "0" if request.param == "vector" else "1")
+    monkeypatch.setenv("LIBMOE_PERM_RANKCOPY", "1" if request.param == "rankcopy" else "0")
     return request.param
 
 
@@ -56,6 +61,9 @@ def copy_kind(request, monkeypatch):
     (1, 1, 1, 1.0, 8, False), (1, 4, 2, 0.5, 8, True), (33, 3, 1, 0.7, 4, False), (1000, 8, 2, 0.5, 40, False),
     (1000, 8, 2, 1.25, 64, True), (4099, 16, 4, 0.9, 24, True), (777, 1024, 32, 2.0, 16, True),
     (2000, 64, 6, 0.0, 8, True), (513, 5, 5, 1.0, 64, False),
+    (20011, 64, 6, 1.2, 16, True),                 # 2502 chunks of 8 tokens: 313 per counting CTA, the last 311
+    (300, 8, 2, 0.9, 10240, True),                 # 20 KB rows: the largest the rank-and-copy slots take
+    (300, 8, 2, 0.9, 10248, True),                 # one 16-byte vector more: rank, then the bulk copy
     (70001, 256, 8, 1.1, 8, True)])                # many index blocks: the scans run as separate kernels
 def test_expert_major(T, E, k, cf, d, bf16, copy_kind):
     idx = routed(T, E, k, skew=1.0)

@@ -79,6 +79,12 @@ def test_noalloc_matches_workspace_path_on_two_calls_in_a_row():
     # call 3: back to expert-major with drops, fp32 rows
     idx3, _ = O.route_topk(synth.normal_f32(9, 1, (3000, 16)), 4)
     compare(synth.normal_f32(9, 2, (3000, 20)), idx3, 16, 0.7)
+    # call 4: the clustered top-6 routing, large enough for the two-launch
+    # expert-major path (counting cluster, then rank and copy per chunk)
+    w4 = W.FINE
+    idx4, _ = O.route_topk(W.make_logits(w4), w4.k)
+    assert idx4.size >= 32768
+    compare(W.make_x(w4)[:, :256], idx4, w4.E, w4.capacity_factor)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
