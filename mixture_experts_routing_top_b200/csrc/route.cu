@@ -363,7 +363,8 @@ __global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __
     const int rows = (int)min((long long)tpb, (long long)T - t0);
     const float* src = logits + t0 * E;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    pdl_trigger();
+    pdl_trigger();                // the next kernel may be scheduled; it waits for this one
+    pdl_wait();                   // the kernel before may still read the workspace
     // this CTA's tokens start with no expert's membership bit set
     for (int i = threadIdx.x; i < rows * mask_words; i += blockDim.x) tokmask[t0 * mask_words + i] = 0u;
     // logits into shared memory (read from global once) and each row's max
@@ -380,12 +381,19 @@ __global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __
         if (lane == 0) rowv[r] = (double)m;
     }
     __syncthreads();
-    // every exp(l - m) in fp64, in parallel
+    // every exp(l - m) in fp64, in parallel; element f = r E + c, its row and
+    // column stepped along with f (no division per element)
     const int n = rows * E;
+    {
+        const int dr = blockDim.x / E, dc = blockDim.x - dr * E;
+        int r = threadIdx.x / E, c = threadIdx.x - r * E;
 #pragma unroll 4
-    for (int f = threadIdx.x; f < n; f += blockDim.x) {
-        const int r = f / E, c = f - r * E;
-        ex[r * ld + c] = exp((double)lg[r * ld + c] - rowv[r]);
+        for (int f = threadIdx.x; f < n; f += blockDim.x) {
+            ex[r * ld + c] = exp((double)lg[r * ld + c] - rowv[r]);
+            r += dr;
+            c += dc;
+            if (c >= E) { c -= E; ++r; }
+        }
     }
     __syncthreads();
     // ascending-expert sums, one thread per token
@@ -401,12 +409,19 @@ __global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __
     __syncthreads();
     // keys, transposed and coalesced, as their high and low 32-bit halves
     // (the selection reads the high halves first and the low ones rarely)
+    {
+        // element f = c rows + r (consecutive threads on consecutive tokens)
+        const int dc = blockDim.x / rows, dr = blockDim.x - dc * rows;
+        int c = threadIdx.x / rows, r = threadIdx.x - c * rows;
 #pragma unroll 4
-    for (int f = threadIdx.x; f < rows * E; f += blockDim.x) {
-        const int c = f / rows, r = f - c * rows;
-        const unsigned long long kb = key_bits((double)lg[r * ld + c] - rowv[r]);
-        keys_hi[(long long)c * T + t0 + r] = (unsigned)(kb >> 32);
-        keys_lo[(long long)c * T + t0 + r] = (unsigned)kb;
+        for (int f = threadIdx.x; f < n; f += blockDim.x) {
+            const unsigned long long kb = key_bits((double)lg[r * ld + c] - rowv[r]);
+            keys_hi[(long long)c * T + t0 + r] = (unsigned)(kb >> 32);
+            keys_lo[(long long)c * T + t0 + r] = (unsigned)kb;
+            c += dc;
+            r += dr;
+            if (r >= rows) { r -= rows; ++c; }
+        }
     }
 }
 
@@ -615,25 +630,32 @@ __device__ __forceinline__ void warp_find_boundary(const int* hist, int nbins, i
 
 // Shared-memory-resident variant (T <= kEcSmemTokens): the high 32 bits of
 // expert e's T keys are loaded once (coalesced, 8 loads in flight per
-// thread) and every radix pass and both compaction passes read them from
-// shared memory.  The threshold is resolved on the high half first; only if
-// the boundary bucket still has to be split are the low halves of the keys
-// whose high half equals the threshold's read from global memory (a second
-// radix over those tokens).  Same selection as ec_select_kernel.
+// thread) into shared memory.  Radix passes over all T keys (8-bit digits,
+// each warp counting into its own 256-bin histogram) run only until the
+// boundary bucket holds at most kEcCand keys; those tokens are then listed
+// once, and the remaining digits - of the high halves, then of the low
+// halves (read from global memory for the listed tokens only) - are
+// resolved over that list.  The selection is then written in one
+// classification pass over all tokens, whose per-32-token masks (above the
+// threshold, at it) are kept in shared memory for the pass that writes the
+// rows in token order.  Same selection as ec_select_kernel.
 constexpr int kEcSmemTokens = 49152;
+constexpr int kEcCand = 8192;                      // listed boundary-bucket tokens (the histograms' 32 KB)
 
 __global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned* __restrict__ keys_hi,
                                                               const unsigned* __restrict__ keys_lo, int T, int E, int C,
                                                               int32_t* __restrict__ ec_token,
                                                               unsigned* __restrict__ tokmask, int mask_words) {
-    extern __shared__ unsigned hi_keys[];          // [T], then 32 per-warp histograms of 256 bins
+    extern __shared__ unsigned hi_keys[];          // [T], then a 32 KB region: the per-warp histograms of the
+                                                   // full passes, then the token list, then the masks
     __shared__ int hist[256];
     __shared__ unsigned s_min, s_max, s_prefix, s_mask;
     __shared__ unsigned s_lprefix, s_lmask;
-    __shared__ int s_need, s_done, s_hi, s_level, s_bin, s_bneed, s_bcount;
+    __shared__ int s_need, s_done, s_hi, s_level, s_bin, s_bneed, s_bcount, s_ncand;
     __shared__ int w_above[32], w_tie[32];
     const int e = blockIdx.x;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    const unsigned lt = (1u << lane) - 1u;
     const unsigned* khi = keys_hi + (long long)e * T;
     const unsigned* klo = keys_lo + (long long)e * T;
     if (threadIdx.x == 0) { s_min = 0xFFFFFFFFu; s_max = 0u; }
@@ -663,6 +685,7 @@ __global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned* __
     if (threadIdx.x == 0) {
         s_need = C;
         s_level = 0;
+        s_bcount = T;                              // the bucket of the common prefix: every key
         const unsigned diff = s_min ^ s_max;
         if (diff == 0) { s_prefix = s_min; s_mask = 0xFFFFFFFFu; s_hi = -1; }
         else {
@@ -676,87 +699,105 @@ __global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned* __
         s_lprefix = 0; s_lmask = 0;
     }
     __syncthreads();
-    // level 0: radix on the high halves (shared memory only), each warp
-    // counting into its own 256-bin histogram (no cross-warp contention,
-    // no per-key warp vote), summed bin by bin afterwards
-    int* whist = reinterpret_cast<int*>(hi_keys + ((T + 3) & ~3));   // [32][256]
-    while (!s_done && s_hi >= 0) {
+    int* region = reinterpret_cast<int*>(hi_keys + ((T + 3) & ~3));   // 32 KB
+    // one radix step on `digit_of` over n items: histogram, boundary bucket,
+    // prefix update (h: the next bit to resolve; lo: digits of the low halves)
+    auto resolve = [&](auto item_key, int n, bool per_warp, bool lo) {
         const int hb = s_hi;
         const int shift = max(hb - 7, 0);
         const unsigned bins_mask = (1u << (hb - shift + 1)) - 1u;
-        for (int i = threadIdx.x; i < 32 * 256; i += blockDim.x) whist[i] = 0;
+        const unsigned prefix = lo ? s_lprefix : s_prefix, mask = lo ? s_lmask : s_mask;
+        if (per_warp) {
+            for (int i = threadIdx.x; i < 32 * 256; i += blockDim.x) region[i] = 0;
+        } else {
+            for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+        }
         __syncthreads();
-        const unsigned prefix = s_prefix, mask = s_mask;
-        int* mine = whist + wid * 256;
-        for (int t0 = 0; t0 < T; t0 += 4 * blockDim.x) {
+        int* mine = per_warp ? region + wid * 256 : hist;
+        for (int i0 = 0; i0 < n; i0 += 4 * blockDim.x) {
             unsigned h[4];
+            bool in[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const int t = t0 + q * blockDim.x + threadIdx.x;
-                h[q] = t < T ? hi_keys[t] : 0u;
+                const int i = i0 + q * blockDim.x + threadIdx.x;
+                in[q] = i < n && item_key(i, h[q]);
             }
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int t = t0 + q * blockDim.x + threadIdx.x;
-                if (t < T && (h[q] & mask) == prefix) atomicAdd(&mine[(h[q] >> shift) & bins_mask], 1);
-            }
+            for (int q = 0; q < 4; ++q)
+                if (in[q] && (h[q] & mask) == prefix) atomicAdd(&mine[(h[q] >> shift) & bins_mask], 1);
         }
         __syncthreads();
-        for (int b = threadIdx.x; b < 256; b += blockDim.x) {
-            int sum = 0;
+        if (per_warp) {
+            for (int bn = threadIdx.x; bn < 256; bn += blockDim.x) {
+                int sum = 0;
 #pragma unroll 8
-            for (int w = 0; w < 32; ++w) sum += whist[w * 256 + b];
-            hist[b] = sum;
+                for (int w = 0; w < 32; ++w) sum += region[w * 256 + bn];
+                hist[bn] = sum;
+            }
+            __syncthreads();
         }
-        __syncthreads();
         if (wid == 0) warp_find_boundary(hist, (int)bins_mask + 1, s_need, &s_bin, &s_bneed, &s_bcount);
         __syncthreads();
         if (threadIdx.x == 0) {
-            const int dgt = s_bin;
-            s_prefix = prefix | ((unsigned)dgt << shift);
-            s_mask = mask | (bins_mask << shift);
+            const unsigned np = prefix | ((unsigned)s_bin << shift), nm = mask | (bins_mask << shift);
+            if (lo) { s_lprefix = np; s_lmask = nm; } else { s_prefix = np; s_mask = nm; }
             s_need = s_bneed;
-            if (s_bcount == s_bneed) s_done = 1;
+            if (s_bcount == s_bneed || (lo && shift == 0)) s_done = 1;
             s_hi = shift - 1;
         }
         __syncthreads();
-    }
-    // level 1: split the boundary bucket on the low halves (global loads of
-    // the few tokens whose high half equals the threshold's)
-    if (!s_done) {
-        if (threadIdx.x == 0) { s_level = 1; s_hi = 31; s_lprefix = 0; s_lmask = 0; }
+    };
+    auto all_hi = [&](int i, unsigned& h) { h = hi_keys[i]; return true; };
+    // full passes while the boundary bucket is too large to list
+    while (!s_done && s_hi >= 0 && s_bcount > kEcCand) resolve(all_hi, T, true, false);
+    bool listed = false;
+    if (!s_done && s_bcount <= kEcCand) {
+        // list the boundary bucket's tokens (token order is not needed here)
+        if (threadIdx.x == 0) s_ncand = 0;
         __syncthreads();
-        const unsigned hprefix = s_prefix;
-        while (!s_done && s_hi >= 0) {
-            const int hb = s_hi;
-            const int shift = max(hb - 7, 0);
-            const unsigned bins_mask = (1u << (hb - shift + 1)) - 1u;
-            for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-            __syncthreads();
-            const unsigned lprefix = s_lprefix, lmask = s_lmask;
-            for (int t0 = 0; t0 < T; t0 += blockDim.x) {
-                const int t = t0 + threadIdx.x;
-                int digit = -1;
-                if (t < T && hi_keys[t] == hprefix) {
-                    const unsigned lo = klo[t];
-                    if ((lo & lmask) == lprefix) digit = (int)((lo >> shift) & bins_mask);
-                }
-                const unsigned peers = __match_any_sync(0xffffffffu, digit);
-                if (digit >= 0 && (peers & ((1u << lane) - 1u)) == 0) atomicAdd(&hist[digit], __popc(peers));
-            }
-            __syncthreads();
-            if (wid == 0) warp_find_boundary(hist, (int)bins_mask + 1, s_need, &s_bin, &s_bneed, &s_bcount);
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                const int dgt = s_bin;
-                s_lprefix = lprefix | ((unsigned)dgt << shift);
-                s_lmask = lmask | (bins_mask << shift);
-                s_need = s_bneed;
-                if (s_bcount == s_bneed || shift == 0) s_done = 1;
-                s_hi = shift - 1;
-            }
-            __syncthreads();
+        const unsigned prefix = s_prefix, mask = s_mask;
+        for (int t0 = 0; t0 < T; t0 += blockDim.x) {
+            const int t = t0 + threadIdx.x;
+            const bool in = t < T && (hi_keys[t] & mask) == prefix;
+            const unsigned b = __ballot_sync(0xffffffffu, in);
+            int base = 0;
+            if (lane == 0 && b) base = atomicAdd(&s_ncand, __popc(b));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            const int slot = base + __popc(b & lt);
+            if (in && slot < kEcCand) region[slot] = t;
         }
+        __syncthreads();
+        listed = true;
+        const int nc = min(s_ncand, kEcCand);
+        auto cand_hi = [&](int i, unsigned& h) { h = hi_keys[region[i]]; return true; };
+        while (!s_done && s_hi >= 0) resolve(cand_hi, nc, false, false);
+        if (!s_done) {
+            // the high halves are exhausted: digits of the low halves of the
+            // listed tokens whose high half is the threshold's
+            if (threadIdx.x == 0) { s_level = 1; s_hi = 31; }
+            __syncthreads();
+            const unsigned hp = s_prefix;
+            auto cand_lo = [&](int i, unsigned& h) {
+                const int t = region[i];
+                if (hi_keys[t] != hp) return false;
+                h = klo[t];
+                return true;
+            };
+            while (!s_done && s_hi >= 0) resolve(cand_lo, nc, false, true);
+        }
+    }
+    if (!s_done && !listed) {
+        // more than kEcCand tokens share the threshold's high half (inputs
+        // with many equal keys): digits of the low halves over all tokens
+        if (threadIdx.x == 0) { s_level = 1; s_hi = 31; }
+        __syncthreads();
+        const unsigned hp = s_prefix;
+        auto all_lo = [&](int t, unsigned& h) {
+            if (hi_keys[t] != hp) return false;
+            h = klo[t];
+            return true;
+        };
+        while (!s_done && s_hi >= 0) resolve(all_lo, T, false, true);
     }
     const unsigned prefix = s_prefix, mask = s_mask, lprefix = s_lprefix, lmask = s_lmask;
     const int need = s_need, level = s_level;
@@ -770,34 +811,40 @@ __global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned* __
         if (lo != lprefix) return lo > lprefix ? 1 : 0;
         return 2;
     };
-    const int S = (T + nw - 1) / nw;
-    const int seg0 = min(wid * S, T), seg1 = min(seg0 + S, T);
-    const unsigned lt = (1u << lane) - 1u;
+    // each warp a contiguous run of 32-token words; the words' masks stay in
+    // shared memory (the list is no longer needed) for the writing pass
+    const int nwords = (T + 31) >> 5;
+    unsigned* m_above = reinterpret_cast<unsigned*>(region);
+    unsigned* m_tie = m_above + nwords;
+    const int wper = (nwords + nw - 1) / nw;
+    const int w0 = min(wid * wper, nwords), w1 = min(w0 + wper, nwords);
     int n_above = 0, n_tie = 0;
-    for (int c = seg0; c < seg1; c += 32) {
-        const int t = c + lane;
-        const int cl = t < seg1 ? classify(t) : 0;
-        n_above += __popc(__ballot_sync(0xffffffffu, cl == 1));
-        n_tie += __popc(__ballot_sync(0xffffffffu, cl == 2));
+    for (int w = w0; w < w1; ++w) {
+        const int t = 32 * w + lane;
+        const int cl = t < T ? classify(t) : 0;
+        const unsigned ab = __ballot_sync(0xffffffffu, cl == 1);
+        const unsigned tb = __ballot_sync(0xffffffffu, cl == 2);
+        if (lane == 0) { m_above[w] = ab; m_tie[w] = tb; }
+        n_above += __popc(ab);
+        n_tie += __popc(tb);
     }
     if (lane == 0) { w_above[wid] = n_above; w_tie[wid] = n_tie; }
     __syncthreads();
     int above_base = 0, tie_base = 0;
     for (int q = 0; q < wid; ++q) { above_base += w_above[q]; tie_base += w_tie[q]; }
     int sel_base = above_base + min(tie_base, need);
-    for (int c = seg0; c < seg1; c += 32) {
-        const int t = c + lane;
-        const int cl = t < seg1 ? classify(t) : 0;
-        const unsigned tie_mask = __ballot_sync(0xffffffffu, cl == 2);
-        const int tie_rank = tie_base + __popc(tie_mask & lt);
-        const bool sel = cl == 1 || (cl == 2 && tie_rank < need);
+    for (int w = w0; w < w1; ++w) {
+        const int t = 32 * w + lane;
+        const unsigned ab = m_above[w], tb = m_tie[w];
+        const int tie_rank = tie_base + __popc(tb & lt);
+        const bool sel = ((ab >> lane) & 1u) || (((tb >> lane) & 1u) && tie_rank < need);
         const unsigned sel_mask = __ballot_sync(0xffffffffu, sel);
         if (sel) {
             const long long r = (long long)e * C + sel_base + __popc(sel_mask & lt);
             ec_token[r] = t;
             atomicOr(&tokmask[(long long)t * mask_words + (e >> 5)], 1u << (e & 31));
         }
-        tie_base += __popc(tie_mask);
+        tie_base += __popc(tb);
         sel_base += __popc(sel_mask);
     }
 }
@@ -1003,8 +1050,9 @@ extern "C" moe_status moe_route_ec(const float* logits, int T, int E, int C, int
         const int tpb = ec_tokens_per_block(E);
         const size_t smem = (size_t)tpb * ((E + 2) * sizeof(double) + (E + 1) * sizeof(float));
         if (!set_smem_limit((const void*)ec_lse_keys_kernel, smem)) return MOE_ERR_CUDA;
-        ec_lse_keys_kernel<<<ceil_div(T, tpb), kEcThreads, smem, s>>>(logits, T, E, tpb, lse, keys_hi, keys_lo, mask,
-                                                                      mw);
+        if (launch_pdl(ec_lse_keys_kernel, ceil_div(T, tpb), kEcThreads, smem, s, logits, T, E, tpb, lse, keys_hi,
+                       keys_lo, mask, mw) != cudaSuccess)
+            return MOE_ERR_CUDA;
         MOE_LAUNCH_CHECK();
     }
     cudaError_t rc;
@@ -1019,7 +1067,8 @@ extern "C" moe_status moe_route_ec(const float* logits, int T, int E, int C, int
     }
     if (rc != cudaSuccess) return MOE_ERR_CUDA;
     MOE_LAUNCH_CHECK();
-    ec_count_scan_kernel<<<kScanCtas, 1024, 0, s>>>(mask, T, mw, tok_ptr);
+    if (launch_pdl(ec_count_scan_kernel, kScanCtas, 1024, 0, s, (const unsigned*)mask, T, mw, tok_ptr) != cudaSuccess)
+        return MOE_ERR_CUDA;
     MOE_LAUNCH_CHECK();
     const long long rows = (long long)E * C;
     if (launch_pdl(ec_fill_kernel, (int)((rows + 255) / 256), 256, 0, s, (const int32_t*)ec_token, T, E, C,
