@@ -342,6 +342,9 @@ __device__ __forceinline__ unsigned long long key_bits(double x) {
 }
 
 // A CTA takes `tpb` consecutive tokens (one contiguous span of logits).
+// It writes each token's lse and, transposed ([e][t]), either the keys'
+// selection bins (the binned selection) or the keys' high and low 32-bit
+// halves (the selection from global memory, for larger T).
 // Everything order-independent runs in parallel over the CTA's tokens x
 // experts: the copy into shared memory, each row's max, every
 // exp(l - m) in fp64; only the additions run one thread per token, over the
@@ -350,10 +353,22 @@ __device__ __forceinline__ unsigned long long key_bits(double x) {
 // consecutive threads on consecutive tokens.
 constexpr int kEcThreads = 256;
 
+// Selection bins of the expert-choice keys: key = l - lse <= 0, bin =
+// floor(-256 key) clamped to kEcBins - 1 (bins 1/256 wide over [-16, 0],
+// every key below -16 in the last).  A larger key never has a larger bin:
+// every key in a bin before the boundary bin beats every key in or after
+// it, so only the boundary bin's keys are compared exactly.
+constexpr int kEcBins = 4096;
+__device__ __forceinline__ int ec_bin(double key) {
+    const double y = -key * 256.0;
+    return y >= (double)(kEcBins - 1) ? kEcBins - 1 : (y > 0.0 ? (int)y : 0);
+}
+
 __global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __restrict__ logits, int T, int E, int tpb,
                                                                  double* __restrict__ lse_out,
                                                                  unsigned* __restrict__ keys_hi,
                                                                  unsigned* __restrict__ keys_lo,
+                                                                 uint16_t* __restrict__ bins,
                                                                  unsigned* __restrict__ tokmask, int mask_words) {
     extern __shared__ double ex[];                 // [tpb][E+1] exps (padded rows), [tpb] row max / lse, then
     const int ld = E + 1;                          // [tpb][E+1] the logits as floats (padded rows)
@@ -415,9 +430,14 @@ __global__ void __launch_bounds__(kEcThreads) ec_lse_keys_kernel(const float* __
         int c = threadIdx.x / rows, r = threadIdx.x - c * rows;
 #pragma unroll 4
         for (int f = threadIdx.x; f < n; f += blockDim.x) {
-            const unsigned long long kb = key_bits((double)lg[r * ld + c] - rowv[r]);
-            keys_hi[(long long)c * T + t0 + r] = (unsigned)(kb >> 32);
-            keys_lo[(long long)c * T + t0 + r] = (unsigned)kb;
+            const double key = (double)lg[r * ld + c] - rowv[r];
+            if (bins) {
+                bins[(long long)c * T + t0 + r] = (uint16_t)ec_bin(key);
+            } else {
+                const unsigned long long kb = key_bits(key);
+                keys_hi[(long long)c * T + t0 + r] = (unsigned)(kb >> 32);
+                keys_lo[(long long)c * T + t0 + r] = (unsigned)kb;
+            }
             c += dc;
             r += dr;
             if (r >= rows) { r -= rows; ++c; }
@@ -628,224 +648,192 @@ __device__ __forceinline__ void warp_find_boundary(const int* hist, int nbins, i
     }
 }
 
-// Shared-memory-resident variant (T <= kEcSmemTokens): the high 32 bits of
-// expert e's T keys are loaded once (coalesced, 8 loads in flight per
-// thread) into shared memory.  Radix passes over all T keys (8-bit digits,
-// each warp counting into its own 256-bin histogram) run only until the
-// boundary bucket holds at most kEcCand keys; those tokens are then listed
-// once, and the remaining digits - of the high halves, then of the low
-// halves (read from global memory for the listed tokens only) - are
-// resolved over that list.  The selection is then written in one
-// classification pass over all tokens, whose per-32-token masks (above the
-// threshold, at it) are kept in shared memory for the pass that writes the
-// rows in token order.  Same selection as ec_select_kernel.
-constexpr int kEcSmemTokens = 49152;
-constexpr int kEcCand = 8192;                      // listed boundary-bucket tokens (the histograms' 32 KB)
+// Binned selection (T <= kEcBinTokens): one 1024-thread CTA per expert.
+// The expert's T key bins are loaded once into shared memory and counted;
+// the boundary bin is the bin, from the best, where the running count
+// reaches C.  Tokens in earlier bins are selected, in later bins not.  The
+// boundary bin is taken whole when it holds exactly the C - (earlier) keys
+// still needed; otherwise its tokens' exact keys (l - lse in fp64,
+// recomputed from the logits and the lse as the key kernel computes them)
+// decide: ranked pairwise (key descending, then token ascending) when the
+// bin holds at most kEcBrute tokens, else by an 8-bit radix select over the
+// 64-bit order-preserving keys (ties at the end resolved in token order).
+// The selection is written in token order: one classification pass over
+// all tokens keeps per-32-token masks (selected, at the threshold) in
+// shared memory, then a second pass writes the rows.  Also sets the
+// token-membership bits used to build the token CSR.
+constexpr int kEcBinTokens = 65536;
+constexpr int kEcBrute = 256;
 
-__global__ void __launch_bounds__(1024) ec_select_smem_kernel(const unsigned* __restrict__ keys_hi,
-                                                              const unsigned* __restrict__ keys_lo, int T, int E, int C,
+__global__ void __launch_bounds__(1024) ec_select_bins_kernel(const uint16_t* __restrict__ bins,
+                                                              const float* __restrict__ logits,
+                                                              const double* __restrict__ lse, int T, int E, int C,
                                                               int32_t* __restrict__ ec_token,
                                                               unsigned* __restrict__ tokmask, int mask_words) {
-    extern __shared__ unsigned hi_keys[];          // [T], then a 32 KB region: the per-warp histograms of the
-                                                   // full passes, then the token list, then the masks
-    __shared__ int hist[256];
-    __shared__ unsigned s_min, s_max, s_prefix, s_mask;
-    __shared__ unsigned s_lprefix, s_lmask;
-    __shared__ int s_need, s_done, s_hi, s_level, s_bin, s_bneed, s_bcount, s_ncand;
-    __shared__ int w_above[32], w_tie[32];
+    extern __shared__ __align__(16) unsigned char ec_sm[];
+    const int nwords = (T + 31) >> 5;
+    int* hist = reinterpret_cast<int*>(ec_sm);                              // [kEcBins]
+    unsigned long long* ckey = reinterpret_cast<unsigned long long*>(hist + kEcBins);   // [kEcBrute]
+    int* ctok = reinterpret_cast<int*>(ckey + kEcBrute);                    // [kEcBrute]
+    unsigned* m_sel = reinterpret_cast<unsigned*>(ctok + kEcBrute);         // [nwords] selected
+    unsigned* m_tie = m_sel + nwords;                                       // [nwords] at the threshold
+    unsigned* chosen = m_tie + nwords;                                      // [nwords] ranked pairwise and kept
+    uint16_t* bs = reinterpret_cast<uint16_t*>(chosen + nwords);            // [T]
+    __shared__ int sh[32];
+    __shared__ int s_bin, s_need, s_bcount, s_nc, s_done, s_rbin, s_rneed, s_rcount;
+    __shared__ unsigned long long s_prefix, s_mask;
+    __shared__ int w_sel[32], w_tie[32];
     const int e = blockIdx.x;
     const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
     const unsigned lt = (1u << lane) - 1u;
-    const unsigned* khi = keys_hi + (long long)e * T;
-    const unsigned* klo = keys_lo + (long long)e * T;
-    if (threadIdx.x == 0) { s_min = 0xFFFFFFFFu; s_max = 0u; }
+    for (int i = threadIdx.x; i < kEcBins; i += blockDim.x) hist[i] = 0;
+    for (int i = threadIdx.x; i < nwords; i += blockDim.x) chosen[i] = 0u;
     __syncthreads();
-    pdl_wait();
-    unsigned lmin = 0xFFFFFFFFu, lmax = 0u;
+    pdl_wait();                                    // the bins come from the kernel before
+    const uint16_t* src = bins + (long long)e * T;
     for (int t0 = 0; t0 < T; t0 += 8 * blockDim.x) {
-        unsigned u[8];
+        int u[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
             const int t = t0 + q * blockDim.x + threadIdx.x;
-            u[q] = t < T ? khi[t] : 0u;
+            u[q] = t < T ? (int)src[t] : -1;
         }
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-            const int t = t0 + q * blockDim.x + threadIdx.x;
-            if (t < T) {
-                hi_keys[t] = u[q];
-                lmin = min(lmin, u[q]);
-                lmax = max(lmax, u[q]);
+            if (u[q] < 0) continue;
+            bs[t0 + q * blockDim.x + threadIdx.x] = (uint16_t)u[q];
+            atomicAdd(&hist[u[q]], 1);
+        }
+    }
+    __syncthreads();
+    {
+        // each thread 4 consecutive bins; the one whose bins hold the C-th key finds the boundary bin
+        constexpr int per = kEcBins / 1024;
+        int c[per], sum = 0;
+#pragma unroll
+        for (int j = 0; j < per; ++j) {
+            c[j] = hist[per * threadIdx.x + j];
+            sum += c[j];
+        }
+        int total;
+        int cum = block_exclusive_scan(sum, &total, sh);
+        if (cum < C && cum + sum >= C) {
+#pragma unroll
+            for (int j = 0; j < per; ++j) {
+                if (cum + c[j] >= C) {
+                    s_bin = per * threadIdx.x + j;
+                    s_need = C - cum;
+                    s_bcount = c[j];
+                    break;
+                }
+                cum += c[j];
             }
         }
     }
-    atomicMin(&s_min, lmin);
-    atomicMax(&s_max, lmax);
     __syncthreads();
-    if (threadIdx.x == 0) {
-        s_need = C;
-        s_level = 0;
-        s_bcount = T;                              // the bucket of the common prefix: every key
-        const unsigned diff = s_min ^ s_max;
-        if (diff == 0) { s_prefix = s_min; s_mask = 0xFFFFFFFFu; s_hi = -1; }
-        else {
-            const int hb = 31 - __clz(diff);
-            const unsigned low = (hb == 31) ? 0xFFFFFFFFu : ((1u << (hb + 1)) - 1u);
-            s_mask = ~low;
-            s_prefix = s_min & ~low;
-            s_hi = hb;
-        }
-        s_done = 0;
-        s_lprefix = 0; s_lmask = 0;
-    }
-    __syncthreads();
-    int* region = reinterpret_cast<int*>(hi_keys + ((T + 3) & ~3));   // 32 KB
-    // one radix step on `digit_of` over n items: histogram, boundary bucket,
-    // prefix update (h: the next bit to resolve; lo: digits of the low halves)
-    auto resolve = [&](auto item_key, int n, bool per_warp, bool lo) {
-        const int hb = s_hi;
-        const int shift = max(hb - 7, 0);
-        const unsigned bins_mask = (1u << (hb - shift + 1)) - 1u;
-        const unsigned prefix = lo ? s_lprefix : s_prefix, mask = lo ? s_lmask : s_mask;
-        if (per_warp) {
-            for (int i = threadIdx.x; i < 32 * 256; i += blockDim.x) region[i] = 0;
-        } else {
-            for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-        }
+    const int bstar = s_bin;
+    int need = s_need;
+    const int bcount = s_bcount;
+    const int mode = bcount == need ? 0 : (bcount <= kEcBrute ? 1 : 2);
+    auto exact_key = [&](int t) { return key_bits((double)logits[(long long)t * E + e] - lse[t]); };
+    if (mode == 1) {
+        // the boundary bin's tokens and exact keys, then pairwise ranks
+        if (threadIdx.x == 0) s_nc = 0;
         __syncthreads();
-        int* mine = per_warp ? region + wid * 256 : hist;
-        for (int i0 = 0; i0 < n; i0 += 4 * blockDim.x) {
-            unsigned h[4];
-            bool in[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const int i = i0 + q * blockDim.x + threadIdx.x;
-                in[q] = i < n && item_key(i, h[q]);
-            }
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (in[q] && (h[q] & mask) == prefix) atomicAdd(&mine[(h[q] >> shift) & bins_mask], 1);
-        }
-        __syncthreads();
-        if (per_warp) {
-            for (int bn = threadIdx.x; bn < 256; bn += blockDim.x) {
-                int sum = 0;
-#pragma unroll 8
-                for (int w = 0; w < 32; ++w) sum += region[w * 256 + bn];
-                hist[bn] = sum;
-            }
-            __syncthreads();
-        }
-        if (wid == 0) warp_find_boundary(hist, (int)bins_mask + 1, s_need, &s_bin, &s_bneed, &s_bcount);
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            const unsigned np = prefix | ((unsigned)s_bin << shift), nm = mask | (bins_mask << shift);
-            if (lo) { s_lprefix = np; s_lmask = nm; } else { s_prefix = np; s_mask = nm; }
-            s_need = s_bneed;
-            if (s_bcount == s_bneed || (lo && shift == 0)) s_done = 1;
-            s_hi = shift - 1;
-        }
-        __syncthreads();
-    };
-    auto all_hi = [&](int i, unsigned& h) { h = hi_keys[i]; return true; };
-    // full passes while the boundary bucket is too large to list
-    while (!s_done && s_hi >= 0 && s_bcount > kEcCand) resolve(all_hi, T, true, false);
-    bool listed = false;
-    if (!s_done && s_bcount <= kEcCand) {
-        // list the boundary bucket's tokens (token order is not needed here)
-        if (threadIdx.x == 0) s_ncand = 0;
-        __syncthreads();
-        const unsigned prefix = s_prefix, mask = s_mask;
         for (int t0 = 0; t0 < T; t0 += blockDim.x) {
             const int t = t0 + threadIdx.x;
-            const bool in = t < T && (hi_keys[t] & mask) == prefix;
-            const unsigned b = __ballot_sync(0xffffffffu, in);
+            const bool in = t < T && bs[t] == bstar;
+            const unsigned bm = __ballot_sync(0xffffffffu, in);
             int base = 0;
-            if (lane == 0 && b) base = atomicAdd(&s_ncand, __popc(b));
+            if (lane == 0 && bm) base = atomicAdd(&s_nc, __popc(bm));
             base = __shfl_sync(0xffffffffu, base, 0);
-            const int slot = base + __popc(b & lt);
-            if (in && slot < kEcCand) region[slot] = t;
+            const int slot = base + __popc(bm & lt);
+            if (in && slot < kEcBrute) {
+                ctok[slot] = t;
+                ckey[slot] = exact_key(t);
+            }
         }
         __syncthreads();
-        listed = true;
-        const int nc = min(s_ncand, kEcCand);
-        auto cand_hi = [&](int i, unsigned& h) { h = hi_keys[region[i]]; return true; };
-        while (!s_done && s_hi >= 0) resolve(cand_hi, nc, false, false);
-        if (!s_done) {
-            // the high halves are exhausted: digits of the low halves of the
-            // listed tokens whose high half is the threshold's
-            if (threadIdx.x == 0) { s_level = 1; s_hi = 31; }
+        const int nc = min(s_nc, kEcBrute);
+        if ((int)threadIdx.x < nc) {
+            const unsigned long long k0 = ckey[threadIdx.x];
+            const int t = ctok[threadIdx.x];
+            int rank = 0;
+            for (int j = 0; j < nc; ++j) {
+                const unsigned long long kj = ckey[j];
+                rank += (kj > k0 || (kj == k0 && ctok[j] < t)) ? 1 : 0;
+            }
+            if (rank < need) atomicOr(&chosen[t >> 5], 1u << (t & 31));
+        }
+        __syncthreads();
+    } else if (mode == 2) {
+        // radix over the boundary bin's 64-bit keys, from the top byte
+        if (threadIdx.x == 0) { s_prefix = 0ull; s_mask = 0ull; s_done = 0; s_rneed = need; }
+        __syncthreads();
+        for (int shift = 56; shift >= 0 && !s_done; shift -= 8) {
+            const unsigned long long prefix = s_prefix, mask = s_mask;
+            for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
             __syncthreads();
-            const unsigned hp = s_prefix;
-            auto cand_lo = [&](int i, unsigned& h) {
-                const int t = region[i];
-                if (hi_keys[t] != hp) return false;
-                h = klo[t];
-                return true;
-            };
-            while (!s_done && s_hi >= 0) resolve(cand_lo, nc, false, true);
+            for (int t0 = 0; t0 < T; t0 += blockDim.x) {
+                const int t = t0 + threadIdx.x;
+                if (t < T && bs[t] == bstar) {
+                    const unsigned long long k0 = exact_key(t);
+                    if ((k0 & mask) == prefix) atomicAdd(&hist[(int)((k0 >> shift) & 255ull)], 1);
+                }
+            }
+            __syncthreads();
+            if (wid == 0) warp_find_boundary(hist, 256, s_rneed, &s_rbin, &s_rneed, &s_rcount);
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                s_prefix = prefix | ((unsigned long long)s_rbin << shift);
+                s_mask = mask | (255ull << shift);
+                if (s_rcount == s_rneed) s_done = 1;
+            }
+            __syncthreads();
         }
+        need = s_rneed;
     }
-    if (!s_done && !listed) {
-        // more than kEcCand tokens share the threshold's high half (inputs
-        // with many equal keys): digits of the low halves over all tokens
-        if (threadIdx.x == 0) { s_level = 1; s_hi = 31; }
-        __syncthreads();
-        const unsigned hp = s_prefix;
-        auto all_lo = [&](int t, unsigned& h) {
-            if (hi_keys[t] != hp) return false;
-            h = klo[t];
-            return true;
-        };
-        while (!s_done && s_hi >= 0) resolve(all_lo, T, false, true);
-    }
-    const unsigned prefix = s_prefix, mask = s_mask, lprefix = s_lprefix, lmask = s_lmask;
-    const int need = s_need, level = s_level;
-    // classify a token: 1 above the threshold, 2 tie at it, 0 below
+    const unsigned long long prefix = s_prefix, mask = s_mask;
+    // 1 selected, 2 at the threshold (radix mode: tie order decides), 0 not
     auto classify = [&](int t) -> int {
-        const unsigned h = hi_keys[t] & mask;
-        if (h != prefix) return h > prefix ? 1 : 0;
-        if (level == 0) return 2;
-        if (hi_keys[t] != prefix) return hi_keys[t] > prefix ? 1 : 0;   // differs below the high mask
-        const unsigned lo = klo[t] & lmask;
-        if (lo != lprefix) return lo > lprefix ? 1 : 0;
+        const int b = bs[t];
+        if (b != bstar) return b < bstar ? 1 : 0;
+        if (mode == 0) return 1;
+        if (mode == 1) return (int)((chosen[t >> 5] >> (t & 31)) & 1u);
+        const unsigned long long km = exact_key(t) & mask;
+        if (km != prefix) return km > prefix ? 1 : 0;
         return 2;
     };
-    // each warp a contiguous run of 32-token words; the words' masks stay in
-    // shared memory (the list is no longer needed) for the writing pass
-    const int nwords = (T + 31) >> 5;
-    unsigned* m_above = reinterpret_cast<unsigned*>(region);
-    unsigned* m_tie = m_above + nwords;
     const int wper = (nwords + nw - 1) / nw;
     const int w0 = min(wid * wper, nwords), w1 = min(w0 + wper, nwords);
-    int n_above = 0, n_tie = 0;
+    int n_sel = 0, n_tie = 0;
     for (int w = w0; w < w1; ++w) {
         const int t = 32 * w + lane;
         const int cl = t < T ? classify(t) : 0;
-        const unsigned ab = __ballot_sync(0xffffffffu, cl == 1);
+        const unsigned sb = __ballot_sync(0xffffffffu, cl == 1);
         const unsigned tb = __ballot_sync(0xffffffffu, cl == 2);
-        if (lane == 0) { m_above[w] = ab; m_tie[w] = tb; }
-        n_above += __popc(ab);
+        if (lane == 0) { m_sel[w] = sb; m_tie[w] = tb; }
+        n_sel += __popc(sb);
         n_tie += __popc(tb);
     }
-    if (lane == 0) { w_above[wid] = n_above; w_tie[wid] = n_tie; }
+    if (lane == 0) { w_sel[wid] = n_sel; w_tie[wid] = n_tie; }
     __syncthreads();
-    int above_base = 0, tie_base = 0;
-    for (int q = 0; q < wid; ++q) { above_base += w_above[q]; tie_base += w_tie[q]; }
-    int sel_base = above_base + min(tie_base, need);
+    int sel_before = 0, tie_base = 0;
+    for (int q = 0; q < wid; ++q) { sel_before += w_sel[q]; tie_base += w_tie[q]; }
+    int out_base = sel_before + min(tie_base, need);
     for (int w = w0; w < w1; ++w) {
         const int t = 32 * w + lane;
-        const unsigned ab = m_above[w], tb = m_tie[w];
+        const unsigned sb = m_sel[w], tb = m_tie[w];
         const int tie_rank = tie_base + __popc(tb & lt);
-        const bool sel = ((ab >> lane) & 1u) || (((tb >> lane) & 1u) && tie_rank < need);
+        const bool sel = ((sb >> lane) & 1u) || (((tb >> lane) & 1u) && tie_rank < need);
         const unsigned sel_mask = __ballot_sync(0xffffffffu, sel);
         if (sel) {
-            const long long r = (long long)e * C + sel_base + __popc(sel_mask & lt);
+            const long long r = (long long)e * C + out_base + __popc(sel_mask & lt);
             ec_token[r] = t;
             atomicOr(&tokmask[(long long)t * mask_words + (e >> 5)], 1u << (e & 31));
         }
         tie_base += __popc(tb);
-        sel_base += __popc(sel_mask);
+        out_base += __popc(sel_mask);
     }
 }
 
@@ -1046,20 +1034,24 @@ extern "C" moe_status moe_route_ec(const float* logits, int T, int E, int C, int
     unsigned* keys_lo = keys_hi + (size_t)T * E;
     unsigned* mask = (unsigned*)(ws + L.mask);
     const int mw = (E + 31) / 32;
+    const bool binned = T <= kEcBinTokens;
+    uint16_t* bins = binned ? reinterpret_cast<uint16_t*>(keys_hi) : nullptr;   // the keys' space holds the bins
     {
         const int tpb = ec_tokens_per_block(E);
         const size_t smem = (size_t)tpb * ((E + 2) * sizeof(double) + (E + 1) * sizeof(float));
         if (!set_smem_limit((const void*)ec_lse_keys_kernel, smem)) return MOE_ERR_CUDA;
         if (launch_pdl(ec_lse_keys_kernel, ceil_div(T, tpb), kEcThreads, smem, s, logits, T, E, tpb, lse, keys_hi,
-                       keys_lo, mask, mw) != cudaSuccess)
+                       keys_lo, bins, mask, mw) != cudaSuccess)
             return MOE_ERR_CUDA;
         MOE_LAUNCH_CHECK();
     }
     cudaError_t rc;
-    if (T <= kEcSmemTokens) {
-        const size_t smem = sizeof(unsigned) * (size_t)((T + 3) & ~3) + sizeof(int) * 32 * 256;
-        if (!set_smem_limit((const void*)ec_select_smem_kernel, smem)) return MOE_ERR_CUDA;
-        rc = launch_pdl(ec_select_smem_kernel, E, 1024, smem, s, (const unsigned*)keys_hi, (const unsigned*)keys_lo, T,
+    if (binned) {
+        const size_t nwords = (size_t)(T + 31) / 32;
+        const size_t smem = sizeof(int) * kEcBins + (sizeof(unsigned long long) + sizeof(int)) * kEcBrute +
+                            3 * sizeof(unsigned) * nwords + sizeof(uint16_t) * (size_t)T;
+        if (!set_smem_limit((const void*)ec_select_bins_kernel, smem)) return MOE_ERR_CUDA;
+        rc = launch_pdl(ec_select_bins_kernel, E, 1024, smem, s, (const uint16_t*)bins, logits, (const double*)lse, T,
                         E, C, ec_token, mask, mw);
     } else {
         rc = launch_pdl(ec_select_kernel, E, 1024, 0, s, (const unsigned*)keys_hi, (const unsigned*)keys_lo, T, E, C,

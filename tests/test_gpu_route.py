@@ -101,15 +101,28 @@ def check_ec(logits, C):
 
 
 @pytest.mark.parametrize("T,E,C", [(1, 1, 1), (40, 4, 10), (1000, 7, 333), (3000, 64, 100), (2048, 33, 2048),
-                                   (5000, 128, 79), (50001, 8, 7001)])   # the last: selection from global memory
+                                   (5000, 128, 79), (50001, 8, 7001),
+                                   (70001, 4, 9000)])   # the last: T above the binned selection, keys in global memory
 def test_expert_choice_random(T, E, C):
     check_ec(synth.normal_f32(5, 1, (T, E)), C)
 
 
 def test_expert_choice_ties():
+    # boundary bins of equal keys: the radix over the full keys, ties in token order
     rng = np.random.default_rng(1)
     check_ec(rng.integers(-1, 2, size=(3000, 16)).astype(np.float32), 700)
     check_ec(np.zeros((257, 3), np.float32), 100)
+
+
+def test_expert_choice_one_crowded_bin():
+    # logits within 1e-4 of each other: every key of an expert in one 1/256-wide
+    # bin, all distinct, so the boundary bin's 3000 keys go through the radix
+    check_ec((1e-4 * synth.normal_f32(5, 3, (3000, 16))).astype(np.float32), 700)
+    # two experts, logits scaled so that the boundary bins hold a few hundred
+    # keys: 243 and 248 (ranked pairwise; the second taken whole), then 331
+    # and 321 (above the pairwise limit of 256: the radix)
+    for a in (0.15, 0.12):
+        check_ec((a * synth.normal_f32(5, 4, (20000, 2))).astype(np.float32), 5000)
 
 
 def test_expert_choice_workload():
