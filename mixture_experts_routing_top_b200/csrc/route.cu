@@ -649,19 +649,23 @@ __device__ __forceinline__ void warp_find_boundary(const int* hist, int nbins, i
 }
 
 // Binned selection (T <= kEcBinTokens): one 1024-thread CTA per expert.
-// The expert's T key bins are loaded once into shared memory and counted;
-// the boundary bin is the bin, from the best, where the running count
-// reaches C.  Tokens in earlier bins are selected, in later bins not.  The
-// boundary bin is taken whole when it holds exactly the C - (earlier) keys
-// still needed; otherwise its tokens' exact keys (l - lse in fp64,
-// recomputed from the logits and the lse as the key kernel computes them)
-// decide: ranked pairwise (key descending, then token ascending) when the
-// bin holds at most kEcBrute tokens, else by an 8-bit radix select over the
-// 64-bit order-preserving keys (ties at the end resolved in token order).
-// The selection is written in token order: one classification pass over
-// all tokens keeps per-32-token masks (selected, at the threshold) in
-// shared memory, then a second pass writes the rows.  Also sets the
-// token-membership bits used to build the token CSR.
+// The expert's T key bins are loaded once into shared memory (two per
+// 32-bit load) and counted; the boundary bin is the bin, from the best,
+// where the running count reaches C.  Tokens in earlier bins are selected,
+// in later bins not.  The boundary bin is taken whole when it holds exactly
+// the C - (earlier) keys still needed; otherwise its tokens' exact keys
+// (l - lse in fp64, recomputed from the logits and the lse as the key
+// kernel computes them) decide: ranked pairwise (key descending, then token
+// ascending) when the bin holds at most kEcBrute tokens, else by an 8-bit
+// radix select over the 64-bit order-preserving keys (ties at the end
+// resolved in token order).  Each warp owns a contiguous run of 64-token
+// groups, a lane two adjacent tokens of each: one pass counts the warp's
+// selected tokens and lists the boundary bin's, a second writes the rows in
+// token order.  (The radix case classifies token by token, 32 tokens a
+// word.)  Global loads that depend on a token (its exact key, its gate
+// exp(key)) are made after the passes, all at once, so that no warp waits
+// on them inside a pass.  Also sets the token-membership bits used to build
+// the token CSR.
 constexpr int kEcBinTokens = 65536;
 constexpr int kEcBrute = 256;
 
@@ -669,16 +673,18 @@ __global__ void __launch_bounds__(1024) ec_select_bins_kernel(const uint16_t* __
                                                               const float* __restrict__ logits,
                                                               const double* __restrict__ lse, int T, int E, int C,
                                                               int32_t* __restrict__ ec_token,
+                                                              float* __restrict__ ec_gate,
                                                               unsigned* __restrict__ tokmask, int mask_words) {
     extern __shared__ __align__(16) unsigned char ec_sm[];
     const int nwords = (T + 31) >> 5;
+    const int ngroups = (T + 63) >> 6;
     int* hist = reinterpret_cast<int*>(ec_sm);                              // [kEcBins]
     unsigned long long* ckey = reinterpret_cast<unsigned long long*>(hist + kEcBins);   // [kEcBrute]
     int* ctok = reinterpret_cast<int*>(ckey + kEcBrute);                    // [kEcBrute]
-    unsigned* m_sel = reinterpret_cast<unsigned*>(ctok + kEcBrute);         // [nwords] selected
-    unsigned* m_tie = m_sel + nwords;                                       // [nwords] at the threshold
-    unsigned* chosen = m_tie + nwords;                                      // [nwords] ranked pairwise and kept
-    uint16_t* bs = reinterpret_cast<uint16_t*>(chosen + nwords);            // [T]
+    unsigned* m_sel = reinterpret_cast<unsigned*>(ctok + kEcBrute);         // [nwords] (radix case)
+    unsigned* m_tie = m_sel + nwords;                                       // [nwords] (radix case)
+    unsigned* chosen = m_tie + nwords;                                      // [nwords] boundary-bin tokens kept
+    uint16_t* bs = reinterpret_cast<uint16_t*>(chosen + nwords);            // [64 ngroups], zero past T
     __shared__ int sh[32];
     __shared__ int s_bin, s_need, s_bcount, s_nc, s_done, s_rbin, s_rneed, s_rcount;
     __shared__ unsigned long long s_prefix, s_mask;
@@ -688,23 +694,47 @@ __global__ void __launch_bounds__(1024) ec_select_bins_kernel(const uint16_t* __
     const unsigned lt = (1u << lane) - 1u;
     for (int i = threadIdx.x; i < kEcBins; i += blockDim.x) hist[i] = 0;
     for (int i = threadIdx.x; i < nwords; i += blockDim.x) chosen[i] = 0u;
+    if (threadIdx.x < 32) w_sel[threadIdx.x] = 0;
     __syncthreads();
     pdl_wait();                                    // the bins come from the kernel before
     const uint16_t* src = bins + (long long)e * T;
-    for (int t0 = 0; t0 < T; t0 += 8 * blockDim.x) {
-        int u[8];
+    unsigned* bs2 = reinterpret_cast<unsigned*>(bs);                        // bin pairs
+    if ((T & 1) == 0) {
+        // pairs of bins, 4-byte aligned (e T is even)
+        const unsigned* src2 = reinterpret_cast<const unsigned*>(src);
+        const int npairs = T >> 1;
+        for (int p0 = 0; p0 < npairs; p0 += 16 * blockDim.x) {
+            unsigned u[16];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            const int t = t0 + q * blockDim.x + threadIdx.x;
-            u[q] = t < T ? (int)src[t] : -1;
+            for (int q = 0; q < 16; ++q) {
+                const int p = p0 + q * blockDim.x + threadIdx.x;
+                u[q] = p < npairs ? src2[p] : 0xFFFFFFFFu;
+            }
+#pragma unroll
+            for (int q = 0; q < 16; ++q) {
+                if (u[q] == 0xFFFFFFFFu) continue;
+                bs2[p0 + q * blockDim.x + threadIdx.x] = u[q];
+                atomicAdd(&hist[u[q] & 0xFFFFu], 1);
+                atomicAdd(&hist[u[q] >> 16], 1);
+            }
         }
+    } else {
+        for (int t0 = 0; t0 < T; t0 += 8 * blockDim.x) {
+            int u[8];
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            if (u[q] < 0) continue;
-            bs[t0 + q * blockDim.x + threadIdx.x] = (uint16_t)u[q];
-            atomicAdd(&hist[u[q]], 1);
+            for (int q = 0; q < 8; ++q) {
+                const int t = t0 + q * blockDim.x + threadIdx.x;
+                u[q] = t < T ? (int)src[t] : -1;
+            }
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                if (u[q] < 0) continue;
+                bs[t0 + q * blockDim.x + threadIdx.x] = (uint16_t)u[q];
+                atomicAdd(&hist[u[q]], 1);
+            }
         }
     }
+    for (int t = T + threadIdx.x; t < 64 * ngroups; t += blockDim.x) bs[t] = 0;   // read below, never counted
     __syncthreads();
     {
         // each thread 4 consecutive bins; the one whose bins hold the C-th key finds the boundary bin
@@ -730,76 +760,125 @@ __global__ void __launch_bounds__(1024) ec_select_bins_kernel(const uint16_t* __
             }
         }
     }
+    if (threadIdx.x == 0) s_nc = 0;
     __syncthreads();
     const int bstar = s_bin;
     int need = s_need;
     const int bcount = s_bcount;
     const int mode = bcount == need ? 0 : (bcount <= kEcBrute ? 1 : 2);
-    auto exact_key = [&](int t) { return key_bits((double)logits[(long long)t * E + e] - lse[t]); };
-    if (mode == 1) {
-        // the boundary bin's tokens and exact keys, then pairwise ranks
-        if (threadIdx.x == 0) s_nc = 0;
-        __syncthreads();
-        for (int t0 = 0; t0 < T; t0 += blockDim.x) {
-            const int t = t0 + threadIdx.x;
-            const bool in = t < T && bs[t] == bstar;
-            const unsigned bm = __ballot_sync(0xffffffffu, in);
-            int base = 0;
-            if (lane == 0 && bm) base = atomicAdd(&s_nc, __popc(bm));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            const int slot = base + __popc(bm & lt);
-            if (in && slot < kEcBrute) {
-                ctok[slot] = t;
-                ckey[slot] = exact_key(t);
+    auto key_of = [&](int t) { return (double)logits[(long long)t * E + e] - lse[t]; };
+    auto exact_key = [&](int t) { return key_bits(key_of(t)); };
+    // the warp's groups of 64 tokens; lane l holds tokens 64 g + 2 l and 64 g + 2 l + 1
+    const int gper = (ngroups + nw - 1) / nw;
+    const int g0 = min(wid * gper, ngroups), g1 = min(g0 + gper, ngroups);
+    if (mode != 2) {
+        // count the warp's tokens in bins before the boundary bin (and in it
+        // when it is taken whole); list the boundary bin's tokens
+        int mine = 0;
+        for (int g = g0; g < g1; ++g) {
+            const unsigned pr = bs2[32 * g + lane];
+            const int t = 64 * g + 2 * lane;
+            const int bA = (int)(pr & 0xFFFFu), bB = (int)(pr >> 16);
+            const bool okA = t < T, okB = t + 1 < T;
+            mine += (okA && (bA < bstar || (mode == 0 && bA == bstar))) + (okB && (bB < bstar || (mode == 0 && bB == bstar)));
+            if (mode == 1) {
+                const bool inA = okA && bA == bstar, inB = okB && bB == bstar;
+                const unsigned mA = __ballot_sync(0xffffffffu, inA), mB = __ballot_sync(0xffffffffu, inB);
+                if (mA | mB) {
+                    int base = 0;
+                    if (lane == 0) base = atomicAdd(&s_nc, __popc(mA) + __popc(mB));
+                    base = __shfl_sync(0xffffffffu, base, 0);
+                    int slot = base + __popc(mA & lt) + __popc(mB & lt);
+                    if (inA) {
+                        if (slot < kEcBrute) ctok[slot] = t;
+                        ++slot;
+                    }
+                    if (inB && slot < kEcBrute) ctok[slot] = t + 1;
+                }
             }
         }
+        mine = warp_sum(mine);
+        if (lane == 0) w_tie[wid] = mine;             // tokens before the boundary bin, per warp
         __syncthreads();
-        const int nc = min(s_nc, kEcBrute);
-        if ((int)threadIdx.x < nc) {
-            const unsigned long long k0 = ckey[threadIdx.x];
-            const int t = ctok[threadIdx.x];
-            int rank = 0;
-            for (int j = 0; j < nc; ++j) {
-                const unsigned long long kj = ckey[j];
-                rank += (kj > k0 || (kj == k0 && ctok[j] < t)) ? 1 : 0;
-            }
-            if (rank < need) atomicOr(&chosen[t >> 5], 1u << (t & 31));
-        }
-        __syncthreads();
-    } else if (mode == 2) {
-        // radix over the boundary bin's 64-bit keys, from the top byte
-        if (threadIdx.x == 0) { s_prefix = 0ull; s_mask = 0ull; s_done = 0; s_rneed = need; }
-        __syncthreads();
-        for (int shift = 56; shift >= 0 && !s_done; shift -= 8) {
-            const unsigned long long prefix = s_prefix, mask = s_mask;
-            for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+        if (mode == 1) {
+            // the listed tokens' exact keys, all loads at once, then pairwise ranks
+            const int nc = min(s_nc, kEcBrute);
+            if ((int)threadIdx.x < nc) ckey[threadIdx.x] = exact_key(ctok[threadIdx.x]);
             __syncthreads();
-            for (int t0 = 0; t0 < T; t0 += blockDim.x) {
-                const int t = t0 + threadIdx.x;
-                if (t < T && bs[t] == bstar) {
-                    const unsigned long long k0 = exact_key(t);
-                    if ((k0 & mask) == prefix) atomicAdd(&hist[(int)((k0 >> shift) & 255ull)], 1);
+            if ((int)threadIdx.x < nc) {
+                const unsigned long long k0 = ckey[threadIdx.x];
+                const int t = ctok[threadIdx.x];
+                int rank = 0;
+                for (int j = 0; j < nc; ++j) {
+                    const unsigned long long kj = ckey[j];
+                    rank += (kj > k0 || (kj == k0 && ctok[j] < t)) ? 1 : 0;
+                }
+                if (rank < need) {
+                    atomicOr(&chosen[t >> 5], 1u << (t & 31));
+                    atomicAdd(&w_sel[min((t >> 6) / max(gper, 1), nw - 1)], 1);   // the owning warp
                 }
             }
             __syncthreads();
-            if (wid == 0) warp_find_boundary(hist, 256, s_rneed, &s_rbin, &s_rneed, &s_rcount);
-            __syncthreads();
-            if (threadIdx.x == 0) {
-                s_prefix = prefix | ((unsigned long long)s_rbin << shift);
-                s_mask = mask | (255ull << shift);
-                if (s_rcount == s_rneed) s_done = 1;
-            }
-            __syncthreads();
         }
-        need = s_rneed;
+        int out_base = 0;
+        for (int q = 0; q < wid; ++q) out_base += w_tie[q] + w_sel[q];
+        for (int g = g0; g < g1; ++g) {
+            const unsigned pr = bs2[32 * g + lane];
+            const int t = 64 * g + 2 * lane;
+            const int bA = (int)(pr & 0xFFFFu), bB = (int)(pr >> 16);
+            const unsigned cw = (mode == 1 && t < T) ? chosen[t >> 5] : 0u;
+            const bool selA = t < T && (bA < bstar || (bA == bstar && (mode == 0 || ((cw >> (t & 31)) & 1u))));
+            const bool selB = t + 1 < T && (bB < bstar || (bB == bstar && (mode == 0 || ((cw >> ((t + 1) & 31)) & 1u))));
+            const unsigned mA = __ballot_sync(0xffffffffu, selA), mB = __ballot_sync(0xffffffffu, selB);
+            int pos = out_base + __popc(mA & lt) + __popc(mB & lt);
+            if (selA) {
+                ec_token[(long long)e * C + pos] = t;
+                atomicOr(&tokmask[(long long)t * mask_words + (e >> 5)], 1u << (e & 31));
+                ++pos;
+            }
+            if (selB) {
+                ec_token[(long long)e * C + pos] = t + 1;
+                atomicOr(&tokmask[(long long)(t + 1) * mask_words + (e >> 5)], 1u << (e & 31));
+            }
+            out_base += __popc(mA) + __popc(mB);
+        }
+        __syncthreads();
+        for (int j = threadIdx.x; j < C; j += blockDim.x) {
+            const long long r = (long long)e * C + j;
+            ec_gate[r] = (float)exp(key_of(ec_token[r]));
+        }
+        return;
     }
+    // radix over the boundary bin's 64-bit keys, from the top byte
+    if (threadIdx.x == 0) { s_prefix = 0ull; s_mask = 0ull; s_done = 0; s_rneed = need; }
+    __syncthreads();
+    for (int shift = 56; shift >= 0 && !s_done; shift -= 8) {
+        const unsigned long long prefix = s_prefix, mask = s_mask;
+        for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
+        __syncthreads();
+        for (int t0 = 0; t0 < T; t0 += blockDim.x) {
+            const int t = t0 + threadIdx.x;
+            if (t < T && bs[t] == bstar) {
+                const unsigned long long k0 = exact_key(t);
+                if ((k0 & mask) == prefix) atomicAdd(&hist[(int)((k0 >> shift) & 255ull)], 1);
+            }
+        }
+        __syncthreads();
+        if (wid == 0) warp_find_boundary(hist, 256, s_rneed, &s_rbin, &s_rneed, &s_rcount);
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            s_prefix = prefix | ((unsigned long long)s_rbin << shift);
+            s_mask = mask | (255ull << shift);
+            if (s_rcount == s_rneed) s_done = 1;
+        }
+        __syncthreads();
+    }
+    need = s_rneed;
     const unsigned long long prefix = s_prefix, mask = s_mask;
-    // 1 selected, 2 at the threshold (radix mode: tie order decides), 0 not
+    // 1 selected, 2 at the threshold (tie order decides), 0 not
     auto classify = [&](int t) -> int {
         const int b = bs[t];
         if (b != bstar) return b < bstar ? 1 : 0;
-        if (mode == 0) return 1;
-        if (mode == 1) return (int)((chosen[t >> 5] >> (t & 31)) & 1u);
         const unsigned long long km = exact_key(t) & mask;
         if (km != prefix) return km > prefix ? 1 : 0;
         return 2;
@@ -828,12 +907,16 @@ __global__ void __launch_bounds__(1024) ec_select_bins_kernel(const uint16_t* __
         const bool sel = ((sb >> lane) & 1u) || (((tb >> lane) & 1u) && tie_rank < need);
         const unsigned sel_mask = __ballot_sync(0xffffffffu, sel);
         if (sel) {
-            const long long r = (long long)e * C + out_base + __popc(sel_mask & lt);
-            ec_token[r] = t;
+            ec_token[(long long)e * C + out_base + __popc(sel_mask & lt)] = t;
             atomicOr(&tokmask[(long long)t * mask_words + (e >> 5)], 1u << (e & 31));
         }
         tie_base += __popc(tb);
         out_base += __popc(sel_mask);
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < C; j += blockDim.x) {
+        const long long r = (long long)e * C + j;
+        ec_gate[r] = (float)exp(key_of(ec_token[r]));
     }
 }
 
@@ -900,19 +983,20 @@ ec_count_scan_kernel(const unsigned* __restrict__ tokmask, int T, int mask_words
     if (c == kScanCtas - 1 && threadIdx.x == 0) tok_ptr[T] = all;
 }
 
-// For every buffer row r = e*C + i holding token t: its gate exp(key) and
-// tok_row[tok_ptr[t] + (#experts below e that chose t)] = r.
+// For every buffer row r = e*C + i holding token t:
+// tok_row[tok_ptr[t] + (#experts below e that chose t)] = r, and its gate
+// exp(key) when `gates` (the binned selection writes the gates itself).
 __global__ void ec_fill_kernel(const int32_t* __restrict__ ec_token, int T, int E, int C,
                                const unsigned* __restrict__ tokmask, int mask_words,
                                const int32_t* __restrict__ tok_ptr, const float* __restrict__ logits,
-                               const double* __restrict__ lse, float* __restrict__ ec_gate,
+                               const double* __restrict__ lse, int gates, float* __restrict__ ec_gate,
                                int32_t* __restrict__ tok_row) {
     long long r = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     pdl_wait();
     if (r >= (long long)E * C) return;
     int e = (int)(r / C);
     int t = ec_token[r];
-    ec_gate[r] = (float)exp((double)logits[(long long)t * E + e] - lse[t]);
+    if (gates) ec_gate[r] = (float)exp((double)logits[(long long)t * E + e] - lse[t]);
     const unsigned* m = tokmask + (long long)t * mask_words;
     int below = 0;
     for (int w = 0; w < (e >> 5); ++w) below += __popc(m[w]);
@@ -1047,12 +1131,12 @@ extern "C" moe_status moe_route_ec(const float* logits, int T, int E, int C, int
     }
     cudaError_t rc;
     if (binned) {
-        const size_t nwords = (size_t)(T + 31) / 32;
+        const size_t nwords = (size_t)(T + 31) / 32, ngroups = (size_t)(T + 63) / 64;
         const size_t smem = sizeof(int) * kEcBins + (sizeof(unsigned long long) + sizeof(int)) * kEcBrute +
-                            3 * sizeof(unsigned) * nwords + sizeof(uint16_t) * (size_t)T;
+                            3 * sizeof(unsigned) * nwords + sizeof(uint16_t) * 64 * ngroups;
         if (!set_smem_limit((const void*)ec_select_bins_kernel, smem)) return MOE_ERR_CUDA;
         rc = launch_pdl(ec_select_bins_kernel, E, 1024, smem, s, (const uint16_t*)bins, logits, (const double*)lse, T,
-                        E, C, ec_token, mask, mw);
+                        E, C, ec_token, ec_gate, mask, mw);
     } else {
         rc = launch_pdl(ec_select_kernel, E, 1024, 0, s, (const unsigned*)keys_hi, (const unsigned*)keys_lo, T, E, C,
                         ec_token, mask, mw);
@@ -1064,8 +1148,8 @@ extern "C" moe_status moe_route_ec(const float* logits, int T, int E, int C, int
     MOE_LAUNCH_CHECK();
     const long long rows = (long long)E * C;
     if (launch_pdl(ec_fill_kernel, (int)((rows + 255) / 256), 256, 0, s, (const int32_t*)ec_token, T, E, C,
-                   (const unsigned*)mask, mw, (const int32_t*)tok_ptr, logits, (const double*)lse, ec_gate,
-                   tok_row) != cudaSuccess)
+                   (const unsigned*)mask, mw, (const int32_t*)tok_ptr, logits, (const double*)lse, binned ? 0 : 1,
+                   ec_gate, tok_row) != cudaSuccess)
         return MOE_ERR_CUDA;
     MOE_LAUNCH_CHECK();
     return MOE_OK;
