@@ -119,6 +119,26 @@ __device__ __forceinline__ void topk_insert(float (&bv)[KM], int (&bi)[KM], floa
     }
 }
 
+// The same insertion without branches: every comparison is made against
+// the list as it was (c[j] = l > bv[j], which, the list being sorted, holds
+// for a suffix of positions), then each entry takes its upper neighbour's
+// value, the new one, or keeps its own.  A lane with nothing to insert
+// passes l = -inf (no comparison holds, nothing moves), so a warp can insert
+// its lanes' candidates in step.
+template <int KM>
+__device__ __forceinline__ void topk_insert_uniform(float (&bv)[KM], int (&bi)[KM], float l, int e) {
+    bool c[KM];
+#pragma unroll
+    for (int j = 0; j < KM; ++j) c[j] = l > bv[j];
+#pragma unroll
+    for (int j = KM - 1; j >= 1; --j) {
+        bv[j] = c[j - 1] ? bv[j - 1] : (c[j] ? l : bv[j]);
+        bi[j] = c[j - 1] ? bi[j - 1] : (c[j] ? e : bi[j]);
+    }
+    bv[0] = c[0] ? l : bv[0];
+    bi[0] = c[0] ? e : bi[0];
+}
+
 // exp(l - m) with the rounding error of l - m carried into the result
 // (TwoSum of l and -m, then exp(hi) * (1 + lo)).
 __device__ __forceinline__ float exp_diff(float l, float m) {

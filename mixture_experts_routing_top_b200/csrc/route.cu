@@ -246,14 +246,15 @@ __global__ void __launch_bounds__(32 * kRowWarps, 4) route_topk_rows_kernel(cons
             issue(c + kRowBufs - 1);           // into the slot scanned one iteration ago
             cp_async_wait<kRowBufs - 1>();     // chunk c: this lane's copies have landed
             __syncwarp();                      // ... and the other lanes' copies are visible
+            const float* row = ring + (c % kRowBufs) * (32 * kRowStride) + lane * kRowStride;
+            const int e0 = c * kRowChunk;
+            unsigned msk = 0u;                 // this lane's candidates in the chunk
             if (t < T) {
-                const float* row = ring + (c % kRowBufs) * (32 * kRowStride) + lane * kRowStride;
-                const int e0 = c * kRowChunk;
                 const int nv = min(kRowChunk, E - e0);
                 if (c == 0) {                  // seed the list with the first KM experts
 #pragma unroll
                     for (int i = 0; i < KM; ++i)
-                        if (i < nv) topk_insert<KM>(bv, bi, row[i], i);
+                        if (i < nv) topk_insert_uniform<KM>(bv, bi, row[i], i);
                 }
                 const int skip = c == 0 ? KM : 0;
                 const float tau = bv[KM - 1];
@@ -274,7 +275,7 @@ __global__ void __launch_bounds__(32 * kRowWarps, 4) route_topk_rows_kernel(cons
                     }
                 }
                 const float cm = fmaxf(fmaxf(cm4[0], cm4[1]), fmaxf(cm4[2], cm4[3]));
-                unsigned msk = m4[0] | m4[1] | m4[2] | m4[3];
+                msk = m4[0] | m4[1] | m4[2] | m4[3];
                 if (!norm_topk) {
                     if (cm > m_run) {
                         s *= exp((double)m_run - (double)cm);
@@ -298,12 +299,20 @@ __global__ void __launch_bounds__(32 * kRowWarps, 4) route_topk_rows_kernel(cons
 #pragma unroll
                     for (int u = 0; u < 4; ++u) s += (double)cs[u] - (double)cc[u];
                 }
-                // insert the candidates in expert order (each re-checked against the moving threshold)
-                while (msk) {
+            }
+            // insert the candidates in expert order (each re-checked against the
+            // moving threshold), the warp's lanes in step: each round every lane
+            // inserts its next candidate, or nothing once it has none left
+            while (__any_sync(0xffffffffu, msk != 0u)) {
+                float l = -INFINITY;
+                int ei = -1;
+                if (msk) {
                     const int i = __ffs(msk) - 1;
                     msk &= msk - 1;
-                    topk_insert<KM>(bv, bi, row[i], e0 + i);
+                    l = row[i];
+                    ei = e0 + i;
                 }
+                topk_insert_uniform<KM>(bv, bi, l, ei);
             }
             __syncwarp();                      // slot c % kRowBufs may be refilled
         }
