@@ -1,5 +1,6 @@
 // api.cu - status strings, ABI version and the per-device fault word.
 #include <atomic>
+#include <cstdlib>
 #include <map>
 #include <mutex>
 #include <utility>
@@ -88,6 +89,27 @@ bool set_smem_limit(const void* fn, size_t bytes) {
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) return false;
     raised[std::make_pair(fn, std::make_pair(dev, current_context_id()))] = bytes;
     return true;
+}
+
+int resident_ctas(const void* fn, int threads, size_t smem) {
+    const char* env = getenv("LIBMOE_ONE_WAVE");
+    if (env && env[0] == '0') return 1 << 30;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 1 << 30;
+    static std::mutex mu;
+    static std::map<std::pair<std::pair<const void*, int>, std::pair<size_t, unsigned long long>>, int> known;
+    std::lock_guard<std::mutex> lk(mu);
+    const auto key = std::make_pair(std::make_pair(fn, threads), std::make_pair(smem, (unsigned long long)dev));
+    const auto it = known.find(key);
+    if (it != known.end()) return it->second;
+    int per = 0, sms = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, fn, threads, smem) != cudaSuccess || per < 1 ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
+        (void)cudaGetLastError();
+        return 1 << 30;
+    }
+    known[key] = per * sms;
+    return per * sms;
 }
 
 }  // namespace moe

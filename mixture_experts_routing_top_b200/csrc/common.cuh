@@ -40,6 +40,14 @@ void count_launch();
 // (no-op up to 48 KB).  False if the runtime refused.
 bool set_smem_limit(const void* fn, size_t bytes);
 
+// CTAs of kernel fn (with `threads` threads and `smem` bytes of dynamic
+// shared memory each) that the current device holds at once, looked up once
+// per kernel, shape and device.  A grid-strided kernel launched with at most
+// this many CTAs runs in one wave and its warps share the work evenly; one
+// more wave than that would leave most of the GPU idle at its end.
+// LIBMOE_ONE_WAVE=0 turns the cap off (a very large number).
+int resident_ctas(const void* fn, int threads, size_t smem);
+
 // Programmatic dependent launch.  A kernel launched with programmatic
 // stream serialization may start while the kernel before it in the stream
 // is still running; it must call pdl_wait() before its first global memory

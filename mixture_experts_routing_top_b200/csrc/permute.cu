@@ -751,7 +751,7 @@ perm_count_cluster_kernel(const int32_t* __restrict__ idx, int T, int k, int E, 
     }
     drop = warp_sum(drop);
     if (lane == 0) wdrop[wid] = drop;
-    tc::cluster_sync_relaxed();                // no CTA exits while another still reads its tot[]
+    tc::cluster_sync();                        // the reads of the others' tot[] are performed before any CTA exits
     __syncthreads();                           // pre[], kept_s[] and wdrop[] are complete
     if (r == 0) {
         const int rows = block_exclusive_scan(kept_s, E, wsum);
@@ -937,8 +937,12 @@ moe_status launch_copy_slots(const void* x, int T, int row_bytes, const int32_t*
         if (!err) return MOE_ERR_CUDA;
         const size_t smem = (size_t)kBulkWarps * slot_bytes;
         if (!set_smem_limit((const void*)copy_rows_bulk_kernel, smem)) return MOE_ERR_CUDA;
-        long long nb = ((long long)T + kBulkWarps - 1) / kBulkWarps;
-        const int blocks = (int)(nb < 148 * 16 ? nb : 148 * 16);
+        // one token per warp, as many CTAs as that takes: fresh CTAs replace
+        // finished ones, which moved rows faster than a grid-strided loop
+        // over fewer CTAs (T = 131072 top-8 rows: 0.94 against 0.91 of HBM
+        // with 148 x 16 CTAs and 0.82 with one resident wave)
+        const long long nb = ((long long)T + kBulkWarps - 1) / kBulkWarps;
+        const int blocks = (int)(nb < (1LL << 30) ? nb : (1LL << 30));
         if (launch_pdl(copy_rows_bulk_kernel, blocks, 32 * kBulkWarps, smem, s, (const uint8_t*)x, T, row_bytes,
                        slot_bytes, row_map, k, (uint8_t*)buffer, err) != cudaSuccess)
             return MOE_ERR_CUDA;
@@ -1122,8 +1126,10 @@ extern "C" moe_status moe_gather_rows(const void* x, int dtype, int T, int d, co
     if (bulk_copy_enabled() && slot_bytes <= 32 * 1024) {
         const size_t smem = (size_t)kBulkWarps * slot_bytes;
         if (!set_smem_limit((const void*)copy_rows_csr_bulk_kernel, smem)) return MOE_ERR_CUDA;
-        long long nb = ((long long)T + kBulkWarps - 1) / kBulkWarps;
-        const int blocks = (int)(nb < 148 * 16 ? nb : 148 * 16);
+        // one token per warp (as the permutation's bulk copy): expert-choice
+        // dispatch 0.74 -> 0.80 of HBM against 148 x 16 grid-strided CTAs
+        const long long nb = ((long long)T + kBulkWarps - 1) / kBulkWarps;
+        const int blocks = (int)(nb < (1LL << 30) ? nb : (1LL << 30));
         copy_rows_csr_bulk_kernel<<<blocks, 32 * kBulkWarps, smem, s>>>((const uint8_t*)x, T, (int)row_bytes, slot_bytes,
                                                                         tok_ptr, tok_row, R, (uint8_t*)buffer, err);
         MOE_LAUNCH_CHECK();

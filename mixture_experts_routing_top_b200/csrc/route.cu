@@ -976,7 +976,11 @@ ec_count_scan_kernel(const unsigned* __restrict__ tokmask, int T, int mask_words
         if (q < c) before += v[q];
         all += v[q];
     }
-    tc::cluster_sync_relaxed();               // every read of cta_total is done before any CTA exits
+    // every CTA's reads of the others' cta_total are performed before any
+    // CTA exits: a release arrive (a relaxed one may be observed while the
+    // loads are still in flight, and the sums above are free to be
+    // computed after it)
+    tc::cluster_sync();
     int run = before + ex;
 #pragma unroll
     for (int j = 0; j < kCache; ++j) {

@@ -214,7 +214,11 @@ cosel_cluster_kernel(const int32_t* __restrict__ idx, int k, int T, int E, SymBa
             if (b != a) atomicAdd(hist + (long long)b * E + a, v);
         }
     }
-    tc::cluster_sync_relaxed();                 // no CTA exits while another still reads its counts
+    // no CTA exits while another still reads its counts: every remote load
+    // above feeds the branch on its value (and the atomics) before this
+    // point, so it has completed when the thread arrives, and a relaxed
+    // arrive need not wait for the merge's global atomics
+    tc::cluster_sync_relaxed();
 }
 
 // The symmetric kernel for E >= 128, where it measured faster (T = 131072,

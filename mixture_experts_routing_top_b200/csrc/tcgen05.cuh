@@ -174,9 +174,14 @@ __device__ __forceinline__ void cluster_sync() {
 }
 
 // A cluster barrier that orders no memory: for waiting until every CTA of
-// the cluster is done reading the others' shared memory (loads whose values
-// it has consumed), without also waiting for its own outstanding global
-// writes and atomics to complete, as a release arrive would.
+// the cluster is done reading the others' shared memory, without also
+// waiting for its own outstanding global writes and atomics to complete, as
+// a release arrive would.  Safe only when the value of every remote load
+// feeds an instruction that must execute before the arrive (a branch, a
+// store or an atomic): the arrive itself does not wait for loads in flight,
+// and arithmetic on their values may be scheduled after it.  Otherwise use
+// cluster_sync(), whose release arrive is observed only after the loads are
+// performed.
 __device__ __forceinline__ void cluster_sync_relaxed() {
     asm volatile("barrier.cluster.arrive.relaxed.aligned;\n\tbarrier.cluster.wait.aligned;" ::: "memory");
 }
