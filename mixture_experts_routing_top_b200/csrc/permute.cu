@@ -718,10 +718,32 @@ perm_count_cluster_kernel(const int32_t* __restrict__ idx, int T, int k, int E, 
     const int cs = kRcTok * k;                 // slots per chunk
     const long long s0 = (long long)c0 * cs;
     const long long s1 = min((long long)c1 * kRcTok, (long long)T) * k;
-    for (long long s = s0 + threadIdx.x; s < s1; s += blockDim.x) {
-        const int e = idx[s];
-        if ((unsigned)e >= (unsigned)E) { raise_error(err, kErrIndex); continue; }
-        atomicAdd(&hist[e * ld + (int)(s - s0) / cs], 1);
+    {
+        // slot s0 + j lies in chunk j / cs of this CTA: the chunk index and the
+        // offset in it stepped along with j (no division per slot), four
+        // slots' expert ids loaded before any is counted
+        const int n = (int)(s1 - s0);
+        const int dq = (int)blockDim.x / cs, dr = (int)blockDim.x - dq * cs;
+        int q = (int)threadIdx.x / cs, rm = (int)threadIdx.x - q * cs;
+        for (int j0 = threadIdx.x; j0 < n; j0 += 4 * blockDim.x) {
+            int ev[4], qv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = j0 + u * blockDim.x;
+                ev[u] = j < n ? idx[s0 + j] : -1;
+                qv[u] = q;
+                q += dq;
+                rm += dr;
+                if (rm >= cs) { rm -= cs; ++q; }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int j = j0 + u * blockDim.x;
+                if (j >= n) break;
+                if ((unsigned)ev[u] >= (unsigned)E) { raise_error(err, kErrIndex); continue; }
+                atomicAdd(&hist[ev[u] * ld + qv[u]], 1);
+            }
+        }
     }
     __syncthreads();
     // one flat scan over the expert-major rows (each row ends with a zero
@@ -764,9 +786,16 @@ perm_count_cluster_kernel(const int32_t* __restrict__ idx, int T, int k, int E, 
         }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < ncc * E; i += blockDim.x) {
-        const int c = i / E, e = i - c * E;
-        chunk_base[(long long)c0 * E + i] = hist[e * ld + c] + pre[e];
+    {
+        // element i = c E + e, its chunk and expert stepped along with i
+        const int dc = (int)blockDim.x / E, de = (int)blockDim.x - dc * E;
+        int c = (int)threadIdx.x / E, e = (int)threadIdx.x - c * E;
+        for (int i = threadIdx.x; i < ncc * E; i += blockDim.x) {
+            chunk_base[(long long)c0 * E + i] = hist[e * ld + c] + pre[e];
+            c += dc;
+            e += de;
+            if (e >= E) { e -= E; ++c; }
+        }
     }
 }
 
