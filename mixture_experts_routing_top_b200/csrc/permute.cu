@@ -292,11 +292,14 @@ __device__ void block_scan_prologue(bool fused, const int32_t* __restrict__ cnt,
 // first kept slot of its token in that group (the row's "head"), and the
 // per-block head count of every group.  code[s]: group id for a head,
 // -2 - j for a kept slot whose head is slot j of the same token, -1 for a
-// dropped slot.
+// dropped slot.  With a capacity of at least T k no slot can be dropped
+// (`nodrop`): every valid slot is kept, the expert ranks are not needed, and
+// only the writer block reads the count matrix (for counts and dropped).
 __global__ void __launch_bounds__(kIdxThreads) perm_group_heads_kernel(
     const int32_t* __restrict__ idx, const int32_t* __restrict__ goe, int T, int k, int E, int G, int nblk, int tb, int fused,
-    const int32_t* __restrict__ ecnt, const int32_t* __restrict__ ebase, long long cap, int32_t* __restrict__ counts,
-    int32_t* __restrict__ dropped, int16_t* __restrict__ code, int32_t* __restrict__ gcnt, unsigned* err) {
+    const int32_t* __restrict__ ecnt, const int32_t* __restrict__ ebase, long long cap, int nodrop,
+    int32_t* __restrict__ counts, int32_t* __restrict__ dropped, int16_t* __restrict__ code, int32_t* __restrict__ gcnt,
+    unsigned* err) {
     pdl_trigger();                // the next kernel may be scheduled; it waits for this one
     pdl_wait();                   // inputs come from the kernel before
     extern __shared__ int sm[];
@@ -313,16 +316,29 @@ __global__ void __launch_bounds__(kIdxThreads) perm_group_heads_kernel(
     // the block's experts and the group map into shared memory at once
     for (long long sl = s0 + threadIdx.x; sl < s1; sl += blockDim.x) keys_s[sl - s0] = idx[sl];
     for (int e = threadIdx.x; e < E; e += blockDim.x) goe_s[e] = goe[e];
-    block_scan_prologue(fused, ecnt, ebase, nullptr, E, nblk, cap, base_s, off_s, counts, nullptr, dropped,
-                        (int)blockIdx.x, blockIdx.x == 0);
-    block_stable_ranks(
-        s0, s1, E, base_s, wcnt,
-        [&](long long s) -> int {
-            const int e = keys_s[s - s0];
-            if (e < 0 || e >= E) { raise_error(err, kErrIndex); return -1; }
-            return e;
-        },
-        [&](long long s, int key, int rank) { kept_s[s - s0] = (key >= 0 && rank < cap) ? 1 : 0; });
+    if (nodrop) {
+        if (blockIdx.x == 0)
+            block_scan_prologue(fused, ecnt, ebase, nullptr, E, nblk, cap, base_s, off_s, counts, nullptr, dropped, 0,
+                                true);
+        __syncthreads();
+        for (long long sl = s0 + threadIdx.x; sl < s1; sl += blockDim.x) {
+            const int e = keys_s[sl - s0];
+            const bool ok = e >= 0 && e < E;
+            if (!ok) raise_error(err, kErrIndex);
+            kept_s[sl - s0] = ok ? 1 : 0;
+        }
+    } else {
+        block_scan_prologue(fused, ecnt, ebase, nullptr, E, nblk, cap, base_s, off_s, counts, nullptr, dropped,
+                            (int)blockIdx.x, blockIdx.x == 0);
+        block_stable_ranks(
+            s0, s1, E, base_s, wcnt,
+            [&](long long s) -> int {
+                const int e = keys_s[s - s0];
+                if (e < 0 || e >= E) { raise_error(err, kErrIndex); return -1; }
+                return e;
+            },
+            [&](long long s, int key, int rank) { kept_s[s - s0] = (key >= 0 && rank < cap) ? 1 : 0; });
+    }
     __syncthreads();
     const long long t0 = (long long)blockIdx.x * tb;
     const int ntok = (int)((s1 - s0) / k);
@@ -1112,9 +1128,10 @@ extern "C" moe_status moe_permute(const void* x, int dtype, int T, int d, const 
         int32_t* gtotal = (int32_t*)(ws + L.gtotal);
         const size_t heads_smem = sizeof(int) * ((size_t)nw * E + 3 * (size_t)E + G + (size_t)tb * k) + (size_t)tb * k;
         if (!set_smem_limit((const void*)perm_group_heads_kernel, heads_smem)) return MOE_ERR_CUDA;
+        const int nodrop = cap >= (long long)T * k ? 1 : 0;
         if (launch_pdl(perm_group_heads_kernel, nblk, kIdxThreads, heads_smem, s, expert_idx, group_of_expert, T, k, E, G, nblk, tb,
-                                                                        fused_e, cnt, base, cap, counts, dropped, code,
-                                                                        gcnt, err) != cudaSuccess)
+                                                                        fused_e, cnt, base, cap, nodrop, counts, dropped,
+                                                                        code, gcnt, err) != cudaSuccess)
             return MOE_ERR_CUDA;
         MOE_LAUNCH_CHECK();
         const int fused_g = (long long)G * nblk <= kFuseLimit;
