@@ -180,14 +180,28 @@ __global__ void __launch_bounds__(256) route_topk_vec_kernel(const float* __rest
 // 32 experts through its own shared-memory ring (cp.async, two chunks in
 // flight; lanes copy 128-byte row pieces, 8 lanes per row, rows padded to
 // 36 floats so that 128-bit reads of a lane's own row are conflict-free).
-// Warps never wait for one another.  Every lane scans its own token: one
-// uniform pass over the chunk takes its maximum and marks the experts that
-// beat the current k-th best; the softmax denominator adds the chunk's terms
-// exp(l - m_run) relative to the running maximum (compensated fp32 sums per
-// chunk, the fp64 total rescaled when the maximum grows; skipped when the
-// gates are renormalised over the k); only the marked experts go through
-// the top-k insertion, in expert order.  Ranking ties resolve as in the
-// other variants (lower expert first).
+// Warps never wait for one another.
+//
+// Every lane ranks its own token by one 32-bit key per expert: the
+// order-preserving image of the logit with its low `kbits` bits replaced by
+// (2^kbits - 1 - expert), so keys are distinct, a larger key is a larger
+// logit or, inside one bucket of 2^kbits consecutive images, a lower expert.
+// The lane keeps the k + 1 best keys in a sorted list that a new key enters
+// through a compare-exchange chain of integer max/min (no branch, no
+// predicate per position).  Per chunk, one uniform pass marks the experts
+// that can still enter the list (logit at or above the lowest float of the
+// (k+1)-th key's bucket; for the first chunk at or above the lowest of
+// k + 1 group maxima, which at least k + 1 of its logits reach), and the
+// warp inserts the marked experts in step, one per lane per round.  At the
+// end the k winners are exact unless the k-th and (k+1)-th keys share a
+// bucket: then the lane ranks its row again with full comparisons (rare:
+// two logits within 2^kbits units of the last place at the boundary, or
+// exact ties).  Winners that share a bucket among themselves are put in
+// exact order; their logits are read back for the gates.  With softmax
+// gates the denominator adds the chunk's terms exp(l - m_run) relative to
+// the running maximum (compensated fp32 sums per chunk, the fp64 total
+// rescaled when the maximum grows); renormalised gates need only the k.
+// Ties resolve as in the other variants (lower expert first, -0 == +0).
 constexpr int kRowWarps = 4;                              // warps per CTA
 constexpr int kRowChunk = 32;                             // experts per chunk
 constexpr int kRowStride = 36;                            // floats per staged row
@@ -203,14 +217,40 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
 
-template <int KM>
+// Order-preserving image of a float as an unsigned (a larger float, a larger
+// image), -0 folded into +0 first so that the two are equal.  NaN patterns
+// fall outside [image(-inf), image(+inf)].
+__device__ __forceinline__ unsigned float_order_key(float v) {
+    const unsigned b = __float_as_uint(__fadd_rn(v, 0.0f));
+    return b ^ ((unsigned)((int)b >> 31) | 0x80000000u);
+}
+// The float whose image is `hk` (a bucket's lowest image); -inf at or below
+// the image of -inf (the NaN patterns there, and the empty key 0).
+__device__ __forceinline__ float float_of_order_key(unsigned hk) {
+    if (hk <= 0x007FFFFFu) return -INFINITY;
+    return __uint_as_float((hk & 0x80000000u) ? (hk ^ 0x80000000u) : ~hk);
+}
+// Insert x into the descending list L of distinct keys (x = 0, the empty
+// key, changes nothing).  Entry j becomes max(L[j], min(L[j-1], x)): the
+// entry above it if x went higher, x if x lands here, else itself - every
+// entry from the old list at once, two dependent integer min/max deep.
+template <int N>
+__device__ __forceinline__ void key_insert(unsigned (&L)[N], unsigned x) {
+#pragma unroll
+    for (int j = N - 1; j >= 1; --j) L[j] = max(L[j], min(L[j - 1], x));
+    L[0] = max(L[0], x);
+}
+
+template <int KM, bool NORM>
 __global__ void __launch_bounds__(32 * kRowWarps, 4) route_topk_rows_kernel(const float* __restrict__ logits, int T,
-                                                                            int E, int k, int norm_topk,
+                                                                            int E, int k, int kbits,
                                                                             int32_t* __restrict__ expert_idx,
                                                                             float* __restrict__ gate) {
     pdl_trigger();                // the next kernel may be scheduled; it waits for this one
     pdl_wait();                   // inputs come from the kernel before
     extern __shared__ __align__(16) float row_ring[];
+    constexpr int NL = KM + 1;            // the k best keys and the next one
+    const unsigned idx_max = (1u << kbits) - 1u, hi_mask = ~idx_max;
     const int lane = threadIdx.x & 31;
     float* ring = row_ring + (threadIdx.x >> 5) * kRowWarpFloats;
     const int E4 = E >> 2;
@@ -233,10 +273,9 @@ __global__ void __launch_bounds__(32 * kRowWarps, 4) route_topk_rows_kernel(cons
             }
             cp_async_commit();                 // one group per chunk slot, empty past the last chunk
         };
-        float bv[KM];
-        int bi[KM];
+        unsigned L[NL];
 #pragma unroll
-        for (int j = 0; j < KM; ++j) { bv[j] = -INFINITY; bi[j] = -1; }
+        for (int j = 0; j < NL; ++j) L[j] = 0u;
         float m_run = -INFINITY;           // running maximum (the softmax reference)
         double s = 0.0;                    // sum of exp(l - m_run) so far
         const long long t = t0 + lane;
@@ -251,41 +290,68 @@ __global__ void __launch_bounds__(32 * kRowWarps, 4) route_topk_rows_kernel(cons
             unsigned msk = 0u;                 // this lane's candidates in the chunk
             if (t < T) {
                 const int nv = min(kRowChunk, E - e0);
-                if (c == 0) {                  // seed the list with the first KM experts
+                // the (k+1)-th key so far: the least of the first k + 1 (a
+                // minimum, not L[k], which would put L in local memory)
+                unsigned lk = L[0];
 #pragma unroll
-                    for (int i = 0; i < KM; ++i)
-                        if (i < nv) topk_insert_uniform<KM>(bv, bi, row[i], i);
+                for (int j = 1; j < NL; ++j) lk = min(lk, j <= k ? L[j] : 0xFFFFFFFFu);
+                float tau = float_of_order_key(lk & hi_mask);
+                const float4* row4 = reinterpret_cast<const float4*>(row);
+                if (c == 0 && nv == kRowChunk) {
+                    // NL disjoint groups of the chunk (float4 q; the halves of the
+                    // last one when NL = 9): their maxima are NL logits at or above
+                    // the lowest of them, so the k + 1 best of the chunk are too
+                    // (taken down to its bucket's lowest float, as the keys compare)
+                    float gm[NL];
+#pragma unroll
+                    for (int g = 0; g < NL; ++g) gm[g] = -INFINITY;
+#pragma unroll
+                    for (int q = 0; q < kRowChunk / 4; ++q) {
+                        const float4 a4 = row4[q];
+                        if (NL > 8 && q == 7) {
+                            gm[NL - 2] = fmaxf(a4.x, a4.y);
+                            gm[NL - 1] = fmaxf(a4.z, a4.w);
+                        } else {
+                            const int g = NL > 8 ? q : q * NL / 8;
+                            gm[g] = fmaxf(gm[g], fmaxf(fmaxf(a4.x, a4.y), fmaxf(a4.z, a4.w)));
+                        }
+                    }
+                    float gmin = gm[0];
+#pragma unroll
+                    for (int g = 1; g < NL; ++g) gmin = fminf(gmin, gm[g]);
+                    tau = float_of_order_key(float_order_key(gmin) & hi_mask);
                 }
-                const int skip = c == 0 ? KM : 0;
-                const float tau = bv[KM - 1];
-                // four independent accumulators (one per float4 lane) keep the dependency chains short
-                float cm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
                 unsigned m4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
                 for (int q = 0; q < kRowChunk / 4; ++q) {
-                    const float4 v4 = *reinterpret_cast<const float4*>(row + 4 * q);
-                    const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+                    const float4 a4 = row4[q];
+                    const float v[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        const int i = 4 * q + u;
-                        if (i < nv) {
-                            cm4[u] = fmaxf(cm4[u], v[u]);
-                            if (i >= skip && v[u] > tau) m4[u] |= 1u << i;
-                        }
-                    }
+                    for (int u = 0; u < 4; ++u)
+                        if (4 * q + u < nv && v[u] >= tau) m4[u] |= 1u << (4 * q + u);
                 }
-                const float cm = fmaxf(fmaxf(cm4[0], cm4[1]), fmaxf(cm4[2], cm4[3]));
                 msk = m4[0] | m4[1] | m4[2] | m4[3];
-                if (!norm_topk) {
+                if (!NORM) {
+                    float cm4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+                    for (int q = 0; q < kRowChunk / 4; ++q) {
+                        const float4 a4 = row4[q];
+                        const float v[4] = {a4.x, a4.y, a4.z, a4.w};
+#pragma unroll
+                        for (int u = 0; u < 4; ++u)
+                            if (4 * q + u < nv) cm4[u] = fmaxf(cm4[u], v[u]);
+                    }
+                    const float cm = fmaxf(fmaxf(cm4[0], cm4[1]), fmaxf(cm4[2], cm4[3]));
                     if (cm > m_run) {
                         s *= exp((double)m_run - (double)cm);
                         m_run = cm;
                     }
+                    // four independent accumulators keep the dependency chains short
                     float cs[4] = {0.0f, 0.0f, 0.0f, 0.0f}, cc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
                     for (int q = 0; q < kRowChunk / 4; ++q) {
-                        const float4 v4 = *reinterpret_cast<const float4*>(row + 4 * q);
-                        const float v[4] = {v4.x, v4.y, v4.z, v4.w};
+                        const float4 a4 = row4[q];
+                        const float v[4] = {a4.x, a4.y, a4.z, a4.w};
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
                             if (4 * q + u < nv) {
@@ -300,29 +366,131 @@ __global__ void __launch_bounds__(32 * kRowWarps, 4) route_topk_rows_kernel(cons
                     for (int u = 0; u < 4; ++u) s += (double)cs[u] - (double)cc[u];
                 }
             }
-            // insert the candidates in expert order (each re-checked against the
-            // moving threshold), the warp's lanes in step: each round every lane
-            // inserts its next candidate, or nothing once it has none left
-            while (__any_sync(0xffffffffu, msk != 0u)) {
-                float l = -INFINITY;
-                int ei = -1;
-                if (msk) {
-                    const int i = __ffs(msk) - 1;
-                    msk &= msk - 1;
-                    l = row[i];
-                    ei = e0 + i;
-                }
-                topk_insert_uniform<KM>(bv, bi, l, ei);
+            // the marked experts enter the list in step: each round every lane
+            // inserts its next one, or the empty key once it has none left
+            // (keys are distinct, so any order gives the same list); the next
+            // key is read while the current one is inserted
+            auto pop = [&]() -> unsigned {
+                const int i = max(__ffs(msk) - 1, 0);
+                const unsigned x = (float_order_key(row[i]) & hi_mask) | (idx_max - (unsigned)(e0 + i));
+                const unsigned r = msk ? x : 0u;
+                msk &= msk - 1;
+                return r;
+            };
+            unsigned x = pop();
+            while (__any_sync(0xffffffffu, x != 0u)) {
+                const unsigned nx = pop();
+                key_insert<NL>(L, x);
+                x = nx;
             }
             __syncwarp();                      // slot c % kRowBufs may be refilled
         }
         cp_async_wait<0>();
+        __syncwarp();                          // every lane is done with the ring
+        const float* xr = logits + t * E;
+        float bv[KM];
+        int bi[KM];
+        unsigned ka = L[0], kb = L[0];         // the k-th and (k+1)-th keys (minima, as above)
+#pragma unroll
+        for (int j = 1; j < NL; ++j) {
+            ka = min(ka, j < k ? L[j] : 0xFFFFFFFFu);
+            kb = min(kb, j <= k ? L[j] : 0xFFFFFFFFu);
+        }
+        // the boundary falls inside a bucket: which of its logits win is not known
+        const bool amb = t < T && kb != 0u && ((ka ^ kb) & hi_mask) == 0u;
+#pragma unroll
+        for (int j = 0; j < KM; ++j) {
+            bi[j] = -1;
+            bv[j] = -INFINITY;
+            if (t < T && j < k && L[j] != 0u) {
+                bi[j] = (int)(idx_max - (L[j] & idx_max));
+                bv[j] = __ldg(xr + bi[j]);
+            }
+        }
+        // Such a row: the winners above the boundary bucket stand; the other
+        // places go to the bucket's logits in full order (image, then expert).
+        // The warp copies the row into its ring and marks the bucket's
+        // logits; the row's lane ranks those few.
+        for (unsigned am = __ballot_sync(0xffffffffu, amb); am; am &= am - 1) {
+            const int f = __ffs(am) - 1;
+            const float4* src = reinterpret_cast<const float4*>(logits + (t0 + f) * E);
+            for (int q = lane; q < E4; q += 32) reinterpret_cast<float4*>(ring)[q] = __ldg(src + q);
+            const unsigned hb = __shfl_sync(0xffffffffu, kb & hi_mask, f);
+            __syncwarp();
+            unsigned ok[KM];
+            int above = 0;                     // winners above the bucket (the list's first ones)
+#pragma unroll
+            for (int j = 0; j < KM; ++j) {
+                ok[j] = 0u;
+                if (j < k && (L[j] & hi_mask) > hb) above = j + 1;
+            }
+            if (lane == f) {
+#pragma unroll
+                for (int j = 0; j < KM; ++j)
+                    if (j >= above) bi[j] = -1;
+            }
+            for (int e0b = 0; e0b < E; e0b += 32) {
+                const int e = e0b + lane;
+                const float l = e < E ? ring[e] : 0.0f;
+                const bool in = e < E && l == l && (float_order_key(l) & hi_mask) == hb;
+                unsigned bm = __ballot_sync(0xffffffffu, in);
+                if (lane == f) {
+                    while (bm) {               // in expert order: strictly better displaces
+                        const int i = __ffs(bm) - 1;
+                        bm &= bm - 1;
+                        unsigned u = float_order_key(ring[e0b + i]);
+                        int ue = e0b + i;
+                        bool placed = false;
+#pragma unroll
+                        for (int j = 0; j < KM; ++j) {
+                            if (j >= above && (placed || u > ok[j])) {
+                                placed = true;
+                                const unsigned tu = ok[j];
+                                const int te = bi[j];
+                                ok[j] = u;
+                                bi[j] = ue;
+                                u = tu;
+                                ue = te;
+                            }
+                        }
+                    }
+                }
+            }
+            if (lane == f) {
+#pragma unroll
+                for (int j = 0; j < KM; ++j)
+                    if (j >= above) bv[j] = (j < k && bi[j] >= 0) ? ring[bi[j]] : -INFINITY;
+            }
+            __syncwarp();                      // the ring may be refilled
+        }
         if (t < T) {
+            // winners of one bucket are in expert order: put them in logit order
+            bool share = false;
+#pragma unroll
+            for (int j = 1; j < KM; ++j)
+                if (j < k && bi[j] >= 0 && ((float_order_key(bv[j]) ^ float_order_key(bv[j - 1])) & hi_mask) == 0u)
+                    share = true;
+            if (share) {
+#pragma unroll
+                for (int a = 1; a < KM; ++a) {
+#pragma unroll
+                    for (int b = a; b > 0; --b) {
+                        if (b < k && bi[b] >= 0 && float_order_key(bv[b]) > float_order_key(bv[b - 1])) {
+                            const float tv = bv[b];
+                            bv[b] = bv[b - 1];
+                            bv[b - 1] = tv;
+                            const int ti = bi[b];
+                            bi[b] = bi[b - 1];
+                            bi[b - 1] = ti;
+                        }
+                    }
+                }
+            }
             const float m = bv[0];
             float ej[KM];
 #pragma unroll
             for (int j = 0; j < KM; ++j) ej[j] = j < k ? exp_diff(bv[j], m) : 0.0f;
-            if (norm_topk) {
+            if (NORM) {
                 s = 0.0;
 #pragma unroll
                 for (int j = 0; j < KM; ++j) s += (double)ej[j];
@@ -1048,15 +1216,21 @@ extern "C" moe_status moe_route_topk(const float* logits, int T, int E, int k, i
     if (blocks > 148 * 16) blocks = 148 * 16;
     const int nv = (E + 31) / 32;
     if (E % 4 == 0 && k <= 8 && ((uintptr_t)logits & 15) == 0 && use_rows_variant(T, k)) {
-        for (auto fn : {route_topk_rows_kernel<1>, route_topk_rows_kernel<2>, route_topk_rows_kernel<4>,
-                        route_topk_rows_kernel<8>})
+        for (auto fn : {route_topk_rows_kernel<1, false>, route_topk_rows_kernel<2, false>,
+                        route_topk_rows_kernel<4, false>, route_topk_rows_kernel<8, false>,
+                        route_topk_rows_kernel<1, true>, route_topk_rows_kernel<2, true>,
+                        route_topk_rows_kernel<4, true>, route_topk_rows_kernel<8, true>})
             if (!set_smem_limit((const void*)fn, kRowSmem)) return MOE_ERR_CUDA;
         const long long warps = ((long long)T + 31) / 32;
         long long rb = (warps + kRowWarps - 1) / kRowWarps;
         const int rblocks = (int)(rb < 148 * 8 ? rb : 148 * 8);
-#define MOE_TOPKR_CASE(KM)                                                                              \
-    (void)launch_pdl(route_topk_rows_kernel<KM>, rblocks, 32 * kRowWarps, kRowSmem, s, logits, T, E, k, norm_topk, expert_idx, \
-                                                                         gate)
+        int kbits = 0;                                   // bits that hold an expert index
+        while ((1 << kbits) < E) ++kbits;
+#define MOE_TOPKR_CASE(KM)                                                                                      \
+    (void)(norm_topk ? launch_pdl(route_topk_rows_kernel<KM, true>, rblocks, 32 * kRowWarps, kRowSmem, s, logits, \
+                                  T, E, k, kbits, expert_idx, gate)                                             \
+                     : launch_pdl(route_topk_rows_kernel<KM, false>, rblocks, 32 * kRowWarps, kRowSmem, s, logits, \
+                                  T, E, k, kbits, expert_idx, gate))
         if (k <= 1) MOE_TOPKR_CASE(1);
         else if (k <= 2) MOE_TOPKR_CASE(2);
         else if (k <= 4) MOE_TOPKR_CASE(4);

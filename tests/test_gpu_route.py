@@ -66,6 +66,40 @@ def test_topk_concentrated_and_sorted_rows(topk_kind):
         check_topk(np.tile(np.arange(E, dtype=np.float32), (T, 1)), 8)
 
 
+def test_topk_near_ties_in_the_last_bits(topk_kind):
+    """Logits that differ in their last few bits: at the k-th / (k+1)-th
+    boundary (the thread-per-token kernel ranks those rows again with full
+    comparisons), among the winners (put back in exact order), and rows of
+    values a few hundred units in the last place apart."""
+    rng = np.random.default_rng(5)
+    for E, k in ((256, 8), (64, 6), (128, 4)):
+        T = 600
+        x = synth.normal_f32(14, 1, (T, E), 0.0, 1.0).copy()
+        order = np.argsort(-x, axis=1, kind="stable")
+        rows = np.arange(T)
+        kth = x[rows, order[:, k - 1]]
+        bits = kth.view(np.uint32).astype(np.int64)
+        one_ulp_down = np.where(kth > 0, bits - 1, bits + 1).astype(np.uint32).view(np.float32)
+        a = rows % 3 == 0                      # the (k+1)-th one unit below the k-th
+        x[rows[a], order[a, k]] = one_ulp_down[a]
+        b = rows % 3 == 1                      # the (k+1)-th equal to the k-th
+        x[rows[b], order[b, k]] = kth[b]
+        top = x[rows, order[:, 0]]             # the 2nd best one unit below the best
+        tb = top.view(np.uint32).astype(np.int64)
+        x[rows, order[:, 1]] = np.where(top > 0, tb - 1, tb + 1).astype(np.uint32).view(np.float32)
+        check_topk(x, k)
+        check_topk(x, k, True)
+    for v0 in (1.0, -3.0):
+        base = np.float32(v0).view(np.uint32)
+        x = (base + rng.integers(0, 600, size=(300, 256)).astype(np.uint32)).view(np.float32)
+        check_topk(x, 8)
+    # masked experts (-inf) with more than k finite logits left per row
+    x = synth.normal_f32(15, 1, (500, 64), 0.0, 1.0).copy()
+    x[:, 16:] = -np.inf
+    check_topk(x, 8)
+    check_topk(x, 8, True)
+
+
 @pytest.mark.parametrize("E,k,norm", [(256, 8, True), (64, 6, False), (8, 2, False), (128, 1, False)])
 def test_topk_large_T_default_choice(E, k, norm):
     """T large enough for the thread-per-token kernel to be the default."""
