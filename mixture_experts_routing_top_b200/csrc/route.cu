@@ -949,15 +949,16 @@ __global__ void __launch_bounds__(1024) ec_select_bins_kernel(const uint16_t* __
     const int gper = (ngroups + nw - 1) / nw;
     const int g0 = min(wid * gper, ngroups), g1 = min(g0 + gper, ngroups);
     if (mode != 2) {
-        // count the warp's tokens in bins before the boundary bin (and in it
+        // mark the warp's tokens in bins before the boundary bin (and in it
         // when it is taken whole); list the boundary bin's tokens
-        int mine = 0;
         for (int g = g0; g < g1; ++g) {
             const unsigned pr = bs2[32 * g + lane];
             const int t = 64 * g + 2 * lane;
             const int bA = (int)(pr & 0xFFFFu), bB = (int)(pr >> 16);
             const bool okA = t < T, okB = t + 1 < T;
-            mine += (okA && (bA < bstar || (mode == 0 && bA == bstar))) + (okB && (bB < bstar || (mode == 0 && bB == bstar)));
+            // tokens before the boundary bin (and in it when it is taken whole) are chosen
+            if (okA && (bA < bstar || (mode == 0 && bA == bstar))) atomicOr(&chosen[t >> 5], 1u << (t & 31));
+            if (okB && (bB < bstar || (mode == 0 && bB == bstar))) atomicOr(&chosen[(t + 1) >> 5], 1u << ((t + 1) & 31));
             if (mode == 1) {
                 const bool inA = okA && bA == bstar, inB = okB && bB == bstar;
                 const unsigned mA = __ballot_sync(0xffffffffu, inA), mB = __ballot_sync(0xffffffffu, inB);
@@ -974,8 +975,6 @@ __global__ void __launch_bounds__(1024) ec_select_bins_kernel(const uint16_t* __
                 }
             }
         }
-        mine = warp_sum(mine);
-        if (lane == 0) w_tie[wid] = mine;             // tokens before the boundary bin, per warp
         __syncthreads();
         if (mode == 1) {
             // the listed tokens' exact keys, all loads at once, then pairwise ranks
@@ -990,39 +989,32 @@ __global__ void __launch_bounds__(1024) ec_select_bins_kernel(const uint16_t* __
                     const unsigned long long kj = ckey[j];
                     rank += (kj > k0 || (kj == k0 && ctok[j] < t)) ? 1 : 0;
                 }
-                if (rank < need) {
-                    atomicOr(&chosen[t >> 5], 1u << (t & 31));
-                    atomicAdd(&w_sel[min((t >> 6) / max(gper, 1), nw - 1)], 1);   // the owning warp
-                }
+                if (rank < need) atomicOr(&chosen[t >> 5], 1u << (t & 31));
             }
             __syncthreads();
         }
-        int out_base = 0;
-        for (int q = 0; q < wid; ++q) out_base += w_tie[q] + w_sel[q];
-        for (int g = g0; g < g1; ++g) {
-            const unsigned pr = bs2[32 * g + lane];
-            const int t = 64 * g + 2 * lane;
-            const int bA = (int)(pr & 0xFFFFu), bB = (int)(pr >> 16);
-            const unsigned cw = (mode == 1 && t < T) ? chosen[t >> 5] : 0u;
-            const bool selA = t < T && (bA < bstar || (bA == bstar && (mode == 0 || ((cw >> (t & 31)) & 1u))));
-            const bool selB = t + 1 < T && (bB < bstar || (bB == bstar && (mode == 0 || ((cw >> ((t + 1) & 31)) & 1u))));
-            const unsigned mA = __ballot_sync(0xffffffffu, selA), mB = __ballot_sync(0xffffffffu, selB);
-            int pos = out_base + __popc(mA & lt) + __popc(mB & lt);
-            if (selA) {
-                ec_token[(long long)e * C + pos] = t;
-                atomicOr(&tokmask[(long long)t * mask_words + (e >> 5)], 1u << (e & 31));
+        // the chosen tokens in token order: each thread takes consecutive words
+        // of the membership bits, a block scan of their counts gives its first
+        // output place
+        const int wpt = (nwords + (int)blockDim.x - 1) / (int)blockDim.x;
+        const int w0 = min((int)threadIdx.x * wpt, nwords), w1 = min(w0 + wpt, nwords);
+        int cnt = 0;
+        for (int w = w0; w < w1; ++w) cnt += __popc(chosen[w]);
+        int total;
+        int pos = block_exclusive_scan(cnt, &total, sh);
+        for (int w = w0; w < w1; ++w) {
+            unsigned m = chosen[w];
+            while (m) {
+                const int t = 32 * w + __ffs(m) - 1;
+                m &= m - 1;
+                if (pos < C) {                 // exactly C bits are set
+                    const long long r = (long long)e * C + pos;
+                    ec_token[r] = t;
+                    atomicOr(&tokmask[(long long)t * mask_words + (e >> 5)], 1u << (e & 31));
+                    ec_gate[r] = (float)exp(key_of(t));
+                }
                 ++pos;
             }
-            if (selB) {
-                ec_token[(long long)e * C + pos] = t + 1;
-                atomicOr(&tokmask[(long long)(t + 1) * mask_words + (e >> 5)], 1u << (e & 31));
-            }
-            out_base += __popc(mA) + __popc(mB);
-        }
-        __syncthreads();
-        for (int j = threadIdx.x; j < C; j += blockDim.x) {
-            const long long r = (long long)e * C + j;
-            ec_gate[r] = (float)exp(key_of(ec_token[r]));
         }
         return;
     }
