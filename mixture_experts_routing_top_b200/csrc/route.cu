@@ -1110,7 +1110,12 @@ ec_count_scan_kernel(const unsigned* __restrict__ tokmask, int T, int mask_words
     pdl_wait();
     auto count = [&](long long t) {
         int n = 0;
-        for (int w = 0; w < mask_words; ++w) n += __popc(tokmask[t * mask_words + w]);
+        if (mask_words == 4) {                 // E in (96, 128]: one 16-byte load per token
+            const uint4 u = reinterpret_cast<const uint4*>(tokmask)[t];
+            n = __popc(u.x) + __popc(u.y) + __popc(u.z) + __popc(u.w);
+        } else {
+            for (int w = 0; w < mask_words; ++w) n += __popc(tokmask[t * mask_words + w]);
+        }
         return n;
     };
     int cached[kCache];
@@ -1170,10 +1175,20 @@ __global__ void ec_fill_kernel(const int32_t* __restrict__ ec_token, int T, int 
     int e = (int)(r / C);
     int t = ec_token[r];
     if (gates) ec_gate[r] = (float)exp((double)logits[(long long)t * E + e] - lse[t]);
-    const unsigned* m = tokmask + (long long)t * mask_words;
     int below = 0;
-    for (int w = 0; w < (e >> 5); ++w) below += __popc(m[w]);
-    below += __popc(m[e >> 5] & ((1u << (e & 31)) - 1u));
+    if (mask_words == 4) {
+        const uint4 u = reinterpret_cast<const uint4*>(tokmask)[t];
+        const unsigned wv[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            if (w < (e >> 5)) below += __popc(wv[w]);
+            else if (w == (e >> 5)) below += __popc(wv[w] & ((1u << (e & 31)) - 1u));
+        }
+    } else {
+        const unsigned* m = tokmask + (long long)t * mask_words;
+        for (int w = 0; w < (e >> 5); ++w) below += __popc(m[w]);
+        below += __popc(m[e >> 5] & ((1u << (e & 31)) - 1u));
+    }
     tok_row[tok_ptr[t] + below] = (int32_t)r;
 }
 
