@@ -97,7 +97,8 @@ moe_status moe_selftest_bounded_wait(int arrive, long long limit_ns, int32_t* re
 
 /* TopKRouter ("Routing Mechanisms: Top-K vs Expert Choice"): softmax over
  * each token's E router logits and its k best experts.
- *   logits      [T, E] fp32 (finite values; NaN gives unspecified experts)
+ *   logits      [T, E] fp32 (finite values, or -inf for a masked expert
+ *               while at least k are finite; NaN gives unspecified experts)
  *   expert_idx  [T, k] int32 out: slot j = the (j+1)-th largest logit;
  *               equal logits: the lower expert index ranks first
  *   gate        [T, k] fp32 out: softmax probability of that expert; with
