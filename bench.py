@@ -226,6 +226,17 @@ def workload_config(w, world):
     return cfg
 
 
+def held_under_power_cap(elapsed_ms, clk):
+    """True when a tensor-bound stage ran in the sustained regime: a timed
+    region of a second or more, or a clock record whose median SM clock sat
+    below 90 % of its maximum with the power cap among the reasons."""
+    if elapsed_ms >= 1000.0:
+        return True
+    if not clk or not clk.get("sm_mhz") or not clk.get("sm_max_mhz"):
+        return False
+    return "sw_power_cap" in (clk.get("reasons") or []) and clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"]
+
+
 def throughput(world, tokens_per_rank, steps, max_elapsed_ms):
     """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
     return world * tokens_per_rank * steps / (max_elapsed_ms / 1e3)
@@ -821,10 +832,7 @@ def run_libmoe(args, w, rank, world, local_rank):
         # figure (cuBLAS timed alone) is its peak; in a region of a second or more, or once the power cap
         # has pulled the SM clock well below its maximum, the seconds-long sustained figure is.  The
         # other fraction is kept beside it.
-        held = (elapsed_ms >= 1000.0 or
-                bool(clk and clk.get("sm_mhz") and clk.get("sm_max_mhz") and
-                     "sw_power_cap" in (clk.get("reasons") or []) and clk["sm_mhz"] < 0.9 * clk["sm_max_mhz"]))
-        sustained = held and "bf16_tflops_sustained" in pk
+        sustained = held_under_power_cap(elapsed_ms, clk) and "bf16_tflops_sustained" in pk
         peak = pk["bf16_tflops_sustained"] if sustained else pk["bf16_tflops"]
         ach = report[dom]["TFLOP/s"]
         roof = {"bound": "tensor", "stage": dom, "achieved": ach, "peak": peak, "unit": "TFLOP/s",
