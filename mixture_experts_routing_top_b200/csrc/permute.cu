@@ -317,9 +317,24 @@ __global__ void __launch_bounds__(kIdxThreads) perm_group_heads_kernel(
     for (long long sl = s0 + threadIdx.x; sl < s1; sl += blockDim.x) keys_s[sl - s0] = idx[sl];
     for (int e = threadIdx.x; e < E; e += blockDim.x) goe_s[e] = goe[e];
     if (nodrop) {
-        if (blockIdx.x == 0)
+        if (fused) {
+            // nothing drops, so each expert's count is its total over the
+            // blocks: every block sums the rows of its share of the experts
+            // (a warp per row), so that no one block reads the whole matrix
+            const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+            const int k0 = (int)((long long)E * blockIdx.x / gridDim.x);
+            const int k1 = (int)((long long)E * (blockIdx.x + 1) / gridDim.x);
+            for (int key = k0 + wid; key < k1; key += nw) {
+                int tot = 0;
+                for (int i = lane; i < nblk; i += 32) tot += ecnt[(long long)key * nblk + i];
+                tot = warp_sum(tot);
+                if (lane == 0) counts[key] = tot;
+            }
+            if (blockIdx.x == 0 && threadIdx.x == 0) *dropped = 0;
+        } else if (blockIdx.x == 0) {
             block_scan_prologue(fused, ecnt, ebase, nullptr, E, nblk, cap, base_s, off_s, counts, nullptr, dropped, 0,
                                 true);
+        }
         __syncthreads();
         for (long long sl = s0 + threadIdx.x; sl < s1; sl += blockDim.x) {
             const int e = keys_s[sl - s0];
