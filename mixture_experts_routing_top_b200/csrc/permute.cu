@@ -294,7 +294,8 @@ __device__ void block_scan_prologue(bool fused, const int32_t* __restrict__ cnt,
 // -2 - j for a kept slot whose head is slot j of the same token, -1 for a
 // dropped slot.  With a capacity of at least T k no slot can be dropped
 // (`nodrop`): every valid slot is kept, the expert ranks are not needed, and
-// only the writer block reads the count matrix (for counts and dropped).
+// the count matrix is read only for counts (each expert's total, every block
+// summing the rows of its share of the experts) and dropped (zero).
 __global__ void __launch_bounds__(kIdxThreads) perm_group_heads_kernel(
     const int32_t* __restrict__ idx, const int32_t* __restrict__ goe, int T, int k, int E, int G, int nblk, int tb, int fused,
     const int32_t* __restrict__ ecnt, const int32_t* __restrict__ ebase, long long cap, int nodrop,
